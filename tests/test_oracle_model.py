@@ -1,0 +1,288 @@
+"""Pins of the oracle's forward pass against what the pages and the mathematics fix."""
+import cmath
+import dataclasses
+import math
+
+import numpy as np
+import pytest
+
+import synth
+from conftest import read_golden
+from oracle import model, tables
+
+
+def golden(name):
+    d = dict(l.split() for l in read_golden("published_counts.txt"))
+    return float(d[name])
+
+
+def widths60():
+    return tables.band_tables(44100, 2048, 60)["widths"]
+
+
+# ---------------------------------------------------------------- module wiring
+def test_param_counts_match_pages():
+    w = widths60()
+    assert model.param_count(synth.VOCALS, w) == golden("params_vocals")
+    assert model.param_count(synth.DEUX, w) == golden("params_deux")
+    # the deux mask head alone
+    no_head = model.param_count(dataclasses.replace(synth.DEUX, num_stems=0), w)
+    assert model.param_count(synth.DEUX, w) - no_head == golden("params_deux_mask_head")
+    # the vocals trunk (both axes, all blocks): 23.7 M
+    base = dataclasses.replace(synth.VOCALS, depth=0)
+    trunk = model.param_count(synth.VOCALS, w) - model.param_count(base, w)
+    assert round(trunk / 1e6, 1) == golden("trunk_params_vocals_millions")
+
+
+def test_weight_table_matches_param_count():
+    # the generator's named shapes add up to the same count (shapes of [1536,384],
+    # [1536,1536], [56,1536], [1040,1536] as the pages print)
+    w = widths60()
+    shapes = dict(synth.weight_shapes(synth.VOCALS, w))
+    assert sum(int(np.prod(s)) for s in shapes.values()) == golden("params_vocals")
+    p = "mask_estimators.0.to_freqs."
+    assert shapes[p + "0.0.0.weight"] == (1536, 384)
+    assert shapes[p + "0.0.2.weight"] == (1536, 1536)
+    assert shapes[p + "0.0.4.weight"] == (56, 1536)
+    assert shapes[p + "59.0.4.weight"] == (1040, 1536)
+
+
+def test_mac_accounting_matches_pages():
+    m = model.mac_count(synth.VOCALS, widths60(), 1, 801)
+    for term in ("qkv", "ff1", "ff2"):
+        assert round(m["per_axis"][term] / 1e9, 2) == golden("macs_per_term_G")
+    assert round(m["trunk"] / 1e9, 1) == golden("macs_trunk_G")
+    assert round(m["attn_time"] / 1e9, 2) == golden("macs_attn_time_G")
+    assert round(m["attn_band"] / 1e9, 2) == golden("macs_attn_band_G")
+    D, A = 384, 512
+    assert 2 * 60 * A == golden("macs_band_attn_per_token")
+    assert D * 4 * D == golden("macs_ffn_projection_per_token")
+    # 3.102 TFLOP per chunk: the page's total stands within 0.5 % of the term sum
+    assert 2 * m["total"] / 1e12 == pytest.approx(golden("tflop_per_chunk"), rel=5e-3)
+
+
+def test_frames_of_8s_chunk():
+    spec = synth.stft_stereo(np.zeros((2, 352800)), 2048, 441)
+    assert spec.shape == (2, 1025, int(golden("frames_8s")))
+
+
+# ---------------------------------------------------------------- RMSNorm
+def test_rmsnorm_properties():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((5, 37))
+    g = np.ones(37)
+    y = model.rms_norm(x, g)
+    assert np.allclose(np.linalg.norm(y, axis=1), math.sqrt(37))      # ||N(x)|| = sqrt(d)
+    assert np.allclose(model.rms_norm(3.7 * x, g), y)                   # scale invariant
+    assert not np.allclose(model.rms_norm(x + 1.0, g), y)               # not mean invariant
+    z = model.rms_norm(np.zeros((2, 8)), np.ones(8))
+    assert np.all(z == 0)                                               # zero row -> 0
+    gam = rng.standard_normal(37)
+    assert np.allclose(model.rms_norm(x, gam), y * gam)
+
+
+def test_gelu_erf_values():
+    # GELU(x) = x * Phi(x); Phi(1) = 0.841344746068542948..., Phi(2) = 0.977249868051820...
+    assert model.gelu(np.array(1.0)) == pytest.approx(0.8413447460685429, abs=1e-15)
+    assert model.gelu(np.array(-1.0)) == pytest.approx(-0.15865525393145707, abs=1e-15)
+    assert model.gelu(np.array(2.0)) == pytest.approx(2 * 0.9772498680518208, abs=1e-14)
+    assert model.gelu(np.array(0.0)) == 0.0
+
+
+# ---------------------------------------------------------------- rotary embedding
+def test_rope_equals_complex_rotation():
+    # pair (x_2i, x_2i+1) as the complex number x_2i + i x_2i+1, multiplied by e^{i p theta^(-2i/d)}
+    rng = np.random.default_rng(1)
+    n, dh, theta = 7, 8, 10000.0
+    x = rng.standard_normal((n, dh))
+    y = model.rope(x, theta)
+    for p in range(n):
+        for i in range(dh // 2):
+            z = complex(x[p, 2 * i], x[p, 2 * i + 1]) * cmath.exp(1j * p * theta ** (-2 * i / dh))
+            assert y[p, 2 * i] == pytest.approx(z.real, abs=1e-12)
+            assert y[p, 2 * i + 1] == pytest.approx(z.imag, abs=1e-12)
+
+
+def test_rope_norm_and_relative_position():
+    rng = np.random.default_rng(2)
+    n, dh = 12, 16
+    q = rng.standard_normal((n, dh))
+    k = rng.standard_normal((n, dh))
+    rq = model.rope(q, 10000.0)
+    assert np.allclose(np.linalg.norm(rq.reshape(n, -1, 2), axis=-1),
+                       np.linalg.norm(q.reshape(n, -1, 2), axis=-1))      # per pair norm kept
+    assert np.allclose(rq[0], q[0])                                       # position 0 is identity
+    # <R_m q, R_n k> depends on m - n only: same vectors placed at (m, n) and (m+s, n+s)
+    qv, kv = q[0], k[0]
+    def at(vec, p):
+        tmp = np.zeros((p + 1, dh)); tmp[p] = vec
+        return model.rope(tmp, 10000.0)[p]
+    a = at(qv, 3) @ at(kv, 1)
+    b = at(qv, 9) @ at(kv, 7)
+    assert a == pytest.approx(b, abs=1e-12)
+    # interleaved pairs to halves is one permutation of q's and k's features: q.k unchanged
+    perm = np.concatenate([np.arange(0, dh, 2), np.arange(1, dh, 2)])
+    rk = model.rope(k, 10000.0)
+    assert np.allclose(rq[:, perm] @ rk[:, perm].T, rq @ rk.T)
+
+
+# ---------------------------------------------------------------- attention
+def brute_attend(q, k, v):
+    n, dh = len(q), len(q[0])
+    out = []
+    for i in range(n):
+        s = [sum(q[i][d] * k[j][d] for d in range(dh)) / math.sqrt(dh) for j in range(n)]
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        z = sum(e)
+        out.append([sum(e[j] / z * v[j][d] for j in range(n)) for d in range(len(v[0]))])
+    return np.array(out)
+
+
+def test_attend_brute_force_and_properties():
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((6, 4)) for _ in range(3))
+    assert np.allclose(model.attend(q, k, v), brute_attend(q.tolist(), k.tolist(), v.tolist()), atol=1e-13)
+    s = model.softmax(rng.standard_normal((5, 9)) * 30)
+    assert np.allclose(s.sum(-1), 1.0)
+    # n = 1: output is v
+    assert np.allclose(model.attend(q[:1], k[:1], v[:1]), v[:1])
+    # splitting the queries is exact
+    full = model.attend(q, k, v)
+    assert np.allclose(np.concatenate([model.attend(q[:2], k, v), model.attend(q[2:], k, v)]), full)
+
+
+def brute_attention_layer(x, w, h, dh, theta):
+    """Scalar loops over the definition: pre-norm, qkv features (which, head, d), RoPE on
+    q and k, softmax attention per head, sigmoid gate per head from the normed input,
+    heads concatenated head-major, output projection."""
+    n, D = x.shape
+    g = w["norm.gamma"]
+    a = []
+    for t in range(n):
+        nrm = math.sqrt(sum(x[t, j] ** 2 for j in range(D)))
+        a.append([x[t, j] / max(nrm, 1e-12) * math.sqrt(D) * g[j] for j in range(D)])
+    Wq = w["to_qkv.weight"]
+    def proj(which, head, t):
+        return [sum(Wq[(which * h + head) * dh + d, j] * a[t][j] for j in range(D)) for d in range(dh)]
+    def rot(vec, p):
+        out = list(vec)
+        for i in range(dh // 2):
+            z = complex(vec[2 * i], vec[2 * i + 1]) * cmath.exp(1j * p * theta ** (-2 * i / dh))
+            out[2 * i], out[2 * i + 1] = z.real, z.imag
+        return out
+    cat = [[0.0] * (h * dh) for _ in range(n)]
+    for head in range(h):
+        q = [rot(proj(0, head, t), t) for t in range(n)]
+        k = [rot(proj(1, head, t), t) for t in range(n)]
+        v = [proj(2, head, t) for t in range(n)]
+        o = brute_attend(q, k, v)
+        for t in range(n):
+            gate = sum(w["to_gates.weight"][head, j] * a[t][j] for j in range(D)) + w["to_gates.bias"][head]
+            sg = 1 / (1 + math.exp(-gate))
+            for d in range(dh):
+                cat[t][head * dh + d] = o[t][d] * sg
+    Wo = w["to_out.0.weight"]
+    return np.array([[sum(Wo[i, j] * cat[t][j] for j in range(h * dh)) for i in range(D)] for t in range(n)])
+
+
+def test_attention_layer_brute_force():
+    rng = np.random.default_rng(4)
+    n, D, h, dh = 5, 6, 2, 4
+    w = {"norm.gamma": 1 + 0.1 * rng.standard_normal(D),
+         "to_qkv.weight": rng.standard_normal((3 * h * dh, D)),
+         "to_gates.weight": rng.standard_normal((h, D)), "to_gates.bias": rng.standard_normal(h),
+         "to_out.0.weight": rng.standard_normal((D, h * dh))}
+    x = rng.standard_normal((1, n, D))
+    got = model.attention(x, w, h, dh, 10000.0)[0]
+    assert np.allclose(got, brute_attention_layer(x[0], w, h, dh, 10000.0), atol=1e-11)
+
+
+def test_transformer_output_norm():
+    rng = np.random.default_rng(5)
+    cfg = synth.TINY
+    widths = tables.band_tables(44100, 256, 8)["widths"]
+    W = synth.make_weights(cfg, widths, seed=0, fp16=False)
+    tw = {k[len("layers.0.0."):]: v.astype(np.float64) for k, v in W.items() if k.startswith("layers.0.0.")}
+    tw["norm.gamma"] = np.ones(cfg.dim)
+    y = model.transformer(rng.standard_normal((3, 5, cfg.dim)), tw, cfg.heads, cfg.dim_head, 10000.0)
+    assert np.allclose(np.linalg.norm(y, axis=-1), math.sqrt(cfg.dim))
+
+
+# ---------------------------------------------------------------- mask head and average
+def test_glu_zero_gate_is_half_value():
+    cfg = synth.TINY
+    tab = tables.band_tables(44100, 256, 8)
+    W = {k: v.astype(np.float64) for k, v in synth.make_weights(cfg, tab["widths"], fp16=False).items()}
+    for k, d in enumerate(tab["widths"]):
+        p = f"mask_estimators.0.to_freqs.{k}.0.4."
+        W[p + "weight"][d:] = 0
+        W[p + "bias"][d:] = 0
+    X = np.random.default_rng(6).standard_normal((4, 8, cfg.dim))
+    m = model.mask_estimator(X, tab, W)
+    # reference value half: y = W4 tanh(W2 tanh(W0 x + b0) + b2) + b4 with the first d rows
+    off = 0
+    for k, d in enumerate(tab["widths"]):
+        p = f"mask_estimators.0.to_freqs.{k}.0."
+        h1 = np.tanh(X[:, k] @ W[p + "0.weight"].T + W[p + "0.bias"])
+        assert np.all(np.abs(h1) < 1)
+        h2 = np.tanh(h1 @ W[p + "2.weight"].T + W[p + "2.bias"])
+        val = h2 @ W[p + "4.weight"][:d].T + W[p + "4.bias"][:d]
+        assert np.allclose(m[:, off:off + d], 0.5 * val)
+        off += d
+
+
+def test_overlap_average_partition_of_unity_and_one_hot():
+    tab = tables.band_tables(44100, 2048, 60)
+    T, R = 3, 2050
+    m = np.full((T, int(tab["widths"].sum())), 0.37)
+    assert np.allclose(model.overlap_average(m, tab, R), 0.37)
+    # one band's features at 1, all else 0: its rows get 1 / (bands over the bin)
+    k = 20
+    off = np.concatenate([[0], np.cumsum(tab["widths"])])
+    m = np.zeros_like(m)
+    m[:, off[k]:off[k + 1]] = 1.0
+    out = model.overlap_average(m, tab, R)
+    for f in range(tab["first_bin"][k], tab["last_bin"][k] + 1):
+        assert np.allclose(out[2 * f: 2 * f + 2], 1.0 / tab["bands_per_bin"][f])
+    assert out[: 2 * tab["first_bin"][k]].sum() == 0
+    assert out[2 * tab["last_bin"][k] + 2:].sum() == 0
+
+
+# ---------------------------------------------------------------- whole forward
+def tiny_case(B=1, T=32, seed=2):
+    cfg = synth.TINY
+    widths = tables.band_tables(44100, 256, 8)["widths"]
+    W = synth.make_weights(cfg, widths, seed=0, fp16=False)
+    x = synth.make_stft_repr(cfg, B, T, seed=seed)
+    return cfg, W, x
+
+
+def test_forward_shapes_and_batching():
+    cfg, W, x = tiny_case(B=2, T=9)
+    out, st = model.forward(x, cfg, W, return_stages=True)
+    assert out.shape == (2, 258, 9, 2)
+    assert st[0]["band_split"].shape == (9, 8, 64)
+    assert st[0]["mask0"].shape == (9, 828)
+    for b in range(2):
+        assert np.allclose(model.forward(x[b:b + 1], cfg, W)[0], out[b])
+
+
+def test_time_transformer_keeps_bands_independent():
+    # before the band transformer, band k's sequence depends on band k's input only
+    cfg, W, x = tiny_case(T=6)
+    _, st = model.forward(x, cfg, W, return_stages=True)
+    tab = tables.band_tables(44100, 256, 8)
+    x2 = x.copy()
+    x2[0, : 2 * tab["first_bin"][1]] *= -1.3        # bins below band 1 belong to band 0 only
+    _, st2 = model.forward(x2, cfg, W, return_stages=True)
+    a, b = st[0]["layer0.time"], st2[0]["layer0.time"]
+    assert not np.allclose(a[:, 0], b[:, 0])
+    assert np.allclose(a[:, 1:], b[:, 1:])
+
+
+def test_forward_fp32_close_to_fp64():
+    cfg, W, x = tiny_case()
+    a = model.forward(x, cfg, W, dtype=np.float64)
+    b = model.forward(x, cfg, W, dtype=np.float32)
+    assert np.abs(a - b).max() / np.abs(a).max() < 1e-4
