@@ -1,0 +1,66 @@
+// Declarations of the tcgen05 GEMM (k_gemm_tc.cu) used by the fp16 schedule.
+#pragma once
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace mrf {
+
+// One group (a band of the mask head, or the single group of a trunk GEMM):
+// C[m, n] = sum_k A[m, k] W[n, k] for m < M, n < N.
+struct GemmGroup {
+  int N;             // output columns of the group
+  int n_tiles;       // ceil(N / BN)
+  int n_tile_start;  // prefix sum of n_tiles over the previous groups
+  int a_off;         // A: first row of the group (mode 0) or the group's coordinate (mode 1)
+  int b_row_off;     // first row of the group's weight in the stacked weight matrix
+  int out_off;       // epilogue output offset of the group
+  int bias_off;      // offset of the group's bias
+  int pad;
+};
+
+enum GemmEpi : int {
+  kTcQkv = 0,     // RoPE + scatter q, k, v (fp16, attention layout) + sigmoid gates
+  kTcResid = 1,   // X += acc (+ bias); writes X fp32, X fp16, row sum of squares
+  kTcGelu = 2,    // out = gelu(acc * rowscale + bias) fp16
+  kTcTanh = 3,    // out = tanh(acc + bias) fp16 (group-strided)
+  kTcGlu = 4,     // interleaved (value, gate) pairs -> value * sigmoid(gate), fp32
+};
+
+struct GemmParams {
+  int M, K, BN, ngroups, total_n_tiles, a_mode, m_tiles;
+  const GemmGroup *groups;
+  unsigned *status;
+  // epilogue
+  const float *ss_in;       // row sums of squares giving the row scale 1 / max(sqrt(ss), eps); null: 1
+  const float *bias;
+  float *X;                 // fp32 residual [M, ld]
+  __half *Xh;               // fp16 copy of X
+  float *ss_out;            // row sums of squares (atomic partials)
+  int ld;
+  __half *out_h;            // fp16 output
+  float *out_f;             // fp32 output
+  int ldo;
+  long long out_group_stride;
+  // q, k, v scatter
+  __half *q, *k, *v;
+  float *gates;
+  const float2 *rope;
+  const float *gbias;
+  int B, T, nb, H, dh, A, axis, n_pad;
+};
+
+// Encode a 3D fp16 tensor map with a 128-byte swizzle and a (64, box1, box2) box.
+// dims/strides in elements; strides[0] is the stride of dim 1, strides[1] of dim 2.
+bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, unsigned long long d1,
+                   unsigned long long d2, unsigned long long s1, unsigned long long s2, unsigned box1,
+                   unsigned box2);
+
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 192;
+size_t gemm_smem_bytes();
+
+void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
+                    int grid, cudaStream_t st);
+
+}  // namespace mrf

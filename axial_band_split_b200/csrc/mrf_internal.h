@@ -1,0 +1,74 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "../../include/mrf.h"
+#include "tables.h"
+
+namespace mrf {
+
+// ------------------------------------------------------------------ device status word
+// Kernels with bounded waits write a nonzero code here instead of hanging or trapping.
+enum DeviceStatus : unsigned { kStatusOk = 0, kStatusTimeout = 1 };
+
+// ------------------------------------------------------------------ SIMT kernels (k_simt.cu)
+// Per-band descriptor of the band split and the mask head.
+struct BandDesc {
+  int width;      // d_in of the band
+  int feat_off;   // first feature of the band in the concatenated feature axis
+  int w_off;      // first element of the band's band-split weight [dim, width]
+  int w3_off;     // first element of the band's last mask layer [2*width, hidden] (fp32 path)
+};
+
+// X[(b*T + t)*nb + k, :] = W_k (x_k / max(|x_k|, eps)) + bias_k, gamma*sqrt(d_in) folded
+// into W_k.  Also writes an fp16 copy and the row sum of squares when given.
+void launch_band_split(const float *in, const int32_t *feat_row, const int32_t *feat_c,
+                       const BandDesc *bands, int nb, const float *w, const float *bias,
+                       int dim, int B, int T, int rows, float *X, __half *Xh, float *ss,
+                       cudaStream_t st, int max_width);
+
+enum SimtEpi : int {
+  kEpiStore = 0,      // C = acc (+ bias)
+  kEpiResidual = 1,   // C += acc (+ bias)
+  kEpiGelu = 2,       // C = gelu(acc + bias)
+  kEpiTanh = 3,       // C = tanh(acc + bias)
+  kEpiSigmoid = 4,    // C = sigmoid(acc + bias)
+  kEpiGlu = 5,        // value/gate halves of N: C[:, e] = v_e * sigmoid(g_e), N/2 outputs
+};
+
+// One group of a grouped fp32 GEMM: C[m, n] = sum_k A[m, k] * W[n, k] for m < M, n < N.
+struct SimtGroup {
+  long long a_off, w_off, c_off, bias_off;
+  int lda, ldc, N, pad;
+};
+void launch_gemm_f32(const float *A, const float *W, const float *bias, float *C,
+                     const SimtGroup *groups_dev, int ngroups, int M, int K, int max_n,
+                     int epi, cudaStream_t st);
+
+// y = x / max(|x|, eps) * gain (per column), rows of width D; y may alias x.
+void launch_rownorm_f32(const float *x, const float *gain, float *y, long long rows, int D,
+                        cudaStream_t st);
+
+// qkv [tok, 3*A] fp32 -> q, k, v [seq*heads, n, dh] with RoPE on q and k.
+// axis 0: sequences over time (seq = b*nb + band, pos = t); axis 1: over bands.
+void launch_rope_split_f32(const float *qkv, const float2 *rope, float *q, float *k, float *v,
+                           int B, int T, int nb, int heads, int dh, int axis, cudaStream_t st);
+
+// o[tok, head*dh + d] = gate[tok, head] * softmax(q k^T / sqrt(dh)) v
+void launch_attention_f32(const float *q, const float *k, const float *v, const float *gate,
+                          float *o, int B, int T, int nb, int heads, int dh, int axis,
+                          cudaStream_t st);
+
+// masks[b, r, t, c] = row_weight[r] * sum of the (<= 2) source features of (r, c)
+void launch_overlap_average(const float *m, int ldm, const int32_t *src0, const int32_t *src1,
+                            const float *row_weight, float *masks, int B, int T, int rows,
+                            cudaStream_t st);
+
+void launch_fill_f32(float *p, float v, long long n, cudaStream_t st);
+
+}  // namespace mrf

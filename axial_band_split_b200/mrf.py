@@ -1,0 +1,210 @@
+"""Python binding of libmrf (include/mrf.h): argument marshalling only.
+
+Every step of the forward runs in the library's CUDA kernels; PyTorch is used here for
+device memory and streams.  The binding raises if libmrf.so is missing or a call fails:
+there is no fallback path.
+
+    from axial_band_split_b200 import mrf
+    model = mrf.Model(cfg, weights, max_batch=1, max_frames=1100)   # weights: name -> ndarray
+    masks = model.forward(stft_repr)            # torch CUDA float32 [B, F*2, T, 2]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmrf.so")
+
+MRF_FP16 = 0
+MRF_FP32_DEBUG = 2
+STATUS = {0: "MRF_OK", -1: "MRF_EINVAL", -2: "MRF_ESHAPE", -3: "MRF_ENOMEM", -4: "MRF_ECUDA",
+          -5: "MRF_EUNSUPPORTED", -6: "MRF_ETIMEOUT", -7: "MRF_EWEIGHTS"}
+
+# every symbol include/mrf.h declares
+EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
+           "mrf_last_error", "mrf_band_tables", "mrf_set_timing", "mrf_kernel_times",
+           "mrf_set_graph", "mrf_launches_per_forward"]
+
+
+class MrfError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class mrf_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "sample_rate", "n_fft", "audio_channels", "num_bands", "dim", "depth", "heads", "dim_head",
+        "ff_mult", "mask_hidden", "mask_depth", "num_stems", "zero_dc", "max_batch", "max_frames")] + \
+        [("rope_theta", ctypes.c_float), ("compute", ctypes.c_int)]
+
+
+class mrf_tensor(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("dtype", ctypes.c_int), ("ndim", ctypes.c_int),
+                ("shape", ctypes.c_int64 * 4), ("host_data", ctypes.c_void_p)]
+
+
+class mrf_kernel_time(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int), ("ms", ctypes.c_double)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libmrf.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"{_LIB_PATH} is missing: run `python -m axial_band_split_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I, V = ctypes.c_void_p, ctypes.c_int, None
+        L.mrf_create.argtypes = [ctypes.POINTER(mrf_config), ctypes.POINTER(mrf_tensor), I, ctypes.POINTER(P)]
+        L.mrf_create.restype = I
+        L.mrf_forward.argtypes = [P, P, P, I, I, P]
+        L.mrf_forward.restype = I
+        L.mrf_forward_host.argtypes = [P, P, P, I, I, P]
+        L.mrf_forward_host.restype = I
+        L.mrf_sync_status.argtypes = [P, P]
+        L.mrf_sync_status.restype = I
+        L.mrf_destroy.argtypes = [P]
+        L.mrf_destroy.restype = V
+        L.mrf_last_error.argtypes = [P]
+        L.mrf_last_error.restype = ctypes.c_char_p
+        L.mrf_band_tables.argtypes = [ctypes.POINTER(mrf_config)] + [P] * 6
+        L.mrf_band_tables.restype = I
+        L.mrf_set_timing.argtypes = [P, I]
+        L.mrf_set_timing.restype = I
+        L.mrf_set_graph.argtypes = [P, I]
+        L.mrf_set_graph.restype = I
+        L.mrf_kernel_times.argtypes = [P, ctypes.POINTER(mrf_kernel_time), I, ctypes.POINTER(I)]
+        L.mrf_kernel_times.restype = I
+        L.mrf_launches_per_forward.argtypes = [P, I, I]
+        L.mrf_launches_per_forward.restype = I
+        _lib = L
+    return _lib
+
+
+def _check(status, handle=None):
+    if status != 0:
+        raise MrfError(status, lib().mrf_last_error(handle).decode(errors="replace"))
+
+
+def make_config(cfg, max_batch=1, max_frames=1100, compute=MRF_FP16):
+    """mrf_config from any object with the model fields (sample_rate, n_fft, ...)."""
+    c = mrf_config()
+    c.sample_rate, c.n_fft, c.audio_channels = cfg.sample_rate, cfg.n_fft, cfg.audio_channels
+    c.num_bands, c.dim, c.depth, c.heads, c.dim_head = cfg.num_bands, cfg.dim, cfg.depth, cfg.heads, cfg.dim_head
+    c.ff_mult, c.mask_hidden, c.mask_depth = cfg.ff_mult, cfg.dim * cfg.mask_hidden_mult, cfg.mask_depth
+    c.num_stems, c.zero_dc = cfg.num_stems, int(cfg.zero_dc)
+    c.max_batch, c.max_frames = max_batch, max_frames
+    c.rope_theta, c.compute = cfg.rope_theta, compute
+    return c
+
+
+def band_tables(cfg):
+    """The library's band tables for cfg: dict of numpy arrays (first_bin, last_bin, width,
+    feat_row, row_weight)."""
+    c = make_config(cfg)
+    n_feat = ctypes.c_int(0)
+    _check(lib().mrf_band_tables(ctypes.byref(c), None, None, None, None, None, ctypes.byref(n_feat)))
+    nb, rows = cfg.num_bands, (cfg.n_fft // 2 + 1) * cfg.audio_channels
+    out = {"first_bin": np.zeros(nb, np.int32), "last_bin": np.zeros(nb, np.int32),
+           "width": np.zeros(nb, np.int32), "feat_row": np.zeros(n_feat.value, np.int32),
+           "row_weight": np.zeros(rows, np.float32)}
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(lib().mrf_band_tables(ctypes.byref(c), ptr(out["first_bin"]), ptr(out["last_bin"]),
+                                 ptr(out["width"]), ptr(out["feat_row"]), ptr(out["row_weight"]), None))
+    return out
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+class Model:
+    """A created libmrf handle: weights on the device, workspace for max_batch x max_frames."""
+
+    def __init__(self, cfg, weights, max_batch=1, max_frames=1100, compute=MRF_FP16):
+        self.cfg = cfg
+        self.rows = (cfg.n_fft // 2 + 1) * cfg.audio_channels
+        c = make_config(cfg, max_batch, max_frames, compute)
+        keep, table = [], (mrf_tensor * len(weights))()
+        for i, (name, a) in enumerate(weights.items()):
+            a = np.ascontiguousarray(a)
+            if a.dtype not in (np.float32, np.float16):
+                a = a.astype(np.float32)
+            keep.append(a)
+            bname = name.encode()
+            keep.append(bname)
+            t = table[i]
+            t.name = bname
+            t.dtype = 0 if a.dtype == np.float32 else 1
+            t.ndim = a.ndim
+            for d in range(a.ndim):
+                t.shape[d] = a.shape[d]
+            t.host_data = a.ctypes.data
+        h = ctypes.c_void_p()
+        _check(lib().mrf_create(ctypes.byref(c), table, len(weights), ctypes.byref(h)))
+        self._h = h
+
+    @property
+    def handle(self):
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().mrf_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def forward(self, stft_repr, out=None, stream=None):
+        """masks for a CUDA float32 tensor [B, F*2, T, 2] (queued on `stream`)."""
+        import torch
+        assert stft_repr.is_cuda and stft_repr.dtype == torch.float32 and stft_repr.is_contiguous()
+        B, R, T, two = stft_repr.shape
+        if out is None:
+            out = torch.empty_like(stft_repr)
+        _check(lib().mrf_forward(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
+                                 ctypes.c_void_p(out.data_ptr()), B, T, _stream_ptr(stream)), self._h)
+        return out
+
+    def forward_host(self, stft_repr, out=None, stream=None):
+        """masks for a host float32 array/tensor, copies inside the call; waits for the stream."""
+        import torch
+        x = stft_repr if isinstance(stft_repr, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(stft_repr))
+        B, R, T, _ = x.shape
+        if out is None:
+            out = torch.empty_like(x)
+        _check(lib().mrf_forward_host(self._h, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                                      B, T, _stream_ptr(stream)), self._h)
+        return out
+
+    def sync_status(self, stream=None):
+        _check(lib().mrf_sync_status(self._h, _stream_ptr(stream)), self._h)
+
+    def set_timing(self, on: bool):
+        _check(lib().mrf_set_timing(self._h, int(on)), self._h)
+
+    def set_graph(self, on: bool):
+        _check(lib().mrf_set_graph(self._h, int(on)), self._h)
+
+    def kernel_times(self):
+        """{kernel name: (launches, total ms)} since the last call (timing mode)."""
+        n = ctypes.c_int(0)
+        buf = (mrf_kernel_time * 64)()
+        _check(lib().mrf_kernel_times(self._h, buf, 64, ctypes.byref(n)), self._h)
+        return {buf[i].name.decode(): (buf[i].launches, buf[i].ms) for i in range(n.value)}
+
+    def launches_per_forward(self, B, T):
+        return lib().mrf_launches_per_forward(self._h, B, T)

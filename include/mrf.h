@@ -1,0 +1,165 @@
+/*
+ * mrf.h - C ABI of the Mel-Band RoFormer core forward on NVIDIA B200 (sm_100a).
+ *
+ * The library computes the network between STFT and iSTFT of Mel-Band RoFormer:
+ * a complex stereo STFT in, per-bin complex masks out.  The contract follows the model
+ * card "musetric/vocal-separation-roformer-onnx", section "Signature": stft_repr float32
+ * [B, F*2, T, 2] (batch, freq*2 + channel, time, re/im) in, masks float32 of the same
+ * shape out, "already gathered/averaged" from the mel bands.  The method is described in
+ * "Mel-Band RoFormer — architecture, inference hot path & RTX 3050 feasibility", section
+ * "The forward chain" (mel-band gather, BandSplit, depth x (time transformer, band
+ * transformer), mask estimator, overlap scatter-add and average), and as a GPU-oriented
+ * rewrite in "@audio/neural-separate 0.4.0 → 0.5.0", package/scripts/export-roformer.py,
+ * class Core.
+ *
+ * Conventions for every entry point:
+ *  - A status code is returned; nothing is thrown, nothing aborts.  mrf_last_error()
+ *    gives a text for the last failure.
+ *  - Host pointers are read during the call only; the caller keeps ownership.
+ *  - Device pointers (stft_repr, masks) are owned by the caller and must stay valid until
+ *    the work queued on the stream has finished.
+ *  - A handle may be used by one host thread at a time.
+ */
+#ifndef MRF_H
+#define MRF_H
+
+#include <stdint.h>
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MRF_OK = 0,
+  MRF_EINVAL = -1,        /* null pointer or value out of range */
+  MRF_ESHAPE = -2,        /* B or T outside [1, max_batch] x [1, max_frames], or a weight shape mismatch */
+  MRF_ENOMEM = -3,        /* device or host allocation failed (nothing leaked) */
+  MRF_ECUDA = -4,         /* a CUDA runtime call failed; mrf_last_error has its text */
+  MRF_EUNSUPPORTED = -5,  /* configuration the kernels do not implement */
+  MRF_ETIMEOUT = -6,      /* a device-side bounded wait expired; the kernel returned early */
+  MRF_EWEIGHTS = -7       /* a required weight is missing, duplicated or has the wrong dtype */
+} mrf_status;
+
+typedef enum {
+  MRF_FP16 = 0,           /* fp16 operands, fp32 accumulation on tcgen05 tensor cores */
+  MRF_FP32_DEBUG = 2      /* fp32 CUDA-core schedule, unfused, for debugging and tight parity */
+} mrf_compute;
+
+typedef enum { MRF_DTYPE_F32 = 0, MRF_DTYPE_F16 = 1 } mrf_dtype;
+
+/* Model configuration: the fields of the checkpoint's config.json.  All sizes explicit. */
+typedef struct {
+  int sample_rate;       /* 44100: defines the Slaney mel band edges */
+  int n_fft;             /* 2048 -> F = n_fft/2 + 1 = 1025 bins */
+  int audio_channels;    /* 2 (stereo; rows are f*2 + s) */
+  int num_bands;         /* 60 mel bands */
+  int dim;               /* 384 */
+  int depth;             /* 6 axial blocks, each a time and a band transformer */
+  int heads;             /* 8 */
+  int dim_head;          /* 64 */
+  int ff_mult;           /* 4: feed-forward inner width ff_mult*dim */
+  int mask_hidden;       /* 4*dim: hidden width of the mask MLP */
+  int mask_depth;        /* 2: tanh layers of the mask MLP before its GLU layer */
+  int num_stems;         /* 1 */
+  int zero_dc;           /* 0: DC rows averaged like any other; 1: DC mask weight 0 */
+  int max_batch;         /* workspace is sized for max_batch x max_frames at create */
+  int max_frames;
+  float rope_theta;      /* 10000 */
+  int compute;           /* mrf_compute */
+} mrf_config;
+
+/* One named weight, PyTorch [out, in] layout, contiguous, in host memory. */
+typedef struct {
+  const char *name;      /* checkpoint path, e.g. "layers.0.1.layers.0.0.to_qkv.weight" */
+  int dtype;             /* mrf_dtype */
+  int ndim;              /* 1 or 2 */
+  int64_t shape[4];
+  const void *host_data;
+} mrf_tensor;
+
+typedef struct mrf_handle mrf_handle;
+
+/*
+ * mrf_create - validate the configuration and the weight table, build the band tables
+ * (Slaney mel bank binarised, DC into band 0, Nyquist into the last band: "Mel-Band
+ * RoFormer — architecture, inference hot path & RTX 3050 feasibility", section "The
+ * mel-band split, exactly"), repack and upload the weights, allocate the workspace for
+ * max_batch x max_frames on the current device.
+ *
+ * Weight names (n_w entries, any order): for each band k,
+ *   band_split.to_features.{k}.0.gamma [d_in_k], .1.weight [dim, d_in_k], .1.bias [dim];
+ * for each block l and axis a (0 = time, 1 = band), under layers.{l}.{a}.:
+ *   layers.0.0.norm.gamma [dim], layers.0.0.to_qkv.weight [3*heads*dim_head, dim],
+ *   layers.0.0.to_gates.weight [heads, dim], layers.0.0.to_gates.bias [heads],
+ *   layers.0.0.to_out.0.weight [dim, heads*dim_head],
+ *   layers.0.1.net.0.gamma [dim], layers.0.1.net.1.weight [ff, dim], .net.1.bias [ff],
+ *   layers.0.1.net.4.weight [dim, ff], .net.4.bias [dim], norm.gamma [dim];
+ * for each band k: mask_estimators.0.to_freqs.{k}.0.{0,2,4}.{weight,bias}.
+ * d_in_k = 2 * bins_k * audio_channels.  Weights are host memory owned by the caller and
+ * are not referenced after the call.  On failure *out is NULL and nothing is leaked.
+ * Errors: MRF_EINVAL, MRF_EUNSUPPORTED, MRF_EWEIGHTS, MRF_ESHAPE, MRF_ENOMEM, MRF_ECUDA.
+ */
+mrf_status mrf_create(const mrf_config *cfg, const mrf_tensor *w, int n_w, mrf_handle **out);
+
+/*
+ * mrf_forward - masks = core(stft_repr), queued on `stream` (a cudaStream_t; NULL is the
+ * legacy default stream).  stft_repr: device float32 [B, F*C, T, 2], contiguous, 16-byte
+ * aligned; masks: device float32, same shape, must not overlap stft_repr.  B in
+ * [1, max_batch], T in [1, max_frames].  Arguments are checked before anything is
+ * launched; on error nothing is queued.  Asynchronous: returns once the work is queued.
+ * Device-side failures (a bounded wait that expired) surface through mrf_sync_status.
+ */
+mrf_status mrf_forward(mrf_handle *h, const float *stft_repr, float *masks, int B, int T,
+                       void *stream);
+
+/*
+ * mrf_forward_host - the same forward from and to HOST memory: copies stft_repr to the
+ * device, runs mrf_forward, copies the masks back, and waits for the stream.  For the
+ * fastest copies the host buffers should be pinned (cudaHostAlloc / torch pin_memory).
+ */
+mrf_status mrf_forward_host(mrf_handle *h, const float *stft_repr_host, float *masks_host,
+                            int B, int T, void *stream);
+
+/*
+ * mrf_sync_status - wait for `stream`, then report the device status word: MRF_OK, or
+ * MRF_ETIMEOUT if a kernel's bounded wait expired (the word is cleared on read), or
+ * MRF_ECUDA for a CUDA error.
+ */
+mrf_status mrf_sync_status(mrf_handle *h, void *stream);
+
+/* mrf_destroy - free everything the handle owns.  NULL is a no-op. */
+void mrf_destroy(mrf_handle *h);
+
+/* Text of the handle's last error, or of the calling thread's last create/table error for NULL. */
+const char *mrf_last_error(const mrf_handle *h);
+
+/*
+ * mrf_band_tables - host-only test hook: the band tables the library builds for cfg
+ * (fields sample_rate, n_fft, audio_channels, num_bands, zero_dc).  Any output may be NULL.
+ *   first_bin, last_bin [num_bands]; width [num_bands] (d_in_k);
+ *   feat_row [sum d_in]: stft_repr row of each band feature (band order, feature
+ *   (j*C + s)*2 + c for the j-th bin of the band); row_weight [F*C]: 1 / (bands covering
+ *   the row's bin), 0 at DC when zero_dc.  *n_feat receives sum d_in.
+ */
+mrf_status mrf_band_tables(const mrf_config *cfg, int32_t *first_bin, int32_t *last_bin,
+                           int32_t *width, int32_t *feat_row, float *row_weight, int32_t *n_feat);
+
+/* Kernel timing, for measurement.  When enabled, mrf_forward launches eagerly (no CUDA
+ * graph) and records a CUDA event pair around every kernel on the forward's stream;
+ * mrf_kernel_times waits for the events and returns, per kernel kind, the number of
+ * launches and the summed milliseconds since the last reset. */
+typedef struct { char name[32]; int launches; double ms; } mrf_kernel_time;
+mrf_status mrf_set_timing(mrf_handle *h, int enable);
+mrf_status mrf_kernel_times(mrf_handle *h, mrf_kernel_time *out, int max_n, int *n_out);
+
+/* Enable (1, default) or disable (0) CUDA graph capture of the forward schedule. */
+mrf_status mrf_set_graph(mrf_handle *h, int enable);
+
+/* Number of kernels one mrf_forward launches for (B, T). */
+int mrf_launches_per_forward(const mrf_handle *h, int B, int T);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MRF_H */
