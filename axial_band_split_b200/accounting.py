@@ -1,0 +1,56 @@
+"""Algorithmic work of one core forward, per kernel kind (roofline numerators).
+
+FLOPs count 2 per multiply-accumulate of the method's dense contractions, nothing padded
+or skipped: the linear layers of "Mel-Band RoFormer — architecture, inference hot path &
+RTX 3050 feasibility", section "FLOP shares" (to_qkv, to_gates, to_out, two feed-forward
+projections per transformer; attention 2*n^2*dh MACs per head for q k^T and again for
+p v), plus the band split and the mask MLP of section "Parameter accounting".  Bytes are
+the minimum DRAM traffic of the memory-bound kernels (each input read once, each output
+written once).
+"""
+from __future__ import annotations
+
+
+def kernel_work(cfg, widths, B: int, T: int):
+    """{kernel name: (kind, total per forward, launches per forward)}; kind is "flop" or "byte"."""
+    D, H, dh = cfg.dim, cfg.heads, cfg.dim_head
+    A = H * dh
+    FF = D * cfg.ff_mult
+    MH = D * cfg.mask_hidden_mult
+    nb = cfg.num_bands
+    L2 = 2 * cfg.depth
+    BT = B * T
+    NT = BT * nb
+    n_feat = int(sum(widths))
+    rows = (cfg.n_fft // 2 + 1) * cfg.audio_channels
+    w = {
+        "gemm_qkv": ("flop", L2 * 2 * NT * D * (3 * A + H), L2),
+        "attn_time_tc": ("flop", cfg.depth * 4 * (B * nb * H) * T * T * dh, cfg.depth),
+        "attn_band_tc": ("flop", cfg.depth * 4 * (BT * H) * nb * nb * dh, cfg.depth),
+        "gemm_out_resid": ("flop", L2 * 2 * NT * A * D, L2),
+        "gemm_ff1_gelu": ("flop", L2 * 2 * NT * D * FF, L2),
+        "gemm_ff2_resid": ("flop", L2 * 2 * NT * FF * D, L2),
+        "gemm_mask_tanh": ("flop", 2 * BT * nb * (D * MH + (cfg.mask_depth - 1) * MH * MH), cfg.mask_depth),
+        "gemm_mask_glu": ("flop", 2 * BT * MH * 2 * n_feat, 1),
+        "band_split": ("flop", 2 * BT * D * n_feat, 1),
+        # x fp32 read + write, x fp16 write, |x|^2 read + write, gain
+        "outnorm": ("byte", L2 * NT * (D * 4 * 2 + D * 2 + 8), L2),
+        # mask features fp32 read once, masks fp32 written once
+        "overlap_average": ("byte", BT * n_feat * 4 + B * rows * T * 2 * 4, 1),
+    }
+    return w
+
+
+def total_flops(cfg, widths, B: int, T: int) -> int:
+    """FLOPs of one forward: every contraction of the method."""
+    return sum(v for k, v, _ in kernel_work(cfg, widths, B, T).values() if k == "flop")
+
+
+def attention_flops(cfg, widths, B, T):
+    w = kernel_work(cfg, widths, B, T)
+    return w["attn_time_tc"][1] + w["attn_band_tc"][1]
+
+
+def audio_seconds(cfg, B: int, T: int) -> float:
+    """Seconds of audio in B windows of T frames: B * T * hop / sample_rate."""
+    return B * T * cfg.hop / cfg.sample_rate

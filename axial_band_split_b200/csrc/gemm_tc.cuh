@@ -59,6 +59,8 @@ bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, un
 constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 192;
 size_t gemm_smem_bytes();
+// Resolve the tensor-map encoder and set the kernels' shared-memory limits (call once, outside capture).
+bool gemm_tc_init();
 
 void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
                     int grid, cudaStream_t st);

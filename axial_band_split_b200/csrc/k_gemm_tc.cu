@@ -375,20 +375,25 @@ bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, un
   return r == CUDA_SUCCESS;
 }
 
+bool gemm_tc_init() {
+  const int smem = (int)gemm_smem_bytes();
+  bool ok = encode_fn() != nullptr;
+  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcQkv>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcResid>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcTanh>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcGlu>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+  return ok;
+}
+
 void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p, int grid,
                     cudaStream_t st) {
   const size_t smem = gemm_smem_bytes();
   switch (epi) {
 #define MRF_GEMM_CASE(E)                                                                         \
-  case E: {                                                                                      \
-    static bool attr = false;                                                                    \
-    if (!attr) {                                                                                 \
-      cudaFuncSetAttribute(gemm_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); \
-      attr = true;                                                                               \
-    }                                                                                            \
+  case E:                                                                                        \
     gemm_tc_kernel<E><<<grid, kGemmThreads, smem, st>>>(tmA, tmB, p);                            \
-    break;                                                                                       \
-  }
+    break;
     MRF_GEMM_CASE(kTcQkv)
     MRF_GEMM_CASE(kTcResid)
     MRF_GEMM_CASE(kTcGelu)

@@ -231,12 +231,19 @@ __global__ void rope_split_kernel(const float *__restrict__ qkv, const float2 *_
   dst[o + 1] = y1;
 }
 
-// ------------------------------------------------------------------ attention (fp32)
-// One warp per query row; keys in chunks of 32 (one per lane), online softmax.
-__global__ void attention_f32_kernel(const float *__restrict__ q, const float *__restrict__ k,
-                                     const float *__restrict__ v, const float *__restrict__ gate,
-                                     float *__restrict__ o, int B, int T, int nb, int H, int dh,
-                                     int axis) {
+// ------------------------------------------------------------------ attention (CUDA cores)
+// One warp per query row; keys in chunks of 32 (one per lane), online softmax.  q, k, v
+// are [(seq*H + head)*n_pad + pos]*dh; o[tok, head*dh + d] = gate[tok, head] * result.
+__device__ __forceinline__ float ld_f(const float *p) { return *p; }
+__device__ __forceinline__ float ld_f(const __half *p) { return __half2float(*p); }
+__device__ __forceinline__ void st_f(float *p, float v) { *p = v; }
+__device__ __forceinline__ void st_f(__half *p, float v) { *p = __float2half_rn(v); }
+
+template <class TI, class TO>
+__global__ void attention_simt_kernel(const TI *__restrict__ q, const TI *__restrict__ k,
+                                      const TI *__restrict__ v, const float *__restrict__ gate,
+                                      TO *__restrict__ o, int B, int T, int nb, int H, int dh,
+                                      int axis, int n_pad) {
   __shared__ float qs[8][64];
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const long long nseq = axis == 0 ? (long long)B * nb : (long long)B * T;
@@ -247,19 +254,19 @@ __global__ void attention_f32_kernel(const float *__restrict__ q, const float *_
   const long long sh = qi / n;  // seq * H + head
   const int head = sh % H;
   const long long seq = sh / H;
-  const float *qr = q + qi * dh;
+  const TI *qr = q + (sh * n_pad + pos) * dh;
   const float scale = rsqrtf((float)dh);
-  for (int d = lane; d < dh; d += 32) qs[warp][d] = qr[d] * scale;
+  for (int d = lane; d < dh; d += 32) qs[warp][d] = ld_f(qr + d) * scale;
   __syncwarp();
-  const float *kb = k + sh * n * dh;
-  const float *vb = v + sh * n * dh;
+  const TI *kb = k + sh * n_pad * dh;
+  const TI *vb = v + sh * n_pad * dh;
   float m = -INFINITY, l = 0.f, o0 = 0.f, o1 = 0.f;
   for (int j0 = 0; j0 < n; j0 += 32) {
     const int j = j0 + lane;
     float s = -INFINITY;
     if (j < n) {
       s = 0.f;
-      for (int d = 0; d < dh; ++d) s = fmaf(qs[warp][d], kb[(long long)j * dh + d], s);
+      for (int d = 0; d < dh; ++d) s = fmaf(qs[warp][d], ld_f(kb + (long long)j * dh + d), s);
     }
     const float mn = fmaxf(m, warp_max(s));
     const float p = (j < n) ? expf(s - mn) : 0.f;
@@ -269,9 +276,9 @@ __global__ void attention_f32_kernel(const float *__restrict__ q, const float *_
     const int cnt = min(32, n - j0);
     for (int jj = 0; jj < cnt; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
-      const float *vr = vb + (long long)(j0 + jj) * dh;
-      if (lane < dh) o0 = fmaf(pj, vr[lane], o0);
-      if (lane + 32 < dh) o1 = fmaf(pj, vr[lane + 32], o1);
+      const TI *vr = vb + (long long)(j0 + jj) * dh;
+      if (lane < dh) o0 = fmaf(pj, ld_f(vr + lane), o0);
+      if (lane + 32 < dh) o1 = fmaf(pj, ld_f(vr + lane + 32), o1);
     }
     m = mn;
   }
@@ -279,9 +286,36 @@ __global__ void attention_f32_kernel(const float *__restrict__ q, const float *_
   if (axis == 0) { const long long b = seq / nb, band = seq % nb; tok = (b * T + pos) * nb + band; }
   else tok = seq * nb + pos;
   const float g = gate[tok * H + head] / l;
-  float *orow = o + tok * (long long)H * dh + head * dh;
-  if (lane < dh) orow[lane] = o0 * g;
-  if (lane + 32 < dh) orow[lane + 32] = o1 * g;
+  TO *orow = o + tok * (long long)H * dh + head * dh;
+  if (lane < dh) st_f(orow + lane, o0 * g);
+  if (lane + 32 < dh) st_f(orow + lane + 32, o1 * g);
+}
+
+// ------------------------------------------------------------------ output norm (fp16 schedule)
+// x = x / max(sqrt(ss), eps) * gain; writes x (fp32), its fp16 copy and the new sum of squares.
+__global__ void outnorm_kernel(float *__restrict__ x, float *__restrict__ ss, const float *__restrict__ gain,
+                               __half *__restrict__ xh, long long rows, int D) {
+  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float r = 1.f / fmaxf(sqrtf(ss[row]), kNormEps);
+  float *xr = x + row * D;
+  __half *hr = xh + row * D;
+  float s = 0.f;
+  for (int j = lane * 4; j < D; j += 128) {
+    float4 a = *reinterpret_cast<float4 *>(xr + j);
+    const float4 g = *reinterpret_cast<const float4 *>(gain + j);
+    a.x *= r * g.x; a.y *= r * g.y; a.z *= r * g.z; a.w *= r * g.w;
+    *reinterpret_cast<float4 *>(xr + j) = a;
+    __half2 h0 = __floats2half2_rn(a.x, a.y), h1 = __floats2half2_rn(a.z, a.w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t *>(&h0);
+    u.y = *reinterpret_cast<uint32_t *>(&h1);
+    *reinterpret_cast<uint2 *>(hr + j) = u;
+    s += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+  }
+  s = warp_sum(s);
+  if (lane == 0) ss[row] = s;
 }
 
 // ------------------------------------------------------------------ overlap average
@@ -347,7 +381,22 @@ void launch_attention_f32(const float *q, const float *k, const float *v, const 
                           float *o, int B, int T, int nb, int heads, int dh, int axis,
                           cudaStream_t st) {
   const long long rows = (long long)B * T * nb * heads;
-  attention_f32_kernel<<<grid1(rows, 8), 256, 0, st>>>(q, k, v, gate, o, B, T, nb, heads, dh, axis);
+  const int n = axis == 0 ? T : nb;
+  attention_simt_kernel<float, float><<<grid1(rows, 8), 256, 0, st>>>(q, k, v, gate, o, B, T, nb, heads, dh,
+                                                                      axis, n);
+}
+
+void launch_attention_simt_f16(const __half *q, const __half *k, const __half *v, const float *gate,
+                               __half *o, int B, int T, int nb, int heads, int dh, int axis, int n_pad,
+                               cudaStream_t st) {
+  const long long rows = (long long)B * T * nb * heads;
+  attention_simt_kernel<__half, __half><<<grid1(rows, 8), 256, 0, st>>>(q, k, v, gate, o, B, T, nb, heads,
+                                                                        dh, axis, n_pad);
+}
+
+void launch_outnorm(float *x, float *ss, const float *gain, __half *xh, long long rows, int D,
+                    cudaStream_t st) {
+  outnorm_kernel<<<grid1(rows, 8), 256, 0, st>>>(x, ss, gain, xh, rows, D);
 }
 
 void launch_overlap_average(const float *m, int ldm, const int32_t *src0, const int32_t *src1,

@@ -408,6 +408,7 @@ void schedule_f32(mrf_handle *h, const float *in, float *out, int B, int T) {
 
 void run_schedule(mrf_handle *h, const float *in, float *out, int B, int T) {
   h->launch_counter = 0;
+  h->sched_error.clear();
   if (h->cfg.compute == MRF_FP32_DEBUG) schedule_f32(h, in, out, B, T);
   else schedule_fp16(h, in, out, B, T);
   h->last_launches = h->launch_counter;
@@ -499,6 +500,7 @@ mrf_status mrf_forward(mrf_handle *h, const float *in, float *out, int B, int T,
   if (h->timing || !h->use_graph) {
     h->cur_stream = st;
     run_schedule(h, in, out, B, T);
+    if (!h->sched_error.empty()) return fail(h, MRF_ECUDA, h->sched_error);
     if (!cuda_ok(h, cudaGetLastError(), "kernel launch", &s)) return s;
     return MRF_OK;
   }
@@ -513,6 +515,10 @@ mrf_status mrf_forward(mrf_handle *h, const float *in, float *out, int B, int T,
     run_schedule(h, in, out, B, T);
     cudaGraph_t graph = nullptr;
     cudaError_t e = cudaStreamEndCapture(h->cap_stream, &graph);
+    if (!h->sched_error.empty()) {
+      if (graph) cudaGraphDestroy(graph);
+      return fail(h, MRF_ECUDA, h->sched_error);
+    }
     if (!cuda_ok(h, e, "end capture", &s)) return s;
     e = cudaGraphInstantiate(&exec, graph, 0);
     cudaGraphDestroy(graph);
@@ -614,6 +620,28 @@ mrf_status mrf_kernel_times(mrf_handle *h, mrf_kernel_time *out, int max_n, int 
   h->pending.clear();
   *n_out = (int)acc.size();
   for (int i = 0; i < (int)acc.size() && i < max_n && out; ++i) out[i] = acc[i];
+  return MRF_OK;
+}
+
+mrf_status mrf_debug_buffer(mrf_handle *h, const char *name, void *dst, size_t max_bytes, size_t *bytes_out) {
+  if (!h || !name || !dst) return fail(h, MRF_EINVAL, "null argument");
+  if (h->last_B < 1) return fail(h, MRF_EINVAL, "no forward has run");
+  const void *src = nullptr;
+  size_t bytes = 0;
+  const std::string n(name);
+  const long long BT = (long long)h->last_B * h->last_T;
+  if (h->cfg.compute == MRF_FP32_DEBUG) {
+    if (n == "X") { src = h->ws.X; bytes = BT * h->cfg.num_bands * h->cfg.dim * sizeof(float); }
+    else if (n == "M") { src = h->ws.Mg; bytes = BT * h->tab.n_feat() * sizeof(float); }
+  } else if (!debug_buffer_fp16(h, n, &src, &bytes)) {
+    src = nullptr;
+  }
+  if (!src) return fail(h, MRF_EINVAL, "unknown buffer " + n);
+  bytes = std::min(bytes, max_bytes);
+  mrf_status s = MRF_OK;
+  if (!cuda_ok(h, cudaDeviceSynchronize(), "device sync", &s)) return s;
+  if (!cuda_ok(h, cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost), "debug copy", &s)) return s;
+  if (bytes_out) *bytes_out = bytes;
   return MRF_OK;
 }
 

@@ -97,6 +97,7 @@ struct mrf_handle {
   std::vector<mrf::GraphEntry> graphs;
   int launch_counter = 0, last_launches = -1, last_B = -1, last_T = -1;
   float *io_in = nullptr, *io_out = nullptr;
+  std::string sched_error;  // set by a schedule that refused to launch
 
   void begin(const char *name);
   void end();
@@ -110,4 +111,5 @@ std::string fp16_supported(const mrf_config &c, const BandTables &t);
 mrf_status pack_fp16(mrf_handle *h, WeightMap &W);
 void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T);
 void destroy_fp16(mrf_handle *h);
+bool debug_buffer_fp16(mrf_handle *h, const std::string &name, const void **ptr, size_t *bytes);
 }  // namespace mrf

@@ -1,13 +1,373 @@
-// fp16 tensor-core schedule (placeholder until the tcgen05 kernels land).
+// fp16 tensor-core schedule: weight packing, workspace and the per-forward launch list.
+//
+// Per forward (N_tok = B*T*bands tokens, token (b*T + t)*bands + k):
+//   band split (gather + norm + Linear)        -> X fp32, X fp16, |x|^2
+//   per transformer (time axis, then band axis, depth times):
+//     QKV+gates GEMM, RoPE epilogue            -> q, k, v fp16 in attention layout, gates
+//     attention                                -> O fp16 (times the gate)
+//     out-projection GEMM, residual epilogue   -> X, X fp16, |x|^2
+//     FF1 GEMM, GELU epilogue                  -> H fp16
+//     FF2 GEMM, residual epilogue              -> X, X fp16, |x|^2
+//     output norm                              -> X, X fp16, |x|^2
+//   mask head: per-band GEMMs (tanh, tanh, GLU) -> m fp32 [B*T, sum d_in]
+//   overlap average                            -> masks
+//
+// Exact rewrites (package/scripts/export-roformer.py of "@audio/neural-separate 0.4.0 →
+// 0.5.0", class Core and its module docstring): each RMSNorm's sqrt(d)*gamma is folded
+// into the weight of the Linear it feeds, leaving the per-row 1/max(|x|, 1e-12) as an
+// epilogue scale; the gates' projection is appended to q, k, v; the mask head's bands
+// are batched as groups of one GEMM; its last layer's value and gate rows are interleaved
+// so that a GLU pair is two adjacent accumulator columns.
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "gemm_tc.cuh"
 #include "mrf_handle.h"
 
 namespace mrf {
 
-std::string fp16_supported(const mrf_config &, const BandTables &) {
-  return "the fp16 tensor-core schedule is not built yet";
+bool launch_attention_tc(const __half *q, const __half *k, const __half *v, const float *gate, __half *o,
+                         int B, int T, int nb, int H, int axis, int n_pad, unsigned *status, cudaStream_t st);
+bool attention_tc_supported(int dh);
+bool attention_tc_init();
+
+struct TrF16 {
+  __half *wqkvg = nullptr, *wo = nullptr, *w1 = nullptr, *w2 = nullptr;
+  float *bg = nullptr, *b1 = nullptr, *b2 = nullptr, *gout = nullptr;
+};
+
+struct Fp16State {
+  std::vector<TrF16> tr;
+  std::vector<__half *> mw;   // mask layers 0 .. mask_depth-1, stacked over bands [nb*MH, K]
+  std::vector<float *> mb;
+  __half *mw_last = nullptr;  // [sum 2*d_in, MH], rows interleaved (value e, gate e)
+  float *mb_last = nullptr;
+  // group tables
+  GemmGroup *g_qkv = nullptr, *g_out = nullptr, *g_ff1 = nullptr, *g_ff2 = nullptr;
+  GemmGroup *g_m0 = nullptr, *g_mid = nullptr, *g_last = nullptr;
+  int n_last_tiles = 0;
+  // workspace
+  float *X = nullptr, *ss = nullptr, *G = nullptr, *Mg = nullptr;
+  __half *Xh = nullptr, *Q = nullptr, *K = nullptr, *V = nullptr, *O = nullptr, *Hh = nullptr,
+         *H1 = nullptr, *H2 = nullptr;
+  long long qkv_elems = 0;
+  int n_pad_time = 0, n_pad_band = 0;
+  int sms = 148;
+  bool tc_attention = true;
+};
+
+namespace {
+
+constexpr int kBnWide = 256, kBnNarrow = 192;
+
+std::vector<__half> to_half(const std::vector<float> &v) {
+  std::vector<__half> o(v.size());
+  for (size_t i = 0; i < v.size(); ++i) o[i] = __float2half_rn(v[i]);
+  return o;
 }
-mrf_status pack_fp16(mrf_handle *, WeightMap &) { return MRF_EUNSUPPORTED; }
-void schedule_fp16(mrf_handle *, const float *, float *, int, int) {}
-void destroy_fp16(mrf_handle *) {}
+
+template <class T>
+T *up(mrf_handle *h, const std::vector<T> &v) {
+  T *p = h->alloc<T>(v.size());
+  if (p && !h->upload(p, v.data(), v.size() * sizeof(T))) return nullptr;
+  return p;
+}
+
+// W [N, K] with column j scaled by s[j] (an RMSNorm's sqrt(K)*gamma folded into the Linear after it).
+std::vector<float> fold_cols(const std::vector<float> &w, const std::vector<float> &gamma, int N, int K) {
+  std::vector<float> o(w.size());
+  const double s = std::sqrt((double)K);
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k) o[(size_t)n * K + k] = (float)((double)w[(size_t)n * K + k] * gamma[k] * s);
+  return o;
+}
+
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+GemmGroup *upload_groups(mrf_handle *h, const std::vector<GemmGroup> &g) { return up(h, g); }
+
+}  // namespace
+
+std::string fp16_supported(const mrf_config &c, const BandTables &t) {
+  (void)t;
+  const int A = c.heads * c.dim_head;
+  if (c.dim % 64) return "fp16 schedule needs dim % 64 == 0";
+  if (A % 64) return "fp16 schedule needs heads*dim_head % 64 == 0";
+  if (c.dim_head % 16) return "fp16 schedule needs dim_head % 16 == 0";
+  if (c.mask_hidden % 64) return "fp16 schedule needs mask_hidden % 64 == 0";
+  return "";
+}
+
+mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
+  const mrf_config &c = h->cfg;
+  const BandTables &t = h->tab;
+  const int nb = c.num_bands, D = c.dim, H = c.heads, dh = c.dim_head, A = H * dh, FF = c.ff_mult * D,
+            MH = c.mask_hidden;
+  const long long MBT = (long long)c.max_batch * c.max_frames, NT = MBT * nb;
+  Fp16State *f = new (std::nothrow) Fp16State();
+  if (!f) return MRF_ENOMEM;
+  h->f16 = f;
+  cudaDeviceGetAttribute(&f->sms, cudaDevAttrMultiProcessorCount, h->device);
+  f->tc_attention = attention_tc_supported(dh);
+  if (!gemm_tc_init() || (f->tc_attention && !attention_tc_init())) {
+    h->err = "tcgen05 kernel initialisation failed (tensor-map encoder or shared-memory limit)";
+    return MRF_ECUDA;
+  }
+  // transformers
+  f->tr.resize(2 * c.depth);
+  for (int l = 0; l < c.depth; ++l)
+    for (int a = 0; a < 2; ++a) {
+      const std::string p = "layers." + std::to_string(l) + "." + std::to_string(a) + ".";
+      TrF16 &x = f->tr[2 * l + a];
+      const auto &ga = W[p + "layers.0.0.norm.gamma"].v;
+      std::vector<float> qkvg = fold_cols(W[p + "layers.0.0.to_qkv.weight"].v, ga, 3 * A, D);
+      std::vector<float> wg = fold_cols(W[p + "layers.0.0.to_gates.weight"].v, ga, H, D);
+      qkvg.insert(qkvg.end(), wg.begin(), wg.end());
+      x.wqkvg = up(h, to_half(qkvg));
+      x.bg = up(h, W[p + "layers.0.0.to_gates.bias"].v);
+      x.wo = up(h, to_half(W[p + "layers.0.0.to_out.0.weight"].v));
+      x.w1 = up(h, to_half(fold_cols(W[p + "layers.0.1.net.1.weight"].v, W[p + "layers.0.1.net.0.gamma"].v, FF, D)));
+      x.b1 = up(h, W[p + "layers.0.1.net.1.bias"].v);
+      x.w2 = up(h, to_half(W[p + "layers.0.1.net.4.weight"].v));
+      x.b2 = up(h, W[p + "layers.0.1.net.4.bias"].v);
+      std::vector<float> go(W[p + "norm.gamma"].v);
+      for (auto &v : go) v = (float)(v * std::sqrt((double)D));
+      x.gout = up(h, go);
+      if (!x.wqkvg || !x.bg || !x.wo || !x.w1 || !x.b1 || !x.w2 || !x.b2 || !x.gout)
+        return MRF_ENOMEM;
+    }
+  // mask head
+  std::vector<std::vector<float>> mw(c.mask_depth), mb(c.mask_depth);
+  std::vector<float> wl, bl;
+  for (int k = 0; k < nb; ++k) {
+    const std::string p = "mask_estimators.0.to_freqs." + std::to_string(k) + ".0.";
+    for (int i = 0; i < c.mask_depth; ++i) {
+      const auto &w = W[p + std::to_string(2 * i) + ".weight"].v;
+      const auto &b = W[p + std::to_string(2 * i) + ".bias"].v;
+      mw[i].insert(mw[i].end(), w.begin(), w.end());
+      mb[i].insert(mb[i].end(), b.begin(), b.end());
+    }
+    const std::string q = p + std::to_string(2 * c.mask_depth);
+    const auto &w = W[q + ".weight"].v;
+    const auto &b = W[q + ".bias"].v;
+    const int wd = t.width[k];
+    for (int e = 0; e < wd; ++e) {
+      wl.insert(wl.end(), w.begin() + (size_t)e * MH, w.begin() + (size_t)(e + 1) * MH);
+      wl.insert(wl.end(), w.begin() + (size_t)(wd + e) * MH, w.begin() + (size_t)(wd + e + 1) * MH);
+      bl.push_back(b[e]);
+      bl.push_back(b[wd + e]);
+    }
+  }
+  for (int i = 0; i < c.mask_depth; ++i) {
+    f->mw.push_back(up(h, to_half(mw[i])));
+    f->mb.push_back(up(h, mb[i]));
+    if (!f->mw.back() || !f->mb.back()) return MRF_ENOMEM;
+  }
+  f->mw_last = up(h, to_half(wl));
+  f->mb_last = up(h, bl);
+  if (!f->mw_last || !f->mb_last) return MRF_ENOMEM;
+  // group tables
+  auto single = [&](int N, int BN) {
+    GemmGroup g{N, cdiv(N, BN), 0, 0, 0, 0, 0, 0};
+    return upload_groups(h, {g});
+  };
+  f->g_qkv = single(3 * A + H, kBnWide);
+  f->g_out = single(D, kBnNarrow);
+  f->g_ff1 = single(FF, kBnWide);
+  f->g_ff2 = single(D, kBnNarrow);
+  std::vector<GemmGroup> g0(nb), g1(nb), g2(nb);
+  int start = 0;
+  for (int k = 0; k < nb; ++k) {
+    g0[k] = {MH, cdiv(MH, kBnWide), k * cdiv(MH, kBnWide), k, k * MH, k, k * MH, 0};
+    g1[k] = {MH, cdiv(MH, kBnWide), k * cdiv(MH, kBnWide), (int)(k * MBT), k * MH, k, k * MH, 0};
+    const int N = 2 * t.width[k];
+    g2[k] = {N, cdiv(N, kBnWide), start, (int)(k * MBT), 2 * t.feat_off[k], t.feat_off[k], 2 * t.feat_off[k], 0};
+    start += g2[k].n_tiles;
+  }
+  f->n_last_tiles = start;
+  f->g_m0 = upload_groups(h, g0);
+  f->g_mid = upload_groups(h, g1);
+  f->g_last = upload_groups(h, g2);
+  if (!f->g_qkv || !f->g_out || !f->g_ff1 || !f->g_ff2 || !f->g_m0 || !f->g_mid || !f->g_last) return MRF_ENOMEM;
+  // workspace
+  f->n_pad_time = cdiv(c.max_frames, 128) * 128;
+  f->n_pad_band = cdiv(nb, 64) * 64;
+  f->qkv_elems = std::max((long long)c.max_batch * nb * H * f->n_pad_time, MBT * H * f->n_pad_band) * dh;
+  f->X = h->alloc<float>(NT * D);
+  f->Xh = h->alloc<__half>(NT * D);
+  f->ss = h->alloc<float>(NT);
+  f->G = h->alloc<float>(NT * H);
+  f->Q = h->alloc<__half>(f->qkv_elems);
+  f->K = h->alloc<__half>(f->qkv_elems);
+  f->V = h->alloc<__half>(f->qkv_elems);
+  f->O = h->alloc<__half>(NT * A);
+  f->Hh = h->alloc<__half>(NT * FF);
+  f->H1 = h->alloc<__half>((long long)nb * MBT * MH);
+  f->H2 = h->alloc<__half>((long long)nb * MBT * MH);
+  f->Mg = h->alloc<float>(MBT * t.n_feat());
+  if (!f->X || !f->Xh || !f->ss || !f->G || !f->Q || !f->K || !f->V || !f->O || !f->Hh || !f->H1 || !f->H2 || !f->Mg)
+    return MRF_ENOMEM;
+  // padded positions of q, k, v are read by the attention tiles: keep them finite (zero)
+  if (cudaMemset(f->Q, 0, f->qkv_elems * 2) != cudaSuccess || cudaMemset(f->K, 0, f->qkv_elems * 2) != cudaSuccess ||
+      cudaMemset(f->V, 0, f->qkv_elems * 2) != cudaSuccess || cudaMemset(f->H1, 0, (size_t)nb * MBT * MH * 2) != cudaSuccess ||
+      cudaMemset(f->H2, 0, (size_t)nb * MBT * MH * 2) != cudaSuccess || cudaMemset(f->Xh, 0, NT * D * 2) != cudaSuccess)
+    return MRF_ECUDA;
+  return MRF_OK;
+}
+
+bool debug_buffer_fp16(mrf_handle *h, const std::string &name, const void **ptr, size_t *bytes) {
+  Fp16State *f = h->f16;
+  if (!f) return false;
+  const long long BT = (long long)h->last_B * h->last_T;
+  if (name == "X") { *ptr = f->X; *bytes = BT * h->cfg.num_bands * h->cfg.dim * sizeof(float); return true; }
+  if (name == "M") { *ptr = f->Mg; *bytes = BT * h->tab.n_feat() * sizeof(float); return true; }
+  return false;
+}
+
+void destroy_fp16(mrf_handle *h) {
+  delete h->f16;
+  h->f16 = nullptr;
+}
+
+namespace {
+
+GemmParams base_params(mrf_handle *h, int M, int K, int BN, const GemmGroup *groups, int ngroups,
+                       int total_n_tiles) {
+  GemmParams p;
+  memset(&p, 0, sizeof p);
+  p.M = M;
+  p.K = K;
+  p.BN = BN;
+  p.groups = groups;
+  p.ngroups = ngroups;
+  p.total_n_tiles = total_n_tiles;
+  p.m_tiles = cdiv(M, 128);
+  p.status = h->status;
+  return p;
+}
+
+void gemm(mrf_handle *h, const char *name, int epi, const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p) {
+  const int tiles = p.m_tiles * p.total_n_tiles;
+  const int grid = std::min(tiles, h->f16->sms);
+  h->begin(name);
+  launch_gemm_tc(epi, a, b, p, grid, h->cur_stream);
+  h->end();
+}
+
+}  // namespace
+
+void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
+  const mrf_config &c = h->cfg;
+  Fp16State *f = h->f16;
+  const int nb = c.num_bands, D = c.dim, H = c.heads, dh = c.dim_head, A = H * dh, FF = c.ff_mult * D,
+            MH = c.mask_hidden;
+  const long long MBT = (long long)c.max_batch * c.max_frames, NT = MBT * nb;
+  const int M = B * T * nb;
+  const int R = h->tab.n_freqs * h->tab.channels;
+  cudaStream_t st = h->cur_stream;
+
+  // tensor maps of the activations (fixed buffers; extents cover the whole workspace)
+  CUtensorMap mXh, mO, mHh, mXband, mH1, mH2;
+  bool ok = make_tmap_f16(&mXh, f->Xh, D, NT, 1, D, NT * D, 128, 1) &&
+            make_tmap_f16(&mO, f->O, A, NT, 1, A, NT * A, 128, 1) &&
+            make_tmap_f16(&mHh, f->Hh, FF, NT, 1, FF, NT * FF, 128, 1) &&
+            make_tmap_f16(&mXband, f->Xh, D, nb, MBT, D, (long long)nb * D, 1, 128) &&
+            make_tmap_f16(&mH1, f->H1, MH, nb * MBT, 1, MH, nb * MBT * MH, 128, 1) &&
+            make_tmap_f16(&mH2, f->H2, MH, nb * MBT, 1, MH, nb * MBT * MH, 128, 1);
+  std::vector<CUtensorMap> wmaps(4 * 2 * c.depth + c.mask_depth + 1);
+  for (int i = 0; ok && i < 2 * c.depth; ++i) {
+    const TrF16 &w = f->tr[i];
+    ok = make_tmap_f16(&wmaps[4 * i + 0], w.wqkvg, D, 3 * A + H, 1, D, (3LL * A + H) * D, kBnWide, 1) &&
+         make_tmap_f16(&wmaps[4 * i + 1], w.wo, A, D, 1, A, (long long)D * A, kBnNarrow, 1) &&
+         make_tmap_f16(&wmaps[4 * i + 2], w.w1, D, FF, 1, D, (long long)FF * D, kBnWide, 1) &&
+         make_tmap_f16(&wmaps[4 * i + 3], w.w2, FF, D, 1, FF, (long long)D * FF, kBnNarrow, 1);
+  }
+  const int wm0 = 8 * c.depth;
+  for (int i = 0; ok && i < c.mask_depth; ++i) {
+    const int K = i == 0 ? D : MH;
+    ok = make_tmap_f16(&wmaps[wm0 + i], f->mw[i], K, (long long)nb * MH, 1, K, (long long)nb * MH * K, kBnWide, 1);
+  }
+  const long long rows_last = 2LL * h->tab.n_feat();
+  ok = ok && make_tmap_f16(&wmaps[wm0 + c.mask_depth], f->mw_last, MH, rows_last, 1, MH, rows_last * MH, kBnWide, 1);
+  if (!ok) {
+    h->sched_error = "tensor-map encoding failed";
+    return;
+  }
+
+  h->begin("band_split");
+  launch_band_split(in, h->d_feat_row, h->d_feat_c, h->d_bands, nb, h->w_bs, h->b_bs, D, B, T, R, f->X, f->Xh,
+                    f->ss, st, h->max_width);
+  h->end();
+
+  for (int i = 0; i < 2 * c.depth; ++i) {
+    const TrF16 &w = f->tr[i];
+    const int axis = i & 1;
+    const CUtensorMap &mWqkv = wmaps[4 * i + 0], &mWo = wmaps[4 * i + 1], &mW1 = wmaps[4 * i + 2],
+                      &mW2 = wmaps[4 * i + 3];
+    const int n_pad = axis == 0 ? f->n_pad_time : f->n_pad_band;
+
+    // q, k, v, gates
+    GemmParams p = base_params(h, M, D, kBnWide, f->g_qkv, 1, cdiv(3 * A + H, kBnWide));
+    p.ss_in = f->ss;
+    p.q = f->Q; p.k = f->K; p.v = f->V; p.gates = f->G; p.rope = h->d_rope; p.gbias = w.bg;
+    p.B = B; p.T = T; p.nb = nb; p.H = H; p.dh = dh; p.A = A; p.axis = axis; p.n_pad = n_pad;
+    gemm(h, "gemm_qkv", kTcQkv, mXh, mWqkv, p);
+
+    h->begin(f->tc_attention ? (axis == 0 ? "attn_time_tc" : "attn_band_tc") : "attn_simt_f16");
+    if (f->tc_attention) {
+      if (!launch_attention_tc(f->Q, f->K, f->V, f->G, f->O, B, T, nb, H, axis, n_pad, h->status, st)) {
+        h->end();
+        h->sched_error = "tensor-map encoding failed (attention)";
+        return;
+      }
+    } else
+      launch_attention_simt_f16(f->Q, f->K, f->V, f->G, f->O, B, T, nb, H, dh, axis, n_pad, st);
+    h->end();
+
+    cudaMemsetAsync(f->ss, 0, sizeof(float) * M, st);
+    p = base_params(h, M, A, kBnNarrow, f->g_out, 1, cdiv(D, kBnNarrow));
+    p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D;
+    gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p);
+
+    p = base_params(h, M, D, kBnWide, f->g_ff1, 1, cdiv(FF, kBnWide));
+    p.ss_in = f->ss; p.bias = w.b1; p.out_h = f->Hh; p.ldo = FF;
+    gemm(h, "gemm_ff1_gelu", kTcGelu, mXh, mW1, p);
+
+    cudaMemsetAsync(f->ss, 0, sizeof(float) * M, st);
+    p = base_params(h, M, FF, kBnNarrow, f->g_ff2, 1, cdiv(D, kBnNarrow));
+    p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D; p.bias = w.b2;
+    gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p);
+
+    h->begin("outnorm");
+    launch_outnorm(f->X, f->ss, w.gout, f->Xh, M, D, st);
+    h->end();
+  }
+
+  // mask head
+  const int BT = B * T;
+  GemmParams p = base_params(h, BT, D, kBnWide, f->g_m0, nb, nb * cdiv(MH, kBnWide));
+  p.a_mode = 1;
+  p.bias = f->mb[0]; p.out_h = f->H1; p.ldo = MH; p.out_group_stride = MBT * MH;
+  gemm(h, "gemm_mask_tanh", kTcTanh, mXband, wmaps[wm0], p);
+  __half *cur = f->H1, *nxt = f->H2;
+  const CUtensorMap *mcur = &mH1, *mnxt = &mH2;
+  for (int i = 1; i < c.mask_depth; ++i) {
+    p = base_params(h, BT, MH, kBnWide, f->g_mid, nb, nb * cdiv(MH, kBnWide));
+    p.bias = f->mb[i]; p.out_h = nxt; p.ldo = MH; p.out_group_stride = MBT * MH;
+    gemm(h, "gemm_mask_tanh", kTcTanh, *mcur, wmaps[wm0 + i], p);
+    std::swap(cur, nxt);
+    std::swap(mcur, mnxt);
+  }
+  p = base_params(h, BT, MH, kBnWide, f->g_last, nb, f->n_last_tiles);
+  p.bias = f->mb_last; p.out_f = f->Mg; p.ldo = h->tab.n_feat();
+  gemm(h, "gemm_mask_glu", kTcGlu, *mcur, wmaps[wm0 + c.mask_depth], p);
+
+  h->begin("overlap_average");
+  launch_overlap_average(f->Mg, h->tab.n_feat(), h->d_src0, h->d_src1, h->d_row_weight, out, B, T, R, st);
+  h->end();
+}
 
 }  // namespace mrf

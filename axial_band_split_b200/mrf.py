@@ -25,7 +25,7 @@ STATUS = {0: "MRF_OK", -1: "MRF_EINVAL", -2: "MRF_ESHAPE", -3: "MRF_ENOMEM", -4:
 # every symbol include/mrf.h declares
 EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
            "mrf_last_error", "mrf_band_tables", "mrf_set_timing", "mrf_kernel_times",
-           "mrf_set_graph", "mrf_launches_per_forward"]
+           "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer"]
 
 
 class MrfError(RuntimeError):
@@ -81,6 +81,8 @@ def lib():
         L.mrf_set_graph.restype = I
         L.mrf_kernel_times.argtypes = [P, ctypes.POINTER(mrf_kernel_time), I, ctypes.POINTER(I)]
         L.mrf_kernel_times.restype = I
+        L.mrf_debug_buffer.argtypes = [P, ctypes.c_char_p, P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)]
+        L.mrf_debug_buffer.restype = I
         L.mrf_launches_per_forward.argtypes = [P, I, I]
         L.mrf_launches_per_forward.restype = I
         _lib = L
@@ -205,6 +207,14 @@ class Model:
         buf = (mrf_kernel_time * 64)()
         _check(lib().mrf_kernel_times(self._h, buf, 64, ctypes.byref(n)), self._h)
         return {buf[i].name.decode(): (buf[i].launches, buf[i].ms) for i in range(n.value)}
+
+    def debug_buffer(self, name, count):
+        """First `count` float32 values of an internal buffer of the last forward ("X", "M")."""
+        out = np.zeros(count, np.float32)
+        n = ctypes.c_size_t(0)
+        _check(lib().mrf_debug_buffer(self._h, name.encode(), out.ctypes.data_as(ctypes.c_void_p),
+                                      out.nbytes, ctypes.byref(n)), self._h)
+        return out[: n.value // 4]
 
     def launches_per_forward(self, B, T):
         return lib().mrf_launches_per_forward(self._h, B, T)

@@ -156,6 +156,16 @@ mrf_status mrf_kernel_times(mrf_handle *h, mrf_kernel_time *out, int max_n, int 
 /* Enable (1, default) or disable (0) CUDA graph capture of the forward schedule. */
 mrf_status mrf_set_graph(mrf_handle *h, int enable);
 
+/*
+ * mrf_debug_buffer - test hook: wait for the device, then copy the start of an internal
+ * buffer of the last forward to host memory.  "X": the residual stream after the last
+ * transformer, float32 [B*T*num_bands, dim], token (b*T + t)*num_bands + k; "M": the mask
+ * estimator output before the overlap average, float32 [B*T, sum d_in].  At most
+ * max_bytes are copied; *bytes_out receives the number copied.
+ */
+mrf_status mrf_debug_buffer(mrf_handle *h, const char *name, void *host_dst, size_t max_bytes,
+                            size_t *bytes_out);
+
 /* Number of kernels one mrf_forward launches for (B, T). */
 int mrf_launches_per_forward(const mrf_handle *h, int B, int T);
 

@@ -94,3 +94,15 @@ def test_null_arguments():
     L.mrf_destroy(None)
     assert L.mrf_launches_per_forward(None, 1, 1) == -1
     assert b"null" in L.mrf_last_error(None)
+
+
+def test_accounting_matches_oracle_mac_count():
+    # the bench's roofline numerators agree with the oracle's pinned MAC accounting
+    from axial_band_split_b200 import accounting
+    from oracle import model as om
+    for cfg, B, T in [(synth.VOCALS, 1, 801), (synth.VOCALS, 1, 1100), (synth.TINY, 2, 32)]:
+        widths = tables.band_tables(cfg.sample_rate, cfg.n_fft, cfg.num_bands)["widths"]
+        m = om.mac_count(cfg, widths, B, T)
+        assert accounting.total_flops(cfg, widths, B, T) == 2 * m["total"]
+        assert accounting.attention_flops(cfg, widths, B, T) == 2 * (m["attn_time"] + m["attn_band"])
+    assert accounting.audio_seconds(synth.VOCALS, 1, 1100) == pytest.approx(11.0)

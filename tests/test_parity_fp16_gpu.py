@@ -1,0 +1,84 @@
+"""fp16 tensor-core schedule against the float64 oracle, through the C ABI (GPU).
+
+Bar (mask domain, all elements): max|diff| <= 2e-2 and SNR >= 40 dB, where
+SNR = 10 log10(sum ref^2 / sum (got - ref)^2).  Weights are rounded to fp16 once and the
+oracle uses the rounded values, so only the fp16 activations and fp32 accumulation of
+the CUDA path count as error."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import synth
+from parity import case, oracle_masks, rel_err, snr_db
+from oracle import model as oracle_model
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+MAX_ABS = 2e-2
+MIN_SNR = 40.0
+
+
+def run(cfg, B, T, W, x, max_batch=None, max_frames=None, graph=True, debug=()):
+    from axial_band_split_b200 import mrf
+    m = mrf.Model(cfg, W, max_batch=max_batch or B, max_frames=max_frames or T, compute=mrf.MRF_FP16)
+    m.set_graph(graph)
+    out = m.forward(torch.from_numpy(x).cuda())
+    m.sync_status()
+    torch.cuda.synchronize()
+    res = out.cpu().numpy()
+    dbg = {}
+    nb = cfg.num_bands
+    if "X" in debug:
+        dbg["X"] = m.debug_buffer("X", B * T * nb * cfg.dim).reshape(B, T, nb, cfg.dim)
+    if "M" in debug:
+        dbg["M"] = m.debug_buffer("M", B * T * 100000).reshape(B, T, -1)
+    m.close()
+    return res, dbg
+
+
+def check(got, ref, what=""):
+    err = float(np.abs(got - ref).max())
+    snr = snr_db(got, ref)
+    assert err <= MAX_ABS and snr >= MIN_SNR, f"{what} max|diff|={err:.3e} snr={snr:.1f} dB"
+    return err, snr
+
+
+def test_mask_head_only_depth0():
+    # no transformer: band split -> mask head -> average (localises GEMM/epilogue errors)
+    cfg = dataclasses.replace(synth.VOCALS, depth=0)
+    B, T = 1, 133
+    W, x = case(cfg, B, T, True)
+    got, dbg = run(cfg, B, T, W, x, debug=("X", "M"))
+    ref, st = oracle_model.forward(x, cfg, W, return_stages=True)
+    check(dbg["X"][0], st[0]["band_split"], "band split")
+    check(dbg["M"][0], st[0]["mask0"], "mask head")
+    check(got, ref, "masks")
+
+
+def test_vocals_depth1_ragged():
+    cfg = dataclasses.replace(synth.VOCALS, depth=1)
+    B, T = 1, 150
+    W, x = case(cfg, B, T, True)
+    got, dbg = run(cfg, B, T, W, x, debug=("X",))
+    ref, st = oracle_model.forward(x, cfg, W, return_stages=True)
+    check(dbg["X"][0], st[0]["layer0.band"], "trunk")
+    check(got, ref, "masks")
+
+
+@pytest.mark.parametrize("B,T", [(1, 32), (2, 17), (1, 1)])
+def test_tiny_fp16(B, T):
+    cfg = synth.TINY
+    W, x = case(cfg, B, T, True)
+    got, _ = run(cfg, B, T, W, x, max_batch=2, max_frames=40)
+    check(got, oracle_masks(cfg, B, T, True), "masks")
+
+
+def test_vocals_full_depth_T300():
+    cfg = synth.VOCALS
+    B, T = 1, 300
+    W, x = case(cfg, B, T, True)
+    got, _ = run(cfg, B, T, W, x)
+    check(got, oracle_masks(cfg, B, T, True), "masks")
