@@ -1,0 +1,370 @@
+#!/usr/bin/env python3
+"""Throughput of the Mel-Band RoFormer core forward on B200 (audio-seconds per second).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the vocals model shape (dim 384, depth 6, 8 heads of 64, 60 mel bands over
+n_fft 2048, mask MLP hidden 1536) on one static window of T = 1100 frames (11.0 s of
+44.1 kHz stereo), B = 1, fp16 operands with fp32 accumulation, random-init weights
+N(0, 0.02) rounded to fp16, stft_repr of seeded synthetic audio (tone stacks + pink
+noise at -20 dBFS).  A step is one full core forward (band split, 6 x (time, band)
+transformer, mask head, overlap average) through mrf_forward, inputs resident on the
+device; the L2 is flushed (256 MiB write) before every timed step, outside its events.
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own replica on its own
+windows (the forward has no exchange step): value = all ranks' audio / max rank time.
+
+--impl reference times the float64 NumPy oracle on the host cores (rank 0 only), on a
+bounded sample of the same model (a window of --ref-frames frames per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "audio-sec separated per sec (core fwd, fp16) at T=1100; attention TFLOP/s vs peak"
+UNIT = "audio-s/s"
+# "musetric/vocal-separation-roformer-onnx", section "What the row cap changed": the core
+# forward at T = 1100 in 1.85 s per 11 s window (desktop NVIDIA, WebGPU, fp16): 11.0 / 1.85.
+PAGES_AUDIO_S_PER_S = 11.0 / 1.85
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--frames", type=int, default=1100)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--ref-frames", type=int, default=32, help="window of one reference-arm step")
+    ap.add_argument("--cpu-sample-frames", type=int, default=110, help="window of the oracle CPU baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--plain", action="store_true",
+                    help="profiling run: warmup + steps eager forwards only, no timing or report")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def workload(cfg, B, T):
+    return {"workload": f"vocals core forward, B={B}, T={T} ({B * T * cfg.hop / cfg.sample_rate:.2f} s audio)",
+            "dim": cfg.dim, "depth": cfg.depth, "heads": cfg.heads, "dim_head": cfg.dim_head,
+            "bands": cfg.num_bands, "n_fft": cfg.n_fft, "batch": B, "frames": T,
+            "weights": "random-init N(0,0.02), fp16-rounded"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"mrf_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if not self.proc or not os.path.exists(self.path):
+            return None
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = max(smax, float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "axial_band_split_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return None
+    k = d.get("kernels", {}).get(kernel)
+    return k.get("dram_bytes_per_launch") if k else None
+
+
+def cpu_baseline(cfg, frames, rank):
+    """The float64 oracle as it stands, timed on this host's cores on one forward of a
+    `frames`-long window of the same model (a bounded sample of the workload)."""
+    import numpy as np
+    import synth
+    from oracle import model as om
+    from oracle import tables as ot
+    widths = ot.band_tables(cfg.sample_rate, cfg.n_fft, cfg.num_bands)["widths"]
+    W = synth.make_weights(cfg, widths, fp16=True)
+    x = synth.make_stft_repr(cfg, 1, frames)
+    t0 = time.perf_counter()
+    om.forward(x, cfg, W)
+    dt = time.perf_counter() - t0
+    audio = frames * cfg.hop / cfg.sample_rate
+    return {"value": audio / dt, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"one float64 forward of the vocals model on a B=1, T={frames} window "
+                      f"({audio:.2f} s audio) in {dt:.1f} s on the host's cores (NumPy/OpenBLAS)"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import synth
+    from oracle import model as om
+    from oracle import tables as ot
+    cfg = synth.VOCALS
+    T = args.ref_frames
+    widths = ot.band_tables(cfg.sample_rate, cfg.n_fft, cfg.num_bands)["widths"]
+    W = synth.make_weights(cfg, widths, fp16=True)
+    x = synth.make_stft_repr(cfg, 1, T)
+    for _ in range(args.warmup):
+        om.forward(x, cfg, W)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        om.forward(x, cfg, W)
+    dt = time.perf_counter() - t0
+    audio = args.steps * T * cfg.hop / cfg.sample_rate
+    value = audio / dt
+    sample = (f"float64 NumPy oracle, vocals model, one B=1 T={T} window ({T * cfg.hop / cfg.sample_rate:.2f} s "
+              f"audio) per step, on the host's cores")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload(cfg, 1, T), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from axial_band_split_b200 import accounting, build, mrf
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    import synth
+    cfg = synth.VOCALS
+    B, T = args.batch, args.frames
+    widths = mrf.band_tables(cfg)["width"]
+    W = {k: v.astype(np.float16) for k, v in synth.make_weights(cfg, widths, fp16=True).items()}
+    model = mrf.Model(cfg, W, max_batch=B, max_frames=T, compute=mrf.MRF_FP16)
+    x_host = synth.make_stft_repr(cfg, B, T, seed=1 + rank)
+    x = torch.from_numpy(x_host).cuda()
+    out = torch.empty_like(x)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    def timed(fn, steps):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        barrier()
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        barrier()
+        ms = sum(a.elapsed_time(b) for a, b in ev)
+        return ms
+
+    fwd = lambda: model.forward(x, out)
+    if args.plain:
+        model.set_graph(False)
+        for _ in range(args.warmup + args.steps):
+            fwd()
+        model.sync_status()
+        torch.cuda.synchronize()
+        print(f"plain run ok: {args.warmup + args.steps} forwards, {model.launches_per_forward(B, T)} launches each")
+        model.close()
+        return 0
+    for _ in range(args.warmup):
+        fwd()
+    model.sync_status()
+    with ClockSampler(local) as clk:
+        ms = timed(fwd, args.steps)
+    model.sync_status()
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t.item())
+    launches = model.launches_per_forward(B, T)
+    audio_total = world * args.steps * accounting.audio_seconds(cfg, B, T)
+    value = audio_total / (ms_max / 1e3)
+
+    # per-kernel times: the same steps launched eagerly with an event pair around each kernel
+    model.set_timing(True)
+    ktimed = timed(fwd, args.steps)
+    kt = model.kernel_times()
+    model.set_timing(False)
+    model.sync_status()
+
+    # end to end through the public host-buffer entry point: H2D + forward + D2H per step
+    xin = torch.from_numpy(x_host).pin_memory()
+    xout = torch.empty_like(xin).pin_memory()
+    e2e_fn = lambda: model.forward_host(xin, xout, stream=stream)
+    e2e_fn()
+    ms_e2e = timed(e2e_fn, args.steps)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    io_bytes = int(x_host.nbytes)
+
+    if rank != 0:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return 0
+
+    peaks, peak_src = load_peaks()
+    work = accounting.kernel_work(cfg, widths, B, T)
+    per_kernel = {}
+    for name, (n, tot) in kt.items():
+        kind, amount, nl = work.get(name, ("?", 0, n))
+        per_launch = amount / max(nl, 1)
+        avg = tot / max(n, 1)
+        per_kernel[name] = {"launches_per_step": n / args.steps, "ms_per_step": tot / args.steps,
+                            "share": tot / max(sum(v[1] for v in kt.values()), 1e-9),
+                            "achieved": (per_launch / (avg / 1e3) / (1e12 if kind == "flop" else 1e9)) if avg > 0 else None,
+                            "unit": "TFLOP/s" if kind == "flop" else "GB/s"}
+    dom = max(kt.items(), key=lambda kv: kv[1][1])[0]
+    kind, amount, nl = work[dom]
+    avg_ms = kt[dom][1] / kt[dom][0]
+    if kind == "flop" and dom != "band_split":
+        bound, unit = "tensor", "TFLOP/s"
+        peak = peaks["bf16_tflops_sustained"]
+        achieved = amount / nl / (avg_ms / 1e3) / 1e12
+    elif kind == "flop":
+        bound, unit = "alu", "TFLOP/s"
+        peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        achieved = amount / nl / (avg_ms / 1e3) / 1e12
+    else:
+        bound, unit = "hbm", "GB/s"
+        peak = peaks["hbm_gbs"]
+        achieved = amount / nl / (avg_ms / 1e3) / 1e9
+    attn_ms = sum(kt[k][1] for k in ("attn_time_tc", "attn_band_tc") if k in kt) / args.steps
+    gemm_ms = sum(v[1] for k, v in kt.items() if k.startswith("gemm_")) / args.steps
+    attn_fl = accounting.attention_flops(cfg, widths, B, T)
+    gemm_fl = sum(v[1] for k, v in work.items() if k.startswith("gemm_"))
+    total_fl = accounting.total_flops(cfg, widths, B, T)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": value / PAGES_AUDIO_S_PER_S, "dtype": "f16", "data": "synthetic",
+        "config": dict(workload(cfg, B, T), l2="flushed by a 256 MiB write before every timed step",
+                       parallelism=f"replicas x{world}"),
+        "roofline": {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "peak_source": peak_src + (" sustained" if bound == "tensor" else ""),
+                     "traffic": traffic_for(dom), "algorithmic_per_launch": amount / nl},
+        "attention": {"tflops": attn_fl / (attn_ms / 1e3) / 1e12 if attn_ms else None,
+                      "frac_of_peak": (attn_fl / (attn_ms / 1e3) / 1e12) / peaks["bf16_tflops_sustained"] if attn_ms else None},
+        "gemm": {"tflops": gemm_fl / (gemm_ms / 1e3) / 1e12 if gemm_ms else None,
+                 "frac_of_peak": (gemm_fl / (gemm_ms / 1e3) / 1e12) / peaks["bf16_tflops_sustained"] if gemm_ms else None},
+        "forward": {"tflops": total_fl / (ms_max / args.steps / 1e3) / 1e12,
+                    "frac_of_peak_burst": total_fl / (ms_max / args.steps / 1e3) / 1e12 / peaks["bf16_tflops"]},
+        "kernels": per_kernel,
+        "kernel_timing_ms_per_step": ktimed / args.steps,
+        "e2e": {"value": world * args.steps * accounting.audio_seconds(cfg, B, T) / (ms_e2e / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_sample_frames, rank)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    model.close()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
