@@ -33,6 +33,9 @@ def kernel_work(cfg, widths, B: int, T: int):
         "gemm_mask_tanh": ("flop", 2 * BT * nb * (D * MH + (cfg.mask_depth - 1) * MH * MH), cfg.mask_depth),
         "gemm_mask_glu": ("flop", 2 * BT * MH * 2 * n_feat, 1),
         "band_split": ("flop", 2 * BT * D * n_feat, 1),
+        "gemm_band_split": ("flop", 2 * BT * D * n_feat, 1),
+        # stft_repr read once, normalised fp16 band features written once
+        "band_gather": ("byte", B * rows * T * 2 * 4 + BT * n_feat * 2, 1),
         # x fp32 read + write, x fp16 write, |x|^2 read + write, gain
         "outnorm": ("byte", L2 * NT * (D * 4 * 2 + D * 2 + 8), L2),
         # mask features fp32 read once, masks fp32 written once
@@ -43,7 +46,8 @@ def kernel_work(cfg, widths, B: int, T: int):
 
 def total_flops(cfg, widths, B: int, T: int) -> int:
     """FLOPs of one forward: every contraction of the method."""
-    return sum(v for k, v, _ in kernel_work(cfg, widths, B, T).values() if k == "flop")
+    return sum(v for name, (k, v, _) in kernel_work(cfg, widths, B, T).items()
+               if k == "flop" and name != "band_split")
 
 
 def attention_flops(cfg, widths, B, T):

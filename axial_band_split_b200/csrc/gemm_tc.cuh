@@ -16,7 +16,7 @@ struct GemmGroup {
   int b_row_off;     // first row of the group's weight in the stacked weight matrix
   int out_off;       // epilogue output offset of the group
   int bias_off;      // offset of the group's bias
-  int pad;
+  int kblocks;       // 64-wide K blocks of the group (0: K / 64 of the launch)
 };
 
 enum GemmEpi : int {
@@ -25,6 +25,7 @@ enum GemmEpi : int {
   kTcGelu = 2,    // out = gelu(acc * rowscale + bias) fp16
   kTcTanh = 3,    // out = tanh(acc + bias) fp16 (group-strided)
   kTcGlu = 4,     // interleaved (value, gate) pairs -> value * sigmoid(gate), fp32
+  kTcBandSplit = 5,  // X = acc + bias for token m*nb + group (band); X fp32, X fp16, row sum of squares
 };
 
 struct GemmParams {
@@ -57,7 +58,7 @@ bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, un
                    unsigned box2);
 
 constexpr int kGemmStages = 4;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
 size_t gemm_smem_bytes();
 // Resolve the tensor-map encoder and set the kernels' shared-memory limits (call once, outside capture).
 bool gemm_tc_init();

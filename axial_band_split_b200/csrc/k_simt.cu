@@ -117,6 +117,47 @@ __global__ void __launch_bounds__(kBsThreads) band_split_kernel(
   }
 }
 
+// Gather + normalise only (fp16 schedule): per band k and frame bt, the band's features
+// divided by their L2 norm, fp16, into A[(k * frame_stride + bt) * k_stride + e] for
+// e < k_pad(k) (zeros past the band's width), the A operand of the band-split GEMM.
+__global__ void __launch_bounds__(kBsThreads) band_gather_kernel(
+    const float *__restrict__ in, const int32_t *__restrict__ feat_row, const int32_t *__restrict__ feat_c,
+    const BandDesc *__restrict__ bands, int B, int T, int R, long long frame_stride, int k_stride,
+    __half *__restrict__ A) {
+  extern __shared__ float xs[];  // [kBsFrames][width]
+  const int k = blockIdx.y;
+  const BandDesc bd = bands[k];
+  const int W = bd.width, Wp = (W + 63) & ~63;
+  const long long frames = (long long)B * T;
+  const long long f0 = (long long)blockIdx.x * kBsFrames;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < kBsFrames * W; i += kBsThreads) {
+    const int f = i / W, e = i % W;
+    const long long bt = f0 + f;
+    float v = 0.f;
+    if (bt < frames) {
+      const long long b = bt / T, t = bt % T;
+      v = in[((b * R + feat_row[bd.feat_off + e]) * T + t) * 2 + feat_c[bd.feat_off + e]];
+    }
+    xs[i] = v;
+  }
+  __syncthreads();
+  for (int f = warp; f < kBsFrames; f += kBsThreads / 32) {
+    float s = 0.f;
+    for (int e = lane; e < W; e += 32) s += xs[f * W + e] * xs[f * W + e];
+    s = warp_sum(s);
+    const float r = 1.f / fmaxf(sqrtf(s), kNormEps);
+    for (int e = lane; e < W; e += 32) xs[f * W + e] *= r;
+  }
+  __syncthreads();
+  for (int i = tid; i < kBsFrames * Wp; i += kBsThreads) {
+    const int f = i / Wp, e = i % Wp;
+    const long long bt = f0 + f;
+    if (bt >= frames) continue;
+    A[((long long)k * frame_stride + bt) * k_stride + e] = __float2half_rn(e < W ? xs[f * W + e] : 0.f);
+  }
+}
+
 // ------------------------------------------------------------------ grouped SIMT GEMM
 constexpr int kGt = 64, kGk = 16;
 
@@ -357,6 +398,15 @@ void launch_band_split(const float *in, const int32_t *feat_row, const int32_t *
   const size_t smem = sizeof(float) * kBsFrames * max_width;
   band_split_kernel<<<grid, kBsThreads, smem, st>>>(in, feat_row, feat_c, bands, nb, w, bias, dim,
                                                    B, T, rows, X, Xh, ss);
+}
+
+void launch_band_gather(const float *in, const int32_t *feat_row, const int32_t *feat_c, const BandDesc *bands,
+                        int nb, int B, int T, int rows, long long frame_stride, int k_stride, __half *A,
+                        int max_width, cudaStream_t st) {
+  const long long frames = (long long)B * T;
+  dim3 grid(grid1(frames, kBsFrames), nb);
+  band_gather_kernel<<<grid, kBsThreads, sizeof(float) * kBsFrames * max_width, st>>>(
+      in, feat_row, feat_c, bands, B, T, rows, frame_stride, k_stride, A);
 }
 
 void launch_gemm_f32(const float *A, const float *W, const float *bias, float *C,

@@ -41,12 +41,16 @@ struct TrF16 {
 
 struct Fp16State {
   std::vector<TrF16> tr;
+  __half *w_bs = nullptr;     // band split [nb*D, k_bs], gamma*sqrt(d_in) folded, zero-padded
+  __half *A_bs = nullptr;     // normalised band features [nb][MBT][k_bs]
+  int k_bs = 0;
+  GemmGroup *g_bs = nullptr;
   std::vector<__half *> mw;   // mask layers 0 .. mask_depth-1, stacked over bands [nb*MH, K]
   std::vector<float *> mb;
   __half *mw_last = nullptr;  // [sum 2*d_in, MH], rows interleaved (value e, gate e)
   float *mb_last = nullptr;
   // group tables
-  GemmGroup *g_qkv = nullptr, *g_out = nullptr, *g_ff1 = nullptr, *g_ff2 = nullptr;
+  GemmGroup *g_qkv = nullptr, *g_qkv_time = nullptr, *g_out = nullptr, *g_ff1 = nullptr, *g_ff2 = nullptr;
   GemmGroup *g_m0 = nullptr, *g_mid = nullptr, *g_last = nullptr;
   int n_last_tiles = 0;
   // workspace
@@ -116,6 +120,28 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
     h->err = "tcgen05 kernel initialisation failed (tensor-map encoder or shared-memory limit)";
     return MRF_ECUDA;
   }
+  // band split: per band [D, d_in] with gamma*sqrt(d_in) folded, zero-padded to k_bs columns
+  f->k_bs = cdiv(h->max_width, 64) * 64;
+  {
+    std::vector<float> wb((size_t)nb * D * f->k_bs, 0.f);
+    for (int k = 0; k < nb; ++k) {
+      const std::string p = "band_split.to_features." + std::to_string(k) + ".";
+      const auto &g = W[p + "0.gamma"].v;
+      const auto &w = W[p + "1.weight"].v;
+      const int wd = t.width[k];
+      const double sc = std::sqrt((double)wd);
+      for (int n = 0; n < D; ++n)
+        for (int e = 0; e < wd; ++e)
+          wb[((size_t)k * D + n) * f->k_bs + e] = (float)((double)w[(size_t)n * wd + e] * g[e] * sc);
+    }
+    f->w_bs = up(h, to_half(wb));
+    std::vector<GemmGroup> gb(nb);
+    for (int k = 0; k < nb; ++k)
+      gb[k] = {D, cdiv(D, kBnNarrow), k * cdiv(D, kBnNarrow), (int)(k * MBT), k * D, k, k * D, cdiv(t.width[k], 64)};
+    f->g_bs = upload_groups(h, gb);
+    f->A_bs = h->alloc<__half>((size_t)nb * MBT * f->k_bs);
+    if (!f->w_bs || !f->g_bs || !f->A_bs) return MRF_ENOMEM;
+  }
   // transformers
   f->tr.resize(2 * c.depth);
   for (int l = 0; l < c.depth; ++l)
@@ -178,7 +204,10 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->g_out = single(D, kBnNarrow);
   f->g_ff1 = single(FF, kBnWide);
   f->g_ff2 = single(D, kBnNarrow);
-  std::vector<GemmGroup> g0(nb), g1(nb), g2(nb);
+  std::vector<GemmGroup> gq(nb), g0(nb), g1(nb), g2(nb);
+  const int nq = cdiv(3 * A + H, kBnWide);
+  for (int k = 0; k < nb; ++k) gq[k] = {3 * A + H, nq, k * nq, k, 0, k, 0, 0};
+  f->g_qkv_time = upload_groups(h, gq);
   int start = 0;
   for (int k = 0; k < nb; ++k) {
     g0[k] = {MH, cdiv(MH, kBnWide), k * cdiv(MH, kBnWide), k, k * MH, k, k * MH, 0};
@@ -191,7 +220,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->g_m0 = upload_groups(h, g0);
   f->g_mid = upload_groups(h, g1);
   f->g_last = upload_groups(h, g2);
-  if (!f->g_qkv || !f->g_out || !f->g_ff1 || !f->g_ff2 || !f->g_m0 || !f->g_mid || !f->g_last) return MRF_ENOMEM;
+  if (!f->g_qkv || !f->g_qkv_time || !f->g_out || !f->g_ff1 || !f->g_ff2 || !f->g_m0 || !f->g_mid || !f->g_last) return MRF_ENOMEM;
   // workspace
   f->n_pad_time = cdiv(c.max_frames, 128) * 128;
   f->n_pad_band = cdiv(nb, 64) * 64;
@@ -277,6 +306,9 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
             make_tmap_f16(&mXband, f->Xh, D, nb, MBT, D, (long long)nb * D, 1, 128) &&
             make_tmap_f16(&mH1, f->H1, MH, nb * MBT, 1, MH, nb * MBT * MH, 128, 1) &&
             make_tmap_f16(&mH2, f->H2, MH, nb * MBT, 1, MH, nb * MBT * MH, 128, 1);
+  CUtensorMap mAbs, mWbs;
+  ok = ok && make_tmap_f16(&mAbs, f->A_bs, f->k_bs, (long long)nb * MBT, 1, f->k_bs, (long long)nb * MBT * f->k_bs, 128, 1) &&
+       make_tmap_f16(&mWbs, f->w_bs, f->k_bs, (long long)nb * D, 1, f->k_bs, (long long)nb * D * f->k_bs, kBnNarrow, 1);
   std::vector<CUtensorMap> wmaps(4 * 2 * c.depth + c.mask_depth + 1);
   for (int i = 0; ok && i < 2 * c.depth; ++i) {
     const TrF16 &w = f->tr[i];
@@ -297,10 +329,15 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     return;
   }
 
-  h->begin("band_split");
-  launch_band_split(in, h->d_feat_row, h->d_feat_c, h->d_bands, nb, h->w_bs, h->b_bs, D, B, T, R, f->X, f->Xh,
-                    f->ss, st, h->max_width);
+  h->begin("band_gather");
+  launch_band_gather(in, h->d_feat_row, h->d_feat_c, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, h->max_width, st);
   h->end();
+  cudaMemsetAsync(f->ss, 0, sizeof(float) * M, st);
+  {
+    GemmParams p = base_params(h, B * T, f->k_bs, kBnNarrow, f->g_bs, nb, nb * cdiv(D, kBnNarrow));
+    p.bias = h->b_bs; p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D; p.nb = nb;
+    gemm(h, "gemm_band_split", kTcBandSplit, mAbs, mWbs, p);
+  }
 
   for (int i = 0; i < 2 * c.depth; ++i) {
     const TrF16 &w = f->tr[i];
@@ -309,12 +346,15 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
                       &mW2 = wmaps[4 * i + 3];
     const int n_pad = axis == 0 ? f->n_pad_time : f->n_pad_band;
 
-    // q, k, v, gates
-    GemmParams p = base_params(h, M, D, kBnWide, f->g_qkv, 1, cdiv(3 * A + H, kBnWide));
+    // q, k, v, gates; on the time axis the rows run band-major (frame m of band g) so that
+    // consecutive rows of a tile are consecutive positions of one sequence
+    GemmParams p = axis == 0 ? base_params(h, B * T, D, kBnWide, f->g_qkv_time, nb, nb * cdiv(3 * A + H, kBnWide))
+                             : base_params(h, M, D, kBnWide, f->g_qkv, 1, cdiv(3 * A + H, kBnWide));
+    p.a_mode = axis == 0 ? 1 : 0;
     p.ss_in = f->ss;
     p.q = f->Q; p.k = f->K; p.v = f->V; p.gates = f->G; p.rope = h->d_rope; p.gbias = w.bg;
     p.B = B; p.T = T; p.nb = nb; p.H = H; p.dh = dh; p.A = A; p.axis = axis; p.n_pad = n_pad;
-    gemm(h, "gemm_qkv", kTcQkv, mXh, mWqkv, p);
+    gemm(h, "gemm_qkv", kTcQkv, axis == 0 ? mXband : mXh, mWqkv, p);
 
     h->begin(f->tc_attention ? (axis == 0 ? "attn_time_tc" : "attn_band_tc") : "attn_simt_f16");
     if (f->tc_attention) {
