@@ -49,6 +49,7 @@ struct GemmParams {
   const float2 *rope;
   const float *gbias;
   int B, T, nb, H, dh, A, axis, n_pad;
+  float q_scale;            // q is multiplied by this after RoPE (the attention's softmax scale)
 };
 
 // Encode a 3D fp16 tensor map with a 128-byte swizzle and a (64, box1, box2) box.

@@ -48,6 +48,21 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe: x = n + f with n = round(x) (magic-number rounding), 2^f by a
+// degree-3 minimax polynomial on [-1/2, 1/2] (relative error 7.5e-5, coefficients from
+// fit_exp2_poly.py), and 2^n added into the exponent bits.  x <= 8 here; below -126 the
+// result is flushed to 0 like ex2.approx.ftz.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;          // 1.5 * 2^23: round to nearest integer
+  const float n = t - 12582912.f;
+  const float f = x - n;
+  float p = fmaf(0.055171669f, f, 0.242611122f);
+  p = fmaf(p, f, 0.693260985f);
+  p = fmaf(p, f, 0.999928074f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -222,7 +237,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + 128 * t + lane_off, tO = tmem + 256 + 64 * t + lane_off;
-    const float sl2 = 1.4426950408889634f * rsqrtf((float)kDh);
     uint8_t *prow = smem + AttnSmem::p + t * 2 * kTile + r * 128;
     const int prob = r >> 6;  // band axis: which of the tile's two problems
     int g = 0;
@@ -236,16 +250,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         int lo, hi;
         if (a.axis == 0) { lo = 0; hi = min(kKeys, a.n - j * kKeys); }
         else { lo = prob * 64; hi = prob * 64 + a.n; }
+        const bool full_blk = lo == 0 && hi == kKeys;  // no masking needed (warp-uniform on the time axis)
         float mx = -INFINITY;
+        if (full_blk) {
 #pragma unroll
-        for (int c = 0; c < kKeys; c += 32) {
-          float v[32];
-          tc::tmem_ld32(tS + c, v);
+          for (int c = 0; c < kKeys; c += 32) {
+            float v[32];
+            tc::tmem_ld32(tS + c, v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c + i >= lo && c + i < hi) mx = fmaxf(mx, v[i]);
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, v[i]);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < kKeys; c += 32) {
+            float v[32];
+            tc::tmem_ld32(tS + c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c + i >= lo && c + i < hi) mx = fmaxf(mx, v[i]);
+          }
         }
-        const float m_cand = fmaxf(m_run, mx * sl2);
+        // scores arrive in log2 units (q was scaled by log2(e) / sqrt(dh) in its projection)
+        const float m_cand = fmaxf(m_run, mx);
         // P_t and O_t are free once the previous block's P*V has completed
         if (j > 0 && !tc::mbar_wait(pv_done + t, (g - 1) & 1, a.status, 39, abort)) { ok = false; break; }
         const bool need = m_cand > m_run + kRescaleLog2;
@@ -272,8 +298,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t h[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2) {
-            const float p0 = (c + i >= lo && c + i < hi) ? ex2(v[i] * sl2 - m_run) : 0.f;
-            const float p1 = (c + i + 1 >= lo && c + i + 1 < hi) ? ex2(v[i + 1] * sl2 - m_run) : 0.f;
+            float p0, p1;
+            // one pair in four on the FMA pipe, the rest on MUFU
+            if (((i >> 1) & 3) == 3) { p0 = exp2_fma(v[i] - m_run); p1 = exp2_fma(v[i + 1] - m_run); }
+            else { p0 = ex2(v[i] - m_run); p1 = ex2(v[i + 1] - m_run); }
+            if (!full_blk) {
+              if (!(c + i >= lo && c + i < hi)) p0 = 0.f;
+              if (!(c + i + 1 >= lo && c + i + 1 < hi)) p1 = 0.f;
+            }
             sum += p0 + p1;
             h[i >> 1] = pack_h2(p0, p1);
           }

@@ -429,11 +429,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int head = (c0 - which * p.A) >> 6;
             const int d0 = c0 & 63;
             if (which < 2) {
+              const float sc = which == 0 ? p.q_scale : 1.f;
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const float x0 = v[2 * i], x1 = v[2 * i + 1];
-                v[2 * i] = x0 * cs[i].x - x1 * cs[i].y;
-                v[2 * i + 1] = x1 * cs[i].x + x0 * cs[i].y;
+                v[2 * i] = (x0 * cs[i].x - x1 * cs[i].y) * sc;
+                v[2 * i + 1] = (x1 * cs[i].x + x0 * cs[i].y) * sc;
               }
             }
             __half *dst = which == 0 ? p.q : which == 1 ? p.k : p.v;
@@ -456,12 +457,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int j = 0; j < 8; ++j) o[j] = v[j8 + j];
               if (which < 2) {
+                const float sc = which == 0 ? p.q_scale : 1.f;
 #pragma unroll
                 for (int j = 0; j < 8; j += 2) {
                   const float2 cc = p.rope[(long long)qr.pos * half_dh + ((dd + j) >> 1)];
                   const float x0 = o[j], x1 = o[j + 1];
-                  o[j] = x0 * cc.x - x1 * cc.y;
-                  o[j + 1] = x1 * cc.x + x0 * cc.y;
+                  o[j] = (x0 * cc.x - x1 * cc.y) * sc;
+                  o[j + 1] = (x1 * cc.x + x0 * cc.y) * sc;
                 }
               }
               __half *dst = which == 0 ? p.q : which == 1 ? p.k : p.v;

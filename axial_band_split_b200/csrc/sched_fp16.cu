@@ -354,6 +354,8 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     p.ss_in = f->ss;
     p.q = f->Q; p.k = f->K; p.v = f->V; p.gates = f->G; p.rope = h->d_rope; p.gbias = w.bg;
     p.B = B; p.T = T; p.nb = nb; p.H = H; p.dh = dh; p.A = A; p.axis = axis; p.n_pad = n_pad;
+    // the tensor-core attention takes scores in log2 units: fold log2(e) / sqrt(dh) into q
+    p.q_scale = f->tc_attention ? (float)(1.4426950408889634 / std::sqrt((double)dh)) : 1.f;
     gemm(h, "gemm_qkv", kTcQkv, axis == 0 ? mXband : mXh, mWqkv, p);
 
     h->begin(f->tc_attention ? (axis == 0 ? "attn_time_tc" : "attn_band_tc") : "attn_simt_f16");
