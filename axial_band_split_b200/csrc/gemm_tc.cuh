@@ -52,6 +52,13 @@ struct GemmParams {
   float q_scale;            // q is multiplied by this after RoPE (the attention's softmax scale)
 };
 
+enum TmapDtype : int { kTmF16 = 0, kTmF32 = 1 };
+
+// Encode a tensor map of rank 1..3: dims and strides in elements (strides of dims 1..rank-1),
+// box in elements, swizzle 0 / 32 / 64 / 128 bytes.
+bool make_tmap(CUtensorMap *map, const void *base, int dtype, int rank, const unsigned long long *dims,
+               const unsigned long long *strides_el, const unsigned *box, int swizzle_bytes);
+
 // Encode a 3D fp16 tensor map with a 128-byte swizzle and a (64, box1, box2) box.
 // dims/strides in elements; strides[0] is the stride of dim 1, strides[1] of dim 2.
 bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, unsigned long long d1,
@@ -60,11 +67,15 @@ bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, un
 
 constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 320;
-size_t gemm_smem_bytes();
 // Resolve the tensor-map encoder and set the kernels' shared-memory limits (call once, outside capture).
 bool gemm_tc_init();
 
-void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p,
-                    int grid, cudaStream_t st);
+// tmC / tmD: output tensor maps of the epilogues that store through bulk tensor stores
+// (kTcResid: X fp32 [M, ld] box 32x32 swizzle 128 and X fp16 box 32x32 swizzle 64;
+//  kTcBandSplit: the same as 3D (ld, nb, frames) boxes 32x1x32; kTcGelu: out fp16 [M, ldo]
+//  box 32x32 swizzle 64; kTcTanh: out fp16 (ldo, frames, groups) box 32x32x1 swizzle 64;
+//  kTcGlu: out fp32 [frames, ldo] box 16x32 swizzle 64).  Unused maps may be any valid map.
+void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
+                    const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st);
 
 }  // namespace mrf

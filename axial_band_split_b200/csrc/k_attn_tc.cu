@@ -63,10 +63,6 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
@@ -320,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l += sum;
         tc::tc_fence_before();
-        fence_proxy_async();
+        tc::fence_proxy_async();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(p_full + t);
       }

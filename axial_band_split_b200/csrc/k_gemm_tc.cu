@@ -14,9 +14,14 @@
 //              (two warps per TMEM lane quarter, alternating 32-column chunks)
 //   warp 8     TMA producer (one lane) and TMEM allocator
 //   warp 9     MMA issuer (one lane): 4 x tcgen05.mma (M=128, N<=256, K=16) per 64-wide K block
-// Shared memory: kGemmStages stages of A (128 x 64) and B (256 x 64) tiles, 128-byte swizzle.
-// Tensor memory: two 256-column fp32 accumulators, so the epilogue of tile i overlaps the
-// main loop of tile i+1.
+// Shared memory: kGemmStages stages of A (128 x 64) and B (BN x 64) tiles, 128-byte swizzle,
+// then per-epilogue-warp output boxes.  Tensor memory: two 256-column fp32 accumulators, so
+// the epilogue of tile i overlaps the main loop of tile i+1.
+//
+// Epilogue stores: each warp writes its 32 rows x 32 columns into a shared-memory box in the
+// tensor map's swizzled layout and one lane issues a bulk tensor store (cp.async.bulk.tensor),
+// so global writes leave the SM as whole lines; rows past M are clipped by the tensor map.
+// The q, k, v scatter keeps plain stores through an 80-byte-row staging buffer.
 #include <cudaTypedefs.h>
 
 #include <cmath>
@@ -30,19 +35,27 @@ namespace mrf {
 
 namespace {
 
-constexpr int BM = 128, BK = 64, BN_MAX = 256;
+constexpr int BM = 128, BK = 64;
 constexpr int A_STAGE = BM * BK * 2;        // 16 KB
-constexpr int B_STAGE = BN_MAX * BK * 2;    // 32 KB
 constexpr int TMEM_COLS = 512;
 constexpr float kEps = 1e-12f;
-
 constexpr int kEpiWarps = 8;
 
+// Widest B tile of an epilogue kind, and the shared memory each epilogue warp needs.
+__host__ __device__ constexpr int bn_max(int epi) { return (epi == kTcResid || epi == kTcBandSplit) ? 192 : 256; }
+__host__ __device__ constexpr int warp_stage_bytes(int epi) {
+  return epi == kTcQkv ? 32 * 80                                           // row staging (80-byte rows)
+         : (epi == kTcResid || epi == kTcBandSplit) ? 4096 + 2048         // fp32 box + fp16 box
+                                                    : 2 * 2048;           // two 2 KB boxes
+}
+
+template <int EPI>
 struct SmemLayout {
+  static constexpr int b_stage = bn_max(EPI) * BK * 2;
   static constexpr int a_off = 0;
   static constexpr int b_off = kGemmStages * A_STAGE;
-  static constexpr int stg_off = b_off + kGemmStages * B_STAGE;
-  static constexpr int bar_off = stg_off + kEpiWarps * 32 * 80;
+  static constexpr int stg_off = b_off + kGemmStages * b_stage;             // 1024-aligned
+  static constexpr int bar_off = stg_off + kEpiWarps * warp_stage_bytes(EPI);
   static constexpr int total = bar_off + 256;
 };
 
@@ -87,14 +100,8 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams &p, int tile) {
   return ti;
 }
 
-// ------------------------------------------------------------------ epilogues
-// Epilogue warp w owns TMEM lane quarter w % 4 (rows 32 (w % 4) .. +31 of the tile) and
-// the 32-column chunks c = w / 4, w / 4 + 2, ... of the tile.  Global stores and the
-// residual loads go through a per-warp staging buffer so that every warp instruction
-// moves whole 64-byte row segments (4 lanes per row, 8 rows per instruction).
-
-constexpr int kStageRow = 80;                   // 64 data bytes + 16 pad (conflict-free)
-constexpr int kStageWarp = 32 * kStageRow;
+// ------------------------------------------------------------------ epilogue helpers
+constexpr int kStageRow = 80;  // q, k, v row staging: 64 data bytes + 16 pad (conflict-free)
 
 __device__ __forceinline__ float row_scale(const GemmParams &p, long long row) {
   if (!p.ss_in) return 1.f;
@@ -119,7 +126,8 @@ __device__ __forceinline__ float erf_as(float x) {
 
 __device__ __forceinline__ float gelu_(float x) { return 0.5f * x * (1.f + erf_as(x * 0.70710678118654752f)); }
 
-// Each lane passes its row's destination (null: skip) and 64 bytes; written coalesced.
+// q, k, v: each lane passes its row's destination (null: skip) and 64 bytes; written
+// coalesced through the staging buffer (4 lanes per row, 8 rows per instruction).
 __device__ __forceinline__ void warp_store64(uint8_t *stg, int lane, uint8_t *dst, const uint4 (&d)[4]) {
   uint8_t *my = stg + lane * kStageRow;
 #pragma unroll
@@ -136,30 +144,6 @@ __device__ __forceinline__ void warp_store64(uint8_t *stg, int lane, uint8_t *ds
   __syncwarp();
 }
 
-// Coalesced 64-byte-per-row load, phase A: issue the global loads (lane holds pieces of rows
-// i*8 + lane/4).  Phase B: redistribute through staging so each lane gets its own row.
-__device__ __forceinline__ void warp_load64_issue(int lane, const uint8_t *src, uint4 (&pc)[4]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = i * 8 + (lane >> 2), q = lane & 3;
-    const uint8_t *rs = reinterpret_cast<const uint8_t *>(
-        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src), r));
-    pc[i] = rs ? *reinterpret_cast<const uint4 *>(rs + q * 16) : make_uint4(0, 0, 0, 0);
-  }
-}
-
-__device__ __forceinline__ void warp_load64_finish(uint8_t *stg, int lane, const uint4 (&pc)[4], uint4 (&d)[4]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = i * 8 + (lane >> 2), q = lane & 3;
-    *reinterpret_cast<uint4 *>(stg + r * kStageRow + q * 16) = pc[i];
-  }
-  __syncwarp();
-#pragma unroll
-  for (int q = 0; q < 4; ++q) d[q] = *reinterpret_cast<const uint4 *>(stg + lane * kStageRow + q * 16);
-  __syncwarp();
-}
-
 __device__ __forceinline__ void pack16(const float *v, uint4 (&d)[4]) {
   // 32 floats -> 32 fp16 (64 bytes)
 #pragma unroll
@@ -168,22 +152,27 @@ __device__ __forceinline__ void pack16(const float *v, uint4 (&d)[4]) {
                       pack_h2(v[8 * q + 4], v[8 * q + 5]), pack_h2(v[8 * q + 6], v[8 * q + 7]));
 }
 
-__device__ __forceinline__ void as_u4(const float *v, uint4 (&d)[4]) {
-  // 16 floats (64 bytes)
+// Box rows in shared memory, in the layouts the tensor maps' swizzle modes define:
+// 128-byte rows with SWIZZLE_128B (16-byte chunk index ^= row % 8) and 64-byte rows with
+// SWIZZLE_64B (chunk index ^= (row / 2) % 4).  Both are conflict-free for row-per-lane access.
+__device__ __forceinline__ void box128_put_row(uint8_t *box, int row, const float *v) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
-    d[q] = make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]), __float_as_uint(v[4 * q + 2]),
-                      __float_as_uint(v[4 * q + 3]));
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<float4 *>(box + row * 128 + ((q ^ (row & 7)) << 4)) =
+        make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
-__device__ __forceinline__ void from_u4(const uint4 (&d)[4], float *v) {
+__device__ __forceinline__ void box128_get_row(const uint8_t *box, int row, float *v) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    v[4 * q] = __uint_as_float(d[q].x);
-    v[4 * q + 1] = __uint_as_float(d[q].y);
-    v[4 * q + 2] = __uint_as_float(d[q].z);
-    v[4 * q + 3] = __uint_as_float(d[q].w);
+  for (int q = 0; q < 8; ++q) {
+    const float4 a = *reinterpret_cast<const float4 *>(box + row * 128 + ((q ^ (row & 7)) << 4));
+    v[4 * q] = a.x; v[4 * q + 1] = a.y; v[4 * q + 2] = a.z; v[4 * q + 3] = a.w;
   }
+}
+
+__device__ __forceinline__ void box64_put_row(uint8_t *box, int row, const uint4 (&d)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4 *>(box + row * 64 + ((q ^ ((row >> 1) & 3)) << 4)) = d[q];
 }
 
 // Token of row m of group g: band-major rows (a_mode 1) are frame m of band g.
@@ -212,16 +201,27 @@ __device__ __forceinline__ QkvRow qkv_row(const GemmParams &p, int m, int g) {
   return r;
 }
 
+__device__ __forceinline__ void load_bias32(const float *b, float *bv) {
+  const float4 *b4 = reinterpret_cast<const float4 *>(b);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 x = b4[j];
+    bv[4 * j] = x.x; bv[4 * j + 1] = x.y; bv[4 * j + 2] = x.z; bv[4 * j + 3] = x.w;
+  }
+}
+
 // ------------------------------------------------------------------ the kernel
 template <int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                    const GemmParams p) {
+  using L = SmemLayout<EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sA = smem + SmemLayout::a_off;
-  uint8_t *sB = smem + SmemLayout::b_off;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + SmemLayout::bar_off);
+  uint8_t *sA = smem + L::a_off;
+  uint8_t *sB = smem + L::b_off;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::bar_off);
   uint64_t *full = bars;                       // [stages]
   uint64_t *empty = bars + kGemmStages;        // [stages]
   uint64_t *tfull = bars + 2 * kGemmStages;    // [2]
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc::mbar_arrive_expect_tx(full + stage, bytes);
           if (p.a_mode == 0) tc::tma_load_3d(sA + stage * A_STAGE, &tmA, full + stage, kb * BK, gr.a_off + m0, 0);
           else tc::tma_load_3d(sA + stage * A_STAGE, &tmA, full + stage, kb * BK, gr.a_off, m0);
-          tc::tma_load_3d(sB + stage * B_STAGE, &tmB, full + stage, kb * BK, n0, 0);
+          tc::tma_load_3d(sB + stage * L::b_stage, &tmB, full + stage, kb * BK, n0, 0);
           if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!tc::mbar_wait(full + stage, phase, p.status, 12, abort)) { ok = false; break; }
           tc::tc_fence_after();
           const uint32_t a_addr = tc::smem_u32(sA + stage * A_STAGE);
-          const uint32_t b_addr = tc::smem_u32(sB + stage * B_STAGE);
+          const uint32_t b_addr = tc::smem_u32(sB + stage * L::b_stage);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             tc::mma_f16(d_tmem, tc::sw128_kmajor_desc(a_addr + kk * 32), tc::sw128_kmajor_desc(b_addr + kk * 32),
@@ -314,15 +314,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ---------------- epilogue warps 0-7
     const int quarter = warp & 3, half = warp >> 2;
-    uint8_t *stg = smem + SmemLayout::stg_off + warp * kStageWarp;
+    uint8_t *stg = smem + L::stg_off + warp * warp_stage_bytes(EPI);
+    int nstore = 0;  // boxes this warp has stored (double-buffer parity)
     int local = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       const TileInfo ti = decode_tile(p, tile);
       const GemmGroup &gr = p.groups[ti.g];
       const int acc = local & 1;
       const uint32_t aphase = (local >> 1) & 1;
-      const int row = quarter * 32 + lane;
-      const int m = ti.mb * BM + row;
+      const int m0w = ti.mb * BM + quarter * 32;  // first row of this warp's 32
+      const int m = m0w + lane;
       const bool valid = m < p.M;
       const int nbase = ti.nblk * p.BN;
       const int n_eff = min(p.BN, gr.N - nbase);
@@ -343,14 +344,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       } else if (EPI == kTcGelu) {
         if (valid) rs = row_scale(p, m);
       }
+      // residual prefetch (kTcResid): lane covers rows i*4 + lane/8, 16-byte piece lane%8
       uint4 pre[8];
       int c = half;
       if (EPI == kTcResid && c < nchunks) {
-        const float *xr = p.X + (long long)m * p.ld + nbase + 32 * c;
-        warp_load64_issue(lane, valid ? reinterpret_cast<const uint8_t *>(xr) : nullptr,
-                          *reinterpret_cast<uint4(*)[4]>(&pre[0]));
-        warp_load64_issue(lane, valid ? reinterpret_cast<const uint8_t *>(xr + 16) : nullptr,
-                          *reinterpret_cast<uint4(*)[4]>(&pre[4]));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = i * 4 + (lane >> 3);
+          pre[i] = (m0w + r < p.M)
+                       ? *reinterpret_cast<const uint4 *>(p.X + (long long)(m0w + r) * p.ld + nbase + 32 * c + (lane & 7) * 4)
+                       : make_uint4(0, 0, 0, 0);
+        }
       }
       if (!tc::mbar_wait(tfull + acc, aphase, p.status, 14, abort)) break;
       tc::tc_fence_after();
@@ -359,56 +363,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int c0 = nbase + 32 * c;
         const bool full_chunk = c0 + 32 <= gr.N;
         float v[32];
-        if (EPI == kTcBandSplit) {
-          tc::tmem_ld32(tbase + 32 * c, v);
-          const long long tok = (long long)m * p.nb + ti.g;
-          const float *bias = p.bias + gr.bias_off + c0;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            v[j] += bias[j];
-            sq += v[j] * v[j];
-          }
-          float *xr = p.X + tok * p.ld + c0;
-          __half *hr = p.Xh + tok * p.ld + c0;
-          uint4 d[4];
-          as_u4(v, d);
-          warp_store64(stg, lane, valid ? reinterpret_cast<uint8_t *>(xr) : nullptr, d);
-          as_u4(v + 16, d);
-          warp_store64(stg, lane, valid ? reinterpret_cast<uint8_t *>(xr + 16) : nullptr, d);
-          pack16(v, d);
-          warp_store64(stg, lane, valid ? reinterpret_cast<uint8_t *>(hr) : nullptr, d);
-          continue;
-        }
-        if (EPI == kTcResid) {
-          // residual of this chunk (prefetched), then prefetch the next one
-          uint4 r0[4], r1[4];
-          warp_load64_finish(stg, lane, *reinterpret_cast<uint4(*)[4]>(&pre[0]), r0);
-          warp_load64_finish(stg, lane, *reinterpret_cast<uint4(*)[4]>(&pre[4]), r1);
-          if (c + 2 < nchunks) {
-            const float *xr = p.X + (long long)m * p.ld + c0 + 64;
-            warp_load64_issue(lane, valid ? reinterpret_cast<const uint8_t *>(xr) : nullptr,
-                              *reinterpret_cast<uint4(*)[4]>(&pre[0]));
-            warp_load64_issue(lane, valid ? reinterpret_cast<const uint8_t *>(xr + 16) : nullptr,
-                              *reinterpret_cast<uint4(*)[4]>(&pre[4]));
-          }
+        if (EPI == kTcResid || EPI == kTcBandSplit) {
+          uint8_t *xb = stg, *hb = stg + 4096;
+          // the previous boxes' stores must have read their sources
+          if (lane == 0) tc::bulk_wait_read<0>();
+          __syncwarp();
           float x[32];
-          from_u4(r0, x);
-          from_u4(r1, x + 16);
+          if (EPI == kTcResid) {
+            // residual rows: coalesced pieces -> swizzled box -> own row
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int r = i * 4 + (lane >> 3), q = lane & 7;
+              *reinterpret_cast<uint4 *>(xb + r * 128 + ((q ^ (r & 7)) << 4)) = pre[i];
+            }
+            __syncwarp();
+            box128_get_row(xb, lane, x);
+            if (c + 2 < nchunks) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int r = i * 4 + (lane >> 3);
+                pre[i] = (m0w + r < p.M)
+                             ? *reinterpret_cast<const uint4 *>(p.X + (long long)(m0w + r) * p.ld + c0 + 64 + (lane & 7) * 4)
+                             : make_uint4(0, 0, 0, 0);
+              }
+            }
+            if (p.bias) {
+              float bv[32];
+              load_bias32(p.bias + c0, bv);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) x[j] += bv[j];
+            }
+            __syncwarp();  // every lane has read its row before the box is rewritten
+          } else {
+            load_bias32(p.bias + gr.bias_off + c0, x);
+          }
           tc::tmem_ld32(tbase + 32 * c, v);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            x[j] += v[j] + (p.bias ? p.bias[c0 + j] : 0.f);
+            x[j] += v[j];
             sq += x[j] * x[j];
           }
-          float *xr = p.X + (long long)m * p.ld + c0;
-          __half *hr = p.Xh + (long long)m * p.ld + c0;
+          box128_put_row(xb, lane, x);
           uint4 d[4];
-          as_u4(x, d);
-          warp_store64(stg, lane, valid ? reinterpret_cast<uint8_t *>(xr) : nullptr, d);
-          as_u4(x + 16, d);
-          warp_store64(stg, lane, valid ? reinterpret_cast<uint8_t *>(xr + 16) : nullptr, d);
           pack16(x, d);
-          warp_store64(stg, lane, valid ? reinterpret_cast<uint8_t *>(hr) : nullptr, d);
+          box64_put_row(hb, lane, d);
+          tc::fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            if (EPI == kTcResid) {
+              tc::tma_store_2d(&tmC, xb, c0, m0w);
+              tc::tma_store_2d(&tmD, hb, c0, m0w);
+            } else {
+              tc::tma_store_3d(&tmC, xb, c0, ti.g, m0w);
+              tc::tma_store_3d(&tmD, hb, c0, ti.g, m0w);
+            }
+            tc::bulk_commit();
+          }
           continue;
         }
         tc::tmem_ld32(tbase + 32 * c, v);
@@ -471,23 +481,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         } else if (EPI == kTcGelu || EPI == kTcTanh) {
-          const float *bias = p.bias + gr.bias_off + c0;
-          __half *dst = p.out_h + gr.out_off * p.out_group_stride + (long long)m * p.ldo + c0;
+          // N is a multiple of 32 for these layers: every chunk is full
+          uint8_t *box = stg + (nstore & 1) * 2048;
+          if (lane == 0) tc::bulk_wait_read<1>();
+          __syncwarp();
+          float bv[32];
+          load_bias32(p.bias + gr.bias_off + c0, bv);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float y = v[j] * rs + (c0 + j < gr.N ? bias[j] : 0.f);
+            const float y = fmaf(v[j], rs, bv[j]);
             v[j] = EPI == kTcGelu ? gelu_(y) : tanhf(y);
           }
-          if (full_chunk) {
-            uint4 d[4];
-            pack16(v, d);
-            warp_store64(stg, lane, valid ? reinterpret_cast<uint8_t *>(dst) : nullptr, d);
-          } else if (valid) {
-            for (int j = 0; j < 32 && c0 + j < gr.N; ++j) dst[j] = __float2half_rn(v[j]);
+          uint4 d[4];
+          pack16(v, d);
+          box64_put_row(box, lane, d);
+          tc::fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            if (EPI == kTcGelu) tc::tma_store_2d(&tmC, box, c0, m0w);
+            else tc::tma_store_3d(&tmC, box, c0, m0w, gr.out_off);
+            tc::bulk_commit();
           }
-        } else {  // kTcGlu
+          ++nstore;
+        } else {  // kTcGlu: interleaved (value, gate) pairs -> 16 fp32 outputs per row
           const float *bias = p.bias + gr.bias_off + c0;
-          float *dst = p.out_f + (long long)m * p.ldo + gr.out_off + (c0 >> 1);
           float o[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
@@ -497,10 +514,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             o[j >> 1] = val * sigmoidf_(gt);
           }
           if (full_chunk) {
-            uint4 d[4];
-            as_u4(o, d);
-            warp_store64(stg, lane, valid ? reinterpret_cast<uint8_t *>(dst) : nullptr, d);
+            uint8_t *box = stg + (nstore & 1) * 2048;
+            if (lane == 0) tc::bulk_wait_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<float4 *>(box + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) =
+                  make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+            tc::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tc::tma_store_2d(&tmC, box, gr.out_off + (c0 >> 1), m0w);
+              tc::bulk_commit();
+            }
+            ++nstore;
           } else if (valid) {
+            float *dst = p.out_f + (long long)m * p.ldo + gr.out_off + (c0 >> 1);
             for (int j = 0; 2 * j + 1 < gr.N - c0; ++j) dst[j] = o[j];
           }
         }
@@ -511,6 +540,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tempty + acc);
     }
+    // outstanding bulk stores must finish reading shared memory before the CTA exits
+    if (lane == 0) tc::bulk_wait_all();
+    __syncwarp();
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -532,44 +564,59 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+template <int EPI>
+constexpr size_t smem_bytes() { return SmemLayout<EPI>::total + 1024; }
+
 }  // namespace
 
-size_t gemm_smem_bytes() { return SmemLayout::total + 1024; }
+bool make_tmap(CUtensorMap *map, const void *base, int dtype, int rank, const unsigned long long *dims,
+               const unsigned long long *strides_el, const unsigned *box, int swizzle_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const int esz = dtype == kTmF32 ? 4 : 2;
+  cuuint64_t d[3] = {1, 1, 1}, st[2] = {0, 0};
+  cuuint32_t b[3] = {1, 1, 1}, es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides_el[i] * esz;
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(map, dtype == kTmF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank,
+                  const_cast<void *>(base), d, st, b, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, unsigned long long d1,
                    unsigned long long d2, unsigned long long s1, unsigned long long s2, unsigned box1,
                    unsigned box2) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {s1 * 2, s2 * 2};
-  cuuint32_t box[3] = {64, box1, box2};
-  cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  const unsigned long long dims[3] = {d0, d1, d2}, st[2] = {s1, s2};
+  const unsigned box[3] = {64, box1, box2};
+  return make_tmap(map, base, kTmF16, 3, dims, st, box, 128);
 }
 
 bool gemm_tc_init() {
-  const int smem = (int)gemm_smem_bytes();
   bool ok = encode_fn() != nullptr;
-  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcQkv>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcResid>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcGelu>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcTanh>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcGlu>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
-  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<kTcBandSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+#define MRF_GEMM_ATTR(E)                                                                                       \
+  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,              \
+                                  (int)smem_bytes<E>()) == cudaSuccess;
+  MRF_GEMM_ATTR(kTcQkv)
+  MRF_GEMM_ATTR(kTcResid)
+  MRF_GEMM_ATTR(kTcGelu)
+  MRF_GEMM_ATTR(kTcTanh)
+  MRF_GEMM_ATTR(kTcGlu)
+  MRF_GEMM_ATTR(kTcBandSplit)
+#undef MRF_GEMM_ATTR
   return ok;
 }
 
-void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const GemmParams &p, int grid,
-                    cudaStream_t st) {
-  const size_t smem = gemm_smem_bytes();
+void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
+                    const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st) {
   switch (epi) {
-#define MRF_GEMM_CASE(E)                                                                         \
-  case E:                                                                                        \
-    gemm_tc_kernel<E><<<grid, kGemmThreads, smem, st>>>(tmA, tmB, p);                            \
+#define MRF_GEMM_CASE(E)                                                                  \
+  case E:                                                                                 \
+    gemm_tc_kernel<E><<<grid, kGemmThreads, smem_bytes<E>(), st>>>(tmA, tmB, tmC, tmD, p); \
     break;
     MRF_GEMM_CASE(kTcQkv)
     MRF_GEMM_CASE(kTcResid)

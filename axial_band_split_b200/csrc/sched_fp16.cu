@@ -278,12 +278,21 @@ GemmParams base_params(mrf_handle *h, int M, int K, int BN, const GemmGroup *gro
   return p;
 }
 
-void gemm(mrf_handle *h, const char *name, int epi, const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p) {
+void gemm(mrf_handle *h, const char *name, int epi, const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p,
+          const CUtensorMap *c = nullptr, const CUtensorMap *d = nullptr) {
   const int tiles = p.m_tiles * p.total_n_tiles;
   const int grid = std::min(tiles, h->f16->sms);
   h->begin(name);
-  launch_gemm_tc(epi, a, b, p, grid, h->cur_stream);
+  launch_gemm_tc(epi, a, b, c ? *c : a, d ? *d : a, p, grid, h->cur_stream);
   h->end();
+}
+
+// Output maps of the bulk-store epilogues (extents exactly the rows of this forward).
+bool map2(CUtensorMap *m, const void *base, int dtype, unsigned long long cols, unsigned long long rows,
+          unsigned long long ld, unsigned box0, int swz) {
+  const unsigned long long dims[2] = {cols, rows}, st[1] = {ld};
+  const unsigned box[2] = {box0, 32};
+  return make_tmap(m, base, dtype, 2, dims, st, box, swz);
 }
 
 }  // namespace
@@ -324,6 +333,22 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   }
   const long long rows_last = 2LL * h->tab.n_feat();
   ok = ok && make_tmap_f16(&wmaps[wm0 + c.mask_depth], f->mw_last, MH, rows_last, 1, MH, rows_last * MH, kBnWide, 1);
+  // bulk-store output maps
+  CUtensorMap mXo, mXho, mXbs, mXhbs, mHo, mH1o, mH2o, mMg;
+  {
+    const unsigned long long BT = (unsigned long long)B * T;
+    const unsigned long long dx[3] = {(unsigned long long)D, (unsigned long long)nb, BT};
+    const unsigned long long sx[2] = {(unsigned long long)D, (unsigned long long)nb * D};
+    const unsigned bx[3] = {32, 1, 32};
+    const unsigned long long dh3[3] = {(unsigned long long)MH, BT, (unsigned long long)nb};
+    const unsigned long long sh3[2] = {(unsigned long long)MH, (unsigned long long)MBT * MH};
+    const unsigned bh[3] = {32, 32, 1};
+    ok = ok && map2(&mXo, f->X, kTmF32, D, M, D, 32, 128) && map2(&mXho, f->Xh, kTmF16, D, M, D, 32, 64) &&
+         make_tmap(&mXbs, f->X, kTmF32, 3, dx, sx, bx, 128) && make_tmap(&mXhbs, f->Xh, kTmF16, 3, dx, sx, bx, 64) &&
+         map2(&mHo, f->Hh, kTmF16, FF, M, FF, 32, 64) && make_tmap(&mH1o, f->H1, kTmF16, 3, dh3, sh3, bh, 64) &&
+         make_tmap(&mH2o, f->H2, kTmF16, 3, dh3, sh3, bh, 64) &&
+         map2(&mMg, f->Mg, kTmF32, h->tab.n_feat(), BT, h->tab.n_feat(), 16, 64);
+  }
   if (!ok) {
     h->sched_error = "tensor-map encoding failed";
     return;
@@ -336,7 +361,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   {
     GemmParams p = base_params(h, B * T, f->k_bs, kBnNarrow, f->g_bs, nb, nb * cdiv(D, kBnNarrow));
     p.bias = h->b_bs; p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D; p.nb = nb;
-    gemm(h, "gemm_band_split", kTcBandSplit, mAbs, mWbs, p);
+    gemm(h, "gemm_band_split", kTcBandSplit, mAbs, mWbs, p, &mXbs, &mXhbs);
   }
 
   for (int i = 0; i < 2 * c.depth; ++i) {
@@ -372,16 +397,16 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     cudaMemsetAsync(f->ss, 0, sizeof(float) * M, st);
     p = base_params(h, M, A, kBnNarrow, f->g_out, 1, cdiv(D, kBnNarrow));
     p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D;
-    gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p);
+    gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p, &mXo, &mXho);
 
     p = base_params(h, M, D, kBnWide, f->g_ff1, 1, cdiv(FF, kBnWide));
     p.ss_in = f->ss; p.bias = w.b1; p.out_h = f->Hh; p.ldo = FF;
-    gemm(h, "gemm_ff1_gelu", kTcGelu, mXh, mW1, p);
+    gemm(h, "gemm_ff1_gelu", kTcGelu, mXh, mW1, p, &mHo);
 
     cudaMemsetAsync(f->ss, 0, sizeof(float) * M, st);
     p = base_params(h, M, FF, kBnNarrow, f->g_ff2, 1, cdiv(D, kBnNarrow));
     p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D; p.bias = w.b2;
-    gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p);
+    gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p, &mXo, &mXho);
 
     h->begin("outnorm");
     launch_outnorm(f->X, f->ss, w.gout, f->Xh, M, D, st);
@@ -393,19 +418,21 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   GemmParams p = base_params(h, BT, D, kBnWide, f->g_m0, nb, nb * cdiv(MH, kBnWide));
   p.a_mode = 1;
   p.bias = f->mb[0]; p.out_h = f->H1; p.ldo = MH; p.out_group_stride = MBT * MH;
-  gemm(h, "gemm_mask_tanh", kTcTanh, mXband, wmaps[wm0], p);
+  gemm(h, "gemm_mask_tanh", kTcTanh, mXband, wmaps[wm0], p, &mH1o);
   __half *cur = f->H1, *nxt = f->H2;
   const CUtensorMap *mcur = &mH1, *mnxt = &mH2;
+  const CUtensorMap *ocur = &mH1o, *onxt = &mH2o;
   for (int i = 1; i < c.mask_depth; ++i) {
     p = base_params(h, BT, MH, kBnWide, f->g_mid, nb, nb * cdiv(MH, kBnWide));
     p.bias = f->mb[i]; p.out_h = nxt; p.ldo = MH; p.out_group_stride = MBT * MH;
-    gemm(h, "gemm_mask_tanh", kTcTanh, *mcur, wmaps[wm0 + i], p);
+    gemm(h, "gemm_mask_tanh", kTcTanh, *mcur, wmaps[wm0 + i], p, onxt);
     std::swap(cur, nxt);
     std::swap(mcur, mnxt);
+    std::swap(ocur, onxt);
   }
   p = base_params(h, BT, MH, kBnWide, f->g_last, nb, f->n_last_tiles);
   p.bias = f->mb_last; p.out_f = f->Mg; p.ldo = h->tab.n_feat();
-  gemm(h, "gemm_mask_glu", kTcGlu, *mcur, wmaps[wm0 + c.mask_depth], p);
+  gemm(h, "gemm_mask_glu", kTcGlu, *mcur, wmaps[wm0 + c.mask_depth], p, &mMg);
 
   h->begin("overlap_average");
   launch_overlap_average(f->Mg, h->tab.n_feat(), h->d_src0, h->d_src1, h->d_row_weight, out, B, T, R, st);

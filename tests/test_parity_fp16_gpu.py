@@ -42,6 +42,7 @@ def run(cfg, B, T, W, x, max_batch=None, max_frames=None, graph=True, debug=()):
 def check(got, ref, what=""):
     err = float(np.abs(got - ref).max())
     snr = snr_db(got, ref)
+    print(f"{what}: max|diff|={err:.3e} snr={snr:.1f} dB max|ref|={float(np.abs(ref).max()):.3e}")
     assert err <= MAX_ABS and snr >= MIN_SNR, f"{what} max|diff|={err:.3e} snr={snr:.1f} dB"
     return err, snr
 
