@@ -20,7 +20,7 @@ struct GemmGroup {
 };
 
 enum GemmEpi : int {
-  kTcQkv = 0,     // RoPE + scatter q, k, v (fp16, attention layout) + sigmoid gates
+  kTcQkv = 0,     // row norm, RoPE on q and k, softmax scale on q, sigmoid gates; token-major fp16 rows
   kTcResid = 1,   // X += acc (+ bias); writes X fp32, X fp16, row sum of squares
   kTcGelu = 2,    // out = gelu(acc * rowscale + bias) fp16
   kTcTanh = 3,    // out = tanh(acc + bias) fp16 (group-strided)
@@ -43,18 +43,23 @@ struct GemmParams {
   float *out_f;             // fp32 output
   int ldo;
   long long out_group_stride;
-  // q, k, v scatter
-  __half *q, *k, *v;
-  float *gates;
+  // q, k, v, gates rows
   const float2 *rope;
   const float *gbias;
-  int B, T, nb, H, dh, A, axis, n_pad;
+  int B, T, nb, H, dh, A, axis;
   float q_scale;            // q is multiplied by this after RoPE (the attention's softmax scale)
+  // deferred output norm of the previous transformer (kTcResid): the residual input x is
+  // scaled by res_gain[col] / max(sqrt(res_ss[row]), eps) before the add (null: no scaling)
+  const float *res_ss;
+  const float *res_gain;
+  // kTcResid: also accumulate sum_j (out_gain[j] * x_j)^2 per row into ssg_out (null: skip)
+  float *ssg_out;
+  const float *out_gain;
 };
 
 enum TmapDtype : int { kTmF16 = 0, kTmF32 = 1 };
 
-// Encode a tensor map of rank 1..3: dims and strides in elements (strides of dims 1..rank-1),
+// Encode a tensor map of rank 1..5: dims and strides in elements (strides of dims 1..rank-1),
 // box in elements, swizzle 0 / 32 / 64 / 128 bytes.
 bool make_tmap(CUtensorMap *map, const void *base, int dtype, int rank, const unsigned long long *dims,
                const unsigned long long *strides_el, const unsigned *box, int swizzle_bytes);
@@ -71,7 +76,7 @@ constexpr int kGemmThreads = 320;
 bool gemm_tc_init();
 
 // tmC / tmD: output tensor maps of the epilogues that store through bulk tensor stores
-// (kTcResid: X fp32 [M, ld] box 32x32 swizzle 128 and X fp16 box 32x32 swizzle 64;
+// (kTcQkv: [q | k | v | gates] fp16 [M, ld] box 32x32 swizzle 64; kTcResid: X fp32 [M, ld] box 32x32 swizzle 128 and X fp16 box 32x32 swizzle 64;
 //  kTcBandSplit: the same as 3D (ld, nb, frames) boxes 32x1x32; kTcGelu: out fp16 [M, ldo]
 //  box 32x32 swizzle 64; kTcTanh: out fp16 (ldo, frames, groups) box 32x32x1 swizzle 64;
 //  kTcGlu: out fp32 [frames, ldo] box 16x32 swizzle 64).  Unused maps may be any valid map.

@@ -10,11 +10,14 @@
 // queries into blocks is exact (model card "musetric/vocal-separation-roformer-onnx",
 // section "How these graphs are written").
 //
+// q, k, v are read from the token-major projection output [token][q | k | v | gates]
+// through 4-D tensor maps (d, head, band, frame).
 // Persistent CTAs; a work item is two 128-row query tiles t = 0, 1 processed in ping-pong:
 //   time axis - two consecutive query tiles of one (band, head) sequence; the keys stream
 //               in blocks of 128 and each K/V block serves both tiles;
-//   band axis - each tile holds two 64-row problems (n <= 64) with their own single K/V
-//               block, masked block-diagonally.
+//   band axis - each tile holds the band sequences of two frames for one head (64 rows
+//               each, bands past n read as zeros) with their own single K/V block, masked
+//               block-diagonally.
 // Warps 0-3 and 4-7: softmax of tile 0 and tile 1 (one query row per thread); warp 8: TMA;
 // warp 9: MMA issue.  Tensor memory (512 columns): S_t at 128 t, O_t at 256 + 64 t.
 // O accumulates in tensor memory across key blocks; a row's running max is raised (and
@@ -22,6 +25,7 @@
 // the unnormalised p stay below 256 and most blocks need no correction.
 #include <cmath>
 
+#include "gemm_tc.cuh"
 #include "mrf_internal.h"
 #include "tc_ptx.cuh"
 
@@ -30,6 +34,7 @@ namespace mrf {
 namespace {
 
 constexpr int kDh = 64, kRows = 128, kKeys = 128, kStages = 2;
+static_assert(kKeys == 128, "the softmax reads a score row as two 64-column halves");
 constexpr int kTile = kRows * kDh * 2;  // 16 KB: one 128 x 64 fp16 tile
 constexpr int kThreads = 320;
 constexpr float kRescaleLog2 = 8.f;
@@ -48,20 +53,46 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe: x = n + f with n = round(x) (magic-number rounding), 2^f by a
-// degree-3 minimax polynomial on [-1/2, 1/2] (relative error 7.5e-5, coefficients from
-// fit_exp2_poly.py), and 2^n added into the exponent bits.  x <= 8 here; below -126 the
-// result is flushed to 0 like ex2.approx.ftz.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;          // 1.5 * 2^23: round to nearest integer
-  const float n = t - 12582912.f;
-  const float f = x - n;
-  float p = fmaf(0.055171669f, f, 0.242611122f);
-  p = fmaf(p, f, 0.693260985f);
-  p = fmaf(p, f, 0.999928074f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
+
+// packed pair add (one f32x2 instruction)
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long x = (static_cast<unsigned long long>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+  unsigned long long y = (static_cast<unsigned long long>(__float_as_uint(b.y)) << 32) | __float_as_uint(b.x);
+  unsigned long long z;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
+  return make_float2(__uint_as_float(static_cast<unsigned>(z)), __uint_as_float(static_cast<unsigned>(z >> 32)));
+}
+
+// 64 consecutive fp32 columns of this thread's TMEM lane: two loads, one wait.  The wait
+// takes the destination registers as operands so no use can be scheduled above it.
+#define MRF_R8(b) "=r"(r[b]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), "=r"(r[b + 5]), \
+                  "=r"(r[b + 6]), "=r"(r[b + 7])
+#define MRF_P8(b) "+r"(r[b]), "+r"(r[b + 1]), "+r"(r[b + 2]), "+r"(r[b + 3]), "+r"(r[b + 4]), "+r"(r[b + 5]), \
+                  "+r"(r[b + 6]), "+r"(r[b + 7])
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+#pragma unroll
+  for (int c = 0; c < 64; c += 32) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : MRF_R8(c), MRF_R8(c + 8), MRF_R8(c + 16), MRF_R8(c + 24)
+        : "r"(taddr + c));
+  }
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : MRF_P8(0), MRF_P8(8), MRF_P8(16), MRF_P8(24) : : "memory");
+  asm volatile("" : MRF_P8(32), MRF_P8(40), MRF_P8(48), MRF_P8(56));
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+#undef MRF_R8
+
 
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
@@ -69,36 +100,37 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 }
 
 struct AttnArgs {
-  const float *gate;
+  const __half *qkv;   // token-major [tok][ld]: q | k | v | sigmoid gates
   __half *o;
   unsigned *status;
-  int B, T, nb, H, axis, n_pad, n, q_tiles, pairs, items, n_blocks;
-  long long problems;
+  int B, T, nb, H, axis, ld, n, q_tiles, pairs, items, n_blocks, BT;
 };
 
-// Rows of the item's query tiles and key blocks.
+// Tensor-map coordinates (d, head, band, frame) of an item's two query tiles; key blocks
+// add j*128 frames on the time axis.  Time axis: the tiles are frames frame0[t] .. +127 of
+// one (band, head) sequence.  Band axis: tile t covers frames frame0[t] and frame0[t] + 1,
+// bands 0..63 of each (bands past nb read as zeros).
 struct Item {
-  long long q_row[2], k_row[2];
-  long long sh;  // time axis: sequence * H + head; band axis: first problem of the item
-  int qt0;       // time axis: index of tile 0 within the sequence
+  int head, band, qt0;
+  int frame0[2];
 };
 
-__device__ __forceinline__ Item item_rows(const AttnArgs &a, int item) {
+__device__ __forceinline__ Item item_coords(const AttnArgs &a, int item) {
   Item it;
   if (a.axis == 0) {
-    it.sh = item / a.pairs;
+    const int sh = item / a.pairs;       // ((b * nb) + band) * H + head
     it.qt0 = 2 * (item % a.pairs);
-    for (int t = 0; t < 2; ++t) {
-      it.q_row[t] = it.sh * a.n_pad + (long long)(it.qt0 + t) * kRows;
-      it.k_row[t] = it.sh * a.n_pad;
-    }
+    it.head = sh % a.H;
+    const int seq = sh / a.H;
+    it.band = seq % a.nb;
+    const int b = seq / a.nb;
+    for (int t = 0; t < 2; ++t) it.frame0[t] = b * a.T + (it.qt0 + t) * kRows;
   } else {
-    it.sh = 4LL * item;
+    it.head = item % a.H;
+    it.band = 0;
     it.qt0 = 0;
-    for (int t = 0; t < 2; ++t) {
-      it.q_row[t] = (it.sh + 2 * t) * a.n_pad;  // n_pad == 64
-      it.k_row[t] = it.q_row[t];
-    }
+    const int f = 4 * (item / a.H);
+    for (int t = 0; t < 2; ++t) it.frame0[t] = f + 2 * t;
   }
   return it;
 }
@@ -151,20 +183,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       int li = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
-        const Item it = item_rows(a, item);
+        const Item it = item_coords(a, item);
         if (!tc::mbar_wait(q_empty, (li & 1) ^ 1, a.status, 30, abort)) break;
         tc::mbar_arrive_expect_tx(q_full, 2 * kTile);
         for (int t = 0; t < 2; ++t)
-          tc::tma_load_3d(smem + AttnSmem::q + t * kTile, &tq, q_full, 0, (int)it.q_row[t], 0);
+          tc::tma_load_4d(smem + AttnSmem::q + t * kTile, &tq, q_full, 0, it.head, it.band, it.frame0[t]);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
           const int s = g % kStages;
           if (!tc::mbar_wait(kv_empty + s, ((g / kStages) & 1) ^ 1, a.status, 31, abort)) { ok = false; break; }
           tc::mbar_arrive_expect_tx(kv_full + s, kv_bytes);
           for (int t = 0; t < (shared_kv ? 1 : 2); ++t) {
-            const int r = (int)(it.k_row[t] + (long long)j * kKeys);
+            const int f = shared_kv ? it.frame0[0] - it.qt0 * kRows + j * kKeys : it.frame0[t];
             uint8_t *dst = smem + AttnSmem::kv + (s * 4 + 2 * t) * kTile;
-            tc::tma_load_3d(dst, &tk, kv_full + s, 0, r, 0);
-            tc::tma_load_3d(dst + kTile, &tv, kv_full + s, 0, r, 0);
+            tc::tma_load_4d(dst, &tk, kv_full + s, 0, it.head, it.band, f);
+            tc::tma_load_4d(dst + kTile, &tv, kv_full + s, 0, it.head, it.band, f);
           }
         }
       }
@@ -246,72 +278,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         int lo, hi;
         if (a.axis == 0) { lo = 0; hi = min(kKeys, a.n - j * kKeys); }
         else { lo = prob * 64; hi = prob * 64 + a.n; }
-        const bool full_blk = lo == 0 && hi == kKeys;  // no masking needed (warp-uniform on the time axis)
+        // the score row in two 64-column reads (scores arrive in log2 units: q was scaled by
+        // log2(e) / sqrt(dh) in its projection)
+        const bool masked = !(lo == 0 && hi == kKeys);
         float mx = -INFINITY;
-        if (full_blk) {
 #pragma unroll
-          for (int c = 0; c < kKeys; c += 32) {
-            float v[32];
-            tc::tmem_ld32(tS + c, v);
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          float sv[64];
+          tmem_ld64(tS + 64 * hlf, sv);
+          if (masked) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, v[i]);
+            for (int i = 0; i < 64; ++i)
+              if (64 * hlf + i < lo || 64 * hlf + i >= hi) sv[i] = -INFINITY;
           }
-        } else {
 #pragma unroll
-          for (int c = 0; c < kKeys; c += 32) {
-            float v[32];
-            tc::tmem_ld32(tS + c, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (c + i >= lo && c + i < hi) mx = fmaxf(mx, v[i]);
-          }
+          for (int i = 0; i < 64; i += 2) mx = max3(mx, sv[i], sv[i + 1]);
         }
-        // scores arrive in log2 units (q was scaled by log2(e) / sqrt(dh) in its projection)
         const float m_cand = fmaxf(m_run, mx);
         // P_t and O_t are free once the previous block's P*V has completed
         if (j > 0 && !tc::mbar_wait(pv_done + t, (g - 1) & 1, a.status, 39, abort)) { ok = false; break; }
         const bool need = m_cand > m_run + kRescaleLog2;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2(m_run - m_cand) : 1.f;
-          if (need) { l *= alpha; m_run = m_cand; }
-          if (j > 0) {
-            tc::tc_fence_after();
+        const bool any_need = __any_sync(0xffffffffu, need);
+        const float alpha = need ? ex2(m_run - m_cand) : 1.f;
+        if (need) { l *= alpha; m_run = m_cand; }
+        // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU
+        float2 acc2 = make_float2(0.f, 0.f);
+        const float2 negm = make_float2(-m_run, -m_run);
 #pragma unroll
-            for (int c = 0; c < kDh; c += 32) {
-              float v[32];
-              tc::tmem_ld32(tO + c, v);
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          float sv[64];
+          tmem_ld64(tS + 64 * hlf, sv);
+          if (masked) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] *= alpha;
-              tc::tmem_st32(tO + c, v);
-            }
+            for (int i = 0; i < 64; ++i)
+              if (64 * hlf + i < lo || 64 * hlf + i >= hi) sv[i] = -INFINITY;
           }
+          uint32_t hh[32];
+#pragma unroll
+          for (int i = 0; i < 64; i += 2) {
+            const float2 d = add2(make_float2(sv[i], sv[i + 1]), negm);
+            const float2 pp = make_float2(ex2(d.x), ex2(d.y));
+            acc2 = add2(acc2, pp);
+            hh[i >> 1] = pack_h2(pp.x, pp.y);
+          }
+          // 128-byte swizzle: 16-byte chunk index XOR (row % 8); column block hlf holds keys 64 hlf ..
+          uint8_t *blk = prow + hlf * kTile;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4 *>(blk + ((q ^ (r & 7)) << 4)) =
+                make_uint4(hh[4 * q], hh[4 * q + 1], hh[4 * q + 2], hh[4 * q + 3]);
         }
-        float sum = 0.f;
+        const float sum = acc2.x + acc2.y;
+        // O row rescaled in place when this row's max was raised (after P, to keep the
+        // score row and the O chunk out of registers at the same time)
+        if (any_need && j > 0) {
+          tc::tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kKeys; c += 32) {
-          float v[32];
-          tc::tmem_ld32(tS + c, v);
-          uint32_t h[16];
+          for (int c = 0; c < kDh; c += 32) {
+            float v[32];
+            tc::tmem_ld32(tO + c, v);
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float p0, p1;
-            // one pair in four on the FMA pipe, the rest on MUFU
-            if (((i >> 1) & 3) == 3) { p0 = exp2_fma(v[i] - m_run); p1 = exp2_fma(v[i + 1] - m_run); }
-            else { p0 = ex2(v[i] - m_run); p1 = ex2(v[i + 1] - m_run); }
-            if (!full_blk) {
-              if (!(c + i >= lo && c + i < hi)) p0 = 0.f;
-              if (!(c + i + 1 >= lo && c + i + 1 < hi)) p1 = 0.f;
-            }
-            sum += p0 + p1;
-            h[i >> 1] = pack_h2(p0, p1);
-          }
-          // 128-byte swizzle: 16-byte chunk index XOR (row % 8); two column blocks of 64 keys
-          uint8_t *blk = prow + (c >> 6) * kTile;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int chunk = ((c & 63) >> 3) + q;
-            *reinterpret_cast<uint4 *>(blk + ((chunk ^ (r & 7)) << 4)) =
-                make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+            tc::tmem_st32(tO + c, v);
           }
         }
         l += sum;
@@ -337,26 +365,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(o_free + t);
-      const Item it = item_rows(a, item);
+      const Item it = item_coords(a, item);
       long long tok = -1;
-      int head = 0;
+      const int head = it.head;
       if (a.axis == 0) {
         const int pos = (it.qt0 + t) * kRows + r;
-        if (pos < a.n) {
-          head = (int)(it.sh % a.H);
-          const long long seq = it.sh / a.H;  // b * nb + band
-          tok = ((seq / a.nb) * a.T + pos) * a.nb + (seq % a.nb);
-        }
+        if (pos < a.n) tok = (long long)(it.frame0[t] + r) * a.nb + it.band;
       } else {
-        const long long shr = it.sh + 2 * t + prob;
-        const int pos = r & 63;
-        if (pos < a.n && shr < a.problems) {
-          head = (int)(shr % a.H);
-          tok = (shr / a.H) * a.nb + pos;
-        }
+        const int f = it.frame0[t] + prob, k = r & 63;
+        if (k < a.n && f < a.BT) tok = (long long)f * a.nb + k;
       }
       if (tok >= 0) {
-        const float gsc = a.gate[tok * a.H + head] / l;
+        const float gsc = __half2float(a.qkv[tok * a.ld + 3 * a.H * kDh + head]) / l;
         __half *dst = a.o + tok * (long long)a.H * kDh + head * kDh;
 #pragma unroll
         for (int d = 0; d < kDh; d += 8) {
@@ -379,10 +399,6 @@ int g_num_sms = 0;
 
 }  // namespace
 
-bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, unsigned long long d1,
-                   unsigned long long d2, unsigned long long s1, unsigned long long s2, unsigned box1,
-                   unsigned box2);
-
 bool attention_tc_supported(int dh) { return dh == kDh; }
 
 bool attention_tc_init() {
@@ -393,32 +409,39 @@ bool attention_tc_init() {
                               (int)(AttnSmem::total + 1024)) == cudaSuccess;
 }
 
-bool launch_attention_tc(const __half *q, const __half *k, const __half *v, const float *gate, __half *o, int B,
-                         int T, int nb, int H, int axis, int n_pad, unsigned *status, cudaStream_t st) {
+bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int axis,
+                         unsigned *status, cudaStream_t st) {
   AttnArgs a;
-  a.gate = gate;
+  a.qkv = qkv;
   a.o = o;
   a.status = status;
-  a.B = B; a.T = T; a.nb = nb; a.H = H; a.axis = axis; a.n_pad = n_pad;
+  a.B = B; a.T = T; a.nb = nb; a.H = H; a.axis = axis; a.ld = ld;
+  a.BT = B * T;
   a.n = axis == 0 ? T : nb;
   a.q_tiles = (a.n + kRows - 1) / kRows;
-  long long rows;
+  unsigned box[4];
   if (axis == 0) {
-    a.problems = (long long)B * nb * H;
     a.pairs = (a.q_tiles + 1) / 2;
-    a.items = (int)(a.problems * a.pairs);
+    a.items = B * nb * H * a.pairs;
     a.n_blocks = (a.n + kKeys - 1) / kKeys;
+    box[0] = kDh; box[1] = 1; box[2] = 1; box[3] = kRows;      // 128 frames of one (band, head)
   } else {
-    a.problems = (long long)B * T * H;
+    if (nb > 64) return false;
     a.pairs = 0;
-    a.items = (int)((a.problems + 3) / 4);
+    a.items = H * ((a.BT + 3) / 4);
     a.n_blocks = 1;
+    box[0] = kDh; box[1] = 1; box[2] = 64; box[3] = 2;         // bands 0..63 of two frames
   }
-  rows = a.problems * n_pad;
+  // (d, head, band, frame) over the token-major buffer; q, k, v differ by their column offset
+  const unsigned long long dims[4] = {(unsigned long long)kDh, (unsigned long long)H, (unsigned long long)nb,
+                                      (unsigned long long)a.BT};
+  const unsigned long long str[3] = {(unsigned long long)kDh, (unsigned long long)ld,
+                                     (unsigned long long)nb * ld};
+  const size_t A = (size_t)H * kDh;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap_f16(&tq, q, kDh, rows, 1, kDh, rows * kDh, kRows, 1) ||
-      !make_tmap_f16(&tk, k, kDh, rows, 1, kDh, rows * kDh, kKeys, 1) ||
-      !make_tmap_f16(&tv, v, kDh, rows, 1, kDh, rows * kDh, kKeys, 1))
+  if (!make_tmap(&tq, qkv, kTmF16, 4, dims, str, box, 128) ||
+      !make_tmap(&tk, qkv + A, kTmF16, 4, dims, str, box, 128) ||
+      !make_tmap(&tv, qkv + 2 * A, kTmF16, 4, dims, str, box, 128))
     return false;
   const size_t smem = AttnSmem::total + 1024;
   const int grid = (int)std::min<long long>(a.items, g_num_sms > 0 ? g_num_sms : 148);

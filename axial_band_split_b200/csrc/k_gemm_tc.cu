@@ -21,7 +21,6 @@
 // Epilogue stores: each warp writes its 32 rows x 32 columns into a shared-memory box in the
 // tensor map's swizzled layout and one lane issues a bulk tensor store (cp.async.bulk.tensor),
 // so global writes leave the SM as whole lines; rows past M are clipped by the tensor map.
-// The q, k, v scatter keeps plain stores through an 80-byte-row staging buffer.
 #include <cudaTypedefs.h>
 
 #include <cmath>
@@ -44,9 +43,8 @@ constexpr int kEpiWarps = 8;
 // Widest B tile of an epilogue kind, and the shared memory each epilogue warp needs.
 __host__ __device__ constexpr int bn_max(int epi) { return (epi == kTcResid || epi == kTcBandSplit) ? 192 : 256; }
 __host__ __device__ constexpr int warp_stage_bytes(int epi) {
-  return epi == kTcQkv ? 32 * 80                                           // row staging (80-byte rows)
-         : (epi == kTcResid || epi == kTcBandSplit) ? 4096 + 2048         // fp32 box + fp16 box
-                                                    : 2 * 2048;           // two 2 KB boxes
+  return (epi == kTcResid || epi == kTcBandSplit) ? 4096 + 2048          // fp32 box + fp16 box
+                                                  : 2 * 2048;            // two 2 KB boxes
 }
 
 template <int EPI>
@@ -64,16 +62,6 @@ __device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + __expf
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
-}
-
-// Store 8 consecutive floats as fp16 (16 bytes).
-__device__ __forceinline__ void st_h8(__half *dst, const float *v) {
-  uint4 u;
-  u.x = pack_h2(v[0], v[1]);
-  u.y = pack_h2(v[2], v[3]);
-  u.z = pack_h2(v[4], v[5]);
-  u.w = pack_h2(v[6], v[7]);
-  *reinterpret_cast<uint4 *>(dst) = u;
 }
 
 __device__ __forceinline__ int find_group(const GemmGroup *g, int n, int tile, int m_tiles) {
@@ -101,8 +89,6 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams &p, int tile) {
 }
 
 // ------------------------------------------------------------------ epilogue helpers
-constexpr int kStageRow = 80;  // q, k, v row staging: 64 data bytes + 16 pad (conflict-free)
-
 __device__ __forceinline__ float row_scale(const GemmParams &p, long long row) {
   if (!p.ss_in) return 1.f;
   return 1.f / fmaxf(sqrtf(p.ss_in[row]), kEps);
@@ -125,24 +111,6 @@ __device__ __forceinline__ float erf_as(float x) {
 }
 
 __device__ __forceinline__ float gelu_(float x) { return 0.5f * x * (1.f + erf_as(x * 0.70710678118654752f)); }
-
-// q, k, v: each lane passes its row's destination (null: skip) and 64 bytes; written
-// coalesced through the staging buffer (4 lanes per row, 8 rows per instruction).
-__device__ __forceinline__ void warp_store64(uint8_t *stg, int lane, uint8_t *dst, const uint4 (&d)[4]) {
-  uint8_t *my = stg + lane * kStageRow;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4 *>(my + q * 16) = d[q];
-  __syncwarp();
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = i * 8 + (lane >> 2), q = lane & 3;
-    uint8_t *rd = reinterpret_cast<uint8_t *>(
-        __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(dst), r));
-    const uint4 v = *reinterpret_cast<const uint4 *>(stg + r * kStageRow + q * 16);
-    if (rd) *reinterpret_cast<uint4 *>(rd + q * 16) = v;
-  }
-  __syncwarp();
-}
 
 __device__ __forceinline__ void pack16(const float *v, uint4 (&d)[4]) {
   // 32 floats -> 32 fp16 (64 bytes)
@@ -343,7 +311,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else if (EPI == kTcGelu) {
         if (valid) rs = row_scale(p, m);
+      } else if (EPI == kTcTanh) {
+        if (valid && p.ss_in) rs = row_scale(p, token_of(p, m, ti.g));
       }
+      float res_s = 1.f;  // deferred norm of the residual input (kTcResid)
+      if (EPI == kTcResid && p.res_ss && valid) res_s = 1.f / fmaxf(sqrtf(p.res_ss[m]), kEps);
       // residual prefetch (kTcResid): lane covers rows i*4 + lane/8, 16-byte piece lane%8
       uint4 pre[8];
       int c = half;
@@ -358,7 +330,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       if (!tc::mbar_wait(tfull + acc, aphase, p.status, 14, abort)) break;
       tc::tc_fence_after();
-      float sq = 0.f;
+      float sq = 0.f, sqg = 0.f;
       for (; c < nchunks; c += 2) {
         const int c0 = nbase + 32 * c;
         const bool full_chunk = c0 + 32 <= gr.N;
@@ -378,6 +350,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             __syncwarp();
             box128_get_row(xb, lane, x);
+            if (p.res_ss) {
+              float gv[32];
+              load_bias32(p.res_gain + c0, gv);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) x[j] *= res_s * gv[j];
+            }
             if (c + 2 < nchunks) {
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
@@ -403,6 +381,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             x[j] += v[j];
             sq += x[j] * x[j];
           }
+          if (EPI == kTcResid && p.ssg_out) {
+            float gv[32];
+            load_bias32(p.out_gain + c0, gv);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float y = gv[j] * x[j];
+              sqg += y * y;
+            }
+          }
           box128_put_row(xb, lane, x);
           uint4 d[4];
           pack16(x, d);
@@ -423,63 +410,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc::tmem_ld32(tbase + 32 * c, v);
         if (EPI == kTcQkv) {
+          // one token-major row [q | k | v | gates]: scale by the row's norm, rotate q and k,
+          // fold the softmax scale into q, squash the gates
           const int A3 = 3 * p.A;
-          if (c0 >= A3) {  // sigmoid gates
-            if (valid)
-              for (int j = 0; j < 32; ++j) {
-                const int h = c0 + j - A3;
-                if (h < p.H) p.gates[qr.tok * p.H + h] = sigmoidf_(v[j] * rs + p.gbias[h]);
-              }
-            continue;
-          }
+          if (c0 >= A3) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= rs;
-          if (p.dh == 64) {
+            for (int j = 0; j < 32; ++j) {
+              const int h = c0 + j - A3;
+              v[j] = h < p.H ? sigmoidf_(v[j] * rs + p.gbias[h]) : 0.f;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= rs;
             const int which = c0 / p.A;
-            const int head = (c0 - which * p.A) >> 6;
-            const int d0 = c0 & 63;
             if (which < 2) {
               const float sc = which == 0 ? p.q_scale : 1.f;
+              if (p.dh == 64) {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float x0 = v[2 * i], x1 = v[2 * i + 1];
-                v[2 * i] = (x0 * cs[i].x - x1 * cs[i].y) * sc;
-                v[2 * i + 1] = (x1 * cs[i].x + x0 * cs[i].y) * sc;
-              }
-            }
-            __half *dst = which == 0 ? p.q : which == 1 ? p.k : p.v;
-            uint4 d[4];
-            pack16(v, d);
-            warp_store64(stg, lane,
-                         valid ? reinterpret_cast<uint8_t *>(dst + ((qr.seq * p.H + head) * p.n_pad + qr.pos) * 64 + d0)
-                               : nullptr,
-                         d);
-          } else if (valid) {
-            const int half_dh = p.dh >> 1;
+                for (int i = 0; i < 16; ++i) {
+                  const float x0 = v[2 * i], x1 = v[2 * i + 1];
+                  v[2 * i] = (x0 * cs[i].x - x1 * cs[i].y) * sc;
+                  v[2 * i + 1] = (x1 * cs[i].x + x0 * cs[i].y) * sc;
+                }
+              } else {
+                const int half_dh = p.dh >> 1;
 #pragma unroll
-            for (int j8 = 0; j8 < 32; j8 += 8) {
-              const int col = c0 + j8;
-              const int which = col / p.A;
-              const int rem = col - which * p.A;
-              const int head = rem / p.dh;
-              const int dd = rem - head * p.dh;
-              float o[8];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) o[j] = v[j8 + j];
-              if (which < 2) {
-                const float sc = which == 0 ? p.q_scale : 1.f;
-#pragma unroll
-                for (int j = 0; j < 8; j += 2) {
-                  const float2 cc = p.rope[(long long)qr.pos * half_dh + ((dd + j) >> 1)];
-                  const float x0 = o[j], x1 = o[j + 1];
-                  o[j] = (x0 * cc.x - x1 * cc.y) * sc;
-                  o[j + 1] = (x1 * cc.x + x0 * cc.y) * sc;
+                for (int i = 0; i < 16; ++i) {
+                  const int dd = (c0 - which * p.A + 2 * i) % p.dh;
+                  const float2 cc = p.rope[(long long)qr.pos * half_dh + (dd >> 1)];
+                  const float x0 = v[2 * i], x1 = v[2 * i + 1];
+                  v[2 * i] = (x0 * cc.x - x1 * cc.y) * sc;
+                  v[2 * i + 1] = (x1 * cc.x + x0 * cc.y) * sc;
                 }
               }
-              __half *dst = which == 0 ? p.q : which == 1 ? p.k : p.v;
-              st_h8(dst + ((qr.seq * p.H + head) * p.n_pad + qr.pos) * p.dh + dd, o);
             }
           }
+          uint8_t *box = stg + (nstore & 1) * 2048;
+          if (lane == 0) tc::bulk_wait_read<1>();
+          __syncwarp();
+          uint4 d[4];
+          pack16(v, d);
+          box64_put_row(box, lane, d);
+          tc::fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tc::tma_store_2d(&tmC, box, c0, m0w);
+            tc::bulk_commit();
+          }
+          ++nstore;
         } else if (EPI == kTcGelu || EPI == kTcTanh) {
           // N is a multiple of 32 for these layers: every chunk is full
           uint8_t *box = stg + (nstore & 1) * 2048;
@@ -535,6 +513,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       if (EPI == kTcResid && valid && p.ss_out && half < nchunks) atomicAdd(p.ss_out + m, sq);
+      if (EPI == kTcResid && valid && p.ssg_out && half < nchunks) atomicAdd(p.ssg_out + m, sqg);
       if (EPI == kTcBandSplit && valid && half < nchunks) atomicAdd(p.ss_out + (long long)m * p.nb + ti.g, sq);
       tc::tc_fence_before();
       __syncwarp();
@@ -574,8 +553,9 @@ bool make_tmap(CUtensorMap *map, const void *base, int dtype, int rank, const un
   auto fn = encode_fn();
   if (!fn) return false;
   const int esz = dtype == kTmF32 ? 4 : 2;
-  cuuint64_t d[3] = {1, 1, 1}, st[2] = {0, 0};
-  cuuint32_t b[3] = {1, 1, 1}, es[3] = {1, 1, 1};
+  cuuint64_t d[5] = {1, 1, 1, 1, 1}, st[4] = {0, 0, 0, 0};
+  cuuint32_t b[5] = {1, 1, 1, 1, 1}, es[5] = {1, 1, 1, 1, 1};
+  if (rank < 1 || rank > 5) return false;
   for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; }
   for (int i = 0; i + 1 < rank; ++i) st[i] = strides_el[i] * esz;
   const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B

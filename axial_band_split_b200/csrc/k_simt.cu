@@ -332,6 +332,59 @@ __global__ void attention_simt_kernel(const TI *__restrict__ q, const TI *__rest
   if (lane + 32 < dh) st_f(orow + lane + 32, o1 * g);
 }
 
+// Same on the fp16 schedule's token-major projection rows qkv[tok][ld] = [q | k | v | gates]
+// (gates already squashed by the sigmoid), for head widths the tensor-core kernel does not take.
+__global__ void attention_tokmajor_kernel(const __half *__restrict__ qkv, int ld, __half *__restrict__ o, int B,
+                                          int T, int nb, int H, int dh, int axis) {
+  __shared__ float qs[8][64];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const long long nseq = axis == 0 ? (long long)B * nb : (long long)B * T;
+  const int n = axis == 0 ? T : nb;
+  const long long qi = (long long)blockIdx.x * 8 + warp;
+  if (qi >= nseq * H * n) return;
+  const int A = H * dh;
+  const int pos = qi % n;
+  const long long sh = qi / n;
+  const int head = sh % H;
+  const long long seq = sh / H;
+  // token of position p of this sequence
+  auto tok_of = [&](int p_) -> long long {
+    if (axis == 0) { const long long b = seq / nb, band = seq % nb; return (b * T + p_) * nb + band; }
+    return seq * nb + p_;
+  };
+  const long long tq = tok_of(pos);
+  const float scale = rsqrtf((float)dh);
+  for (int d = lane; d < dh; d += 32) qs[warp][d] = __half2float(qkv[tq * ld + head * dh + d]) * scale;
+  __syncwarp();
+  float m = -INFINITY, l = 0.f, o0 = 0.f, o1 = 0.f;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    float s = -INFINITY;
+    if (j < n) {
+      const __half *kr = qkv + tok_of(j) * ld + A + head * dh;
+      s = 0.f;
+      for (int d = 0; d < dh; ++d) s = fmaf(qs[warp][d], __half2float(kr[d]), s);
+    }
+    const float mn = fmaxf(m, warp_max(s));
+    const float p = (j < n) ? expf(s - mn) : 0.f;
+    const float corr = expf(m - mn);
+    l = l * corr + warp_sum(p);
+    o0 *= corr; o1 *= corr;
+    const int cnt = min(32, n - j0);
+    for (int jj = 0; jj < cnt; ++jj) {
+      const float pj = __shfl_sync(0xffffffffu, p, jj);
+      const __half *vr = qkv + tok_of(j0 + jj) * ld + 2 * A + head * dh;
+      if (lane < dh) o0 = fmaf(pj, __half2float(vr[lane]), o0);
+      if (lane + 32 < dh) o1 = fmaf(pj, __half2float(vr[lane + 32]), o1);
+    }
+    m = mn;
+  }
+  const float g = __half2float(qkv[tq * ld + 3 * A + head]) / l;
+  __half *orow = o + tq * (long long)A + head * dh;
+  if (lane < dh) orow[lane] = __float2half_rn(o0 * g);
+  if (lane + 32 < dh) orow[lane + 32] = __float2half_rn(o1 * g);
+}
+
 // ------------------------------------------------------------------ output norm (fp16 schedule)
 // x = x / max(sqrt(ss), eps) * gain; writes x (fp32), its fp16 copy and the new sum of squares.
 __global__ void outnorm_kernel(float *__restrict__ x, float *__restrict__ ss, const float *__restrict__ gain,
@@ -436,12 +489,10 @@ void launch_attention_f32(const float *q, const float *k, const float *v, const 
                                                                       axis, n);
 }
 
-void launch_attention_simt_f16(const __half *q, const __half *k, const __half *v, const float *gate,
-                               __half *o, int B, int T, int nb, int heads, int dh, int axis, int n_pad,
-                               cudaStream_t st) {
+void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int T, int nb, int heads, int dh,
+                               int axis, cudaStream_t st) {
   const long long rows = (long long)B * T * nb * heads;
-  attention_simt_kernel<__half, __half><<<grid1(rows, 8), 256, 0, st>>>(q, k, v, gate, o, B, T, nb, heads,
-                                                                        dh, axis, n_pad);
+  attention_tokmajor_kernel<<<grid1(rows, 8), 256, 0, st>>>(qkv, ld, o, B, T, nb, heads, dh, axis);
 }
 
 void launch_outnorm(float *x, float *ss, const float *gain, __half *xh, long long rows, int D,

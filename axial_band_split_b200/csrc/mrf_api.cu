@@ -640,7 +640,11 @@ mrf_status mrf_debug_buffer(mrf_handle *h, const char *name, void *dst, size_t m
   bytes = std::min(bytes, max_bytes);
   mrf_status s = MRF_OK;
   if (!cuda_ok(h, cudaDeviceSynchronize(), "device sync", &s)) return s;
-  if (!cuda_ok(h, cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost), "debug copy", &s)) return s;
+  cudaPointerAttributes attr{};
+  const bool host_src = cudaPointerGetAttributes(&attr, src) == cudaSuccess && attr.type != cudaMemoryTypeDevice;
+  cudaGetLastError();
+  if (host_src) memcpy(dst, src, bytes);
+  else if (!cuda_ok(h, cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost), "debug copy", &s)) return s;
   if (bytes_out) *bytes_out = bytes;
   return MRF_OK;
 }

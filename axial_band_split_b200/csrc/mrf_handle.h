@@ -112,4 +112,5 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W);
 void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T);
 void destroy_fp16(mrf_handle *h);
 bool debug_buffer_fp16(mrf_handle *h, const std::string &name, const void **ptr, size_t *bytes);
+
 }  // namespace mrf

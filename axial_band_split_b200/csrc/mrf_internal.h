@@ -70,10 +70,9 @@ void launch_attention_f32(const float *q, const float *k, const float *v, const 
                           float *o, int B, int T, int nb, int heads, int dh, int axis,
                           cudaStream_t st);
 
-// Same on fp16 q, k, v with a per-sequence stride of n_pad positions; fp16 output.
-void launch_attention_simt_f16(const __half *q, const __half *k, const __half *v, const float *gate,
-                               __half *o, int B, int T, int nb, int heads, int dh, int axis, int n_pad,
-                               cudaStream_t st);
+// Same on the fp16 schedule's token-major rows qkv[tok][ld] = [q | k | v | sigmoid gates]; fp16 output.
+void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int T, int nb, int heads, int dh,
+                               int axis, cudaStream_t st);
 
 // x = x / max(sqrt(ss), eps) * gain (D % 128 == 0); writes x, its fp16 copy and ss = |x|^2.
 void launch_outnorm(float *x, float *ss, const float *gain, __half *xh, long long rows, int D,

@@ -29,8 +29,8 @@
 
 namespace mrf {
 
-bool launch_attention_tc(const __half *q, const __half *k, const __half *v, const float *gate, __half *o,
-                         int B, int T, int nb, int H, int axis, int n_pad, unsigned *status, cudaStream_t st);
+bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int axis,
+                         unsigned *status, cudaStream_t st);
 bool attention_tc_supported(int dh);
 bool attention_tc_init();
 
@@ -50,15 +50,15 @@ struct Fp16State {
   __half *mw_last = nullptr;  // [sum 2*d_in, MH], rows interleaved (value e, gate e)
   float *mb_last = nullptr;
   // group tables
-  GemmGroup *g_qkv = nullptr, *g_qkv_time = nullptr, *g_out = nullptr, *g_ff1 = nullptr, *g_ff2 = nullptr;
+  GemmGroup *g_qkv = nullptr, *g_out = nullptr, *g_ff1 = nullptr, *g_ff2 = nullptr;
   GemmGroup *g_m0 = nullptr, *g_mid = nullptr, *g_last = nullptr;
   int n_last_tiles = 0;
   // workspace
-  float *X = nullptr, *ss = nullptr, *G = nullptr, *Mg = nullptr;
-  __half *Xh = nullptr, *Q = nullptr, *K = nullptr, *V = nullptr, *O = nullptr, *Hh = nullptr,
-         *H1 = nullptr, *H2 = nullptr;
-  long long qkv_elems = 0;
-  int n_pad_time = 0, n_pad_band = 0;
+  float *X = nullptr, *ss = nullptr, *Mg = nullptr;
+  // deferred output norm: |x|^2 and |g x|^2 of the last FF2 output (g = sqrt(D) gamma_out)
+  float *ssx = nullptr, *ssg = nullptr;
+  __half *Xh = nullptr, *QKV = nullptr, *O = nullptr, *Hh = nullptr, *H1 = nullptr, *H2 = nullptr;
+  int ldq = 0;  // row length of QKV: [q | k | v | gates], padded to a multiple of 8
   int sms = 148;
   bool tc_attention = true;
 };
@@ -152,6 +152,15 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
       std::vector<float> qkvg = fold_cols(W[p + "layers.0.0.to_qkv.weight"].v, ga, 3 * A, D);
       std::vector<float> wg = fold_cols(W[p + "layers.0.0.to_gates.weight"].v, ga, H, D);
       qkvg.insert(qkvg.end(), wg.begin(), wg.end());
+      if (2 * l + a > 0) {
+        // the previous transformer's output norm is deferred: its sqrt(D) * gamma scales x
+        // column-wise, folded here into every q, k, v and gate weight column
+        const int pl = a == 1 ? l : l - 1, pa = a == 1 ? 0 : 1;
+        const auto &gp = W["layers." + std::to_string(pl) + "." + std::to_string(pa) + ".norm.gamma"].v;
+        const double sd = std::sqrt((double)D);
+        for (int n = 0; n < 3 * A + H; ++n)
+          for (int k = 0; k < D; ++k) qkvg[(size_t)n * D + k] = (float)((double)qkvg[(size_t)n * D + k] * gp[k] * sd);
+      }
       x.wqkvg = up(h, to_half(qkvg));
       x.bg = up(h, W[p + "layers.0.0.to_gates.bias"].v);
       x.wo = up(h, to_half(W[p + "layers.0.0.to_out.0.weight"].v));
@@ -187,6 +196,14 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
       bl.push_back(b[wd + e]);
     }
   }
+  if (c.depth > 0) {
+    // the last transformer's output norm is deferred: fold its sqrt(D) * gamma into the
+    // mask MLP's first layer (its 1 / |x| is a row scale in that layer's epilogue)
+    const auto &gl = W["layers." + std::to_string(c.depth - 1) + ".1.norm.gamma"].v;
+    const double sd = std::sqrt((double)D);
+    for (size_t r = 0; r < mw[0].size() / D; ++r)
+      for (int k = 0; k < D; ++k) mw[0][r * D + k] = (float)((double)mw[0][r * D + k] * gl[k] * sd);
+  }
   for (int i = 0; i < c.mask_depth; ++i) {
     f->mw.push_back(up(h, to_half(mw[i])));
     f->mb.push_back(up(h, mb[i]));
@@ -204,10 +221,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->g_out = single(D, kBnNarrow);
   f->g_ff1 = single(FF, kBnWide);
   f->g_ff2 = single(D, kBnNarrow);
-  std::vector<GemmGroup> gq(nb), g0(nb), g1(nb), g2(nb);
-  const int nq = cdiv(3 * A + H, kBnWide);
-  for (int k = 0; k < nb; ++k) gq[k] = {3 * A + H, nq, k * nq, k, 0, k, 0, 0};
-  f->g_qkv_time = upload_groups(h, gq);
+  std::vector<GemmGroup> g0(nb), g1(nb), g2(nb);
   int start = 0;
   for (int k = 0; k < nb; ++k) {
     g0[k] = {MH, cdiv(MH, kBnWide), k * cdiv(MH, kBnWide), k, k * MH, k, k * MH, 0};
@@ -220,28 +234,24 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->g_m0 = upload_groups(h, g0);
   f->g_mid = upload_groups(h, g1);
   f->g_last = upload_groups(h, g2);
-  if (!f->g_qkv || !f->g_qkv_time || !f->g_out || !f->g_ff1 || !f->g_ff2 || !f->g_m0 || !f->g_mid || !f->g_last) return MRF_ENOMEM;
+  if (!f->g_qkv || !f->g_out || !f->g_ff1 || !f->g_ff2 || !f->g_m0 || !f->g_mid || !f->g_last) return MRF_ENOMEM;
   // workspace
-  f->n_pad_time = cdiv(c.max_frames, 128) * 128;
-  f->n_pad_band = cdiv(nb, 64) * 64;
-  f->qkv_elems = std::max((long long)c.max_batch * nb * H * f->n_pad_time, MBT * H * f->n_pad_band) * dh;
+  f->ldq = cdiv(3 * A + H, 8) * 8;
   f->X = h->alloc<float>(NT * D);
   f->Xh = h->alloc<__half>(NT * D);
   f->ss = h->alloc<float>(NT);
-  f->G = h->alloc<float>(NT * H);
-  f->Q = h->alloc<__half>(f->qkv_elems);
-  f->K = h->alloc<__half>(f->qkv_elems);
-  f->V = h->alloc<__half>(f->qkv_elems);
+  f->ssx = h->alloc<float>(NT);
+  f->ssg = h->alloc<float>(NT);
+  f->QKV = h->alloc<__half>(NT * f->ldq);
   f->O = h->alloc<__half>(NT * A);
   f->Hh = h->alloc<__half>(NT * FF);
   f->H1 = h->alloc<__half>((long long)nb * MBT * MH);
   f->H2 = h->alloc<__half>((long long)nb * MBT * MH);
   f->Mg = h->alloc<float>(MBT * t.n_feat());
-  if (!f->X || !f->Xh || !f->ss || !f->G || !f->Q || !f->K || !f->V || !f->O || !f->Hh || !f->H1 || !f->H2 || !f->Mg)
+  if (!f->X || !f->Xh || !f->ss || !f->ssx || !f->ssg || !f->QKV || !f->O || !f->Hh || !f->H1 || !f->H2 || !f->Mg)
     return MRF_ENOMEM;
-  // padded positions of q, k, v are read by the attention tiles: keep them finite (zero)
-  if (cudaMemset(f->Q, 0, f->qkv_elems * 2) != cudaSuccess || cudaMemset(f->K, 0, f->qkv_elems * 2) != cudaSuccess ||
-      cudaMemset(f->V, 0, f->qkv_elems * 2) != cudaSuccess || cudaMemset(f->H1, 0, (size_t)nb * MBT * MH * 2) != cudaSuccess ||
+  // rows past a forward's B*T are read by ragged tiles (and discarded): keep them finite
+  if (cudaMemset(f->QKV, 0, NT * f->ldq * 2) != cudaSuccess || cudaMemset(f->H1, 0, (size_t)nb * MBT * MH * 2) != cudaSuccess ||
       cudaMemset(f->H2, 0, (size_t)nb * MBT * MH * 2) != cudaSuccess || cudaMemset(f->Xh, 0, NT * D * 2) != cudaSuccess)
     return MRF_ECUDA;
   return MRF_OK;
@@ -251,7 +261,27 @@ bool debug_buffer_fp16(mrf_handle *h, const std::string &name, const void **ptr,
   Fp16State *f = h->f16;
   if (!f) return false;
   const long long BT = (long long)h->last_B * h->last_T;
-  if (name == "X") { *ptr = f->X; *bytes = BT * h->cfg.num_bands * h->cfg.dim * sizeof(float); return true; }
+  if (name == "X") {
+    // the residual stream after the last transformer, with its deferred output norm applied
+    const int D = h->cfg.dim;
+    const long long rows = BT * h->cfg.num_bands;
+    static thread_local std::vector<float> hx;
+    hx.resize((size_t)rows * D);
+    if (cudaMemcpy(hx.data(), f->X, hx.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess) return false;
+    if (h->cfg.depth > 0) {
+      std::vector<float> s2(rows), g(D);
+      if (cudaMemcpy(s2.data(), f->ssx, rows * 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
+          cudaMemcpy(g.data(), f->tr.back().gout, D * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return false;
+      for (long long r = 0; r < rows; ++r) {
+        const float inv = 1.f / std::max(std::sqrt(s2[r]), 1e-12f);
+        for (int k = 0; k < D; ++k) hx[(size_t)r * D + k] *= inv * g[k];
+      }
+    }
+    *ptr = hx.data();
+    *bytes = hx.size() * 4;
+    return true;
+  }
   if (name == "M") { *ptr = f->Mg; *bytes = BT * h->tab.n_feat() * sizeof(float); return true; }
   return false;
 }
@@ -334,7 +364,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   const long long rows_last = 2LL * h->tab.n_feat();
   ok = ok && make_tmap_f16(&wmaps[wm0 + c.mask_depth], f->mw_last, MH, rows_last, 1, MH, rows_last * MH, kBnWide, 1);
   // bulk-store output maps
-  CUtensorMap mXo, mXho, mXbs, mXhbs, mHo, mH1o, mH2o, mMg;
+  CUtensorMap mXo, mXho, mXbs, mXhbs, mHo, mH1o, mH2o, mMg, mQKVo;
   {
     const unsigned long long BT = (unsigned long long)B * T;
     const unsigned long long dx[3] = {(unsigned long long)D, (unsigned long long)nb, BT};
@@ -347,7 +377,8 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
          make_tmap(&mXbs, f->X, kTmF32, 3, dx, sx, bx, 128) && make_tmap(&mXhbs, f->Xh, kTmF16, 3, dx, sx, bx, 64) &&
          map2(&mHo, f->Hh, kTmF16, FF, M, FF, 32, 64) && make_tmap(&mH1o, f->H1, kTmF16, 3, dh3, sh3, bh, 64) &&
          make_tmap(&mH2o, f->H2, kTmF16, 3, dh3, sh3, bh, 64) &&
-         map2(&mMg, f->Mg, kTmF32, h->tab.n_feat(), BT, h->tab.n_feat(), 16, 64);
+         map2(&mMg, f->Mg, kTmF32, h->tab.n_feat(), BT, h->tab.n_feat(), 16, 64) &&
+         map2(&mQKVo, f->QKV, kTmF16, 3 * A + H, M, f->ldq, 32, 64);
   }
   if (!ok) {
     h->sched_error = "tensor-map encoding failed";
@@ -357,10 +388,10 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   h->begin("band_gather");
   launch_band_gather(in, h->d_feat_row, h->d_feat_c, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, h->max_width, st);
   h->end();
-  cudaMemsetAsync(f->ss, 0, sizeof(float) * M, st);
+  cudaMemsetAsync(f->ssg, 0, sizeof(float) * M, st);
   {
     GemmParams p = base_params(h, B * T, f->k_bs, kBnNarrow, f->g_bs, nb, nb * cdiv(D, kBnNarrow));
-    p.bias = h->b_bs; p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D; p.nb = nb;
+    p.bias = h->b_bs; p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ssg; p.ld = D; p.nb = nb;
     gemm(h, "gemm_band_split", kTcBandSplit, mAbs, mWbs, p, &mXbs, &mXhbs);
   }
 
@@ -369,54 +400,50 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     const int axis = i & 1;
     const CUtensorMap &mWqkv = wmaps[4 * i + 0], &mWo = wmaps[4 * i + 1], &mW1 = wmaps[4 * i + 2],
                       &mW2 = wmaps[4 * i + 3];
-    const int n_pad = axis == 0 ? f->n_pad_time : f->n_pad_band;
-
-    // q, k, v, gates; on the time axis the rows run band-major (frame m of band g) so that
-    // consecutive rows of a tile are consecutive positions of one sequence
-    GemmParams p = axis == 0 ? base_params(h, B * T, D, kBnWide, f->g_qkv_time, nb, nb * cdiv(3 * A + H, kBnWide))
-                             : base_params(h, M, D, kBnWide, f->g_qkv, 1, cdiv(3 * A + H, kBnWide));
-    p.a_mode = axis == 0 ? 1 : 0;
-    p.ss_in = f->ss;
-    p.q = f->Q; p.k = f->K; p.v = f->V; p.gates = f->G; p.rope = h->d_rope; p.gbias = w.bg;
-    p.B = B; p.T = T; p.nb = nb; p.H = H; p.dh = dh; p.A = A; p.axis = axis; p.n_pad = n_pad;
+    // [q | k | v | gates] per token (RoPE positions along this transformer's axis)
+    GemmParams p = base_params(h, M, D, kBnWide, f->g_qkv, 1, cdiv(3 * A + H, kBnWide));
+    p.ss_in = f->ssg;  // |g x|^2 of the previous output (band split: |x|^2)
+    p.rope = h->d_rope; p.gbias = w.bg;
+    p.B = B; p.T = T; p.nb = nb; p.H = H; p.dh = dh; p.A = A; p.axis = axis;
     // the tensor-core attention takes scores in log2 units: fold log2(e) / sqrt(dh) into q
     p.q_scale = f->tc_attention ? (float)(1.4426950408889634 / std::sqrt((double)dh)) : 1.f;
-    gemm(h, "gemm_qkv", kTcQkv, axis == 0 ? mXband : mXh, mWqkv, p);
+    gemm(h, "gemm_qkv", kTcQkv, mXh, mWqkv, p, &mQKVo);
 
     h->begin(f->tc_attention ? (axis == 0 ? "attn_time_tc" : "attn_band_tc") : "attn_simt_f16");
     if (f->tc_attention) {
-      if (!launch_attention_tc(f->Q, f->K, f->V, f->G, f->O, B, T, nb, H, axis, n_pad, h->status, st)) {
+      if (!launch_attention_tc(f->QKV, f->ldq, f->O, B, T, nb, H, axis, h->status, st)) {
         h->end();
         h->sched_error = "tensor-map encoding failed (attention)";
         return;
       }
     } else
-      launch_attention_simt_f16(f->Q, f->K, f->V, f->G, f->O, B, T, nb, H, dh, axis, n_pad, st);
+      launch_attention_simt_f16(f->QKV, f->ldq, f->O, B, T, nb, H, dh, axis, st);
     h->end();
 
     cudaMemsetAsync(f->ss, 0, sizeof(float) * M, st);
     p = base_params(h, M, A, kBnNarrow, f->g_out, 1, cdiv(D, kBnNarrow));
     p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D;
+    if (i > 0) { p.res_ss = f->ssx; p.res_gain = f->tr[i - 1].gout; }  // the previous output norm
     gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p, &mXo, &mXho);
 
     p = base_params(h, M, D, kBnWide, f->g_ff1, 1, cdiv(FF, kBnWide));
     p.ss_in = f->ss; p.bias = w.b1; p.out_h = f->Hh; p.ldo = FF;
     gemm(h, "gemm_ff1_gelu", kTcGelu, mXh, mW1, p, &mHo);
 
-    cudaMemsetAsync(f->ss, 0, sizeof(float) * M, st);
+    cudaMemsetAsync(f->ssx, 0, sizeof(float) * M, st);
+    cudaMemsetAsync(f->ssg, 0, sizeof(float) * M, st);
     p = base_params(h, M, FF, kBnNarrow, f->g_ff2, 1, cdiv(D, kBnNarrow));
-    p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D; p.bias = w.b2;
+    p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ssx; p.ld = D; p.bias = w.b2;
+    p.ssg_out = f->ssg; p.out_gain = w.gout;  // the output norm is left to the consumers
     gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p, &mXo, &mXho);
-
-    h->begin("outnorm");
-    launch_outnorm(f->X, f->ss, w.gout, f->Xh, M, D, st);
-    h->end();
   }
 
   // mask head
   const int BT = B * T;
   GemmParams p = base_params(h, BT, D, kBnWide, f->g_m0, nb, nb * cdiv(MH, kBnWide));
   p.a_mode = 1;
+  p.ss_in = c.depth > 0 ? f->ssx : nullptr;  // 1 / |x| of the deferred last output norm
+  p.nb = nb;
   p.bias = f->mb[0]; p.out_h = f->H1; p.ldo = MH; p.out_group_stride = MBT * MH;
   gemm(h, "gemm_mask_tanh", kTcTanh, mXband, wmaps[wm0], p, &mH1o);
   __half *cur = f->H1, *nxt = f->H2;
@@ -440,3 +467,4 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
 }
 
 }  // namespace mrf
+

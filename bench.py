@@ -139,17 +139,22 @@ def kernel_source_hash():
 
 
 def traffic_for(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary
+    profiles/traffic.txt, if it was taken on the current kernel sources; else None.
+    Format: '# comment' lines, 'source_hash <hash>', then '<kernel> <bytes per launch>'."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
+    vals = {}
     with open(p) as f:
-        d = json.load(f)
-    if d.get("source_hash") != kernel_source_hash():
+        for line in f:
+            parts = line.split("#")[0].split()
+            if len(parts) == 2:
+                vals[parts[0]] = parts[1]
+    if vals.get("source_hash") != kernel_source_hash():
         return None
-    k = d.get("kernels", {}).get(kernel)
-    return k.get("dram_bytes_per_launch") if k else None
+    v = vals.get(kernel)
+    return float(v) if v is not None else None
 
 
 def cpu_baseline(cfg, frames, rank):
