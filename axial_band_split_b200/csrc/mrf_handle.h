@@ -113,4 +113,14 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T);
 void destroy_fp16(mrf_handle *h);
 bool debug_buffer_fp16(mrf_handle *h, const std::string &name, const void **ptr, size_t *bytes);
 
+// The fp16 schedule's per-forward workspace pointers, and their layout in one
+// caller-provided region (sched_fp16.cu); used by mrf_forward_static.
+struct Fp16Workspace {
+  float *X, *ss, *Mg;
+  __half *Xh, *QKV, *O, *Hh, *H1, *H2, *A_bs;
+  float *ssx, *ssg;
+};
+size_t fp16_workspace_layout(mrf_handle *h, void *base, bool apply, Fp16Workspace *saved, size_t *qkv_offset,
+                             size_t *qkv_bytes);
+void fp16_restore_workspace(mrf_handle *h, const Fp16Workspace &s);
 }  // namespace mrf

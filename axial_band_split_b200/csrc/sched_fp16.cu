@@ -468,3 +468,56 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
 
 }  // namespace mrf
 
+namespace mrf {
+
+// ------------------------------------------------------------------ caller-provided workspace
+// Lay the fp16 schedule's per-forward workspace out in one region of `bytes` at `base`
+// (256-byte aligned pieces, the same sizes as the handle's own workspace) and, if `apply`,
+// point the schedule at it; returns the bytes needed.  `saved` receives the handle's own
+// pointers so that fp16_restore_workspace can put them back.
+size_t fp16_workspace_layout(mrf_handle *h, void *base, bool apply, Fp16Workspace *saved,
+                             size_t *qkv_offset, size_t *qkv_bytes) {
+  Fp16State *f = h->f16;
+  const mrf_config &c = h->cfg;
+  const int nb = c.num_bands, D = c.dim, H = c.heads, A = H * c.dim_head, FF = c.ff_mult * D, MH = c.mask_hidden;
+  const long long MBT = (long long)c.max_batch * c.max_frames, NT = MBT * nb;
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off += (n + 255) & ~size_t(255);
+    return o;
+  };
+  const size_t oA = take((size_t)nb * MBT * f->k_bs * 2), oX = take(NT * D * 4), oXh = take(NT * D * 2),
+               oss = take(NT * 4), ossx = take(NT * 4), ossg = take(NT * 4);
+  const size_t oQ = take(NT * f->ldq * 2);
+  const size_t oO = take(NT * A * 2), oHh = take(NT * FF * 2), oH1 = take((size_t)nb * MBT * MH * 2),
+               oH2 = take((size_t)nb * MBT * MH * 2), oMg = take(MBT * h->tab.n_feat() * 4);
+  (void)H;
+  if (qkv_offset) *qkv_offset = oQ;
+  if (qkv_bytes) *qkv_bytes = oO - oQ;
+  if (apply && f) {
+    if (saved) *saved = {f->X, f->ss, f->Mg, f->Xh, f->QKV, f->O, f->Hh, f->H1, f->H2, f->A_bs, f->ssx, f->ssg};
+    uint8_t *b = static_cast<uint8_t *>(base);
+    f->A_bs = reinterpret_cast<__half *>(b + oA);
+    f->X = reinterpret_cast<float *>(b + oX);
+    f->Xh = reinterpret_cast<__half *>(b + oXh);
+    f->ss = reinterpret_cast<float *>(b + oss);
+    f->ssx = reinterpret_cast<float *>(b + ossx);
+    f->ssg = reinterpret_cast<float *>(b + ossg);
+    f->QKV = reinterpret_cast<__half *>(b + oQ);
+    f->O = reinterpret_cast<__half *>(b + oO);
+    f->Hh = reinterpret_cast<__half *>(b + oHh);
+    f->H1 = reinterpret_cast<__half *>(b + oH1);
+    f->H2 = reinterpret_cast<__half *>(b + oH2);
+    f->Mg = reinterpret_cast<float *>(b + oMg);
+  }
+  return off;
+}
+
+void fp16_restore_workspace(mrf_handle *h, const Fp16Workspace &s) {
+  Fp16State *f = h->f16;
+  f->X = s.X; f->ss = s.ss; f->Mg = s.Mg; f->Xh = s.Xh; f->QKV = s.QKV;
+  f->O = s.O; f->Hh = s.Hh; f->H1 = s.H1; f->H2 = s.H2; f->A_bs = s.A_bs; f->ssx = s.ssx; f->ssg = s.ssg;
+}
+
+}  // namespace mrf

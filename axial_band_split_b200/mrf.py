@@ -25,7 +25,7 @@ STATUS = {0: "MRF_OK", -1: "MRF_EINVAL", -2: "MRF_ESHAPE", -3: "MRF_ENOMEM", -4:
 # every symbol include/mrf.h declares
 EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
            "mrf_last_error", "mrf_band_tables", "mrf_set_timing", "mrf_kernel_times",
-           "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer"]
+           "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer", "mrf_forward_static"]
 
 
 class MrfError(RuntimeError):
@@ -65,6 +65,8 @@ def lib():
         L.mrf_create.restype = I
         L.mrf_forward.argtypes = [P, P, P, I, I, P]
         L.mrf_forward.restype = I
+        L.mrf_forward_static.argtypes = [P, P, P, I, I, P]
+        L.mrf_forward_static.restype = I
         L.mrf_forward_host.argtypes = [P, P, P, I, I, P]
         L.mrf_forward_host.restype = I
         L.mrf_sync_status.argtypes = [P, P]
@@ -179,6 +181,16 @@ class Model:
             out = torch.empty_like(stft_repr)
         _check(lib().mrf_forward(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
                                  ctypes.c_void_p(out.data_ptr()), B, T, _stream_ptr(stream)), self._h)
+        return out
+
+    def forward_static(self, stft_repr, out, stream=None):
+        """mrf_forward_static: the same forward with the library's fixed device scratch
+        instead of the handle's workspace; allocates nothing (out must be given)."""
+        import torch
+        assert stft_repr.is_cuda and stft_repr.dtype == torch.float32 and stft_repr.is_contiguous()
+        B, R, T, _ = stft_repr.shape
+        _check(lib().mrf_forward_static(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
+                                        ctypes.c_void_p(out.data_ptr()), B, T, _stream_ptr(stream)), self._h)
         return out
 
     def forward_host(self, stft_repr, out=None, stream=None):

@@ -122,6 +122,31 @@ mrf_status mrf_forward_host(mrf_handle *h, const float *stft_repr_host, float *m
                             int B, int T, void *stream);
 
 /*
+ * mrf_forward_static - the same fp16 forward as mrf_forward, for callers that must not
+ * allocate device memory while they run the model: a real-time audio callback that may not
+ * block in the allocator, or a host framework that owns every device allocation and
+ * forbids others during processing.  (The pages have no counterpart: this is an
+ * integration entry point, not a step of the method.)
+ *
+ * The per-call workspace lives in a 64 MiB array compiled into the library (every device
+ * that loads the library holds it until the process exits); nothing is allocated by this
+ * call: no cudaMalloc, no cudaFree, no graph instantiation (it launches eagerly).  The
+ * handle must come from mrf_create with compute = MRF_FP16, and its whole workspace for
+ * max_batch x max_frames must fit in 64 MiB, else MRF_ESHAPE with the size in the message
+ * (the tiny model fits at T <= ~2000; the vocals model only at a few tens of frames).
+ * stft_repr and masks as for mrf_forward; the handle's device must be current.
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture.  Every call
+ * uses the same array, which keeps the last call's contents (each call clears the
+ * accumulators it needs at zero and writes every other buffer before reading it): calls
+ * that overlap on the GPU, from any handle or thread, race and corrupt each other's
+ * results.  Serialise them (one stream, or events).
+ */
+mrf_status mrf_forward_static(mrf_handle *h, const float *stft_repr, float *masks, int B, int T,
+                              void *stream);
+
+/*
  * mrf_sync_status - wait for `stream`, then report the device status word: MRF_OK, or
  * MRF_ETIMEOUT if a kernel's bounded wait expired (the word is cleared on read), or
  * MRF_ECUDA for a CUDA error.
