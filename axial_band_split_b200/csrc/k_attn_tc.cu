@@ -236,6 +236,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tc_fence_after();
         issue_s(0, s);
         issue_s(1, s);
+        // q is read only by S = q k^T: release its buffer once the item's last S is issued,
+        // so the next item's q loads under this item's softmax and P v
+        if (a.n_blocks == 1) tc::mma_commit(q_empty);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
           s = g % kStages;
           const bool last = j + 1 == a.n_blocks;
@@ -250,11 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (t == 0 && !tc::mbar_wait(kv_full + s1, ((g + 1) / kStages) & 1, a.status, 36, abort)) { ok = false; break; }
               tc::tc_fence_after();
               issue_s(t, s1);
+              if (t == 1 && j + 2 == a.n_blocks) tc::mma_commit(q_empty);
             }
           }
           if (!ok) break;
         }
-        if (ok) tc::mma_commit(q_empty);
       }
       tc::mma_commit(done);
       tc::mbar_wait(done, 0, a.status, 37, abort);
