@@ -19,7 +19,9 @@
 //               each, bands past n read as zeros) with their own single K/V block, masked
 //               block-diagonally.
 // Warps 0-3 and 4-7: softmax of tile 0 and tile 1 (one query row per thread); warp 8: TMA;
-// warp 9: MMA issue.  Tensor memory (512 columns): S_t at 128 t, O_t at 256 + 64 t.
+// warp 9: MMA issue.  Tensor memory (512 columns): S_t at 128 t, O_t at 256 + 64 t, and P_t
+// (the softmax's fp16 probabilities, two per 32-bit column) at 384 + 64 t, which the P*V
+// MMA reads as its A operand straight from tensor memory.
 // O accumulates in tensor memory across key blocks; a row's running max is raised (and
 // its O row rescaled in place) only when a block's max exceeds it by more than 2^8, so
 // the unnormalised p stay below 256 and most blocks need no correction.
@@ -42,8 +44,7 @@ constexpr float kRescaleLog2 = 8.f;
 struct AttnSmem {
   static constexpr int q = 0;                              // [2 tiles]
   static constexpr int kv = q + 2 * kTile;                 // [stage][tile][K, V]
-  static constexpr int p = kv + kStages * 4 * kTile;       // [2 tiles] 128 x 128 fp16 (two column blocks)
-  static constexpr int bar = p + 2 * 2 * kTile;
+  static constexpr int bar = kv + kStages * 4 * kTile;
   static constexpr int total = bar + 256;
 };
 
@@ -93,6 +94,25 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
 }
 #undef MRF_R8
 
+
+// 4 consecutive 32-bit TMEM columns of this thread's lane; no wait.  (Four-register
+// pieces: a 16-register source group must sit in one aligned register block, which the
+// allocator could only provide by spilling.)
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// D (+)= A * B with A (M x K, fp16, two values per 32-bit column) in tensor memory.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u));
+}
 
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
@@ -219,14 +239,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mma_commit(s_full + t);
       };
       auto issue_pv = [&](int t, int s, bool acc) {
-        const uint32_t p_addr = tc::smem_u32(smem + AttnSmem::p + t * 2 * kTile);
         const uint32_t v_addr = tc::smem_u32(smem + AttnSmem::kv + (s * 4 + (shared_kv ? 0 : 2 * t) + 1) * kTile);
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint32_t pa = p_addr + (kk >> 2) * kTile + (kk & 3) * 32;
-          tc::mma_f16(tmem + 256 + 64 * t, tc::sw128_kmajor_desc(pa), tc::sw128_mnmajor_desc(v_addr + kk * 2048),
-                      id_pv, acc || kk != 0);
-        }
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          mma_f16_ts(tmem + 256 + 64 * t, tmem + 384 + 64 * t + 8 * kk, tc::sw128_mnmajor_desc(v_addr + kk * 2048),
+                     id_pv, acc || kk != 0);
         tc::mma_commit(pv_done + t);
       };
       for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
@@ -268,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = (warp & 3) * 32 + lane;
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + 128 * t + lane_off, tO = tmem + 256 + 64 * t + lane_off;
-    uint8_t *prow = smem + AttnSmem::p + t * 2 * kTile + r * 128;
+    const uint32_t tP = tmem + 384 + 64 * t + lane_off;  // P_t: 64 columns of packed fp16
     const int prob = r >> 6;  // band axis: which of the tile's two problems
     int g = 0;
     int li = 0;
@@ -294,8 +311,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 64; ++i)
               if (64 * hlf + i < lo || 64 * hlf + i >= hi) sv[i] = -INFINITY;
           }
+          // four independent max chains over 16 values each, joined at the end
+          float ma = sv[0], mb = sv[16], mc = sv[32], md = sv[48];
 #pragma unroll
-          for (int i = 0; i < 64; i += 2) mx = max3(mx, sv[i], sv[i + 1]);
+          for (int i = 1; i < 16; i += 2) {
+            ma = max3(ma, sv[i], sv[i + 1 < 16 ? i + 1 : i]);
+            mb = max3(mb, sv[16 + i], sv[16 + (i + 1 < 16 ? i + 1 : i)]);
+            mc = max3(mc, sv[32 + i], sv[32 + (i + 1 < 16 ? i + 1 : i)]);
+            md = max3(md, sv[48 + i], sv[48 + (i + 1 < 16 ? i + 1 : i)]);
+          }
+          mx = max3(mx, max3(ma, mb, mc), md);
         }
         const float m_cand = fmaxf(m_run, mx);
         // P_t and O_t are free once the previous block's P*V has completed
@@ -305,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float alpha = need ? ex2(m_run - m_cand) : 1.f;
         if (need) { l *= alpha; m_run = m_cand; }
         // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU
-        float2 acc2 = make_float2(0.f, 0.f);
+        float2 sa = make_float2(0.f, 0.f), sb = sa, sc = sa, sd = sa;  // four independent sum chains
         const float2 negm = make_float2(-m_run, -m_run);
 #pragma unroll
         for (int hlf = 0; hlf < 2; ++hlf) {
@@ -316,22 +341,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 64; ++i)
               if (64 * hlf + i < lo || 64 * hlf + i >= hi) sv[i] = -INFINITY;
           }
-          uint32_t hh[32];
 #pragma unroll
-          for (int i = 0; i < 64; i += 2) {
-            const float2 d = add2(make_float2(sv[i], sv[i + 1]), negm);
-            const float2 pp = make_float2(ex2(d.x), ex2(d.y));
-            acc2 = add2(acc2, pp);
-            hh[i >> 1] = pack_h2(pp.x, pp.y);
+          for (int q32 = 0; q32 < 64; q32 += 32) {
+            uint32_t hh[16];
+#pragma unroll
+            for (int i = q32; i < q32 + 32; i += 2) {
+              const float2 d = add2(make_float2(sv[i], sv[i + 1]), negm);
+              const float2 pp = make_float2(ex2(d.x), ex2(d.y));
+              switch ((i >> 1) & 3) {
+                case 0: sa = add2(sa, pp); break;
+                case 1: sb = add2(sb, pp); break;
+                case 2: sc = add2(sc, pp); break;
+                default: sd = add2(sd, pp); break;
+              }
+              hh[(i - q32) >> 1] = pack_h2(pp.x, pp.y);
+            }
+            // P into tensor memory, two fp16 per column: keys 64 hlf + q32 .. + 31
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              tmem_st4(tP + 32 * hlf + (q32 >> 1) + 4 * q, hh[4 * q], hh[4 * q + 1], hh[4 * q + 2], hh[4 * q + 3]);
           }
-          // 128-byte swizzle: 16-byte chunk index XOR (row % 8); column block hlf holds keys 64 hlf ..
-          uint8_t *blk = prow + hlf * kTile;
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<uint4 *>(blk + ((q ^ (r & 7)) << 4)) =
-                make_uint4(hh[4 * q], hh[4 * q + 1], hh[4 * q + 2], hh[4 * q + 3]);
         }
-        const float sum = acc2.x + acc2.y;
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        const float2 s01 = add2(sa, sb), s23 = add2(sc, sd);
+        const float2 s4 = add2(s01, s23);
+        const float sum = s4.x + s4.y;
         // O row rescaled in place when this row's max was raised (after P, to keep the
         // score row and the O chunk out of registers at the same time)
         if (any_need && j > 0) {
@@ -347,7 +381,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         l += sum;
         tc::tc_fence_before();
-        tc::fence_proxy_async();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(p_full + t);
       }
