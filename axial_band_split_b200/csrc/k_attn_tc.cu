@@ -18,8 +18,9 @@
 //   band axis - each tile holds the band sequences of two frames for one head (64 rows
 //               each, bands past n read as zeros) with their own single K/V block, masked
 //               block-diagonally.
-// Warps 0-3 and 4-7: softmax of tile 0 and tile 1 (one query row per thread); warp 8: TMA;
-// warp 9: MMA issue.  Tensor memory (512 columns): S_t at 128 t, O_t at 256 + 64 t, and P_t
+// Warps 0-3 and 4-7: softmax of tile 0 and tile 1 (one query row per thread, the whole
+// 128-score row in registers); warp 8: TMA; warp 9: MMA issue; warps 10-11 idle.  The third
+// warpgroup gives registers up to the two softmax warpgroups (setmaxnreg).  Tensor memory (512 columns): S_t at 128 t, O_t at 256 + 64 t, and P_t
 // (the softmax's fp16 probabilities, two per 32-bit column) at 384 + 64 t, which the P*V
 // MMA reads as its A operand straight from tensor memory.
 // O accumulates in tensor memory across key blocks; a row's running max is raised (and
@@ -35,16 +36,25 @@ namespace mrf {
 
 namespace {
 
-constexpr int kDh = 64, kRows = 128, kKeys = 128, kStages = 2;
+constexpr int kDh = 64, kRows = 128, kKeys = 128;
+// K/V ring: 12 tiles of 16 KB.  Time axis: one K and one V tile per stage, shared by both
+// query tiles (6 stages); band axis: a K and a V tile per query tile (3 stages).
+constexpr int kRingTiles = 12, kMaxStages = 6;
 static_assert(kKeys == 128, "the softmax reads a score row as two 64-column halves");
 constexpr int kTile = kRows * kDh * 2;  // 16 KB: one 128 x 64 fp16 tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// register split: launched at 168 per thread (384 threads, one CTA per SM); the TMA/MMA
+// warpgroup drops to kRegsIo and the softmax warpgroups rise to kRegsSoftmax, within the
+// launch's total: 2 * 128 * 208 + 128 * 72 = 62464 <= 384 * 168 = 64512.  (An increase
+// beyond what the launch holds would wait forever; the init checks the launch count.)
+constexpr int kRegsLaunch = 168, kRegsSoftmax = 208, kRegsIo = 72;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * kRegsLaunch, "register split over budget");
 constexpr float kRescaleLog2 = 8.f;
 
 struct AttnSmem {
   static constexpr int q = 0;                              // [2 tiles]
   static constexpr int kv = q + 2 * kTile;                 // [stage][tile][K, V]
-  static constexpr int bar = kv + kStages * 4 * kTile;
+  static constexpr int bar = kv + kRingTiles * kTile;
   static constexpr int total = bar + 256;
 };
 
@@ -70,16 +80,17 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
   return make_float2(__uint_as_float(static_cast<unsigned>(z)), __uint_as_float(static_cast<unsigned>(z >> 32)));
 }
 
-// 64 consecutive fp32 columns of this thread's TMEM lane: two loads, one wait.  The wait
-// takes the destination registers as operands so no use can be scheduled above it.
+// Consecutive fp32 columns of this thread's TMEM lane.  The wait takes the destination
+// registers as operands so no use can be scheduled above it.
 #define MRF_R8(b) "=r"(r[b]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), "=r"(r[b + 5]), \
                   "=r"(r[b + 6]), "=r"(r[b + 7])
 #define MRF_P8(b) "+r"(r[b]), "+r"(r[b + 1]), "+r"(r[b + 2]), "+r"(r[b + 3]), "+r"(r[b + 4]), "+r"(r[b + 5]), \
                   "+r"(r[b + 6]), "+r"(r[b + 7])
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r[64];
+// 128 consecutive fp32 columns: four loads, one wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
+  uint32_t r[128];
 #pragma unroll
-  for (int c = 0; c < 64; c += 32) {
+  for (int c = 0; c < 128; c += 32) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -89,10 +100,13 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
   }
   asm volatile("tcgen05.wait::ld.sync.aligned;" : MRF_P8(0), MRF_P8(8), MRF_P8(16), MRF_P8(24) : : "memory");
   asm volatile("" : MRF_P8(32), MRF_P8(40), MRF_P8(48), MRF_P8(56));
+  asm volatile("" : MRF_P8(64), MRF_P8(72), MRF_P8(80), MRF_P8(88));
+  asm volatile("" : MRF_P8(96), MRF_P8(104), MRF_P8(112), MRF_P8(120));
 #pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
 }
 #undef MRF_R8
+#undef MRF_P8
 
 
 // 4 consecutive 32-bit TMEM columns of this thread's lane; no wait.  (Four-register
@@ -162,25 +176,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + AttnSmem::bar);
   uint64_t *q_full = bars + 0, *q_empty = bars + 1;
-  uint64_t *kv_full = bars + 2;     // [kStages]
-  uint64_t *kv_empty = bars + 4;    // [kStages]
-  uint64_t *s_full = bars + 6;      // [2]
-  uint64_t *p_full = bars + 8;      // [2]
-  uint64_t *pv_done = bars + 10;    // [2]
-  uint64_t *o_free = bars + 12;     // [2]
-  uint64_t *done = bars + 14;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 15);
+  uint64_t *kv_full = bars + 2;     // [kMaxStages]
+  uint64_t *kv_empty = bars + 8;    // [kMaxStages]
+  uint64_t *s_full = bars + 14;     // [2]
+  uint64_t *p_full = bars + 16;     // [2]
+  uint64_t *pv_done = bars + 18;    // [2]
+  uint64_t *o_free = bars + 20;     // [2]
+  uint64_t *s_free = bars + 22;     // [2]
+  uint64_t *done = bars + 24;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 25);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool shared_kv = a.axis == 0;
+  const int stage_tiles = shared_kv ? 2 : 4, n_stages = kRingTiles / stage_tiles;
   if (threadIdx.x == 0) {
     abort_flag = 0;
     tc::mbar_init(q_full, 1);
     tc::mbar_init(q_empty, 1);
-    for (int s = 0; s < kStages; ++s) { tc::mbar_init(kv_full + s, 1); tc::mbar_init(kv_empty + s, 1); }
+    for (int s = 0; s < n_stages; ++s) { tc::mbar_init(kv_full + s, 1); tc::mbar_init(kv_empty + s, 1); }
     for (int t = 0; t < 2; ++t) {
       tc::mbar_init(s_full + t, 1);
+      tc::mbar_init(s_free + t, 4);
       tc::mbar_init(p_full + t, 4);
       tc::mbar_init(pv_done + t, 1);
       tc::mbar_init(o_free + t, 4);
@@ -194,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int *abort = &abort_flag;
-
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIo));
   if (warp == 8) {
     // ---------------- TMA producer
     if (lane == 0) {
@@ -209,12 +227,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t)
           tc::tma_load_4d(smem + AttnSmem::q + t * kTile, &tq, q_full, 0, it.head, it.band, it.frame0[t]);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
-          const int s = g % kStages;
-          if (!tc::mbar_wait(kv_empty + s, ((g / kStages) & 1) ^ 1, a.status, 31, abort)) { ok = false; break; }
+          const int s = g % n_stages;
+          if (!tc::mbar_wait(kv_empty + s, ((g / n_stages) & 1) ^ 1, a.status, 31, abort)) { ok = false; break; }
           tc::mbar_arrive_expect_tx(kv_full + s, kv_bytes);
           for (int t = 0; t < (shared_kv ? 1 : 2); ++t) {
             const int f = shared_kv ? it.frame0[0] - it.qt0 * kRows + j * kKeys : it.frame0[t];
-            uint8_t *dst = smem + AttnSmem::kv + (s * 4 + 2 * t) * kTile;
+            uint8_t *dst = smem + AttnSmem::kv + (s * stage_tiles + 2 * t) * kTile;
             tc::tma_load_4d(dst, &tk, kv_full + s, 0, it.head, it.band, f);
             tc::tma_load_4d(dst + kTile, &tv, kv_full + s, 0, it.head, it.band, f);
           }
@@ -231,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto issue_s = [&](int t, int s) {
         const uint32_t q_addr = tc::smem_u32(smem + AttnSmem::q + t * kTile);
-        const uint32_t k_addr = tc::smem_u32(smem + AttnSmem::kv + (s * 4 + (shared_kv ? 0 : 2 * t)) * kTile);
+        const uint32_t k_addr = tc::smem_u32(smem + AttnSmem::kv + (s * stage_tiles + (shared_kv ? 0 : 2 * t)) * kTile);
 #pragma unroll
         for (int kk = 0; kk < kDh / 16; ++kk)
           tc::mma_f16(tmem + 128 * t, tc::sw128_kmajor_desc(q_addr + kk * 32), tc::sw128_kmajor_desc(k_addr + kk * 32),
@@ -239,39 +257,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mma_commit(s_full + t);
       };
       auto issue_pv = [&](int t, int s, bool acc) {
-        const uint32_t v_addr = tc::smem_u32(smem + AttnSmem::kv + (s * 4 + (shared_kv ? 0 : 2 * t) + 1) * kTile);
+        const uint32_t v_addr = tc::smem_u32(smem + AttnSmem::kv + (s * stage_tiles + (shared_kv ? 0 : 2 * t) + 1) * kTile);
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
           mma_f16_ts(tmem + 256 + 64 * t, tmem + 384 + 64 * t + 8 * kk, tc::sw128_mnmajor_desc(v_addr + kk * 2048),
                      id_pv, acc || kk != 0);
         tc::mma_commit(pv_done + t);
       };
+      // S(t) of a block is issued once the softmax has read S(t) of the block before (its
+      // registers then hold the scores), so the next scores compute under this block's
+      // exponentials; P(t)*V follows once P(t) is in tensor memory.
       for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
         if (!tc::mbar_wait(q_full, li & 1, a.status, 32, abort)) break;
-        int s = g % kStages;
-        if (!tc::mbar_wait(kv_full + s, (g / kStages) & 1, a.status, 33, abort)) break;
-        tc::tc_fence_after();
-        issue_s(0, s);
-        issue_s(1, s);
+        int s = g % n_stages;
+        if (!tc::mbar_wait(kv_full + s, (g / n_stages) & 1, a.status, 33, abort)) break;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (g > 0 && !tc::mbar_wait(s_free + t, (g - 1) & 1, a.status, 41, abort)) ok = false;
+          tc::tc_fence_after();
+          if (ok) issue_s(t, s);
+        }
+        if (!ok) break;
         // q is read only by S = q k^T: release its buffer once the item's last S is issued,
         // so the next item's q loads under this item's softmax and P v
         if (a.n_blocks == 1) tc::mma_commit(q_empty);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
-          s = g % kStages;
+          s = g % n_stages;
           const bool last = j + 1 == a.n_blocks;
-          const int s1 = (g + 1) % kStages;
+          const int s1 = (g + 1) % n_stages;
           for (int t = 0; t < 2; ++t) {
+            if (!last) {
+              if (t == 0 && !tc::mbar_wait(kv_full + s1, ((g + 1) / n_stages) & 1, a.status, 36, abort)) { ok = false; break; }
+              if (!tc::mbar_wait(s_free + t, g & 1, a.status, 41, abort)) { ok = false; break; }
+              tc::tc_fence_after();
+              issue_s(t, s1);
+              if (t == 1 && j + 2 == a.n_blocks) tc::mma_commit(q_empty);
+            }
             if (!tc::mbar_wait(p_full + t, g & 1, a.status, 34, abort)) { ok = false; break; }
             if (j == 0 && !tc::mbar_wait(o_free + t, (li & 1) ^ 1, a.status, 35, abort)) { ok = false; break; }
             tc::tc_fence_after();
             issue_pv(t, s, j != 0);
             if (t == 1) tc::mma_commit(kv_empty + s);
-            if (!last) {
-              if (t == 0 && !tc::mbar_wait(kv_full + s1, ((g + 1) / kStages) & 1, a.status, 36, abort)) { ok = false; break; }
-              tc::tc_fence_after();
-              issue_s(t, s1);
-              if (t == 1 && j + 2 == a.n_blocks) tc::mma_commit(q_empty);
-            }
           }
           if (!ok) break;
         }
@@ -279,7 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mma_commit(done);
       tc::mbar_wait(done, 0, a.status, 37, abort);
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ---------------- softmax warpgroups: tile t = warp / 4, query row r of the tile
     const int t = warp >> 2;
     const int r = (warp & 3) * 32 + lane;
@@ -292,75 +319,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
       float m_run = -INFINITY, l = 0.f;
+      // this row's output token and its head's gate, fetched now so the load's latency is
+      // hidden under the item's key blocks
+      const Item it = item_coords(a, item);
+      long long tok = -1;
+      if (a.axis == 0) {
+        const int pos = (it.qt0 + t) * kRows + r;
+        if (pos < a.n) tok = (long long)(it.frame0[t] + r) * a.nb + it.band;
+      } else {
+        const int f = it.frame0[t] + prob, k = r & 63;
+        if (k < a.n && f < a.BT) tok = (long long)f * a.nb + k;
+      }
+      const __half gate = tok >= 0 ? a.qkv[tok * a.ld + 3 * a.H * kDh + it.head] : __float2half(0.f);
       for (int j = 0; j < a.n_blocks; ++j, ++g) {
         if (!tc::mbar_wait(s_full + t, g & 1, a.status, 38, abort)) { ok = false; break; }
         tc::tc_fence_after();
         int lo, hi;
         if (a.axis == 0) { lo = 0; hi = min(kKeys, a.n - j * kKeys); }
         else { lo = prob * 64; hi = prob * 64 + a.n; }
-        // the score row in two 64-column reads (scores arrive in log2 units: q was scaled by
-        // log2(e) / sqrt(dh) in its projection)
-        const bool masked = !(lo == 0 && hi == kKeys);
-        float mx = -INFINITY;
+        // the whole score row (scores arrive in log2 units: q was scaled by log2(e) / sqrt(dh)
+        // in its projection)
+        float sv[kKeys];
+        tmem_ld128(tS, sv);
+        // S_t may now take the next block's scores
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(s_free + t);
+        if (!(lo == 0 && hi == kKeys)) {
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          float sv[64];
-          tmem_ld64(tS + 64 * hlf, sv);
-          if (masked) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (64 * hlf + i < lo || 64 * hlf + i >= hi) sv[i] = -INFINITY;
-          }
-          // four independent max chains over 16 values each, joined at the end
-          float ma = sv[0], mb = sv[16], mc = sv[32], md = sv[48];
-#pragma unroll
-          for (int i = 1; i < 16; i += 2) {
-            ma = max3(ma, sv[i], sv[i + 1 < 16 ? i + 1 : i]);
-            mb = max3(mb, sv[16 + i], sv[16 + (i + 1 < 16 ? i + 1 : i)]);
-            mc = max3(mc, sv[32 + i], sv[32 + (i + 1 < 16 ? i + 1 : i)]);
-            md = max3(md, sv[48 + i], sv[48 + (i + 1 < 16 ? i + 1 : i)]);
-          }
-          mx = max3(mx, max3(ma, mb, mc), md);
+          for (int i = 0; i < kKeys; ++i)
+            if (i < lo || i >= hi) sv[i] = -INFINITY;
         }
-        const float m_cand = fmaxf(m_run, mx);
+        // four independent max chains over 32 values each, joined at the end
+        float ma = sv[0], mb = sv[32], mc = sv[64], md = sv[96];
+#pragma unroll
+        for (int i = 1; i < 32; i += 2) {
+          const int i2 = i + 1 < 32 ? i + 1 : i;
+          ma = max3(ma, sv[i], sv[i2]);
+          mb = max3(mb, sv[32 + i], sv[32 + i2]);
+          mc = max3(mc, sv[64 + i], sv[64 + i2]);
+          md = max3(md, sv[96 + i], sv[96 + i2]);
+        }
+        const float m_cand = fmaxf(m_run, fmaxf(fmaxf(ma, mb), fmaxf(mc, md)));
         // P_t and O_t are free once the previous block's P*V has completed
         if (j > 0 && !tc::mbar_wait(pv_done + t, (g - 1) & 1, a.status, 39, abort)) { ok = false; break; }
         const bool need = m_cand > m_run + kRescaleLog2;
         const bool any_need = __any_sync(0xffffffffu, need);
         const float alpha = need ? ex2(m_run - m_cand) : 1.f;
         if (need) { l *= alpha; m_run = m_cand; }
-        // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU
+        // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU, and P into
+        // tensor memory two fp16 per column, four columns (8 keys) per store
         float2 sa = make_float2(0.f, 0.f), sb = sa, sc = sa, sd = sa;  // four independent sum chains
         const float2 negm = make_float2(-m_run, -m_run);
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          float sv[64];
-          tmem_ld64(tS + 64 * hlf, sv);
-          if (masked) {
+        for (int i = 0; i < kKeys; i += 8) {
+          uint32_t hh[4];
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (64 * hlf + i < lo || 64 * hlf + i >= hi) sv[i] = -INFINITY;
-          }
-#pragma unroll
-          for (int q32 = 0; q32 < 64; q32 += 32) {
-            uint32_t hh[16];
-#pragma unroll
-            for (int i = q32; i < q32 + 32; i += 2) {
-              const float2 d = add2(make_float2(sv[i], sv[i + 1]), negm);
-              const float2 pp = make_float2(ex2(d.x), ex2(d.y));
-              switch ((i >> 1) & 3) {
-                case 0: sa = add2(sa, pp); break;
-                case 1: sb = add2(sb, pp); break;
-                case 2: sc = add2(sc, pp); break;
-                default: sd = add2(sd, pp); break;
-              }
-              hh[(i - q32) >> 1] = pack_h2(pp.x, pp.y);
+          for (int u = 0; u < 4; ++u) {
+            const float2 d = add2(make_float2(sv[i + 2 * u], sv[i + 2 * u + 1]), negm);
+            const float2 pp = make_float2(ex2(d.x), ex2(d.y));
+            switch (u) {
+              case 0: sa = add2(sa, pp); break;
+              case 1: sb = add2(sb, pp); break;
+              case 2: sc = add2(sc, pp); break;
+              default: sd = add2(sd, pp); break;
             }
-            // P into tensor memory, two fp16 per column: keys 64 hlf + q32 .. + 31
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              tmem_st4(tP + 32 * hlf + (q32 >> 1) + 4 * q, hh[4 * q], hh[4 * q + 1], hh[4 * q + 2], hh[4 * q + 3]);
+            hh[u] = pack_h2(pp.x, pp.y);
           }
+          tmem_st4(tP + (i >> 1), hh[0], hh[1], hh[2], hh[3]);
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         const float2 s01 = add2(sa, sb), s23 = add2(sc, sd);
@@ -401,19 +427,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(o_free + t);
-      const Item it = item_coords(a, item);
-      long long tok = -1;
-      const int head = it.head;
-      if (a.axis == 0) {
-        const int pos = (it.qt0 + t) * kRows + r;
-        if (pos < a.n) tok = (long long)(it.frame0[t] + r) * a.nb + it.band;
-      } else {
-        const int f = it.frame0[t] + prob, k = r & 63;
-        if (k < a.n && f < a.BT) tok = (long long)f * a.nb + k;
-      }
       if (tok >= 0) {
-        const float gsc = __half2float(a.qkv[tok * a.ld + 3 * a.H * kDh + head]) / l;
-        __half *dst = a.o + tok * (long long)a.H * kDh + head * kDh;
+        const float gsc = __half2float(gate) / l;
+        __half *dst = a.o + tok * (long long)a.H * kDh + it.head * kDh;
 #pragma unroll
         for (int d = 0; d < kDh; d += 8) {
           *reinterpret_cast<uint4 *>(dst + d) =
@@ -441,6 +457,8 @@ bool attention_tc_init() {
   int dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, attn_tc_kernel) != cudaSuccess || fa.numRegs < kRegsLaunch) return false;
   return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)(AttnSmem::total + 1024)) == cudaSuccess;
 }
