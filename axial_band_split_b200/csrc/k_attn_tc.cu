@@ -18,11 +18,13 @@
 //   band axis - each tile holds the band sequences of two frames for one head (64 rows
 //               each, bands past n read as zeros) with their own single K/V block, masked
 //               block-diagonally.
-// Warps 0-3 and 4-7: softmax of tile 0 and tile 1 (one query row per thread, the whole
-// 128-score row in registers); warp 8: TMA; warp 9: MMA issue; warps 10-11 idle.  The third
-// warpgroup gives registers up to the two softmax warpgroups (setmaxnreg).  Tensor memory (512 columns): S_t at 128 t, O_t at 256 + 64 t, and P_t
-// (the softmax's fp16 probabilities, two per 32-bit column) at 384 + 64 t, which the P*V
-// MMA reads as its A operand straight from tensor memory.
+// Warps 0-3 and 4-7: softmax of tile 0 and tile 1 (one query row per thread, the row's
+// live scores in registers: 128 on the time axis, the row's own 64-key half on the band
+// axis); warp 8: TMA; warp 9: MMA issue; warps 10-11 idle.  The third warpgroup gives
+// registers up to the two softmax warpgroups (setmaxnreg).
+// Tensor memory (512 columns): S_t at 128 t, O_t at 256 + 64 t, and P_t (the softmax's
+// fp16 probabilities, two per 32-bit column) at 384 + 64 t, which the P*V MMA reads as its
+// A operand straight from tensor memory.
 // O accumulates in tensor memory across key blocks; a row's running max is raised (and
 // its O row rescaled in place) only when a block's max exceeds it by more than 2^8, so
 // the unnormalised p stay below 256 and most blocks need no correction.
@@ -37,9 +39,9 @@ namespace mrf {
 namespace {
 
 constexpr int kDh = 64, kRows = 128, kKeys = 128;
-// K/V ring: 12 tiles of 16 KB.  Time axis: one K and one V tile per stage, shared by both
-// query tiles (6 stages); band axis: a K and a V tile per query tile (3 stages).
-constexpr int kRingTiles = 12, kMaxStages = 6;
+// K/V ring: 10 tiles of 16 KB.  Time axis: one K and one V tile per stage, shared by both
+// query tiles (5 stages); band axis: a K and a V tile per query tile (2 stages).
+constexpr int kRingTiles = 10, kMaxStages = 5;
 static_assert(kKeys == 128, "the softmax reads a score row as two 64-column halves");
 constexpr int kTile = kRows * kDh * 2;  // 16 KB: one 128 x 64 fp16 tile
 constexpr int kThreads = 384;
@@ -54,7 +56,8 @@ constexpr float kRescaleLog2 = 8.f;
 struct AttnSmem {
   static constexpr int q = 0;                              // [2 tiles]
   static constexpr int kv = q + 2 * kTile;                 // [stage][tile][K, V]
-  static constexpr int bar = kv + kRingTiles * kTile;
+  static constexpr int ostage = kv + kRingTiles * kTile;  // [8 warps] 32 rows x 128 B of output
+  static constexpr int bar = ostage + 8 * 4096;
   static constexpr int total = bar + 256;
 };
 
@@ -86,11 +89,13 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
                   "=r"(r[b + 6]), "=r"(r[b + 7])
 #define MRF_P8(b) "+r"(r[b]), "+r"(r[b + 1]), "+r"(r[b + 2]), "+r"(r[b + 3]), "+r"(r[b + 4]), "+r"(r[b + 5]), \
                   "+r"(r[b + 6]), "+r"(r[b + 7])
-// 128 consecutive fp32 columns: four loads, one wait.
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
+// N (64 or 128) consecutive fp32 columns: N / 32 loads, one wait.
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[N]) {
+  static_assert(N == 64 || N == 128, "64 or 128 columns");
   uint32_t r[128];
 #pragma unroll
-  for (int c = 0; c < 128; c += 32) {
+  for (int c = 0; c < N; c += 32) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
@@ -100,10 +105,12 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float (&v)[128]) {
   }
   asm volatile("tcgen05.wait::ld.sync.aligned;" : MRF_P8(0), MRF_P8(8), MRF_P8(16), MRF_P8(24) : : "memory");
   asm volatile("" : MRF_P8(32), MRF_P8(40), MRF_P8(48), MRF_P8(56));
-  asm volatile("" : MRF_P8(64), MRF_P8(72), MRF_P8(80), MRF_P8(88));
-  asm volatile("" : MRF_P8(96), MRF_P8(104), MRF_P8(112), MRF_P8(120));
+  if (N == 128) {
+    asm volatile("" : MRF_P8(64), MRF_P8(72), MRF_P8(80), MRF_P8(88));
+    asm volatile("" : MRF_P8(96), MRF_P8(104), MRF_P8(112), MRF_P8(120));
+  }
 #pragma unroll
-  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
 }
 #undef MRF_R8
 #undef MRF_P8
@@ -128,6 +135,15 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u));
 }
 
+// 5-D bulk tensor store from shared memory (one bulk group per call site commit).
+__device__ __forceinline__ void tma_store_5d(const CUtensorMap *map, const void *src, int c0, int c1, int c2,
+                                             int c3, int c4) {
+  asm volatile("cp.async.bulk.tensor.5d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(tc::smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t *>(&h);
@@ -145,7 +161,7 @@ struct AttnArgs {
 // one (band, head) sequence.  Band axis: tile t covers frames frame0[t] and frame0[t] + 1,
 // bands 0..63 of each (bands past nb read as zeros).
 struct Item {
-  int head, band, qt0;
+  int head, band, qt0, b;
   int frame0[2];
 };
 
@@ -158,10 +174,12 @@ __device__ __forceinline__ Item item_coords(const AttnArgs &a, int item) {
     const int seq = sh / a.H;
     it.band = seq % a.nb;
     const int b = seq / a.nb;
+    it.b = b;
     for (int t = 0; t < 2; ++t) it.frame0[t] = b * a.T + (it.qt0 + t) * kRows;
   } else {
     it.head = item % a.H;
     it.band = 0;
+    it.b = 0;
     it.qt0 = 0;
     const int f = 4 * (item / a.H);
     for (int t = 0; t < 2; ++t) it.frame0[t] = f + 2 * t;
@@ -169,9 +187,92 @@ __device__ __forceinline__ Item item_coords(const AttnArgs &a, int item) {
   return it;
 }
 
+// One key block of one query row: scores from tensor memory (log2 units: q was scaled by
+// log2(e) / sqrt(dh) in its projection), the running max and sum, p = 2^(s - m) into P as
+// fp16, and the O row rescaled in place when its max was raised.  NC live score columns at
+// tS (columns >= hi are masked); P's matching NC / 2 columns at tP.  Returns false if a
+// wait timed out.
+template <int NC>
+__device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t tO, int hi, float &m_run, float &l,
+                                              bool wait_pv, uint64_t *pv_done, uint32_t pv_parity,
+                                              uint64_t *s_free, uint64_t *p_full, int lane, unsigned *status,
+                                              volatile int *abort) {
+  float sv[NC];
+  tmem_ldn<NC>(tS, sv);
+  // S_t may now take the next block's scores
+  tc::tc_fence_before();
+  __syncwarp();
+  if (lane == 0) tc::mbar_arrive(s_free);
+  if (hi < NC) {
+#pragma unroll
+    for (int i = 0; i < NC; ++i)
+      if (i >= hi) sv[i] = -INFINITY;
+  }
+  // four independent max chains, joined at the end
+  constexpr int Q = NC / 4;
+  float ma = sv[0], mb = sv[Q], mc = sv[2 * Q], md = sv[3 * Q];
+#pragma unroll
+  for (int i = 1; i < Q; i += 2) {
+    const int i2 = i + 1 < Q ? i + 1 : i;
+    ma = max3(ma, sv[i], sv[i2]);
+    mb = max3(mb, sv[Q + i], sv[Q + i2]);
+    mc = max3(mc, sv[2 * Q + i], sv[2 * Q + i2]);
+    md = max3(md, sv[3 * Q + i], sv[3 * Q + i2]);
+  }
+  const float m_cand = fmaxf(m_run, fmaxf(fmaxf(ma, mb), fmaxf(mc, md)));
+  // P_t and O_t are free once the previous block's P*V has completed
+  if (wait_pv && !tc::mbar_wait(pv_done, pv_parity, status, 39, abort)) return false;
+  const bool need = m_cand > m_run + kRescaleLog2;
+  const bool any_need = __any_sync(0xffffffffu, need);
+  const float alpha = need ? ex2(m_run - m_cand) : 1.f;
+  if (need) { l *= alpha; m_run = m_cand; }
+  // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU, and P into
+  // tensor memory two fp16 per column, four columns (8 keys) per store
+  float2 sa = make_float2(0.f, 0.f), sb = sa, sc = sa, sd = sa;  // four independent sum chains
+  const float2 negm = make_float2(-m_run, -m_run);
+#pragma unroll
+  for (int i = 0; i < NC; i += 8) {
+    uint32_t hh[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 d = add2(make_float2(sv[i + 2 * u], sv[i + 2 * u + 1]), negm);
+      const float2 pp = make_float2(ex2(d.x), ex2(d.y));
+      switch (u) {
+        case 0: sa = add2(sa, pp); break;
+        case 1: sb = add2(sb, pp); break;
+        case 2: sc = add2(sc, pp); break;
+        default: sd = add2(sd, pp); break;
+      }
+      hh[u] = pack_h2(pp.x, pp.y);
+    }
+    tmem_st4(tP + (i >> 1), hh[0], hh[1], hh[2], hh[3]);
+  }
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+  const float2 s01 = add2(sa, sb), s23 = add2(sc, sd);
+  const float2 s4 = add2(s01, s23);
+  // O row rescaled in place when this row's max was raised
+  if (any_need && wait_pv) {
+    tc::tc_fence_after();
+#pragma unroll
+    for (int c = 0; c < kDh; c += 32) {
+      float v[32];
+      tc::tmem_ld32(tO + c, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] *= alpha;
+      tc::tmem_st32(tO + c, v);
+    }
+  }
+  l += s4.x + s4.y;
+  tc::tc_fence_before();
+  __syncwarp();
+  if (lane == 0) tc::mbar_arrive(p_full);
+  return true;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                   const __grid_constant__ CUtensorMap tv, const AttnArgs a) {
+                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                   const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + AttnSmem::bar);
@@ -282,23 +383,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (a.n_blocks == 1) tc::mma_commit(q_empty);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
           s = g % n_stages;
-          const bool last = j + 1 == a.n_blocks;
-          const int s1 = (g + 1) % n_stages;
-          for (int t = 0; t < 2; ++t) {
-            if (!last) {
-              if (t == 0 && !tc::mbar_wait(kv_full + s1, ((g + 1) / n_stages) & 1, a.status, 36, abort)) { ok = false; break; }
+          // both tiles' next scores first: each waits only for its softmax to have read S,
+          // so they compute under this block's exponentials
+          if (j + 1 < a.n_blocks) {
+            const int s1 = (g + 1) % n_stages;
+            if (!tc::mbar_wait(kv_full + s1, ((g + 1) / n_stages) & 1, a.status, 36, abort)) { ok = false; break; }
+            for (int t = 0; t < 2 && ok; ++t) {
               if (!tc::mbar_wait(s_free + t, g & 1, a.status, 41, abort)) { ok = false; break; }
               tc::tc_fence_after();
               issue_s(t, s1);
-              if (t == 1 && j + 2 == a.n_blocks) tc::mma_commit(q_empty);
             }
+            if (!ok) break;
+            if (j + 2 == a.n_blocks) tc::mma_commit(q_empty);
+          }
+          for (int t = 0; t < 2; ++t) {
             if (!tc::mbar_wait(p_full + t, g & 1, a.status, 34, abort)) { ok = false; break; }
             if (j == 0 && !tc::mbar_wait(o_free + t, (li & 1) ^ 1, a.status, 35, abort)) { ok = false; break; }
             tc::tc_fence_after();
             issue_pv(t, s, j != 0);
-            if (t == 1) tc::mma_commit(kv_empty + s);
           }
           if (!ok) break;
+          tc::mma_commit(kv_empty + s);
         }
       }
       tc::mma_commit(done);
@@ -317,6 +422,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g = 0;
     int li = 0;
     bool ok = true;
+    if (a.axis == 1) {
+      // band axis: a row's P over the other problem's 64 keys stays zero for the whole launch
+#pragma unroll
+      for (int c = 0; c < 32; c += 4) tmem_st4(tP + 32 * (1 - prob) + c, 0u, 0u, 0u, 0u);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    }
     for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
       float m_run = -INFINITY, l = 0.f;
       // this row's output token and its head's gate, fetched now so the load's latency is
@@ -334,81 +445,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < a.n_blocks; ++j, ++g) {
         if (!tc::mbar_wait(s_full + t, g & 1, a.status, 38, abort)) { ok = false; break; }
         tc::tc_fence_after();
-        int lo, hi;
-        if (a.axis == 0) { lo = 0; hi = min(kKeys, a.n - j * kKeys); }
-        else { lo = prob * 64; hi = prob * 64 + a.n; }
-        // the whole score row (scores arrive in log2 units: q was scaled by log2(e) / sqrt(dh)
-        // in its projection)
-        float sv[kKeys];
-        tmem_ld128(tS, sv);
-        // S_t may now take the next block's scores
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(s_free + t);
-        if (!(lo == 0 && hi == kKeys)) {
-#pragma unroll
-          for (int i = 0; i < kKeys; ++i)
-            if (i < lo || i >= hi) sv[i] = -INFINITY;
-        }
-        // four independent max chains over 32 values each, joined at the end
-        float ma = sv[0], mb = sv[32], mc = sv[64], md = sv[96];
-#pragma unroll
-        for (int i = 1; i < 32; i += 2) {
-          const int i2 = i + 1 < 32 ? i + 1 : i;
-          ma = max3(ma, sv[i], sv[i2]);
-          mb = max3(mb, sv[32 + i], sv[32 + i2]);
-          mc = max3(mc, sv[64 + i], sv[64 + i2]);
-          md = max3(md, sv[96 + i], sv[96 + i2]);
-        }
-        const float m_cand = fmaxf(m_run, fmaxf(fmaxf(ma, mb), fmaxf(mc, md)));
-        // P_t and O_t are free once the previous block's P*V has completed
-        if (j > 0 && !tc::mbar_wait(pv_done + t, (g - 1) & 1, a.status, 39, abort)) { ok = false; break; }
-        const bool need = m_cand > m_run + kRescaleLog2;
-        const bool any_need = __any_sync(0xffffffffu, need);
-        const float alpha = need ? ex2(m_run - m_cand) : 1.f;
-        if (need) { l *= alpha; m_run = m_cand; }
-        // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU, and P into
-        // tensor memory two fp16 per column, four columns (8 keys) per store
-        float2 sa = make_float2(0.f, 0.f), sb = sa, sc = sa, sd = sa;  // four independent sum chains
-        const float2 negm = make_float2(-m_run, -m_run);
-#pragma unroll
-        for (int i = 0; i < kKeys; i += 8) {
-          uint32_t hh[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 d = add2(make_float2(sv[i + 2 * u], sv[i + 2 * u + 1]), negm);
-            const float2 pp = make_float2(ex2(d.x), ex2(d.y));
-            switch (u) {
-              case 0: sa = add2(sa, pp); break;
-              case 1: sb = add2(sb, pp); break;
-              case 2: sc = add2(sc, pp); break;
-              default: sd = add2(sd, pp); break;
-            }
-            hh[u] = pack_h2(pp.x, pp.y);
-          }
-          tmem_st4(tP + (i >> 1), hh[0], hh[1], hh[2], hh[3]);
-        }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        const float2 s01 = add2(sa, sb), s23 = add2(sc, sd);
-        const float2 s4 = add2(s01, s23);
-        const float sum = s4.x + s4.y;
-        // O row rescaled in place when this row's max was raised (after P, to keep the
-        // score row and the O chunk out of registers at the same time)
-        if (any_need && j > 0) {
-          tc::tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < kDh; c += 32) {
-            float v[32];
-            tc::tmem_ld32(tO + c, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= alpha;
-            tc::tmem_st32(tO + c, v);
-          }
-        }
-        l += sum;
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(p_full + t);
+        const bool go = a.axis == 0
+                            ? softmax_block<kKeys>(tS, tP, tO, min(kKeys, a.n - j * kKeys), m_run, l, j > 0,
+                                                   pv_done + t, (g - 1) & 1, s_free + t, p_full + t, lane, a.status,
+                                                   abort)
+                            : softmax_block<64>(tS + 64 * prob, tP + 32 * prob, tO, a.n, m_run, l, false,
+                                                pv_done + t, 0, s_free + t, p_full + t, lane, a.status, abort);
+        if (!go) { ok = false; break; }
       }
       if (!ok) break;
       // the item's output: O_t / l * gate once the last P*V has completed
@@ -427,17 +470,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(o_free + t);
-      if (tok >= 0) {
-        const float gsc = __half2float(gate) / l;
-        __half *dst = a.o + tok * (long long)a.H * kDh + it.head * kDh;
+      // staged in shared memory (128-byte swizzle: 16-byte chunk c of row i at c ^ (i % 8))
+      // and written by one bulk tensor store per warp; rows outside the output tensor
+      // (frames past T, bands past nb) are not written
+      const float gsc = tok >= 0 ? __half2float(gate) / l : 0.f;
+      uint8_t *stg = smem + AttnSmem::ostage + warp * 4096;
+      if (lane == 0) tc::bulk_wait_read<0>();
+      __syncwarp();
 #pragma unroll
-        for (int d = 0; d < kDh; d += 8) {
-          *reinterpret_cast<uint4 *>(dst + d) =
-              make_uint4(pack_h2(o[d] * gsc, o[d + 1] * gsc), pack_h2(o[d + 2] * gsc, o[d + 3] * gsc),
-                         pack_h2(o[d + 4] * gsc, o[d + 5] * gsc), pack_h2(o[d + 6] * gsc, o[d + 7] * gsc));
+      for (int c = 0; c < 8; ++c) {
+        const float *oc = o + 8 * c;
+        *reinterpret_cast<uint4 *>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+            make_uint4(pack_h2(oc[0] * gsc, oc[1] * gsc), pack_h2(oc[2] * gsc, oc[3] * gsc),
+                       pack_h2(oc[4] * gsc, oc[5] * gsc), pack_h2(oc[6] * gsc, oc[7] * gsc));
+      }
+      tc::fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        // output coordinates (d, head, band, frame within the window, batch)
+        int c2, c3, c4;
+        if (a.axis == 0) {
+          c2 = it.band; c3 = (it.qt0 + t) * kRows + 32 * (warp & 3); c4 = it.b;
+        } else {
+          const int f = it.frame0[t] + ((warp & 3) >> 1);
+          c2 = 32 * (warp & 1); c3 = f % a.T; c4 = f / a.T;
         }
+        tma_store_5d(&to, stg, 0, it.head, c2, c3, c4);
+        tc::bulk_commit();
       }
     }
+    if (lane == 0) tc::bulk_wait_all();
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -492,14 +554,22 @@ bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int
   const unsigned long long str[3] = {(unsigned long long)kDh, (unsigned long long)ld,
                                      (unsigned long long)nb * ld};
   const size_t A = (size_t)H * kDh;
-  CUtensorMap tq, tk, tv;
+  // output [token][head][d] as (d, head, band, frame within the window, batch); a warp
+  // stores 32 rows: 32 frames of one band (time axis) or 32 bands of one frame (band axis)
+  const unsigned long long odims[5] = {(unsigned long long)kDh, (unsigned long long)H, (unsigned long long)nb,
+                                       (unsigned long long)T, (unsigned long long)B};
+  const unsigned long long ostr[4] = {(unsigned long long)kDh, (unsigned long long)A, (unsigned long long)nb * A,
+                                      (unsigned long long)T * nb * A};
+  const unsigned obox[5] = {(unsigned)kDh, 1u, axis == 0 ? 1u : 32u, axis == 0 ? 32u : 1u, 1u};
+  CUtensorMap tq, tk, tv, to;
   if (!make_tmap(&tq, qkv, kTmF16, 4, dims, str, box, 128) ||
       !make_tmap(&tk, qkv + A, kTmF16, 4, dims, str, box, 128) ||
-      !make_tmap(&tv, qkv + 2 * A, kTmF16, 4, dims, str, box, 128))
+      !make_tmap(&tv, qkv + 2 * A, kTmF16, 4, dims, str, box, 128) ||
+      !make_tmap(&to, o, kTmF16, 5, odims, ostr, obox, 128))
     return false;
   const size_t smem = AttnSmem::total + 1024;
   const int grid = (int)std::min<long long>(a.items, g_num_sms > 0 ? g_num_sms : 148);
-  attn_tc_kernel<<<grid, kThreads, smem, st>>>(tq, tk, tv, a);
+  attn_tc_kernel<<<grid, kThreads, smem, st>>>(tq, tk, tv, to, a);
   return true;
 }
 
