@@ -70,8 +70,6 @@ bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, un
                    unsigned long long d2, unsigned long long s1, unsigned long long s2, unsigned box1,
                    unsigned box2);
 
-constexpr int kGemmStages = 4;
-constexpr int kGemmThreads = 320;
 // Resolve the tensor-map encoder and set the kernels' shared-memory limits (call once, outside capture).
 bool gemm_tc_init();
 

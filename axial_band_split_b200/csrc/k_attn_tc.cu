@@ -76,11 +76,15 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 
 // packed pair add (one f32x2 instruction)
 __device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  unsigned long long x = (static_cast<unsigned long long>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
-  unsigned long long y = (static_cast<unsigned long long>(__float_as_uint(b.y)) << 32) | __float_as_uint(b.x);
-  unsigned long long z;
-  asm("add.f32x2 %0, %1, %2;" : "=l"(z) : "l"(x), "l"(y));
-  return make_float2(__uint_as_float(static_cast<unsigned>(z)), __uint_as_float(static_cast<unsigned>(z >> 32)));
+  float2 r;
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "add.f32x2 rc, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rc;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
 }
 
 // Consecutive fp32 columns of this thread's TMEM lane.  The wait takes the destination

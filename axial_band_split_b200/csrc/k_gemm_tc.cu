@@ -9,12 +9,12 @@
 // "@audio/neural-separate 0.4.0 → 0.5.0", package/scripts/export-roformer.py, class Core
 // (norm scale folded into the next weight, gates joined to q/k/v, bands batched).
 //
-// CTA layout (320 threads, one CTA per SM):
-//   warps 0-7  epilogue: tcgen05.ld of the 128 x BN accumulator, fused epilogue, stores
-//              (two warps per TMEM lane quarter, alternating 32-column chunks)
-//   warp 8     TMA producer (one lane) and TMEM allocator
-//   warp 9     MMA issuer (one lane): 4 x tcgen05.mma (M=128, N<=256, K=16) per 64-wide K block
-// Shared memory: kGemmStages stages of A (128 x 64) and B (BN x 64) tiles, 128-byte swizzle,
+// CTA layout (one CTA per SM; E = 8 or 16 epilogue warps by epilogue kind):
+//   warps 0..E-1  epilogue: tcgen05.ld of the 128 x BN accumulator, fused epilogue, stores
+//                 (E / 4 warps per TMEM lane quarter, taking turns over 32-column chunks)
+//   warp E        TMA producer (one lane) and TMEM allocator
+//   warp E+1      MMA issuer (one lane): 4 x tcgen05.mma (M=128, N<=256, K=16) per 64-wide K block
+// Shared memory: gemm_stages(EPI) stages of A (128 x 64) and B (BN x 64) tiles, 128-byte swizzle,
 // then per-epilogue-warp output boxes.  Tensor memory: two 256-column fp32 accumulators, so
 // the epilogue of tile i overlaps the main loop of tile i+1.
 //
@@ -38,7 +38,14 @@ constexpr int BM = 128, BK = 64;
 constexpr int A_STAGE = BM * BK * 2;        // 16 KB
 constexpr int TMEM_COLS = 512;
 constexpr float kEps = 1e-12f;
-constexpr int kEpiWarps = 8;
+// Epilogue warps per kind: 16 (four per 32-lane quarter of the tile) where the epilogue's
+// arithmetic is the bottleneck and fits 96 registers a thread (the register file of an SM
+// sub-partition then holds five warps): GELU and the band split; 8 elsewhere, where the
+// main loop wants four pipeline stages and the epilogue the 168 registers of a 10-warp
+// CTA.  Pipeline stages fill what shared memory the epilogue staging leaves.
+__host__ __device__ constexpr int epi_warps(int epi) { return (epi == kTcGelu || epi == kTcBandSplit) ? 16 : 8; }
+__host__ __device__ constexpr int gemm_stages(int epi) { return epi_warps(epi) == 8 ? 4 : 3; }
+__host__ __device__ constexpr int gemm_threads(int epi) { return 32 * (epi_warps(epi) + 2); }
 
 // Widest B tile of an epilogue kind, and the shared memory each epilogue warp needs.
 __host__ __device__ constexpr int bn_max(int epi) { return (epi == kTcResid || epi == kTcBandSplit) ? 192 : 256; }
@@ -51,9 +58,9 @@ template <int EPI>
 struct SmemLayout {
   static constexpr int b_stage = bn_max(EPI) * BK * 2;
   static constexpr int a_off = 0;
-  static constexpr int b_off = kGemmStages * A_STAGE;
-  static constexpr int stg_off = b_off + kGemmStages * b_stage;             // 1024-aligned
-  static constexpr int bar_off = stg_off + kEpiWarps * warp_stage_bytes(EPI);
+  static constexpr int b_off = gemm_stages(EPI) * A_STAGE;
+  static constexpr int stg_off = b_off + gemm_stages(EPI) * b_stage;        // 1024-aligned
+  static constexpr int bar_off = stg_off + epi_warps(EPI) * warp_stage_bytes(EPI);
   static constexpr int total = bar_off + 256;
 };
 
@@ -89,28 +96,8 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams &p, int tile) {
 }
 
 // ------------------------------------------------------------------ epilogue helpers
-__device__ __forceinline__ float row_scale(const GemmParams &p, long long row) {
-  if (!p.ss_in) return 1.f;
-  return 1.f / fmaxf(sqrtf(p.ss_in[row]), kEps);
-}
 
-// erf by Abramowitz & Stegun 7.1.26 (|error| <= 1.5e-7), branch-free:
-// erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2), t = 1 / (1 + p z), z >= 0.
-__device__ __forceinline__ float erf_as(float x) {
-  const float z = fabsf(x);
-  float t;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, z, 1.f)));
-  float poly = fmaf(t, 1.061405429f, -1.453152027f);
-  poly = fmaf(t, poly, 1.421413741f);
-  poly = fmaf(t, poly, -0.284496736f);
-  poly = fmaf(t, poly, 0.254829592f);
-  poly *= t;
-  float e;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-z * z * 1.4426950408889634f));
-  return copysignf(fmaf(-poly, e, 1.f), x);
-}
 
-__device__ __forceinline__ float gelu_(float x) { return 0.5f * x * (1.f + erf_as(x * 0.70710678118654752f)); }
 
 // Packed pairs (one f32x2 instruction for two lanes of math).
 __device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
@@ -130,8 +117,10 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigne
   return d;
 }
 
-// GELU of y0 = v0 * rs + b0 and y1 = v1 * rs + b1 with the erf of Abramowitz & Stegun
-// 7.1.26 (as erf_as), the polynomial and the scalings in packed pairs.
+// GELU of y0 = v0 * rs + b0 and y1 = v1 * rs + b1, y * (1 + erf(y / sqrt 2)) / 2, with the
+// erf of Abramowitz & Stegun 7.1.26 (|error| <= 1.5e-7), branch-free:
+// erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2), t = 1 / (1 + p z), z >= 0;
+// the polynomial and the scalings in packed pairs.
 __device__ __forceinline__ float2 gelu2(float v0, float v1, float rs, float b0, float b1) {
   const unsigned long long y = fma2(f2_pack(v0, v1), f2_pack(rs, rs), f2_pack(b0, b1));
   const float2 yy = f2_unpack(y);
@@ -194,23 +183,17 @@ __device__ __forceinline__ long long token_of(const GemmParams &p, int m, int g)
 }
 
 struct QkvRow {
-  long long tok, seq;
+  long long tok;
   int pos;
 };
 
+// A QKV row's token and its rotary position: the frame within the window (time axis) or
+// the band (band axis).  Tokens fit 32 bits (the handle limits B * T * bands).
 __device__ __forceinline__ QkvRow qkv_row(const GemmParams &p, int m, int g) {
   QkvRow r;
   r.tok = token_of(p, m, g);
-  const int band = (int)(r.tok % p.nb);
-  const long long bt = r.tok / p.nb;
-  if (p.axis == 0) {
-    const int b = (int)(bt / p.T);
-    r.pos = (int)(bt % p.T);
-    r.seq = (long long)b * p.nb + band;
-  } else {
-    r.seq = bt;
-    r.pos = band;
-  }
+  const unsigned tok = (unsigned)r.tok, bt = tok / (unsigned)p.nb;
+  r.pos = p.axis == 0 ? (int)(bt % (unsigned)p.T) : (int)(tok - bt * (unsigned)p.nb);
   return r;
 }
 
@@ -225,11 +208,12 @@ __device__ __forceinline__ void load_bias32(const float *b, float *bv) {
 
 // ------------------------------------------------------------------ the kernel
 template <int EPI>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads(EPI), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                    const GemmParams p) {
   using L = SmemLayout<EPI>;
+  constexpr int kEpiWarps = epi_warps(EPI), kSplit = kEpiWarps / 4, kGemmStages = gemm_stages(EPI);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem + L::a_off;
@@ -326,10 +310,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ---------------- epilogue warps 0-7
-    const int quarter = warp & 3, half = warp >> 2;
+    const int quarter = warp & 3, sub = warp >> 2;  // rows 32 quarter.., chunks sub, sub + kSplit, ...
     uint8_t *stg = smem + L::stg_off + warp * warp_stage_bytes(EPI);
     int nstore = 0;  // boxes this warp has stored (double-buffer parity)
     int local = 0;
+    // The row's deferred-norm sum of squares (and, for QKV, its rotary (cos, sin) pairs),
+    // fetched one tile ahead so the loads' latency hides under the previous tile's
+    // epilogue: nothing reads them before the next tile.
+    float ss_pf = 1.f;
+    QkvRow qr_pf{0, 0};
+    float2 cs_pf[16];
+    auto row_fetch = [&](int tile_) {
+      if (tile_ >= total) return;
+      const TileInfo t_ = decode_tile(p, tile_);
+      const int m_ = t_.mb * BM + quarter * 32 + lane;
+      const bool v_ = m_ < p.M;
+      if (EPI == kTcQkv) {
+        qr_pf = qkv_row(p, v_ ? m_ : 0, t_.g);
+        ss_pf = (v_ && p.ss_in) ? p.ss_in[qr_pf.tok] : 1.f;
+        if (p.dh == 64) {
+          const float2 *rp = p.rope + (long long)qr_pf.pos * 32 + (sub & 1) * 16;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) cs_pf[i] = rp[i];
+        }
+      } else if (EPI == kTcGelu) {
+        ss_pf = (v_ && p.ss_in) ? p.ss_in[m_] : 1.f;
+      } else if (EPI == kTcTanh) {
+        ss_pf = (v_ && p.ss_in) ? p.ss_in[token_of(p, m_, t_.g)] : 1.f;
+      } else if (EPI == kTcResid) {
+        ss_pf = (v_ && p.res_ss) ? p.res_ss[m_] : 1.f;
+      }
+    };
+    row_fetch(blockIdx.x);
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       const TileInfo ti = decode_tile(p, tile);
       const GemmGroup &gr = p.groups[ti.g];
@@ -344,26 +356,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * 256;
       // ---- work that does not need the accumulator, before waiting for it
       float rs = 1.f;
-      QkvRow qr{0, 0, 0};
+      QkvRow qr{0, 0};
       float2 cs[16];
+      // 1 / |x| of the row (deferred norm: of the GEMM input, or of the residual for kTcResid)
+      const float rsq = 1.f / fmaxf(sqrtf(ss_pf), kEps);
       if (EPI == kTcQkv) {
-        qr = qkv_row(p, valid ? m : 0, ti.g);
-        if (valid) rs = row_scale(p, qr.tok);
-        if (p.dh == 64) {
-          const float2 *rp = p.rope + (long long)qr.pos * 32 + half * 16;
+        qr = qr_pf;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) cs[i] = rp[i];
-        }
-      } else if (EPI == kTcGelu) {
-        if (valid) rs = row_scale(p, m);
-      } else if (EPI == kTcTanh) {
-        if (valid && p.ss_in) rs = row_scale(p, token_of(p, m, ti.g));
+        for (int i = 0; i < 16; ++i) cs[i] = cs_pf[i];
       }
-      float res_s = 1.f;  // deferred norm of the residual input (kTcResid)
-      if (EPI == kTcResid && p.res_ss && valid) res_s = 1.f / fmaxf(sqrtf(p.res_ss[m]), kEps);
+      if (EPI == kTcQkv || EPI == kTcGelu || EPI == kTcTanh) rs = rsq;
+      const float res_s = rsq;  // kTcResid
+      row_fetch(tile + gridDim.x);
       // residual prefetch (kTcResid): lane covers rows i*4 + lane/8, 16-byte piece lane%8
       uint4 pre[8];
-      int c = half;
+      int c = sub;
       if (EPI == kTcResid && c < nchunks) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -376,7 +383,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!tc::mbar_wait(tfull + acc, aphase, p.status, 14, abort)) break;
       tc::tc_fence_after();
       float sq = 0.f, sqg = 0.f;
-      for (; c < nchunks; c += 2) {
+      for (; c < nchunks; c += kSplit) {
         const int c0 = nbase + 32 * c;
         const bool full_chunk = c0 + 32 <= gr.N;
         float v[32];
@@ -401,12 +408,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
               for (int j = 0; j < 32; ++j) x[j] *= res_s * gv[j];
             }
-            if (c + 2 < nchunks) {
+            if (c + kSplit < nchunks) {
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
                 const int r = i * 4 + (lane >> 3);
                 pre[i] = (m0w + r < p.M)
-                             ? *reinterpret_cast<const uint4 *>(p.X + (long long)(m0w + r) * p.ld + c0 + 64 + (lane & 7) * 4)
+                             ? *reinterpret_cast<const uint4 *>(p.X + (long long)(m0w + r) * p.ld + c0 + 32 * kSplit + (lane & 7) * 4)
                              : make_uint4(0, 0, 0, 0);
               }
             }
@@ -563,9 +570,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (EPI == kTcResid && valid && p.ss_out && half < nchunks) atomicAdd(p.ss_out + m, sq);
-      if (EPI == kTcResid && valid && p.ssg_out && half < nchunks) atomicAdd(p.ssg_out + m, sqg);
-      if (EPI == kTcBandSplit && valid && half < nchunks) atomicAdd(p.ss_out + (long long)m * p.nb + ti.g, sq);
+      if (EPI == kTcResid && valid && p.ss_out && sub < nchunks) atomicAdd(p.ss_out + m, sq);
+      if (EPI == kTcResid && valid && p.ssg_out && sub < nchunks) atomicAdd(p.ssg_out + m, sqg);
+      if (EPI == kTcBandSplit && valid && sub < nchunks) atomicAdd(p.ss_out + (long long)m * p.nb + ti.g, sq);
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tempty + acc);
@@ -647,7 +654,7 @@ void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, con
   switch (epi) {
 #define MRF_GEMM_CASE(E)                                                                  \
   case E:                                                                                 \
-    gemm_tc_kernel<E><<<grid, kGemmThreads, smem_bytes<E>(), st>>>(tmA, tmB, tmC, tmD, p); \
+    gemm_tc_kernel<E><<<grid, gemm_threads(E), smem_bytes<E>(), st>>>(tmA, tmB, tmC, tmD, p); \
     break;
     MRF_GEMM_CASE(kTcQkv)
     MRF_GEMM_CASE(kTcResid)
