@@ -39,8 +39,11 @@ namespace mrf {
 namespace {
 
 constexpr int kDh = 64, kRows = 128, kKeys = 128;
-// K/V ring: 10 tiles of 16 KB.  Time axis: one K and one V tile per stage, shared by both
-// query tiles (5 stages); band axis: a K and a V tile per query tile (2 stages).
+// K/V ring: 10 tiles of 16 KB, filled block by block in order.  A key block takes one K and
+// one V tile when both query tiles share the keys (two tiles of one time-axis sequence) and
+// a K and a V tile per query tile otherwise (band axis; time-axis items that pair the odd
+// last tiles of two sequences).  At most kMaxStages blocks are in flight, each with its own
+// full/empty barrier pair.
 constexpr int kRingTiles = 10, kMaxStages = 5;
 static_assert(kKeys == 128, "the softmax reads a score row as two 64-column halves");
 constexpr int kTile = kRows * kDh * 2;  // 16 KB: one 128 x 64 fp16 tile
@@ -158,37 +161,54 @@ struct AttnArgs {
   __half *o;
   unsigned *status;
   int B, T, nb, H, axis, ld, n, q_tiles, pairs, items, n_blocks, BT;
+  int S, shared_items;  // time axis: sequences (b, band, head); items pairing two tiles of one sequence
 };
 
-// Tensor-map coordinates (d, head, band, frame) of an item's two query tiles; key blocks
-// add j*128 frames on the time axis.  Time axis: the tiles are frames frame0[t] .. +127 of
-// one (band, head) sequence.  Band axis: tile t covers frames frame0[t] and frame0[t] + 1,
-// bands 0..63 of each (bands past nb read as zeros).
-struct Item {
-  int head, band, qt0, b;
-  int frame0[2];
+// Query tile t of an item.  Tensor-map coordinates (d, head, band, frame): the tile's
+// queries start at frame frame0 of (head, band) and its key block j at frame kv0 + j * 128.
+// Time axis: a tile is 128 frames of one (band, head) sequence; an item holds either two
+// consecutive tiles of one sequence (shared keys) or the odd last tiles of two sequences
+// (mixed: separate keys; with an odd sequence count the last item's tile 1 is idle).
+// Band axis: tile t covers frames frame0 and frame0 + 1, bands 0..63 of each (bands past
+// nb read as zeros), with its own keys.
+struct TileC {
+  int head, band, b, qt, frame0, kv0;
+  bool valid;
 };
 
-__device__ __forceinline__ Item item_coords(const AttnArgs &a, int item) {
-  Item it;
+__device__ __forceinline__ bool item_mixed(const AttnArgs &a, int item) {
+  return a.axis != 0 || item >= a.shared_items;
+}
+
+__device__ __forceinline__ TileC tile_coords(const AttnArgs &a, int item, int t) {
+  TileC c;
   if (a.axis == 0) {
-    const int sh = item / a.pairs;       // ((b * nb) + band) * H + head
-    it.qt0 = 2 * (item % a.pairs);
-    it.head = sh % a.H;
-    const int seq = sh / a.H;
-    it.band = seq % a.nb;
-    const int b = seq / a.nb;
-    it.b = b;
-    for (int t = 0; t < 2; ++t) it.frame0[t] = b * a.T + (it.qt0 + t) * kRows;
+    int seq, qt;
+    c.valid = true;
+    if (item < a.shared_items) {
+      seq = item / a.pairs;  // ((b * nb) + band) * H + head
+      qt = 2 * (item % a.pairs) + t;
+    } else {
+      seq = 2 * (item - a.shared_items) + t;
+      if (seq >= a.S) { seq = a.S - 1; c.valid = false; }
+      qt = a.q_tiles - 1;
+    }
+    c.head = seq % a.H;
+    const int bb = seq / a.H;
+    c.band = bb % a.nb;
+    c.b = bb / a.nb;
+    c.qt = qt;
+    c.kv0 = c.b * a.T;
+    c.frame0 = c.kv0 + qt * kRows;
   } else {
-    it.head = item % a.H;
-    it.band = 0;
-    it.b = 0;
-    it.qt0 = 0;
-    const int f = 4 * (item / a.H);
-    for (int t = 0; t < 2; ++t) it.frame0[t] = f + 2 * t;
+    c.head = item % a.H;
+    c.band = 0;
+    c.b = 0;
+    c.qt = 0;
+    c.frame0 = c.kv0 = 4 * (item / a.H) + 2 * t;
+    c.valid = true;
   }
-  return it;
+  return c;
 }
 
 // One key block of one query row: scores from tensor memory (log2 units: q was scaled by
@@ -293,13 +313,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool shared_kv = a.axis == 0;
-  const int stage_tiles = shared_kv ? 2 : 4, n_stages = kRingTiles / stage_tiles;
+
   if (threadIdx.x == 0) {
     abort_flag = 0;
     tc::mbar_init(q_full, 1);
     tc::mbar_init(q_empty, 1);
-    for (int s = 0; s < n_stages; ++s) { tc::mbar_init(kv_full + s, 1); tc::mbar_init(kv_empty + s, 1); }
+    for (int s = 0; s < kMaxStages; ++s) { tc::mbar_init(kv_full + s, 1); tc::mbar_init(kv_empty + s, 1); }
     for (int t = 0; t < 2; ++t) {
       tc::mbar_init(s_full + t, 1);
       tc::mbar_init(s_free + t, 4);
@@ -321,26 +340,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8) {
     // ---------------- TMA producer
     if (lane == 0) {
-      const uint32_t kv_bytes = (shared_kv ? 2 : 4) * kTile;
-      int g = 0;  // key blocks loaded so far
+      int g = 0;              // key blocks loaded so far
+      int oldest = 0;         // oldest block whose ring tiles are not known to be free
+      int used = 0;           // ring tiles held by blocks oldest .. g - 1
+      int ptr = 0;            // next ring tile
+      int held[kMaxStages];   // ring tiles of the block in each slot
       int li = 0;
       bool ok = true;
       for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
-        const Item it = item_coords(a, item);
+        const TileC c0 = tile_coords(a, item, 0), c1 = tile_coords(a, item, 1);
+        const bool mixed = item_mixed(a, item);
         if (!tc::mbar_wait(q_empty, (li & 1) ^ 1, a.status, 30, abort)) break;
         tc::mbar_arrive_expect_tx(q_full, 2 * kTile);
-        for (int t = 0; t < 2; ++t)
-          tc::tma_load_4d(smem + AttnSmem::q + t * kTile, &tq, q_full, 0, it.head, it.band, it.frame0[t]);
+        tc::tma_load_4d(smem + AttnSmem::q, &tq, q_full, 0, c0.head, c0.band, c0.frame0);
+        tc::tma_load_4d(smem + AttnSmem::q + kTile, &tq, q_full, 0, c1.head, c1.band, c1.frame0);
+        const int need = mixed ? 4 : 2;
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
-          const int s = g % n_stages;
-          if (!tc::mbar_wait(kv_empty + s, ((g / n_stages) & 1) ^ 1, a.status, 31, abort)) { ok = false; break; }
-          tc::mbar_arrive_expect_tx(kv_full + s, kv_bytes);
-          for (int t = 0; t < (shared_kv ? 1 : 2); ++t) {
-            const int f = shared_kv ? it.frame0[0] - it.qt0 * kRows + j * kKeys : it.frame0[t];
-            uint8_t *dst = smem + AttnSmem::kv + (s * stage_tiles + 2 * t) * kTile;
-            tc::tma_load_4d(dst, &tk, kv_full + s, 0, it.head, it.band, f);
-            tc::tma_load_4d(dst + kTile, &tv, kv_full + s, 0, it.head, it.band, f);
+          // a free slot and `need` free ring tiles: release the oldest blocks in order
+          while (ok && (g - oldest >= kMaxStages || used + need > kRingTiles)) {
+            const int so = oldest % kMaxStages;
+            if (!tc::mbar_wait(kv_empty + so, (oldest / kMaxStages) & 1, a.status, 31, abort)) ok = false;
+            used -= held[so];
+            ++oldest;
           }
+          if (!ok) break;
+          const int s = g % kMaxStages;
+          held[s] = need;
+          tc::mbar_arrive_expect_tx(kv_full + s, need * kTile);
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (t == 1 && !mixed) break;
+            const TileC &c = t == 0 ? c0 : c1;
+            const int f = c.kv0 + j * kKeys;
+            tc::tma_load_4d(smem + AttnSmem::kv + ((ptr + 2 * t) % kRingTiles) * kTile, &tk, kv_full + s, 0,
+                            c.head, c.band, f);
+            tc::tma_load_4d(smem + AttnSmem::kv + ((ptr + 2 * t + 1) % kRingTiles) * kTile, &tv, kv_full + s, 0,
+                            c.head, c.band, f);
+          }
+          ptr = (ptr + need) % kRingTiles;
+          used += need;
         }
       }
     }
@@ -349,20 +387,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_s = tc::idesc_f16(kRows, kKeys);
       const uint32_t id_pv = tc::idesc_f16(kRows, kDh, true);
-      int g = 0;
+      int g = 0;    // key blocks consumed so far
+      int ptr = 0;  // ring tile of the next item's first block (the producer's order)
       int li = 0;
       bool ok = true;
-      auto issue_s = [&](int t, int s) {
+      bool mixed = false;
+      // block at ring tile `base`: tile t's K at base (+ 2 t when the tiles have separate
+      // keys), its V one tile further
+      auto kv_tile = [&](int base, int t, int which) {
+        return smem + AttnSmem::kv + ((base + (mixed ? 2 * t : 0) + which) % kRingTiles) * kTile;
+      };
+      auto issue_s = [&](int t, int base) {
         const uint32_t q_addr = tc::smem_u32(smem + AttnSmem::q + t * kTile);
-        const uint32_t k_addr = tc::smem_u32(smem + AttnSmem::kv + (s * stage_tiles + (shared_kv ? 0 : 2 * t)) * kTile);
+        const uint32_t k_addr = tc::smem_u32(kv_tile(base, t, 0));
 #pragma unroll
         for (int kk = 0; kk < kDh / 16; ++kk)
           tc::mma_f16(tmem + 128 * t, tc::sw128_kmajor_desc(q_addr + kk * 32), tc::sw128_kmajor_desc(k_addr + kk * 32),
                       id_s, kk != 0);
         tc::mma_commit(s_full + t);
       };
-      auto issue_pv = [&](int t, int s, bool acc) {
-        const uint32_t v_addr = tc::smem_u32(smem + AttnSmem::kv + (s * stage_tiles + (shared_kv ? 0 : 2 * t) + 1) * kTile);
+      auto issue_pv = [&](int t, int base, bool acc) {
+        const uint32_t v_addr = tc::smem_u32(kv_tile(base, t, 1));
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
           mma_f16_ts(tmem + 256 + 64 * t, tmem + 384 + 64 * t + 8 * kk, tc::sw128_mnmajor_desc(v_addr + kk * 2048),
@@ -373,29 +418,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       // registers then hold the scores), so the next scores compute under this block's
       // exponentials; P(t)*V follows once P(t) is in tensor memory.
       for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
+        mixed = item_mixed(a, item);
+        const int need = mixed ? 4 : 2;
         if (!tc::mbar_wait(q_full, li & 1, a.status, 32, abort)) break;
-        int s = g % n_stages;
-        if (!tc::mbar_wait(kv_full + s, (g / n_stages) & 1, a.status, 33, abort)) break;
+        if (!tc::mbar_wait(kv_full + g % kMaxStages, (g / kMaxStages) & 1, a.status, 33, abort)) break;
         for (int t = 0; t < 2 && ok; ++t) {
           if (g > 0 && !tc::mbar_wait(s_free + t, (g - 1) & 1, a.status, 41, abort)) ok = false;
           tc::tc_fence_after();
-          if (ok) issue_s(t, s);
+          if (ok) issue_s(t, ptr);
         }
         if (!ok) break;
         // q is read only by S = q k^T: release its buffer once the item's last S is issued,
         // so the next item's q loads under this item's softmax and P v
         if (a.n_blocks == 1) tc::mma_commit(q_empty);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
-          s = g % n_stages;
+          const int base = (ptr + j * need) % kRingTiles;
           // both tiles' next scores first: each waits only for its softmax to have read S,
           // so they compute under this block's exponentials
           if (j + 1 < a.n_blocks) {
-            const int s1 = (g + 1) % n_stages;
-            if (!tc::mbar_wait(kv_full + s1, ((g + 1) / n_stages) & 1, a.status, 36, abort)) { ok = false; break; }
+            if (!tc::mbar_wait(kv_full + (g + 1) % kMaxStages, ((g + 1) / kMaxStages) & 1, a.status, 36, abort)) {
+              ok = false;
+              break;
+            }
             for (int t = 0; t < 2 && ok; ++t) {
               if (!tc::mbar_wait(s_free + t, g & 1, a.status, 41, abort)) { ok = false; break; }
               tc::tc_fence_after();
-              issue_s(t, s1);
+              issue_s(t, (base + need) % kRingTiles);
             }
             if (!ok) break;
             if (j + 2 == a.n_blocks) tc::mma_commit(q_empty);
@@ -404,11 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!tc::mbar_wait(p_full + t, g & 1, a.status, 34, abort)) { ok = false; break; }
             if (j == 0 && !tc::mbar_wait(o_free + t, (li & 1) ^ 1, a.status, 35, abort)) { ok = false; break; }
             tc::tc_fence_after();
-            issue_pv(t, s, j != 0);
+            issue_pv(t, base, j != 0);
           }
           if (!ok) break;
-          tc::mma_commit(kv_empty + s);
+          tc::mma_commit(kv_empty + g % kMaxStages);
         }
+        ptr = (ptr + a.n_blocks * need) % kRingTiles;
       }
       tc::mma_commit(done);
       tc::mbar_wait(done, 0, a.status, 37, abort);
@@ -436,13 +485,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_run = -INFINITY, l = 0.f;
       // this row's output token and its head's gate, fetched now so the load's latency is
       // hidden under the item's key blocks
-      const Item it = item_coords(a, item);
+      const TileC it = tile_coords(a, item, t);
       long long tok = -1;
       if (a.axis == 0) {
-        const int pos = (it.qt0 + t) * kRows + r;
-        if (pos < a.n) tok = (long long)(it.frame0[t] + r) * a.nb + it.band;
+        const int pos = it.qt * kRows + r;
+        if (it.valid && pos < a.n) tok = (long long)(it.frame0 + r) * a.nb + it.band;
       } else {
-        const int f = it.frame0[t] + prob, k = r & 63;
+        const int f = it.frame0 + prob, k = r & 63;
         if (k < a.n && f < a.BT) tok = (long long)f * a.nb + k;
       }
       const __half gate = tok >= 0 ? a.qkv[tok * a.ld + 3 * a.H * kDh + it.head] : __float2half(0.f);
@@ -490,13 +539,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::fence_proxy_async();
       __syncwarp();
-      if (lane == 0) {
+      if (lane == 0 && it.valid) {
         // output coordinates (d, head, band, frame within the window, batch)
         int c2, c3, c4;
         if (a.axis == 0) {
-          c2 = it.band; c3 = (it.qt0 + t) * kRows + 32 * (warp & 3); c4 = it.b;
+          c2 = it.band; c3 = it.qt * kRows + 32 * (warp & 3); c4 = it.b;
         } else {
-          const int f = it.frame0[t] + ((warp & 3) >> 1);
+          const int f = it.frame0 + ((warp & 3) >> 1);
           c2 = 32 * (warp & 1); c3 = f % a.T; c4 = f / a.T;
         }
         tma_store_5d(&to, stg, 0, it.head, c2, c3, c4);
@@ -541,13 +590,19 @@ bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int
   a.q_tiles = (a.n + kRows - 1) / kRows;
   unsigned box[4];
   if (axis == 0) {
-    a.pairs = (a.q_tiles + 1) / 2;
-    a.items = B * nb * H * a.pairs;
+    // pairs of consecutive tiles of one sequence; an odd last tile pairs with the next
+    // sequence's (separate keys)
+    a.S = B * nb * H;
+    a.pairs = a.q_tiles / 2;
+    a.shared_items = a.S * a.pairs;
+    a.items = a.shared_items + ((a.q_tiles & 1) ? (a.S + 1) / 2 : 0);
     a.n_blocks = (a.n + kKeys - 1) / kKeys;
     box[0] = kDh; box[1] = 1; box[2] = 1; box[3] = kRows;      // 128 frames of one (band, head)
   } else {
     if (nb > 64) return false;
     a.pairs = 0;
+    a.S = 0;
+    a.shared_items = 0;
     a.items = H * ((a.BT + 3) / 4);
     a.n_blocks = 1;
     box[0] = kDh; box[1] = 1; box[2] = 64; box[3] = 2;         // bands 0..63 of two frames

@@ -83,3 +83,23 @@ def test_vocals_full_depth_T300():
     W, x = case(cfg, B, T, True)
     got, _ = run(cfg, B, T, W, x)
     check(got, oracle_masks(cfg, B, T, True), "masks")
+
+
+def test_time_axis_odd_last_tiles_batch2():
+    # T=260: three 128-frame query tiles per sequence; the odd last tiles of two sequences
+    # share an item with separate keys, across both batch elements
+    cfg = dataclasses.replace(synth.VOCALS, depth=1)
+    B, T = 2, 260
+    W, x = case(cfg, B, T, True)
+    got, _ = run(cfg, B, T, W, x)
+    check(got, oracle_masks(cfg, B, T, True), "masks")
+
+
+def test_time_axis_odd_sequence_count():
+    # 7 bands x 1 head of width 64: an odd number of sequences, so the last item's second
+    # query tile has no sequence and must leave the output untouched
+    cfg = dataclasses.replace(synth.TINY, num_bands=7, heads=1, dim_head=64)
+    B, T = 1, 300
+    W, x = case(cfg, B, T, True)
+    got, _ = run(cfg, B, T, W, x)
+    check(got, oracle_masks(cfg, B, T, True), "masks")
