@@ -20,7 +20,7 @@
 //               block-diagonally.
 // Warps 0-3 and 4-7: softmax of tile 0 and tile 1 (one query row per thread, the row's
 // live scores in registers: 128 on the time axis, the row's own 64-key half on the band
-// axis); warp 8: TMA; warp 9: MMA issue; warps 10-11 idle.  The third warpgroup gives
+// axis); warp 8: TMA; warps 9 and 10: MMA issue for tile 0 and tile 1; warp 11 idle.  The third warpgroup gives
 // registers up to the two softmax warpgroups (setmaxnreg).
 // Tensor memory (512 columns): S_t at 128 t, O_t at 256 + 64 t, and P_t (the softmax's
 // fp16 probabilities, two per 32-bit column) at 384 + 64 t, which the P*V MMA reads as its
@@ -161,7 +161,7 @@ struct AttnArgs {
   __half *o;
   unsigned *status;
   int B, T, nb, H, axis, ld, n, q_tiles, pairs, items, n_blocks, BT;
-  int S, shared_items;  // time axis: sequences (b, band, head); items pairing two tiles of one sequence
+  int S;  // time axis: sequences (b, band, head)
 };
 
 // Query tile t of an item.  Tensor-map coordinates (d, head, band, frame): the tile's
@@ -176,20 +176,44 @@ struct TileC {
   bool valid;
 };
 
+// Time-axis items come in groups of two sequences 2k, 2k + 1 (sequence index
+// ((b * nb) + band) * H + head): the pairs of sequence 2k, those of 2k + 1, then (odd tile
+// count) the item of their two last tiles, so all items reading a sequence's keys run close
+// together and find them in L2.  With an odd sequence count the last group has one sequence.
+struct ItemPos {
+  int seq, pair;  // shared: sequence and pair index; mixed: first sequence, pair = -1
+};
+
+__device__ __forceinline__ ItemPos item_pos(const AttnArgs &a, int item) {
+  const int gs = 2 * a.pairs + (a.q_tiles & 1);
+  const int grp = item / gs, r = item - grp * gs;
+  const int n_seq = 2 * grp + 1 < a.S ? 2 : 1;
+  ItemPos ip;
+  if (r < n_seq * a.pairs) {
+    ip.seq = 2 * grp + r / a.pairs;
+    ip.pair = r % a.pairs;
+  } else {
+    ip.seq = 2 * grp;
+    ip.pair = -1;
+  }
+  return ip;
+}
+
 __device__ __forceinline__ bool item_mixed(const AttnArgs &a, int item) {
-  return a.axis != 0 || item >= a.shared_items;
+  return a.axis != 0 || item_pos(a, item).pair < 0;
 }
 
 __device__ __forceinline__ TileC tile_coords(const AttnArgs &a, int item, int t) {
   TileC c;
   if (a.axis == 0) {
+    const ItemPos ip = item_pos(a, item);
     int seq, qt;
     c.valid = true;
-    if (item < a.shared_items) {
-      seq = item / a.pairs;  // ((b * nb) + band) * H + head
-      qt = 2 * (item % a.pairs) + t;
+    if (ip.pair >= 0) {
+      seq = ip.seq;
+      qt = 2 * ip.pair + t;
     } else {
-      seq = 2 * (item - a.shared_items) + t;
+      seq = ip.seq + t;
       if (seq >= a.S) { seq = a.S - 1; c.valid = false; }
       qt = a.q_tiles - 1;
     }
@@ -317,8 +341,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     tc::mbar_init(q_full, 1);
-    tc::mbar_init(q_empty, 1);
-    for (int s = 0; s < kMaxStages; ++s) { tc::mbar_init(kv_full + s, 1); tc::mbar_init(kv_empty + s, 1); }
+    tc::mbar_init(q_empty, 2);  // released by both tiles' MMA issuers
+    for (int s = 0; s < kMaxStages; ++s) { tc::mbar_init(kv_full + s, 1); tc::mbar_init(kv_empty + s, 2); }
     for (int t = 0; t < 2; ++t) {
       tc::mbar_init(s_full + t, 1);
       tc::mbar_init(s_free + t, 4);
@@ -326,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(pv_done + t, 1);
       tc::mbar_init(o_free + t, 4);
     }
-    tc::mbar_init(done, 1);
+    tc::mbar_init(done, 2);
     tc::fence_barrier_init();
   }
   if (warp == 8) tc::tmem_alloc(tmem_slot, 512);
@@ -382,8 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 9) {
-    // ---------------- MMA issuer
+  } else if (warp == 9 || warp == 10) {
+    // ---------------- MMA issuers: warp 9 + t issues tile t's MMAs, so neither tile's S or
+    // P*V waits behind the other tile's softmax (the tensor core queues both streams)
+    const int t = warp - 9;
     if (lane == 0) {
       const uint32_t id_s = tc::idesc_f16(kRows, kKeys);
       const uint32_t id_pv = tc::idesc_f16(kRows, kDh, true);
@@ -416,45 +442,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       // S(t) of a block is issued once the softmax has read S(t) of the block before (its
       // registers then hold the scores), so the next scores compute under this block's
-      // exponentials; P(t)*V follows once P(t) is in tensor memory.
+      // exponentials; P(t)*V follows once P(t) is in tensor memory.  A K/V block and the q
+      // buffer are released when both issuers have committed their last read of them.
       for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
         mixed = item_mixed(a, item);
         const int need = mixed ? 4 : 2;
         if (!tc::mbar_wait(q_full, li & 1, a.status, 32, abort)) break;
         if (!tc::mbar_wait(kv_full + g % kMaxStages, (g / kMaxStages) & 1, a.status, 33, abort)) break;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (g > 0 && !tc::mbar_wait(s_free + t, (g - 1) & 1, a.status, 41, abort)) ok = false;
-          tc::tc_fence_after();
-          if (ok) issue_s(t, ptr);
-        }
-        if (!ok) break;
-        // q is read only by S = q k^T: release its buffer once the item's last S is issued,
-        // so the next item's q loads under this item's softmax and P v
+        if (g > 0 && !tc::mbar_wait(s_free + t, (g - 1) & 1, a.status, 41, abort)) break;
+        tc::tc_fence_after();
+        issue_s(t, ptr);
         if (a.n_blocks == 1) tc::mma_commit(q_empty);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
           const int base = (ptr + j * need) % kRingTiles;
-          // both tiles' next scores first: each waits only for its softmax to have read S,
-          // so they compute under this block's exponentials
           if (j + 1 < a.n_blocks) {
-            if (!tc::mbar_wait(kv_full + (g + 1) % kMaxStages, ((g + 1) / kMaxStages) & 1, a.status, 36, abort)) {
+            if (!tc::mbar_wait(kv_full + (g + 1) % kMaxStages, ((g + 1) / kMaxStages) & 1, a.status, 36, abort) ||
+                !tc::mbar_wait(s_free + t, g & 1, a.status, 41, abort)) {
               ok = false;
               break;
             }
-            for (int t = 0; t < 2 && ok; ++t) {
-              if (!tc::mbar_wait(s_free + t, g & 1, a.status, 41, abort)) { ok = false; break; }
-              tc::tc_fence_after();
-              issue_s(t, (base + need) % kRingTiles);
-            }
-            if (!ok) break;
+            tc::tc_fence_after();
+            issue_s(t, (base + need) % kRingTiles);
             if (j + 2 == a.n_blocks) tc::mma_commit(q_empty);
           }
-          for (int t = 0; t < 2; ++t) {
-            if (!tc::mbar_wait(p_full + t, g & 1, a.status, 34, abort)) { ok = false; break; }
-            if (j == 0 && !tc::mbar_wait(o_free + t, (li & 1) ^ 1, a.status, 35, abort)) { ok = false; break; }
-            tc::tc_fence_after();
-            issue_pv(t, base, j != 0);
+          if (!tc::mbar_wait(p_full + t, g & 1, a.status, 34, abort) ||
+              (j == 0 && !tc::mbar_wait(o_free + t, (li & 1) ^ 1, a.status, 35, abort))) {
+            ok = false;
+            break;
           }
-          if (!ok) break;
+          tc::tc_fence_after();
+          issue_pv(t, base, j != 0);
           tc::mma_commit(kv_empty + g % kMaxStages);
         }
         ptr = (ptr + a.n_blocks * need) % kRingTiles;
@@ -594,15 +611,13 @@ bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int
     // sequence's (separate keys)
     a.S = B * nb * H;
     a.pairs = a.q_tiles / 2;
-    a.shared_items = a.S * a.pairs;
-    a.items = a.shared_items + ((a.q_tiles & 1) ? (a.S + 1) / 2 : 0);
+    a.items = a.S * a.pairs + ((a.q_tiles & 1) ? (a.S + 1) / 2 : 0);
     a.n_blocks = (a.n + kKeys - 1) / kKeys;
     box[0] = kDh; box[1] = 1; box[2] = 1; box[3] = kRows;      // 128 frames of one (band, head)
   } else {
     if (nb > 64) return false;
     a.pairs = 0;
     a.S = 0;
-    a.shared_items = 0;
     a.items = H * ((a.BT + 3) / 4);
     a.n_blocks = 1;
     box[0] = kDh; box[1] = 1; box[2] = 64; box[3] = 2;         // bands 0..63 of two frames
