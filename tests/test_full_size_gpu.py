@@ -1,0 +1,83 @@
+"""Full-size workloads through the C ABI (GPU): the batch of eight 801-frame windows cut from one
+clip, and the longest window of the chunk-length sweep.
+
+The oracle cannot afford these sizes element by element, so they are checked through properties
+that hold at any size: every window of a batch is computed independently, so the batch's masks are
+the single-window masks stacked ("Mel-Band RoFormer — architecture, inference hot path & RTX 3050
+feasibility", section "Verified inference hot path": the per-chunk loop runs the model on each
+window by itself), the captured graph replays the eager launches, and every mask is finite.
+The fp32 row statistics are accumulated with atomic adds, whose order may differ between
+launches, so two runs agree to rounding, not bit for bit."""
+import numpy as np
+import pytest
+
+import synth
+from parity import case, snr_db
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def model(cfg, W, B, T, graph=True):
+    from axial_band_split_b200 import mrf
+    m = mrf.Model(cfg, W, max_batch=B, max_frames=T, compute=mrf.MRF_FP16)
+    m.set_graph(graph)
+    return m
+
+
+def run(m, x):
+    out = m.forward(torch.from_numpy(np.ascontiguousarray(x)).cuda())
+    m.sync_status()
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def close(a, b, what):
+    err = float(np.abs(a - b).max())
+    snr = snr_db(a, b)
+    print(f"{what}: max|diff|={err:.3e} snr={snr:.1f} dB")
+    assert np.isfinite(a).all() and np.isfinite(b).all()
+    assert err <= 5e-3 and snr >= 60.0, f"{what}: max|diff|={err:.3e} snr={snr:.1f} dB"
+
+
+def test_batch8_T801_equals_single_windows():
+    cfg = synth.VOCALS
+    B, T = 8, 801
+    W, x = case(cfg, B, T, True)
+    mb = model(cfg, W, B, T)
+    got = run(mb, x)
+    mb.close()
+    m1 = model(cfg, W, 1, T)
+    for b in (0, 3, 7):
+        close(got[b:b + 1], run(m1, x[b:b + 1]), f"window {b} of 8")
+    m1.close()
+
+
+def test_T4096_graph_matches_eager_and_finite():
+    cfg = synth.VOCALS
+    B, T = 1, 4096
+    W, x = case(cfg, B, T, True)
+    mg = model(cfg, W, B, T, graph=True)
+    a = run(mg, x)
+    mg.set_graph(False)
+    b = run(mg, x)
+    mg.close()
+    close(a, b, "T=4096 graph vs eager")
+
+
+def test_T1100_full_size_vs_oracle():
+    # the benchmarked configuration (B=1, T=1100, captured graph) against the float64 oracle,
+    # every mask element (the oracle takes about a minute on the host cores)
+    from parity import oracle_masks
+    cfg = synth.VOCALS
+    B, T = 1, 1100
+    W, x = case(cfg, B, T, True)
+    m = model(cfg, W, B, T)
+    got = run(m, x)
+    m.close()
+    ref = oracle_masks(cfg, B, T, True)
+    err = float(np.abs(got - ref).max())
+    snr = snr_db(got, ref)
+    print(f"T=1100 masks: max|diff|={err:.3e} snr={snr:.1f} dB max|ref|={float(np.abs(ref).max()):.3e}")
+    assert err <= 2e-2 and snr >= 40.0
