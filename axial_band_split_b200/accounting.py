@@ -23,6 +23,7 @@ def kernel_work(cfg, widths, B: int, T: int):
     NT = BT * nb
     n_feat = int(sum(widths))
     rows = (cfg.n_fft // 2 + 1) * cfg.audio_channels
+    S = cfg.num_stems  # one mask estimator (and overlap average) per stem
     w = {
         "gemm_qkv": ("flop", L2 * 2 * NT * D * (3 * A + H), L2),
         "attn_time_tc": ("flop", cfg.depth * 4 * (B * nb * H) * T * T * dh, cfg.depth),
@@ -30,16 +31,16 @@ def kernel_work(cfg, widths, B: int, T: int):
         "gemm_out_resid": ("flop", L2 * 2 * NT * A * D, L2),
         "gemm_ff1_gelu": ("flop", L2 * 2 * NT * D * FF, L2),
         "gemm_ff2_resid": ("flop", L2 * 2 * NT * FF * D, L2),
-        "gemm_mask_tanh": ("flop", 2 * BT * nb * (D * MH + (cfg.mask_depth - 1) * MH * MH), cfg.mask_depth),
-        "gemm_mask_glu": ("flop", 2 * BT * MH * 2 * n_feat, 1),
+        "gemm_mask_tanh": ("flop", S * 2 * BT * nb * (D * MH + (cfg.mask_depth - 1) * MH * MH), S * cfg.mask_depth),
+        "gemm_mask_glu": ("flop", S * 2 * BT * MH * 2 * n_feat, S),
         "band_split": ("flop", 2 * BT * D * n_feat, 1),
         "gemm_band_split": ("flop", 2 * BT * D * n_feat, 1),
         # stft_repr read once, normalised fp16 band features written once
         "band_gather": ("byte", B * rows * T * 2 * 4 + BT * n_feat * 2, 1),
         # x fp32 read + write, x fp16 write, |x|^2 read + write, gain
         "outnorm": ("byte", L2 * NT * (D * 4 * 2 + D * 2 + 8), L2),
-        # mask features fp32 read once, masks fp32 written once
-        "overlap_average": ("byte", BT * n_feat * 4 + B * rows * T * 2 * 4, 1),
+        # per stem: mask features fp32 read once, masks fp32 written once
+        "overlap_average": ("byte", S * (BT * n_feat * 4 + B * rows * T * 2 * 4), S),
     }
     return w
 

@@ -60,7 +60,7 @@ extern "C" mrf_status mrf_forward_static(mrf_handle *h, const float *in, float *
   }
   const size_t io = (size_t)B * h->tab.n_freqs * h->tab.channels * T * 2 * sizeof(float);
   const char *a = reinterpret_cast<const char *>(in), *b = reinterpret_cast<const char *>(out);
-  if (a < b + io && b < a + io) { h->err = "stft_repr and masks overlap"; return MRF_EINVAL; }
+  if (a < b + io * h->cfg.num_stems && b < a + io) { h->err = "stft_repr and masks overlap"; return MRF_EINVAL; }
   const size_t need = fp16_workspace_layout(h, nullptr, false, nullptr, nullptr, nullptr);
   if (need > kStaticScratchBytes) {
     char buf[256];

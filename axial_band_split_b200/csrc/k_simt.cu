@@ -413,10 +413,14 @@ __global__ void outnorm_kernel(float *__restrict__ x, float *__restrict__ ss, co
 }
 
 // ------------------------------------------------------------------ overlap average
+// masks[b, r, t, c] = wrow[r] * (m[b, t, src0] + m[b, t, src1]) written at out + b * out_bstride
+// + (r T + t) 2 + c; with `spec` (stft_repr [B, R, T, 2]) the complex product of the mask and
+// spec at (b, r, t) is written instead (the separated spectrum).
 __global__ void overlap_average_kernel(const float *__restrict__ m, int ldm,
                                        const int32_t *__restrict__ src0,
                                        const int32_t *__restrict__ src1,
                                        const float *__restrict__ wrow, float *__restrict__ out,
+                                       long long out_bstride, const float *__restrict__ spec,
                                        int B, int T, int R) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long total = (long long)B * R * T * 2;
@@ -425,12 +429,23 @@ __global__ void overlap_average_kernel(const float *__restrict__ m, int ldm,
   const long long t = (i >> 1) % T;
   const long long r = ((i >> 1) / T) % R;
   const long long b = (i >> 1) / ((long long)T * R);
-  const int o = (int)r * 2 + c;
+  const long long j = i - b * (long long)R * T * 2;  // (r T + t) 2 + c
   const float *mr = m + (b * T + t) * ldm;
-  const int s0 = src0[o], s1 = src1[o];
-  float v = mr[s0];
-  if (s1 >= 0) v += mr[s1];
-  out[i] = v * wrow[r];
+  const float w = wrow[r];
+  auto mask = [&](int cc) {
+    const int o = (int)r * 2 + cc;
+    const int s0 = src0[o], s1 = src1[o];
+    float v = mr[s0];
+    if (s1 >= 0) v += mr[s1];
+    return v * w;
+  };
+  if (!spec) {
+    out[b * out_bstride + j] = mask(c);
+    return;
+  }
+  const float m_re = mask(0), m_im = mask(1);
+  const float *x = spec + i - c;
+  out[b * out_bstride + j] = c == 0 ? m_re * x[0] - m_im * x[1] : m_re * x[1] + m_im * x[0];
 }
 
 __global__ void fill_kernel(float *p, float v, long long n) {
@@ -501,11 +516,11 @@ void launch_outnorm(float *x, float *ss, const float *gain, __half *xh, long lon
 }
 
 void launch_overlap_average(const float *m, int ldm, const int32_t *src0, const int32_t *src1,
-                            const float *row_weight, float *masks, int B, int T, int rows,
-                            cudaStream_t st) {
+                            const float *row_weight, float *masks, long long out_bstride, const float *spec,
+                            int B, int T, int rows, cudaStream_t st) {
   const long long n = (long long)B * rows * T * 2;
-  overlap_average_kernel<<<grid1(n, 256), 256, 0, st>>>(m, ldm, src0, src1, row_weight, masks, B,
-                                                        T, rows);
+  overlap_average_kernel<<<grid1(n, 256), 256, 0, st>>>(m, ldm, src0, src1, row_weight, masks, out_bstride,
+                                                        spec, B, T, rows);
 }
 
 void launch_fill_f32(float *p, float v, long long n, cudaStream_t st) {

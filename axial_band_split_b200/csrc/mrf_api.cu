@@ -46,7 +46,7 @@ std::string validate_config(const mrf_config &c) {
   if (c.ff_mult < 1 || c.ff_mult > 8) return "ff_mult out of range";
   if (c.mask_hidden < 16 || c.mask_hidden > 8192) return "mask_hidden out of range";
   if (c.mask_depth < 1 || c.mask_depth > 4) return "mask_depth out of range";
-  if (c.num_stems != 1) return "num_stems other than 1 is not implemented";
+  if (c.num_stems < 1 || c.num_stems > 4) return "num_stems must be in [1, 4]";
   if (c.max_batch < 1 || c.max_frames < 1) return "max_batch and max_frames must be >= 1";
   if ((long long)c.max_batch * c.max_frames > (1LL << 22)) return "max_batch * max_frames too large";
   if (!(c.rope_theta > 1.f)) return "rope_theta must be > 1";
@@ -80,8 +80,9 @@ std::map<std::string, std::vector<int64_t>> expected_weights(const mrf_config &c
       e[p + "layers.0.1.net.4.bias"] = {D};
       e[p + "norm.gamma"] = {D};
     }
+  for (int s = 0; s < c.num_stems; ++s)
   for (int k = 0; k < c.num_bands; ++k) {
-    const std::string p = "mask_estimators.0.to_freqs." + std::to_string(k) + ".0.";
+    const std::string p = "mask_estimators." + std::to_string(s) + ".to_freqs." + std::to_string(k) + ".0.";
     std::vector<int64_t> dims = {D};
     for (int i = 0; i < c.mask_depth; ++i) dims.push_back(MH);
     dims.push_back(2 * (int64_t)t.width[k]);
@@ -287,30 +288,36 @@ mrf_status pack_f32(mrf_handle *h, std::map<std::string, HostW> &W) {
           !x.b2 || !x.g_out)
         return fail(h, MRF_ENOMEM, "device allocation failed (transformer weights)");
     }
-  // mask head: layers 0 .. mask_depth-1 stacked per band, last layer interleaved
-  std::vector<std::vector<float>> mw(c.mask_depth), mb(c.mask_depth);
-  std::vector<float> w_last, b_last;
-  for (int k = 0; k < nb; ++k) {
-    const std::string p = "mask_estimators.0.to_freqs." + std::to_string(k) + ".0.";
-    for (int i = 0; i < c.mask_depth; ++i) {
-      const auto &w = W[p + std::to_string(2 * i) + ".weight"].v;
-      const auto &b = W[p + std::to_string(2 * i) + ".bias"].v;
-      mw[i].insert(mw[i].end(), w.begin(), w.end());
-      mb[i].insert(mb[i].end(), b.begin(), b.end());
+  // mask heads (one per stem): layers 0 .. mask_depth-1 stacked per band, last layer interleaved
+  h->mf.w.resize(c.num_stems);
+  h->mf.b.resize(c.num_stems);
+  h->mf.w_last.resize(c.num_stems);
+  h->mf.b_last.resize(c.num_stems);
+  for (int s = 0; s < c.num_stems; ++s) {
+    std::vector<std::vector<float>> mw(c.mask_depth), mb(c.mask_depth);
+    std::vector<float> w_last, b_last;
+    for (int k = 0; k < nb; ++k) {
+      const std::string p = "mask_estimators." + std::to_string(s) + ".to_freqs." + std::to_string(k) + ".0.";
+      for (int i = 0; i < c.mask_depth; ++i) {
+        const auto &w = W[p + std::to_string(2 * i) + ".weight"].v;
+        const auto &b = W[p + std::to_string(2 * i) + ".bias"].v;
+        mw[i].insert(mw[i].end(), w.begin(), w.end());
+        mb[i].insert(mb[i].end(), b.begin(), b.end());
+      }
+      const std::string q = p + std::to_string(2 * c.mask_depth);
+      interleave_glu(W[q + ".weight"].v, W[q + ".bias"].v, t.width[k], MH, &w_last, &b_last);
     }
-    const std::string q = p + std::to_string(2 * c.mask_depth);
-    interleave_glu(W[q + ".weight"].v, W[q + ".bias"].v, t.width[k], MH, &w_last, &b_last);
+    h->mf.w[s].resize(c.mask_depth);
+    h->mf.b[s].resize(c.mask_depth);
+    for (int i = 0; i < c.mask_depth; ++i) {
+      h->mf.w[s][i] = upload_f32(h, mw[i]);
+      h->mf.b[s][i] = upload_f32(h, mb[i]);
+      if (!h->mf.w[s][i] || !h->mf.b[s][i]) return fail(h, MRF_ENOMEM, "device allocation failed (mask head)");
+    }
+    h->mf.w_last[s] = upload_f32(h, w_last);
+    h->mf.b_last[s] = upload_f32(h, b_last);
+    if (!h->mf.w_last[s] || !h->mf.b_last[s]) return fail(h, MRF_ENOMEM, "device allocation failed (mask head)");
   }
-  h->mf.w.resize(c.mask_depth);
-  h->mf.b.resize(c.mask_depth);
-  for (int i = 0; i < c.mask_depth; ++i) {
-    h->mf.w[i] = upload_f32(h, mw[i]);
-    h->mf.b[i] = upload_f32(h, mb[i]);
-    if (!h->mf.w[i] || !h->mf.b[i]) return fail(h, MRF_ENOMEM, "device allocation failed (mask head)");
-  }
-  h->mf.w_last = upload_f32(h, w_last);
-  h->mf.b_last = upload_f32(h, b_last);
-  if (!h->mf.w_last || !h->mf.b_last) return fail(h, MRF_ENOMEM, "device allocation failed (mask head)");
   // groups of the mask-head GEMMs
   const int D = c.dim;
   std::vector<SimtGroup> g0(nb), g1(nb), g2(nb);
@@ -387,23 +394,27 @@ void schedule_f32(mrf_handle *h, const float *in, float *out, int B, int T) {
     h->begin("rownorm_f32"); launch_rownorm_f32(w.X, x.g_out, w.X, NT, D, st); h->end();
   }
   const int M = B * T, MH = c.mask_hidden;
-  h->begin("gemm_f32");
-  launch_gemm_f32(w.X, h->mf.w[0], h->mf.b[0], w.H1, h->mf.g_first, nb, M, D, MH, kEpiTanh, st);
-  h->end();
-  float *cur = w.H1, *nxt = w.H2;
-  for (int i = 1; i < c.mask_depth; ++i) {
+  const long long per_stem = (long long)R * T * 2;  // one stem's masks of one window
+  for (int s = 0; s < c.num_stems; ++s) {
     h->begin("gemm_f32");
-    launch_gemm_f32(cur, h->mf.w[i], h->mf.b[i], nxt, h->mf.g_mid, nb, M, MH, MH, kEpiTanh, st);
+    launch_gemm_f32(w.X, h->mf.w[s][0], h->mf.b[s][0], w.H1, h->mf.g_first, nb, M, D, MH, kEpiTanh, st);
     h->end();
-    std::swap(cur, nxt);
+    float *cur = w.H1, *nxt = w.H2;
+    for (int i = 1; i < c.mask_depth; ++i) {
+      h->begin("gemm_f32");
+      launch_gemm_f32(cur, h->mf.w[s][i], h->mf.b[s][i], nxt, h->mf.g_mid, nb, M, MH, MH, kEpiTanh, st);
+      h->end();
+      std::swap(cur, nxt);
+    }
+    h->begin("gemm_f32");
+    launch_gemm_f32(cur, h->mf.w_last[s], h->mf.b_last[s], w.Mg, h->mf.g_last, nb, M, MH, 2 * h->max_width,
+                    kEpiGlu, st);
+    h->end();
+    h->begin("overlap_average");
+    launch_overlap_average(w.Mg, h->tab.n_feat(), h->d_src0, h->d_src1, h->d_row_weight, out + s * per_stem,
+                           c.num_stems * per_stem, h->apply_masks ? in : nullptr, B, T, R, st);
+    h->end();
   }
-  h->begin("gemm_f32");
-  launch_gemm_f32(cur, h->mf.w_last, h->mf.b_last, w.Mg, h->mf.g_last, nb, M, MH,
-                  2 * h->max_width, kEpiGlu, st);
-  h->end();
-  h->begin("overlap_average");
-  launch_overlap_average(w.Mg, h->tab.n_feat(), h->d_src0, h->d_src1, h->d_row_weight, out, B, T, R, st);
-  h->end();
 }
 
 void run_schedule(mrf_handle *h, const float *in, float *out, int B, int T) {
@@ -484,19 +495,27 @@ mrf_status mrf_create(const mrf_config *cfg, const mrf_tensor *w, int n_w, mrf_h
   return MRF_OK;
 }
 
-mrf_status mrf_forward(mrf_handle *h, const float *in, float *out, int B, int T, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// mrf_forward (apply = false: masks out) and mrf_forward_separate (apply = true: the masks
+// multiplied into stft_repr).  The output holds B x num_stems x rows x T x 2 floats.
+mrf_status forward_impl(mrf_handle *h, const float *in, float *out, int B, int T, void *stream, bool apply) {
   if (!h) return fail(nullptr, MRF_EINVAL, "null handle");
-  if (!in || !out) return fail(h, MRF_EINVAL, "null stft_repr or masks pointer");
+  if (!in || !out) return fail(h, MRF_EINVAL, "null stft_repr or output pointer");
   if (B < 1 || B > h->cfg.max_batch || T < 1 || T > h->cfg.max_frames)
     return fail(h, MRF_ESHAPE, "B or T outside [1, max_batch] x [1, max_frames]");
   if ((reinterpret_cast<uintptr_t>(in) | reinterpret_cast<uintptr_t>(out)) & 15)
-    return fail(h, MRF_EINVAL, "stft_repr and masks must be 16-byte aligned");
+    return fail(h, MRF_EINVAL, "stft_repr and the output must be 16-byte aligned");
   const size_t bytes = (size_t)B * h->tab.n_freqs * h->tab.channels * T * 2 * sizeof(float);
+  const size_t out_bytes = bytes * h->cfg.num_stems;
   const char *a = reinterpret_cast<const char *>(in), *b = reinterpret_cast<const char *>(out);
-  if (a < b + bytes && b < a + bytes) return fail(h, MRF_EINVAL, "stft_repr and masks overlap");
+  if (a < b + out_bytes && b < a + bytes) return fail(h, MRF_EINVAL, "stft_repr and the output overlap");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaGetLastError();
   mrf_status s = MRF_OK;
+  h->apply_masks = apply;
   if (h->timing || !h->use_graph) {
     h->cur_stream = st;
     run_schedule(h, in, out, B, T);
@@ -504,8 +523,8 @@ mrf_status mrf_forward(mrf_handle *h, const float *in, float *out, int B, int T,
     if (!cuda_ok(h, cudaGetLastError(), "kernel launch", &s)) return s;
     return MRF_OK;
   }
-  // CUDA graph per (B, T, in, out): captured once on an internal stream, replayed on `st`
-  GraphKey key{B, T, in, out};
+  // CUDA graph per (B, T, in, out, apply): captured once on an internal stream, replayed on `st`
+  GraphKey key{B, T, in, out, apply};
   cudaGraphExec_t exec = nullptr;
   for (auto &g : h->graphs)
     if (g.key == key) exec = g.exec;
@@ -535,6 +554,18 @@ mrf_status mrf_forward(mrf_handle *h, const float *in, float *out, int B, int T,
   return MRF_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+mrf_status mrf_forward(mrf_handle *h, const float *in, float *out, int B, int T, void *stream) {
+  return forward_impl(h, in, out, B, T, stream, false);
+}
+
+mrf_status mrf_forward_separate(mrf_handle *h, const float *in, float *out, int B, int T, void *stream) {
+  return forward_impl(h, in, out, B, T, stream, true);
+}
+
 mrf_status mrf_forward_host(mrf_handle *h, const float *in_host, float *out_host, int B, int T,
                             void *stream) {
   if (!h) return fail(nullptr, MRF_EINVAL, "null handle");
@@ -542,18 +573,19 @@ mrf_status mrf_forward_host(mrf_handle *h, const float *in_host, float *out_host
   if (B < 1 || B > h->cfg.max_batch || T < 1 || T > h->cfg.max_frames)
     return fail(h, MRF_ESHAPE, "B or T outside [1, max_batch] x [1, max_frames]");
   const size_t bytes = (size_t)B * h->tab.n_freqs * h->tab.channels * T * 2 * sizeof(float);
+  const size_t out_bytes = bytes * h->cfg.num_stems;
   mrf_status s = MRF_OK;
   if (!h->io_in) {
     const size_t maxb = (size_t)h->cfg.max_batch * h->tab.n_freqs * h->tab.channels * h->cfg.max_frames * 2 * sizeof(float);
     h->io_in = static_cast<float *>(h->alloc_bytes(maxb));
-    h->io_out = static_cast<float *>(h->alloc_bytes(maxb));
+    h->io_out = static_cast<float *>(h->alloc_bytes(maxb * h->cfg.num_stems));
     if (!h->io_in || !h->io_out) return fail(h, MRF_ENOMEM, "device allocation failed (io buffers)");
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (!cuda_ok(h, cudaMemcpyAsync(h->io_in, in_host, bytes, cudaMemcpyHostToDevice, st), "H2D copy", &s)) return s;
   s = mrf_forward(h, h->io_in, h->io_out, B, T, stream);
   if (s != MRF_OK) return s;
-  if (!cuda_ok(h, cudaMemcpyAsync(out_host, h->io_out, bytes, cudaMemcpyDeviceToHost, st), "D2H copy", &s)) return s;
+  if (!cuda_ok(h, cudaMemcpyAsync(out_host, h->io_out, out_bytes, cudaMemcpyDeviceToHost, st), "D2H copy", &s)) return s;
   if (!cuda_ok(h, cudaStreamSynchronize(st), "stream sync", &s)) return s;
   return mrf_sync_status(h, stream);
 }

@@ -16,9 +16,9 @@ struct TrF32 {  // one transformer, fp32 (debug schedule)
   float *g_ff = nullptr, *w1 = nullptr, *b1 = nullptr, *w2 = nullptr, *b2 = nullptr, *g_out = nullptr;
 };
 
-struct MaskF32 {
-  std::vector<float *> w, b;
-  float *w_last = nullptr, *b_last = nullptr;
+struct MaskF32 {  // the mask heads, one per stem: w[stem][layer]
+  std::vector<std::vector<float *>> w, b;
+  std::vector<float *> w_last, b_last;
   SimtGroup *g_first = nullptr, *g_mid = nullptr, *g_last = nullptr;
 };
 
@@ -31,7 +31,10 @@ struct GraphKey {
   int B, T;
   const float *in;
   float *out;
-  bool operator==(const GraphKey &o) const { return B == o.B && T == o.T && in == o.in && out == o.out; }
+  bool apply;  // masks applied to stft_repr (mrf_forward_separate) rather than written
+  bool operator==(const GraphKey &o) const {
+    return B == o.B && T == o.T && in == o.in && out == o.out && apply == o.apply;
+  }
 };
 
 struct GraphEntry {
@@ -92,6 +95,7 @@ struct mrf_handle {
 
   // execution
   bool timing = false, use_graph = true;
+  bool apply_masks = false;  // the schedule being recorded multiplies stft_repr by the masks
   cudaStream_t cur_stream = nullptr, cap_stream = nullptr;
   std::vector<mrf::PendingTiming> pending;
   std::vector<mrf::GraphEntry> graphs;

@@ -79,9 +79,11 @@ void launch_outnorm(float *x, float *ss, const float *gain, __half *xh, long lon
                     cudaStream_t st);
 
 // masks[b, r, t, c] = row_weight[r] * sum of the (<= 2) source features of (r, c)
+// out_bstride: elements between batch items of `masks` (stems x rows x T x 2 when the
+// stems are interleaved); spec: null, or stft_repr to multiply the masks into.
 void launch_overlap_average(const float *m, int ldm, const int32_t *src0, const int32_t *src1,
-                            const float *row_weight, float *masks, int B, int T, int rows,
-                            cudaStream_t st);
+                            const float *row_weight, float *masks, long long out_bstride, const float *spec,
+                            int B, int T, int rows, cudaStream_t st);
 
 void launch_fill_f32(float *p, float v, long long n, cudaStream_t st);
 

@@ -45,10 +45,12 @@ struct Fp16State {
   __half *A_bs = nullptr;     // normalised band features [nb][MBT][k_bs]
   int k_bs = 0;
   GemmGroup *g_bs = nullptr;
-  std::vector<__half *> mw;   // mask layers 0 .. mask_depth-1, stacked over bands [nb*MH, K]
-  std::vector<float *> mb;
-  __half *mw_last = nullptr;  // [sum 2*d_in, MH], rows interleaved (value e, gate e)
-  float *mb_last = nullptr;
+  // mask heads, one per stem: layers 0 .. mask_depth-1 stacked over bands [nb*MH, K] (mw[stem][layer]);
+  // the last layer [sum 2*d_in, MH] with rows interleaved (value e, gate e)
+  std::vector<std::vector<__half *>> mw;
+  std::vector<std::vector<float *>> mb;
+  std::vector<__half *> mw_last;
+  std::vector<float *> mb_last;
   // group tables
   GemmGroup *g_qkv = nullptr, *g_out = nullptr, *g_ff1 = nullptr, *g_ff2 = nullptr;
   GemmGroup *g_m0 = nullptr, *g_mid = nullptr, *g_last = nullptr;
@@ -174,11 +176,12 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
       if (!x.wqkvg || !x.bg || !x.wo || !x.w1 || !x.b1 || !x.w2 || !x.b2 || !x.gout)
         return MRF_ENOMEM;
     }
-  // mask head
+  // mask heads
+  for (int s = 0; s < c.num_stems; ++s) {
   std::vector<std::vector<float>> mw(c.mask_depth), mb(c.mask_depth);
   std::vector<float> wl, bl;
   for (int k = 0; k < nb; ++k) {
-    const std::string p = "mask_estimators.0.to_freqs." + std::to_string(k) + ".0.";
+    const std::string p = "mask_estimators." + std::to_string(s) + ".to_freqs." + std::to_string(k) + ".0.";
     for (int i = 0; i < c.mask_depth; ++i) {
       const auto &w = W[p + std::to_string(2 * i) + ".weight"].v;
       const auto &b = W[p + std::to_string(2 * i) + ".bias"].v;
@@ -204,14 +207,17 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
     for (size_t r = 0; r < mw[0].size() / D; ++r)
       for (int k = 0; k < D; ++k) mw[0][r * D + k] = (float)((double)mw[0][r * D + k] * gl[k] * sd);
   }
+  f->mw.emplace_back();
+  f->mb.emplace_back();
   for (int i = 0; i < c.mask_depth; ++i) {
-    f->mw.push_back(up(h, to_half(mw[i])));
-    f->mb.push_back(up(h, mb[i]));
-    if (!f->mw.back() || !f->mb.back()) return MRF_ENOMEM;
+    f->mw.back().push_back(up(h, to_half(mw[i])));
+    f->mb.back().push_back(up(h, mb[i]));
+    if (!f->mw.back().back() || !f->mb.back().back()) return MRF_ENOMEM;
   }
-  f->mw_last = up(h, to_half(wl));
-  f->mb_last = up(h, bl);
-  if (!f->mw_last || !f->mb_last) return MRF_ENOMEM;
+  f->mw_last.push_back(up(h, to_half(wl)));
+  f->mb_last.push_back(up(h, bl));
+  if (!f->mw_last.back() || !f->mb_last.back()) return MRF_ENOMEM;
+  }
   // group tables
   auto single = [&](int N, int BN) {
     GemmGroup g{N, cdiv(N, BN), 0, 0, 0, 0, 0, 0};
@@ -348,7 +354,8 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   CUtensorMap mAbs, mWbs;
   ok = ok && make_tmap_f16(&mAbs, f->A_bs, f->k_bs, (long long)nb * MBT, 1, f->k_bs, (long long)nb * MBT * f->k_bs, 128, 1) &&
        make_tmap_f16(&mWbs, f->w_bs, f->k_bs, (long long)nb * D, 1, f->k_bs, (long long)nb * D * f->k_bs, kBnNarrow, 1);
-  std::vector<CUtensorMap> wmaps(4 * 2 * c.depth + c.mask_depth + 1);
+  const int n_mask_maps = c.mask_depth + 1;  // per stem
+  std::vector<CUtensorMap> wmaps(4 * 2 * c.depth + c.num_stems * n_mask_maps);
   for (int i = 0; ok && i < 2 * c.depth; ++i) {
     const TrF16 &w = f->tr[i];
     ok = make_tmap_f16(&wmaps[4 * i + 0], w.wqkvg, D, 3 * A + H, 1, D, (3LL * A + H) * D, kBnWide, 1) &&
@@ -357,12 +364,15 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
          make_tmap_f16(&wmaps[4 * i + 3], w.w2, FF, D, 1, FF, (long long)D * FF, kBnNarrow, 1);
   }
   const int wm0 = 8 * c.depth;
-  for (int i = 0; ok && i < c.mask_depth; ++i) {
-    const int K = i == 0 ? D : MH;
-    ok = make_tmap_f16(&wmaps[wm0 + i], f->mw[i], K, (long long)nb * MH, 1, K, (long long)nb * MH * K, kBnWide, 1);
-  }
   const long long rows_last = 2LL * h->tab.n_feat();
-  ok = ok && make_tmap_f16(&wmaps[wm0 + c.mask_depth], f->mw_last, MH, rows_last, 1, MH, rows_last * MH, kBnWide, 1);
+  for (int s = 0; ok && s < c.num_stems; ++s) {
+    const int w0 = wm0 + s * n_mask_maps;
+    for (int i = 0; ok && i < c.mask_depth; ++i) {
+      const int K = i == 0 ? D : MH;
+      ok = make_tmap_f16(&wmaps[w0 + i], f->mw[s][i], K, (long long)nb * MH, 1, K, (long long)nb * MH * K, kBnWide, 1);
+    }
+    ok = ok && make_tmap_f16(&wmaps[w0 + c.mask_depth], f->mw_last[s], MH, rows_last, 1, MH, rows_last * MH, kBnWide, 1);
+  }
   // bulk-store output maps
   CUtensorMap mXo, mXho, mXbs, mXhbs, mHo, mH1o, mH2o, mMg, mQKVo;
   {
@@ -438,32 +448,38 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p, &mXo, &mXho);
   }
 
-  // mask head
+  // mask heads, one per stem, each followed by its overlap average (or, for
+  // mrf_forward_separate, the masks multiplied into stft_repr) into the stem's slice
   const int BT = B * T;
-  GemmParams p = base_params(h, BT, D, kBnWide, f->g_m0, nb, nb * cdiv(MH, kBnWide));
-  p.a_mode = 1;
-  p.ss_in = c.depth > 0 ? f->ssx : nullptr;  // 1 / |x| of the deferred last output norm
-  p.nb = nb;
-  p.bias = f->mb[0]; p.out_h = f->H1; p.ldo = MH; p.out_group_stride = MBT * MH;
-  gemm(h, "gemm_mask_tanh", kTcTanh, mXband, wmaps[wm0], p, &mH1o);
-  __half *cur = f->H1, *nxt = f->H2;
-  const CUtensorMap *mcur = &mH1, *mnxt = &mH2;
-  const CUtensorMap *ocur = &mH1o, *onxt = &mH2o;
-  for (int i = 1; i < c.mask_depth; ++i) {
-    p = base_params(h, BT, MH, kBnWide, f->g_mid, nb, nb * cdiv(MH, kBnWide));
-    p.bias = f->mb[i]; p.out_h = nxt; p.ldo = MH; p.out_group_stride = MBT * MH;
-    gemm(h, "gemm_mask_tanh", kTcTanh, *mcur, wmaps[wm0 + i], p, onxt);
-    std::swap(cur, nxt);
-    std::swap(mcur, mnxt);
-    std::swap(ocur, onxt);
-  }
-  p = base_params(h, BT, MH, kBnWide, f->g_last, nb, f->n_last_tiles);
-  p.bias = f->mb_last; p.out_f = f->Mg; p.ldo = h->tab.n_feat();
-  gemm(h, "gemm_mask_glu", kTcGlu, *mcur, wmaps[wm0 + c.mask_depth], p, &mMg);
+  const long long per_stem = (long long)R * T * 2;  // one stem's masks of one window
+  for (int s = 0; s < c.num_stems; ++s) {
+    const int w0 = wm0 + s * n_mask_maps;
+    GemmParams p = base_params(h, BT, D, kBnWide, f->g_m0, nb, nb * cdiv(MH, kBnWide));
+    p.a_mode = 1;
+    p.ss_in = c.depth > 0 ? f->ssx : nullptr;  // 1 / |x| of the deferred last output norm
+    p.nb = nb;
+    p.bias = f->mb[s][0]; p.out_h = f->H1; p.ldo = MH; p.out_group_stride = MBT * MH;
+    gemm(h, "gemm_mask_tanh", kTcTanh, mXband, wmaps[w0], p, &mH1o);
+    __half *cur = f->H1, *nxt = f->H2;
+    const CUtensorMap *mcur = &mH1, *mnxt = &mH2;
+    const CUtensorMap *ocur = &mH1o, *onxt = &mH2o;
+    for (int i = 1; i < c.mask_depth; ++i) {
+      p = base_params(h, BT, MH, kBnWide, f->g_mid, nb, nb * cdiv(MH, kBnWide));
+      p.bias = f->mb[s][i]; p.out_h = nxt; p.ldo = MH; p.out_group_stride = MBT * MH;
+      gemm(h, "gemm_mask_tanh", kTcTanh, *mcur, wmaps[w0 + i], p, onxt);
+      std::swap(cur, nxt);
+      std::swap(mcur, mnxt);
+      std::swap(ocur, onxt);
+    }
+    p = base_params(h, BT, MH, kBnWide, f->g_last, nb, f->n_last_tiles);
+    p.bias = f->mb_last[s]; p.out_f = f->Mg; p.ldo = h->tab.n_feat();
+    gemm(h, "gemm_mask_glu", kTcGlu, *mcur, wmaps[w0 + c.mask_depth], p, &mMg);
 
-  h->begin("overlap_average");
-  launch_overlap_average(f->Mg, h->tab.n_feat(), h->d_src0, h->d_src1, h->d_row_weight, out, B, T, R, st);
-  h->end();
+    h->begin("overlap_average");
+    launch_overlap_average(f->Mg, h->tab.n_feat(), h->d_src0, h->d_src1, h->d_row_weight, out + s * per_stem,
+                           c.num_stems * per_stem, h->apply_masks ? in : nullptr, B, T, R, st);
+    h->end();
+  }
 }
 
 }  // namespace mrf

@@ -23,7 +23,7 @@ STATUS = {0: "MRF_OK", -1: "MRF_EINVAL", -2: "MRF_ESHAPE", -3: "MRF_ENOMEM", -4:
           -5: "MRF_EUNSUPPORTED", -6: "MRF_ETIMEOUT", -7: "MRF_EWEIGHTS"}
 
 # every symbol include/mrf.h declares
-EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
+EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_separate", "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
            "mrf_last_error", "mrf_band_tables", "mrf_set_timing", "mrf_kernel_times",
            "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer", "mrf_forward_static"]
 
@@ -65,6 +65,8 @@ def lib():
         L.mrf_create.restype = I
         L.mrf_forward.argtypes = [P, P, P, I, I, P]
         L.mrf_forward.restype = I
+        L.mrf_forward_separate.argtypes = [P, P, P, I, I, P]
+        L.mrf_forward_separate.restype = I
         L.mrf_forward_static.argtypes = [P, P, P, I, I, P]
         L.mrf_forward_static.restype = I
         L.mrf_forward_host.argtypes = [P, P, P, I, I, P]
@@ -172,15 +174,35 @@ class Model:
         except Exception:
             pass
 
+    def _out_like(self, x, out):
+        """[B, F*2, T, 2] for one stem, [B, stems, F*2, T, 2] for more."""
+        import torch
+        if out is not None:
+            return out
+        B, R, T, two = x.shape
+        stems = self.cfg.num_stems
+        shape = (B, R, T, two) if stems == 1 else (B, stems, R, T, two)
+        return torch.empty(shape, dtype=x.dtype, device=x.device, pin_memory=not x.is_cuda and x.is_pinned())
+
     def forward(self, stft_repr, out=None, stream=None):
         """masks for a CUDA float32 tensor [B, F*2, T, 2] (queued on `stream`)."""
         import torch
         assert stft_repr.is_cuda and stft_repr.dtype == torch.float32 and stft_repr.is_contiguous()
         B, R, T, two = stft_repr.shape
-        if out is None:
-            out = torch.empty_like(stft_repr)
+        out = self._out_like(stft_repr, out)
         _check(lib().mrf_forward(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
                                  ctypes.c_void_p(out.data_ptr()), B, T, _stream_ptr(stream)), self._h)
+        return out
+
+    def separate(self, stft_repr, out=None, stream=None):
+        """mrf_forward_separate: the separated spectra (masks times stft_repr, complex), same
+        shape as forward's masks."""
+        import torch
+        assert stft_repr.is_cuda and stft_repr.dtype == torch.float32 and stft_repr.is_contiguous()
+        B, R, T, two = stft_repr.shape
+        out = self._out_like(stft_repr, out)
+        _check(lib().mrf_forward_separate(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
+                                          ctypes.c_void_p(out.data_ptr()), B, T, _stream_ptr(stream)), self._h)
         return out
 
     def forward_static(self, stft_repr, out, stream=None):
@@ -198,8 +220,7 @@ class Model:
         import torch
         x = stft_repr if isinstance(stft_repr, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(stft_repr))
         B, R, T, _ = x.shape
-        if out is None:
-            out = torch.empty_like(x)
+        out = self._out_like(x, out)
         _check(lib().mrf_forward_host(self._h, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(out.data_ptr()),
                                       B, T, _stream_ptr(stream)), self._h)
         return out

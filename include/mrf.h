@@ -61,7 +61,7 @@ typedef struct {
   int ff_mult;           /* 4: feed-forward inner width ff_mult*dim */
   int mask_hidden;       /* 4*dim: hidden width of the mask MLP */
   int mask_depth;        /* 2: tanh layers of the mask MLP before its GLU layer */
-  int num_stems;         /* 1 */
+  int num_stems;         /* 1..4: one mask estimator per stem over the shared trunk */
   int zero_dc;           /* 0: DC rows averaged like any other; 1: DC mask weight 0 */
   int max_batch;         /* workspace is sized for max_batch x max_frames at create */
   int max_frames;
@@ -95,7 +95,7 @@ typedef struct mrf_handle mrf_handle;
  *   layers.0.0.to_out.0.weight [dim, heads*dim_head],
  *   layers.0.1.net.0.gamma [dim], layers.0.1.net.1.weight [ff, dim], .net.1.bias [ff],
  *   layers.0.1.net.4.weight [dim, ff], .net.4.bias [dim], norm.gamma [dim];
- * for each band k: mask_estimators.0.to_freqs.{k}.0.{0,2,4}.{weight,bias}.
+ * for each stem s and band k: mask_estimators.{s}.to_freqs.{k}.0.{0,2,4}.{weight,bias}.
  * d_in_k = 2 * bins_k * audio_channels.  Weights are host memory owned by the caller and
  * are not referenced after the call.  On failure *out is NULL and nothing is leaked.
  * Errors: MRF_EINVAL, MRF_EUNSUPPORTED, MRF_EWEIGHTS, MRF_ESHAPE, MRF_ENOMEM, MRF_ECUDA.
@@ -105,17 +105,30 @@ mrf_status mrf_create(const mrf_config *cfg, const mrf_tensor *w, int n_w, mrf_h
 /*
  * mrf_forward - masks = core(stft_repr), queued on `stream` (a cudaStream_t; NULL is the
  * legacy default stream).  stft_repr: device float32 [B, F*C, T, 2], contiguous, 16-byte
- * aligned; masks: device float32, same shape, must not overlap stft_repr.  B in
- * [1, max_batch], T in [1, max_frames].  Arguments are checked before anything is
- * launched; on error nothing is queued.  Asynchronous: returns once the work is queued.
- * Device-side failures (a bounded wait that expired) surface through mrf_sync_status.
+ * aligned; masks: device float32 [B, num_stems, F*C, T, 2] (for one stem the shape of
+ * stft_repr), must not overlap stft_repr.  B in [1, max_batch], T in [1, max_frames].
+ * Arguments are checked before anything is launched; on error nothing is queued.
+ * Asynchronous: returns once the work is queued.  Device-side failures (a bounded wait
+ * that expired) surface through mrf_sync_status.
  */
 mrf_status mrf_forward(mrf_handle *h, const float *stft_repr, float *masks, int B, int T,
                        void *stream);
 
 /*
+ * mrf_forward_separate - the separated spectra: the forward's masks multiplied into the
+ * complex stft_repr, spec[b, s, r, t] = masks[b, s, r, t] * stft_repr[b, r, t] (complex
+ * product of the (re, im) pairs), computed in the overlap-average kernel so the masks are
+ * never written ("Mel-Band RoFormer — architecture, inference hot path & RTX 3050
+ * feasibility", section "The forward chain": multiply the original complex STFT).  Same arguments,
+ * layout, checks and errors as mrf_forward, with spec in place of masks.
+ */
+mrf_status mrf_forward_separate(mrf_handle *h, const float *stft_repr, float *spec, int B, int T,
+                                void *stream);
+
+/*
  * mrf_forward_host - the same forward from and to HOST memory: copies stft_repr to the
- * device, runs mrf_forward, copies the masks back, and waits for the stream.  For the
+ * device, runs mrf_forward, copies the masks back ([B, num_stems, F*C, T, 2] floats), and
+ * waits for the stream.  For the
  * fastest copies the host buffers should be pinned (cudaHostAlloc / torch pin_memory).
  */
 mrf_status mrf_forward_host(mrf_handle *h, const float *stft_repr_host, float *masks_host,

@@ -14,7 +14,9 @@ Each function restates one step as the pages describe it:
   norm -> Linear -> GELU -> Linear with biases; each transformer ends with its own norm;
   attention is softmax(q k^T * scale) v with q, k rotated; the norm clamps ||x|| at 1e-12.
 * "musetric/vocal-separation-roformer-onnx" (page 3), section "Signature": stft_repr
-  [B, F*2, T, 2] in, per-bin complex masks of the same shape out, already averaged.
+  [B, F*2, T, 2] in, per-bin complex masks of the same shape out, already averaged; with
+  more than one stem, one mask per stem over the shared trunk (page 1, "The forward chain":
+  MaskEstimator per stem), and the separated spectra are mask times mixture (complex).
 
 Readings where the pages leave a value open: RoPE theta 10000 on interleaved pairs
 (2i, 2i+1), positions 0..n-1 along the attended axis (the band index on the band axis);
@@ -164,6 +166,20 @@ def overlap_average(m, tab, n_rows: int):
     acc = np.zeros((n_rows, T, 2), dtype=m.dtype)
     np.add.at(acc, (tab["feat_row"], slice(None), tab["feat_c"]), m.T)
     return acc * tab["row_weight"][:, None, None]
+
+
+def apply_masks(stft_repr, masks):
+    """The separated spectra: each stem's complex mask times the mixture's complex STFT
+    (page 1, section "The forward chain": multiply the original complex STFT).  stft_repr
+    (B, R, T, 2) and masks (B, R, T, 2) or (B, stems, R, T, 2), the last axis (re, im)."""
+    x = np.asarray(stft_repr, dtype=np.float64)
+    m = np.asarray(masks, dtype=np.float64)
+    xc = x[..., 0] + 1j * x[..., 1]
+    mc = m[..., 0] + 1j * m[..., 1]
+    if mc.ndim == xc.ndim + 1:  # one mixture under every stem's mask
+        xc = xc[:, None]
+    y = mc * xc
+    return np.stack([y.real, y.imag], axis=-1)
 
 
 def forward(stft_repr, cfg, weights, dtype=np.float64, return_stages: bool = False):

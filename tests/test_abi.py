@@ -62,9 +62,12 @@ def tiny_weights(cfg=synth.TINY):
 def test_create_validates_before_any_device_work():
     cfg = synth.TINY
     W = tiny_weights()
-    with pytest.raises(mrf.MrfError) as e:                      # unsupported stems
+    with pytest.raises(mrf.MrfError) as e:                      # stems out of range
+        mrf.Model(dataclasses.replace(cfg, num_stems=5), W)
+    assert e.value.status == -1
+    with pytest.raises(mrf.MrfError) as e:                      # a second stem without its weights
         mrf.Model(dataclasses.replace(cfg, num_stems=2), W)
-    assert e.value.status == -5
+    assert e.value.status == -7 and "mask_estimators.1." in str(e.value)
     with pytest.raises(mrf.MrfError) as e:                      # odd head width
         mrf.Model(dataclasses.replace(cfg, dim_head=15), W)
     assert e.value.status == -1

@@ -286,3 +286,44 @@ def test_forward_fp32_close_to_fp64():
     a = model.forward(x, cfg, W, dtype=np.float64)
     b = model.forward(x, cfg, W, dtype=np.float32)
     assert np.abs(a - b).max() / np.abs(a).max() < 1e-4
+
+
+def test_apply_masks_unit_and_imaginary_unit():
+    # mask 1 passes the mixture through; mask i turns (re, im) into (-im, re)
+    rng = np.random.Generator(np.random.PCG64(7))
+    x = rng.standard_normal((2, 6, 5, 2))
+    one = np.zeros_like(x)
+    one[..., 0] = 1.0
+    assert np.array_equal(model.apply_masks(x, one), x)
+    i = np.zeros_like(x)
+    i[..., 1] = 1.0
+    y = model.apply_masks(x, i)
+    assert np.array_equal(y[..., 0], -x[..., 1]) and np.array_equal(y[..., 1], x[..., 0])
+
+
+def test_apply_masks_modulus_and_stems_summing_to_one():
+    # |m x| = |m| |x| element by element; stems whose masks sum to 1 give back the mixture
+    rng = np.random.Generator(np.random.PCG64(8))
+    x = rng.standard_normal((1, 4, 3, 2))
+    m = rng.standard_normal((1, 2, 4, 3, 2))
+    y = model.apply_masks(x, m)
+    mod = lambda a: np.hypot(a[..., 0], a[..., 1])
+    assert np.allclose(mod(y), mod(m) * mod(x)[:, None], rtol=1e-12, atol=0)
+    m[:, 1] = -m[:, 0]
+    m[:, 1, ..., 0] += 1.0                                    # m1 = 1 - m0
+    y = model.apply_masks(x, m)
+    assert np.allclose(y.sum(axis=1), x, rtol=0, atol=1e-12)
+
+
+def test_stems_share_the_trunk():
+    # two stems: the same trunk output under two mask heads; stem 0 equals the one-stem model
+    # built from stem 0's weights
+    import dataclasses
+    cfg, W, x = tiny_case()
+    cfg2 = dataclasses.replace(cfg, num_stems=2)
+    W2 = synth.make_weights(cfg2, tables.band_tables(44100, 256, 8)["widths"], fp16=False)
+    two = model.forward(x, cfg2, W2)
+    one = model.forward(x, cfg, {k: v for k, v in W2.items() if not k.startswith("mask_estimators.1.")})
+    assert two.shape == (1, 2) + x.shape[1:]
+    assert np.array_equal(two[:, 0], one)
+    assert not np.allclose(two[:, 1], one)
