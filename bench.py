@@ -129,10 +129,11 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def kernel_source_hash():
+def kernel_source_hash(files=None):
+    """sha256 (16 hex digits) of the named files under csrc/ (all of csrc/ when None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "axial_band_split_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
+    for n in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, n), "rb") as f:
             h.update(n.encode() + f.read())
     return h.hexdigest()[:16]
@@ -140,18 +141,24 @@ def kernel_source_hash():
 
 def traffic_for(kernel):
     """DRAM bytes (read + write) per launch of `kernel` from the committed ncu summary
-    profiles/traffic.txt, if it was taken on the current kernel sources; else None.
-    Format: '# comment' lines, 'source_hash <hash>', then '<kernel> <bytes per launch>'."""
+    profiles/traffic.txt, if it was taken on the current sources of the profiled kernels; else
+    None.  Format: '# comment' lines, 'sources <file> ...' (under csrc/), 'source_hash <hash>'
+    of those files, then '<kernel> <bytes per launch>'."""
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    vals = {}
+    vals, files = {}, None
     with open(p) as f:
         for line in f:
             parts = line.split("#")[0].split()
-            if len(parts) == 2:
+            if parts and parts[0] == "sources":
+                files = parts[1:]
+            elif len(parts) == 2:
                 vals[parts[0]] = parts[1]
-    if vals.get("source_hash") != kernel_source_hash():
+    try:
+        if vals.get("source_hash") != kernel_source_hash(files):
+            return None
+    except OSError:
         return None
     v = vals.get(kernel)
     return float(v) if v is not None else None
