@@ -610,6 +610,7 @@ void mrf_destroy(mrf_handle *h) {
   for (auto &g : h->graphs) cudaGraphExecDestroy(g.exec);
   for (auto &p : h->pending) { cudaEventDestroy(p.e0); cudaEventDestroy(p.e1); }
   for (void *p : h->allocs) cudaFree(p);
+  for (auto &p : h->sig_scratch) cudaFree(p.first);
   if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   destroy_fp16(h);
   delete h;

@@ -101,6 +101,10 @@ struct mrf_handle {
   std::vector<mrf::GraphEntry> graphs;
   int launch_counter = 0, last_launches = -1, last_B = -1, last_T = -1;
   float *io_in = nullptr, *io_out = nullptr;
+  // spectral front / back end (signal_api.cu): FFT tables of n_fft and grow-only scratch
+  float2 *d_tw = nullptr;
+  float *d_win = nullptr;
+  std::vector<std::pair<void *, size_t>> sig_scratch;
   std::string sched_error;  // set by a schedule that refused to launch
 
   void begin(const char *name);

@@ -79,6 +79,29 @@ void launch_outnorm(float *x, float *ss, const float *gain, __half *xh, long lon
                     cudaStream_t st);
 
 // masks[b, r, t, c] = row_weight[r] * sum of the (<= 2) source features of (r, c)
+// ------------------------------------------------------------------ spectral front / back end (k_signal.cu)
+// Up to 16 chunks of the chunk loop gathered at once: chunk k covers samples off[k] .. off[k]
+// + n[k] of the padded mix; past n[k] its own reflection (reflect[k] != 0) or zeros.
+struct ChunkBatch {
+  int count;
+  int off[16], n[16], reflect[16];
+};
+bool signal_kernels_init();
+// x [B, C, L] -> out [B, (n/2+1) C, T, 2], n = 2^log2n <= 4096; tw[i] = exp(-2 pi i i / n), i < n/2;
+// win: the analysis window (n values).
+void launch_stft(const float *x, float *out, const float2 *tw, const float *win, int B, int C, int L, int T,
+                 int log2n, int hop, cudaStream_t st);
+// spec [S, (n/2+1) C, T, 2] -> out [S, C, length]; frames: scratch of S * C * T * n floats.
+void launch_istft(const float *spec, float *frames, float *out, const float2 *tw, const float *win, int S, int C,
+                  int T, int log2n, int hop, int length, cudaStream_t st);
+void launch_pad_reflect(const float *mix, float *xp, int C, int L, int border, cudaStream_t st);
+void launch_gather_chunks(const float *xp, float *chunks, const ChunkBatch &cb, int C, int Lp, int chunk,
+                          cudaStream_t st);
+void launch_accumulate_chunk(const float *est, float *acc, float *counter, int S, int C, int Lp, int chunk, int fade,
+                             int off, int n, bool first, bool last, cudaStream_t st);
+void launch_finalize(const float *acc, const float *counter, float *out, int S, int C, int Lp, int L, int border,
+                     cudaStream_t st);
+
 // out_bstride: elements between batch items of `masks` (stems x rows x T x 2 when the
 // stems are interleaved); spec: null, or stft_repr to multiply the masks into.
 void launch_overlap_average(const float *m, int ldm, const int32_t *src0, const int32_t *src1,

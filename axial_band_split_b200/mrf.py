@@ -23,7 +23,8 @@ STATUS = {0: "MRF_OK", -1: "MRF_EINVAL", -2: "MRF_ESHAPE", -3: "MRF_ENOMEM", -4:
           -5: "MRF_EUNSUPPORTED", -6: "MRF_ETIMEOUT", -7: "MRF_EWEIGHTS"}
 
 # every symbol include/mrf.h declares
-EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_separate", "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
+EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_separate", "mrf_stft", "mrf_istft", "mrf_separate_audio",
+           "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
            "mrf_last_error", "mrf_band_tables", "mrf_set_timing", "mrf_kernel_times",
            "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer", "mrf_forward_static"]
 
@@ -67,6 +68,12 @@ def lib():
         L.mrf_forward.restype = I
         L.mrf_forward_separate.argtypes = [P, P, P, I, I, P]
         L.mrf_forward_separate.restype = I
+        L.mrf_stft.argtypes = [P, P, P, I, I, I, P]
+        L.mrf_stft.restype = I
+        L.mrf_istft.argtypes = [P, P, P, I, I, I, I, P]
+        L.mrf_istft.restype = I
+        L.mrf_separate_audio.argtypes = [P, P, P, I, I, P]
+        L.mrf_separate_audio.restype = I
         L.mrf_forward_static.argtypes = [P, P, P, I, I, P]
         L.mrf_forward_static.restype = I
         L.mrf_forward_host.argtypes = [P, P, P, I, I, P]
@@ -203,6 +210,42 @@ class Model:
         out = self._out_like(stft_repr, out)
         _check(lib().mrf_forward_separate(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
                                           ctypes.c_void_p(out.data_ptr()), B, T, _stream_ptr(stream)), self._h)
+        return out
+
+    def stft(self, audio, hop, out=None, stream=None):
+        """mrf_stft: CUDA float32 audio [B, C, L] -> stft_repr [B, (n_fft/2+1) C, 1 + L // hop, 2]."""
+        import torch
+        assert audio.is_cuda and audio.dtype == torch.float32 and audio.is_contiguous()
+        B, C, L = audio.shape
+        if out is None:
+            out = torch.empty((B, (self.cfg.n_fft // 2 + 1) * C, 1 + L // hop, 2), dtype=audio.dtype,
+                              device=audio.device)
+        _check(lib().mrf_stft(self._h, ctypes.c_void_p(audio.data_ptr()), ctypes.c_void_p(out.data_ptr()), B, L,
+                              hop, _stream_ptr(stream)), self._h)
+        return out
+
+    def istft(self, spec, hop, length, out=None, stream=None):
+        """mrf_istft: CUDA float32 spectra [..., (n_fft/2+1) C, T, 2] -> audio [..., C, length]."""
+        import torch
+        assert spec.is_cuda and spec.dtype == torch.float32 and spec.is_contiguous()
+        lead, FC, T = spec.shape[:-3], spec.shape[-3], spec.shape[-2]
+        C = self.cfg.audio_channels
+        S = int(np.prod(lead)) if lead else 1
+        if out is None:
+            out = torch.empty(tuple(lead) + (C, length), dtype=spec.dtype, device=spec.device)
+        _check(lib().mrf_istft(self._h, ctypes.c_void_p(spec.data_ptr()), ctypes.c_void_p(out.data_ptr()), S, T,
+                               hop, length, _stream_ptr(stream)), self._h)
+        return out
+
+    def separate_audio(self, mix, hop, out=None, stream=None):
+        """mrf_separate_audio: CUDA float32 mix [C, L] -> stems [num_stems, C, L]."""
+        import torch
+        assert mix.is_cuda and mix.dtype == torch.float32 and mix.is_contiguous()
+        C, L = mix.shape
+        if out is None:
+            out = torch.empty((self.cfg.num_stems, C, L), dtype=mix.dtype, device=mix.device)
+        _check(lib().mrf_separate_audio(self._h, ctypes.c_void_p(mix.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                                        L, hop, _stream_ptr(stream)), self._h)
         return out
 
     def forward_static(self, stft_repr, out, stream=None):

@@ -126,6 +126,39 @@ mrf_status mrf_forward_separate(mrf_handle *h, const float *stft_repr, float *sp
                                 void *stream);
 
 /*
+ * mrf_stft - the model's STFT ("Mel-Band RoFormer — architecture, inference hot path & RTX
+ * 3050 feasibility", section "The forward chain": torch.stft, periodic Hann window of n_fft,
+ * center=True with reflect padding of n_fft/2, unnormalised).  audio: device float32
+ * [B, C, L] (C = audio_channels), L > n_fft/2; stft_repr: device float32 [B, (n_fft/2+1)*C,
+ * 1 + L/hop, 2], row f*C + c, (re, im).  n_fft must be a power of two <= 4096.  Queued on
+ * `stream`.  Errors: MRF_EINVAL, MRF_ESHAPE, MRF_EUNSUPPORTED, MRF_ENOMEM, MRF_ECUDA.
+ */
+mrf_status mrf_stft(mrf_handle *h, const float *audio, float *stft_repr, int B, int L, int hop, void *stream);
+
+/*
+ * mrf_istft - torch.istft of the same STFT: per frame the inverse real FFT times the window,
+ * overlap-added at hop, divided by the overlap-added squared window; the first n_fft/2
+ * samples dropped, `length` kept.  spec: device float32 [S, (n_fft/2+1)*C, T, 2]; audio:
+ * device float32 [S, C, length].  Allocates (once, grown on demand) an S*C*T*n_fft scratch.
+ */
+mrf_status mrf_istft(mrf_handle *h, const float *spec, float *audio, int S, int T, int hop, int length,
+                     void *stream);
+
+/*
+ * mrf_separate_audio - full separation of one mix: the chunk loop of "Mel-Band RoFormer —
+ * ...", section "Verified inference hot path" (8 s chunks at a stride of 0.9 chunk; the mix
+ * reflect-padded by the border chunk - stride when longer than two borders; a short last chunk
+ * padded by reflection when more than half a chunk remains, by zeros otherwise; linear fades
+ * of chunk/10 samples, the first chunk's fade-in and the last chunk's fade-out forced to 1;
+ * out += estimate * window, counter += window; out / max(counter, 1e-8), border cropped),
+ * each chunk through mrf_stft, mrf_forward_separate and mrf_istft, up to min(max_batch, 16)
+ * chunks per forward.  mix: device float32 [C, L]; stems: device float32 [num_stems, C, L].
+ * max_frames must hold 1 + 8 sample_rate / hop frames.  Allocates its buffers on first use
+ * (grown on demand, freed by mrf_destroy).
+ */
+mrf_status mrf_separate_audio(mrf_handle *h, const float *mix, float *stems, int L, int hop, void *stream);
+
+/*
  * mrf_forward_host - the same forward from and to HOST memory: copies stft_repr to the
  * device, runs mrf_forward, copies the masks back ([B, num_stems, F*C, T, 2] floats), and
  * waits for the stream.  For the
