@@ -85,3 +85,18 @@ def test_separate_spectra_fp16_and_fp32():
     ref1 = oracle_model.apply_masks(x1, oracle_model.forward(x1, cfg1, W1))
     got1 = run(cfg1, W1, x1, mrf.MRF_FP32_DEBUG, separate=True)
     assert rel_err(got1, ref1) <= 1e-4
+
+
+def test_zero_dc_masks():
+    # zero_dc: the DC rows' mask weight is 0 (the overlap average's row weight), both schedules
+    from axial_band_split_b200 import mrf
+    cfg = dataclasses.replace(synth.TINY, zero_dc=True)
+    W32, x = case(cfg, 1, 32, False)
+    ref = oracle_model.forward(x, cfg, W32)
+    assert np.abs(ref[:, : cfg.audio_channels]).max() == 0          # rows f = 0
+    got32 = run(cfg, W32, x, mrf.MRF_FP32_DEBUG, max_frames=40)
+    assert rel_err(got32, ref) <= 1e-4 and np.abs(got32[:, : cfg.audio_channels]).max() == 0
+    W16, _ = case(cfg, 1, 32, True)
+    got16 = run(cfg, W16, x, mrf.MRF_FP16, max_frames=40)
+    check16(got16, oracle_model.forward(x, cfg, W16), "tiny zero_dc")
+    assert np.abs(got16[:, : cfg.audio_channels]).max() == 0
