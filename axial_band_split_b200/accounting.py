@@ -16,6 +16,7 @@ def kernel_work(cfg, widths, B: int, T: int):
     D, H, dh = cfg.dim, cfg.heads, cfg.dim_head
     A = H * dh
     FF = D * cfg.ff_mult
+    F1 = FF * (2 if getattr(cfg, "ff_act", 0) == 1 else 1)  # GEGLU: value and gate halves
     MH = D * cfg.mask_hidden_mult
     nb = cfg.num_bands
     L2 = 2 * cfg.depth
@@ -29,7 +30,8 @@ def kernel_work(cfg, widths, B: int, T: int):
         "attn_time_tc": ("flop", cfg.depth * 4 * (B * nb * H) * T * T * dh, cfg.depth),
         "attn_band_tc": ("flop", cfg.depth * 4 * (BT * H) * nb * nb * dh, cfg.depth),
         "gemm_out_resid": ("flop", L2 * 2 * NT * A * D, L2),
-        "gemm_ff1_gelu": ("flop", L2 * 2 * NT * D * FF, L2),
+        "gemm_ff1_gelu": ("flop", L2 * 2 * NT * D * F1, L2),
+        "gemm_ff1_geglu": ("flop", L2 * 2 * NT * D * F1, L2),   # the GEGLU variant's launch name
         "gemm_ff2_resid": ("flop", L2 * 2 * NT * FF * D, L2),
         "gemm_mask_tanh": ("flop", S * 2 * BT * nb * (D * MH + (cfg.mask_depth - 1) * MH * MH), S * cfg.mask_depth),
         "gemm_mask_glu": ("flop", S * 2 * BT * MH * 2 * n_feat, S),
@@ -45,10 +47,14 @@ def kernel_work(cfg, widths, B: int, T: int):
     return w
 
 
+# entries that restate others' work (the SIMT band split; FF1 under its GEGLU launch name)
+_ALIASES = ("band_split", "gemm_ff1_geglu")
+
+
 def total_flops(cfg, widths, B: int, T: int) -> int:
     """FLOPs of one forward: every contraction of the method."""
     return sum(v for name, (k, v, _) in kernel_work(cfg, widths, B, T).items()
-               if k == "flop" and name != "band_split")
+               if k == "flop" and name not in _ALIASES)
 
 
 def attention_flops(cfg, widths, B, T):

@@ -26,6 +26,7 @@ enum GemmEpi : int {
   kTcTanh = 3,    // out = tanh(acc + bias) fp16 (group-strided)
   kTcGlu = 4,     // interleaved (value, gate) pairs -> value * sigmoid(gate), fp32
   kTcBandSplit = 5,  // X = acc + bias for token m*nb + group (band); X fp32, X fp16, row sum of squares
+  kTcGeglu = 6,   // interleaved (value, gate) pairs of acc * rowscale + bias -> value * gelu(gate), fp16
 };
 
 struct GemmParams {
@@ -77,7 +78,8 @@ bool gemm_tc_init();
 // (kTcQkv: [q | k | v | gates] fp16 [M, ld] box 32x32 swizzle 64; kTcResid: X fp32 [M, ld] box 32x32 swizzle 128 and X fp16 box 32x32 swizzle 64;
 //  kTcBandSplit: the same as 3D (ld, nb, frames) boxes 32x1x32; kTcGelu: out fp16 [M, ldo]
 //  box 32x32 swizzle 64; kTcTanh: out fp16 (ldo, frames, groups) box 32x32x1 swizzle 64;
-//  kTcGlu: out fp32 [frames, ldo] box 16x32 swizzle 64).  Unused maps may be any valid map.
+//  kTcGlu: out fp32 [frames, ldo] box 16x32 swizzle 64; kTcGeglu: out fp16 [M, ldo] box 16x32,
+//  no swizzle).  Unused maps may be any valid map.
 void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
                     const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st);
 

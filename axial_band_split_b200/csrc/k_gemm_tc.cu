@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) cs_pf[i] = rp[i];
         }
-      } else if (EPI == kTcGelu) {
+      } else if (EPI == kTcGelu || EPI == kTcGeglu) {
         ss_pf = (v_ && p.ss_in) ? p.ss_in[m_] : 1.f;
       } else if (EPI == kTcTanh) {
         ss_pf = (v_ && p.ss_in) ? p.ss_in[token_of(p, m_, t_.g)] : 1.f;
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) cs[i] = cs_pf[i];
       }
-      if (EPI == kTcQkv || EPI == kTcGelu || EPI == kTcTanh) rs = rsq;
+      if (EPI == kTcQkv || EPI == kTcGelu || EPI == kTcGeglu || EPI == kTcTanh) rs = rsq;
       const float res_s = rsq;  // kTcResid
       row_fetch(tile + gridDim.x);
       // residual prefetch (kTcResid): lane covers rows i*4 + lane/8, 16-byte piece lane%8
@@ -493,6 +493,32 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
             tc::bulk_commit();
           }
           ++nstore;
+        } else if (EPI == kTcGeglu) {
+          // interleaved (value e, gate e) columns -> 16 fp16 outputs value * gelu(gate) per row,
+          // stored through a 16 x 32 box (32-byte rows, no swizzle)
+          uint8_t *box = stg + (nstore & 1) * 2048;
+          if (lane == 0) tc::bulk_wait_read<1>();
+          __syncwarp();
+          float bv[32];
+          load_bias32(p.bias + gr.bias_off + c0, bv);
+          float o[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float2 g = tcm::gelu2(v[j + 1], v[j + 3], rs, bv[j + 1], bv[j + 3]);
+            o[j >> 1] = fmaf(v[j], rs, bv[j]) * g.x;
+            o[(j >> 1) + 1] = fmaf(v[j + 2], rs, bv[j + 2]) * g.y;
+          }
+          *reinterpret_cast<uint4 *>(box + lane * 32) =
+              make_uint4(pack_h2(o[0], o[1]), pack_h2(o[2], o[3]), pack_h2(o[4], o[5]), pack_h2(o[6], o[7]));
+          *reinterpret_cast<uint4 *>(box + lane * 32 + 16) =
+              make_uint4(pack_h2(o[8], o[9]), pack_h2(o[10], o[11]), pack_h2(o[12], o[13]), pack_h2(o[14], o[15]));
+          tc::fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tc::tma_store_2d(&tmC, box, c0 >> 1, m0w);
+            tc::bulk_commit();
+          }
+          ++nstore;
         } else {  // kTcGlu: interleaved (value, gate) pairs -> 16 fp32 outputs per row
           const float *bias = p.bias + gr.bias_off + c0;
           float o[16];
@@ -598,6 +624,7 @@ bool gemm_tc_init() {
   MRF_GEMM_ATTR(kTcGelu)
   MRF_GEMM_ATTR(kTcTanh)
   MRF_GEMM_ATTR(kTcGlu)
+  MRF_GEMM_ATTR(kTcGeglu)
   MRF_GEMM_ATTR(kTcBandSplit)
 #undef MRF_GEMM_ATTR
   return ok;
@@ -615,6 +642,7 @@ void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, con
     MRF_GEMM_CASE(kTcGelu)
     MRF_GEMM_CASE(kTcTanh)
     MRF_GEMM_CASE(kTcGlu)
+    MRF_GEMM_CASE(kTcGeglu)
     MRF_GEMM_CASE(kTcBandSplit)
 #undef MRF_GEMM_CASE
     default: break;

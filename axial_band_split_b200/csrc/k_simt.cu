@@ -217,6 +217,12 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(
             dst[n >> 1] = v * sigm(gt);
           }
           break;
+        case kEpiGeglu:
+          if ((j & 1) == 0 && n + 1 < g.N) {
+            const float gt = acc[i][j + 1] + (bs ? bs[n + 1] : 0.f);
+            dst[n >> 1] = v * gelu_erf(gt);
+          }
+          break;
         default: dst[n] = v; break;
       }
     }

@@ -46,6 +46,7 @@ std::string validate_config(const mrf_config &c) {
   if (c.ff_mult < 1 || c.ff_mult > 8) return "ff_mult out of range";
   if (c.mask_hidden < 16 || c.mask_hidden > 8192) return "mask_hidden out of range";
   if (c.mask_depth < 1 || c.mask_depth > 4) return "mask_depth out of range";
+  if (c.ff_act != 0 && c.ff_act != 1) return "ff_act must be 0 (GELU) or 1 (GEGLU)";
   if (c.num_stems < 1 || c.num_stems > 4) return "num_stems must be in [1, 4]";
   if (c.max_batch < 1 || c.max_frames < 1) return "max_batch and max_frames must be >= 1";
   if ((long long)c.max_batch * c.max_frames > (1LL << 22)) return "max_batch * max_frames too large";
@@ -74,8 +75,9 @@ std::map<std::string, std::vector<int64_t>> expected_weights(const mrf_config &c
       e[p + "layers.0.0.to_gates.bias"] = {H};
       e[p + "layers.0.0.to_out.0.weight"] = {D, A};
       e[p + "layers.0.1.net.0.gamma"] = {D};
-      e[p + "layers.0.1.net.1.weight"] = {FF, D};
-      e[p + "layers.0.1.net.1.bias"] = {FF};
+      const int64_t F1 = c.ff_act == 1 ? 2 * FF : FF;  // GEGLU: value and gate halves
+      e[p + "layers.0.1.net.1.weight"] = {F1, D};
+      e[p + "layers.0.1.net.1.bias"] = {F1};
       e[p + "layers.0.1.net.4.weight"] = {D, FF};
       e[p + "layers.0.1.net.4.bias"] = {D};
       e[p + "norm.gamma"] = {D};
@@ -279,8 +281,14 @@ mrf_status pack_f32(mrf_handle *h, std::map<std::string, HostW> &W) {
       x.bg = upload_f32(h, W[p + "layers.0.0.to_gates.bias"].v);
       x.wo = upload_f32(h, W[p + "layers.0.0.to_out.0.weight"].v);
       x.g_ff = upload_f32(h, scaled_gain(W[p + "layers.0.1.net.0.gamma"].v));
-      x.w1 = upload_f32(h, W[p + "layers.0.1.net.1.weight"].v);
-      x.b1 = upload_f32(h, W[p + "layers.0.1.net.1.bias"].v);
+      if (c.ff_act == 1) {  // GEGLU: (value, gate) rows paired for the epilogue
+        const int FFh = c.ff_mult * c.dim;
+        x.w1 = upload_f32(h, interleave_halves(W[p + "layers.0.1.net.1.weight"].v, FFh, c.dim));
+        x.b1 = upload_f32(h, interleave_halves(W[p + "layers.0.1.net.1.bias"].v, FFh, 1));
+      } else {
+        x.w1 = upload_f32(h, W[p + "layers.0.1.net.1.weight"].v);
+        x.b1 = upload_f32(h, W[p + "layers.0.1.net.1.bias"].v);
+      }
       x.w2 = upload_f32(h, W[p + "layers.0.1.net.4.weight"].v);
       x.b2 = upload_f32(h, W[p + "layers.0.1.net.4.bias"].v);
       x.g_out = upload_f32(h, scaled_gain(W[p + "norm.gamma"].v));
@@ -341,7 +349,7 @@ mrf_status pack_f32(mrf_handle *h, std::map<std::string, HostW> &W) {
       {0, 0, 0, 0, D, 3 * A, 3 * A, 0},  // qkv
       {0, 0, 0, 0, D, H, H, 0},          // gates
       {0, 0, 0, 0, A, D, D, 0},          // out
-      {0, 0, 0, 0, D, FF, FF, 0},        // ff1
+      {0, 0, 0, 0, D, FF, c.ff_act == 1 ? 2 * FF : FF, 0},  // ff1 (GEGLU: 2 FF paired columns, FF outputs)
       {0, 0, 0, 0, FF, D, D, 0},         // ff2
   };
   h->d_tgroups = h->alloc<SimtGroup>(5);
@@ -389,7 +397,11 @@ void schedule_f32(mrf_handle *h, const float *in, float *out, int B, int T) {
     h->begin("attention_f32"); launch_attention_f32(w.Q, w.K, w.V, w.G, w.O, B, T, nb, H, dh, axis, st); h->end();
     h->begin("gemm_f32"); launch_gemm_f32(w.O, x.wo, nullptr, w.X, tg + 2, 1, (int)NT, A, D, kEpiResidual, st); h->end();
     h->begin("rownorm_f32"); launch_rownorm_f32(w.X, x.g_ff, w.Xa, NT, D, st); h->end();
-    h->begin("gemm_f32"); launch_gemm_f32(w.Xa, x.w1, x.b1, w.Hf, tg + 3, 1, (int)NT, D, FF, kEpiGelu, st); h->end();
+    if (c.ff_act == 1) {
+      h->begin("gemm_f32"); launch_gemm_f32(w.Xa, x.w1, x.b1, w.Hf, tg + 3, 1, (int)NT, D, 2 * FF, kEpiGeglu, st); h->end();
+    } else {
+      h->begin("gemm_f32"); launch_gemm_f32(w.Xa, x.w1, x.b1, w.Hf, tg + 3, 1, (int)NT, D, FF, kEpiGelu, st); h->end();
+    }
     h->begin("gemm_f32"); launch_gemm_f32(w.Hf, x.w2, x.b2, w.X, tg + 4, 1, (int)NT, FF, D, kEpiResidual, st); h->end();
     h->begin("rownorm_f32"); launch_rownorm_f32(w.X, x.g_out, w.X, NT, D, st); h->end();
   }

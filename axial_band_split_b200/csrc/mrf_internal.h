@@ -45,6 +45,7 @@ enum SimtEpi : int {
   kEpiTanh = 3,       // C = tanh(acc + bias)
   kEpiSigmoid = 4,    // C = sigmoid(acc + bias)
   kEpiGlu = 5,        // value/gate halves of N: C[:, e] = v_e * sigmoid(g_e), N/2 outputs
+  kEpiGeglu = 6,      // columns interleaved (value e, gate e): C[:, e] = v_e * gelu(g_e), N/2 outputs
 };
 
 // One group of a grouped fp32 GEMM: C[m, n] = sum_k A[m, k] * W[n, k] for m < M, n < N.

@@ -166,8 +166,14 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
       x.wqkvg = up(h, to_half(qkvg));
       x.bg = up(h, W[p + "layers.0.0.to_gates.bias"].v);
       x.wo = up(h, to_half(W[p + "layers.0.0.to_out.0.weight"].v));
-      x.w1 = up(h, to_half(fold_cols(W[p + "layers.0.1.net.1.weight"].v, W[p + "layers.0.1.net.0.gamma"].v, FF, D)));
-      x.b1 = up(h, W[p + "layers.0.1.net.1.bias"].v);
+      if (c.ff_act == 1) {  // GEGLU: (value, gate) rows paired for the epilogue
+        x.w1 = up(h, to_half(fold_cols(interleave_halves(W[p + "layers.0.1.net.1.weight"].v, FF, D),
+                                       W[p + "layers.0.1.net.0.gamma"].v, 2 * FF, D)));
+        x.b1 = up(h, interleave_halves(W[p + "layers.0.1.net.1.bias"].v, FF, 1));
+      } else {
+        x.w1 = up(h, to_half(fold_cols(W[p + "layers.0.1.net.1.weight"].v, W[p + "layers.0.1.net.0.gamma"].v, FF, D)));
+        x.b1 = up(h, W[p + "layers.0.1.net.1.bias"].v);
+      }
       x.w2 = up(h, to_half(W[p + "layers.0.1.net.4.weight"].v));
       x.b2 = up(h, W[p + "layers.0.1.net.4.bias"].v);
       std::vector<float> go(W[p + "norm.gamma"].v);
@@ -225,7 +231,8 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   };
   f->g_qkv = single(3 * A + H, kBnWide);
   f->g_out = single(D, kBnNarrow);
-  f->g_ff1 = single(FF, kBnWide);
+  const int F1 = c.ff_act == 1 ? 2 * FF : FF;  // first feed-forward projection's outputs
+  f->g_ff1 = single(F1, kBnWide);
   f->g_ff2 = single(D, kBnNarrow);
   std::vector<GemmGroup> g0(nb), g1(nb), g2(nb);
   int start = 0;
@@ -339,6 +346,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   const int nb = c.num_bands, D = c.dim, H = c.heads, dh = c.dim_head, A = H * dh, FF = c.ff_mult * D,
             MH = c.mask_hidden;
   const long long MBT = (long long)c.max_batch * c.max_frames, NT = MBT * nb;
+  const int F1 = c.ff_act == 1 ? 2 * FF : FF;  // first feed-forward projection's outputs
   const int M = B * T * nb;
   const int R = h->tab.n_freqs * h->tab.channels;
   cudaStream_t st = h->cur_stream;
@@ -360,7 +368,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     const TrF16 &w = f->tr[i];
     ok = make_tmap_f16(&wmaps[4 * i + 0], w.wqkvg, D, 3 * A + H, 1, D, (3LL * A + H) * D, kBnWide, 1) &&
          make_tmap_f16(&wmaps[4 * i + 1], w.wo, A, D, 1, A, (long long)D * A, kBnNarrow, 1) &&
-         make_tmap_f16(&wmaps[4 * i + 2], w.w1, D, FF, 1, D, (long long)FF * D, kBnWide, 1) &&
+         make_tmap_f16(&wmaps[4 * i + 2], w.w1, D, F1, 1, D, (long long)F1 * D, kBnWide, 1) &&
          make_tmap_f16(&wmaps[4 * i + 3], w.w2, FF, D, 1, FF, (long long)D * FF, kBnNarrow, 1);
   }
   const int wm0 = 8 * c.depth;
@@ -374,7 +382,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     ok = ok && make_tmap_f16(&wmaps[w0 + c.mask_depth], f->mw_last[s], MH, rows_last, 1, MH, rows_last * MH, kBnWide, 1);
   }
   // bulk-store output maps
-  CUtensorMap mXo, mXho, mXbs, mXhbs, mHo, mH1o, mH2o, mMg, mQKVo;
+  CUtensorMap mXo, mXho, mXbs, mXhbs, mHo, mHo16, mH1o, mH2o, mMg, mQKVo;
   {
     const unsigned long long BT = (unsigned long long)B * T;
     const unsigned long long dx[3] = {(unsigned long long)D, (unsigned long long)nb, BT};
@@ -385,7 +393,8 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     const unsigned bh[3] = {32, 32, 1};
     ok = ok && map2(&mXo, f->X, kTmF32, D, M, D, 32, 128) && map2(&mXho, f->Xh, kTmF16, D, M, D, 32, 64) &&
          make_tmap(&mXbs, f->X, kTmF32, 3, dx, sx, bx, 128) && make_tmap(&mXhbs, f->Xh, kTmF16, 3, dx, sx, bx, 64) &&
-         map2(&mHo, f->Hh, kTmF16, FF, M, FF, 32, 64) && make_tmap(&mH1o, f->H1, kTmF16, 3, dh3, sh3, bh, 64) &&
+         map2(&mHo, f->Hh, kTmF16, FF, M, FF, 32, 64) && map2(&mHo16, f->Hh, kTmF16, FF, M, FF, 16, 0) &&
+         make_tmap(&mH1o, f->H1, kTmF16, 3, dh3, sh3, bh, 64) &&
          make_tmap(&mH2o, f->H2, kTmF16, 3, dh3, sh3, bh, 64) &&
          map2(&mMg, f->Mg, kTmF32, h->tab.n_feat(), BT, h->tab.n_feat(), 16, 64) &&
          map2(&mQKVo, f->QKV, kTmF16, 3 * A + H, M, f->ldq, 32, 64);
@@ -436,9 +445,10 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     if (i > 0) { p.res_ss = f->ssx; p.res_gain = f->tr[i - 1].gout; }  // the previous output norm
     gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p, &mXo, &mXho);
 
-    p = base_params(h, M, D, kBnWide, f->g_ff1, 1, cdiv(FF, kBnWide));
+    p = base_params(h, M, D, kBnWide, f->g_ff1, 1, cdiv(F1, kBnWide));
     p.ss_in = f->ss; p.bias = w.b1; p.out_h = f->Hh; p.ldo = FF;
-    gemm(h, "gemm_ff1_gelu", kTcGelu, mXh, mW1, p, &mHo);
+    if (c.ff_act == 1) gemm(h, "gemm_ff1_geglu", kTcGeglu, mXh, mW1, p, &mHo16);
+    else gemm(h, "gemm_ff1_gelu", kTcGelu, mXh, mW1, p, &mHo);
 
     cudaMemsetAsync(f->ssx, 0, sizeof(float) * M, st);
     cudaMemsetAsync(f->ssg, 0, sizeof(float) * M, st);

@@ -92,4 +92,13 @@ std::string build_band_tables(int sr, int n_fft, int nb, int C, bool zero_dc, Ba
   return "";
 }
 
+std::vector<float> interleave_halves(const std::vector<float> &w, int half_rows, int cols) {
+  std::vector<float> out(w.size());
+  for (int r = 0; r < half_rows; ++r)
+    for (int h = 0; h < 2; ++h)
+      for (int c = 0; c < cols; ++c)
+        out[((size_t)2 * r + h) * cols + c] = w[((size_t)h * half_rows + r) * cols + c];
+  return out;
+}
+
 }  // namespace mrf

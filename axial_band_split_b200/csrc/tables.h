@@ -29,4 +29,8 @@ struct BandTables {
 std::string build_band_tables(int sample_rate, int n_fft, int n_bands, int channels, bool zero_dc,
                               BandTables *out);
 
+// Rows [v_0 .. v_{n-1}, g_0 .. g_{n-1}] (each `cols` wide) reordered as v_0, g_0, v_1, g_1, ...:
+// the GEGLU projection's value and gate halves paired for an epilogue that reads neighbours.
+std::vector<float> interleave_halves(const std::vector<float> &w, int half_rows, int cols);
+
 }  // namespace mrf

@@ -39,7 +39,7 @@ class mrf_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "sample_rate", "n_fft", "audio_channels", "num_bands", "dim", "depth", "heads", "dim_head",
         "ff_mult", "mask_hidden", "mask_depth", "num_stems", "zero_dc", "max_batch", "max_frames")] + \
-        [("rope_theta", ctypes.c_float), ("compute", ctypes.c_int)]
+        [("rope_theta", ctypes.c_float), ("compute", ctypes.c_int), ("ff_act", ctypes.c_int)]
 
 
 class mrf_tensor(ctypes.Structure):
@@ -114,6 +114,7 @@ def make_config(cfg, max_batch=1, max_frames=1100, compute=MRF_FP16):
     c.num_stems, c.zero_dc = cfg.num_stems, int(cfg.zero_dc)
     c.max_batch, c.max_frames = max_batch, max_frames
     c.rope_theta, c.compute = cfg.rope_theta, compute
+    c.ff_act = getattr(cfg, "ff_act", 0)
     return c
 
 

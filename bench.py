@@ -335,8 +335,8 @@ def run_ours(args):
         peak = peaks["hbm_gbs"]
         achieved = amount / nl / (avg_ms / 1e3) / 1e9
     attn_ms = sum(kt[k][1] for k in ("attn_time_tc", "attn_band_tc") if k in kt) / args.steps
-    # dense projections: the GEMM launches and the fused feed-forward, as this forward ran them
-    gemm_names = [k for k in kt if (k.startswith("gemm_") or k == "mlp_ff") and k in work]
+    # dense projections: the GEMM launches this forward ran
+    gemm_names = [k for k in kt if k.startswith("gemm_") and k in work]
     gemm_ms = sum(kt[k][1] for k in gemm_names) / args.steps
     attn_fl = accounting.attention_flops(cfg, widths, B, T)
     gemm_fl = sum(work[k][1] for k in gemm_names)

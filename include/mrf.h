@@ -67,6 +67,9 @@ typedef struct {
   int max_frames;
   float rope_theta;      /* 10000 */
   int compute;           /* mrf_compute */
+  int ff_act;            /* feed-forward activation: 0 GELU (the pages' models); 1 GEGLU, a variant
+                            whose first projection is [2*ff, dim] with halves (value, gate) and
+                            whose hidden is value * gelu(gate) */
 } mrf_config;
 
 /* One named weight, PyTorch [out, in] layout, contiguous, in host memory. */

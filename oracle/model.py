@@ -108,19 +108,26 @@ def attention(x, w, heads: int, dim_head: int, theta: float):
     return out
 
 
-def feed_forward(x, w):
-    """norm -> Linear(D, FF) + b -> GELU -> Linear(FF, D) + b."""
+def feed_forward(x, w, ff_act: int = 0):
+    """norm -> Linear(D, FF) + b -> GELU -> Linear(FF, D) + b.  ff_act 1 (the GEGLU variant):
+    the first projection is Linear(D, 2 FF) and its halves combine as value * GELU(gate), the
+    first half the value (Shazeer, "GLU Variants Improve Transformer", 2020)."""
     a = rms_norm(x, w["net.0.gamma"])
-    h = gelu(a @ w["net.1.weight"].T + w["net.1.bias"])
+    y = a @ w["net.1.weight"].T + w["net.1.bias"]
+    if ff_act == 1:
+        value, gate = np.split(y, 2, axis=-1)
+        h = value * gelu(gate)
+    else:
+        h = gelu(y)
     return h @ w["net.4.weight"].T + w["net.4.bias"]
 
 
-def transformer(x, w, heads, dim_head, theta):
+def transformer(x, w, heads, dim_head, theta, ff_act: int = 0):
     """x += attn(x); x += ff(x); return norm_out(x).  x (S, n, D)."""
     aw = {k[len("layers.0.0."):]: v for k, v in w.items() if k.startswith("layers.0.0.")}
     fw = {k[len("layers.0.1."):]: v for k, v in w.items() if k.startswith("layers.0.1.")}
     x = attention(x, aw, heads, dim_head, theta) + x
-    x = feed_forward(x, fw) + x
+    x = feed_forward(x, fw, ff_act) + x
     return rms_norm(x, w["norm.gamma"])
 
 
@@ -199,10 +206,11 @@ def forward(stft_repr, cfg, weights, dtype=np.float64, return_stages: bool = Fal
         for l in range(cfg.depth):
             tw = _sub(W, f"layers.{l}.0.")
             bw = _sub(W, f"layers.{l}.1.")
+            ff_act = getattr(cfg, "ff_act", 0)
             X = np.transpose(transformer(np.transpose(X, (1, 0, 2)), tw, cfg.heads,
-                                         cfg.dim_head, cfg.rope_theta), (1, 0, 2))
+                                         cfg.dim_head, cfg.rope_theta, ff_act), (1, 0, 2))
             st[f"layer{l}.time"] = X.copy()
-            X = transformer(X, bw, cfg.heads, cfg.dim_head, cfg.rope_theta)
+            X = transformer(X, bw, cfg.heads, cfg.dim_head, cfg.rope_theta, ff_act)
             st[f"layer{l}.band"] = X.copy()
         per_stem = []
         for s in range(cfg.num_stems):
@@ -223,7 +231,8 @@ def param_count(cfg, widths):
     FF = D * cfg.ff_mult
     MH = D * cfg.mask_hidden_mult
     n = sum(w + D * w + D for w in widths)
-    per_tr = (D + 3 * A * D + H * D + H + D * A) + (D + FF * D + FF + D * FF + D) + D
+    F1 = 2 * FF if getattr(cfg, "ff_act", 0) == 1 else FF   # GEGLU: value and gate halves
+    per_tr = (D + 3 * A * D + H * D + H + D * A) + (D + F1 * D + F1 + D * FF + D) + D
     n += 2 * cfg.depth * per_tr
     for _ in range(cfg.num_stems):
         for w in widths:
@@ -246,7 +255,7 @@ def mac_count(cfg, widths, B: int, T: int):
         "qkv": L * tok * D * 3 * A,
         "gates": L * tok * D * H,
         "out": L * tok * A * D,
-        "ff1": L * tok * D * FF,
+        "ff1": L * tok * D * FF * (2 if getattr(cfg, "ff_act", 0) == 1 else 1),
         "ff2": L * tok * FF * D,
     }
     attn_time = L * (B * nb * H) * 2 * T * T * dh

@@ -45,6 +45,7 @@ class ModelConfig:
     heads: int = 8
     dim_head: int = 64
     ff_mult: int = 4
+    ff_act: int = 0            # feed-forward activation: 0 GELU (the pages), 1 GEGLU (variant)
     mask_hidden_mult: int = 4
     mask_depth: int = 2
     num_stems: int = 1
@@ -115,7 +116,8 @@ def weight_shapes(cfg: ModelConfig, widths):
                     (q + "to_gates.weight", (H, D)), (q + "to_gates.bias", (H,)),
                     (q + "to_out.0.weight", (D, A))]
             f = p + "layers.0.1.net."
-            out += [(f + "0.gamma", (D,)), (f + "1.weight", (FF, D)), (f + "1.bias", (FF,)),
+            F1 = 2 * FF if cfg.ff_act == 1 else FF  # GEGLU: value and gate halves
+            out += [(f + "0.gamma", (D,)), (f + "1.weight", (F1, D)), (f + "1.bias", (F1,)),
                     (f + "4.weight", (D, FF)), (f + "4.bias", (D,))]
             out += [(p + "norm.gamma", (D,))]
     for s in range(cfg.num_stems):

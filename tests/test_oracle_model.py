@@ -327,3 +327,34 @@ def test_stems_share_the_trunk():
     assert two.shape == (1, 2) + x.shape[1:]
     assert np.array_equal(two[:, 0], one)
     assert not np.allclose(two[:, 1], one)
+
+
+def test_geglu_with_unit_value_half_is_the_gelu_block():
+    # GEGLU(y) = value * GELU(gate): with the value half's weights 0 and biases 1 the block is
+    # the GELU block whose first projection is the gate half (a swapped or missing half fails)
+    import dataclasses
+    cfg, W, x = tiny_case(T=5)
+    g = dataclasses.replace(cfg, ff_act=1)
+    widths = tables.band_tables(44100, 256, 8)["widths"]
+    Wg = synth.make_weights(g, widths, seed=0, fp16=False)
+    Wp = dict(Wg)
+    FF = cfg.dim * cfg.ff_mult
+    for l in range(cfg.depth):
+        for a in range(2):
+            p = f"layers.{l}.{a}.layers.0.1.net.1."
+            w, b = Wg[p + "weight"].copy(), Wg[p + "bias"].copy()
+            w[:FF] = 0.0
+            b[:FF] = 1.0
+            Wg[p + "weight"], Wg[p + "bias"] = w, b
+            Wp[p + "weight"], Wp[p + "bias"] = w[FF:], b[FF:]
+    assert np.allclose(model.forward(x, g, Wg), model.forward(x, cfg, Wp), rtol=0, atol=1e-12)
+
+
+def test_geglu_parameter_count():
+    # the first projection doubles: 2 * (D * FF + FF) more per transformer
+    import dataclasses
+    widths = tables.band_tables(44100, 2048, 60)["widths"]
+    base = model.param_count(synth.VOCALS, widths)
+    g = model.param_count(dataclasses.replace(synth.VOCALS, ff_act=1), widths)
+    D, FF = 384, 1536
+    assert g - base == 2 * 6 * (D * FF + FF) and g == 235_299_108

@@ -100,3 +100,25 @@ def test_zero_dc_masks():
     got16 = run(cfg, W16, x, mrf.MRF_FP16, max_frames=40)
     check16(got16, oracle_model.forward(x, cfg, W16), "tiny zero_dc")
     assert np.abs(got16[:, : cfg.audio_channels]).max() == 0
+
+
+@pytest.mark.parametrize("B,T", [(1, 32), (2, 17)])
+def test_geglu_tiny_fp32_and_fp16(B, T):
+    # ff_act 1: the first feed-forward projection is [2 ff, dim], hidden = value * gelu(gate)
+    from axial_band_split_b200 import mrf
+    cfg = dataclasses.replace(synth.TINY, ff_act=1)
+    W32, x = case(cfg, B, T, False)
+    got32 = run(cfg, W32, x, mrf.MRF_FP32_DEBUG, max_batch=2, max_frames=40)
+    assert rel_err(got32, oracle_model.forward(x, cfg, W32)) <= 1e-4
+    W16, _ = case(cfg, B, T, True)
+    got16 = run(cfg, W16, x, mrf.MRF_FP16, max_batch=2, max_frames=40)
+    check16(got16, oracle_model.forward(x, cfg, W16), f"tiny GEGLU B={B} T={T}")
+
+
+def test_geglu_vocals_depth1_fp16():
+    from axial_band_split_b200 import mrf
+    cfg = dataclasses.replace(synth.VOCALS, depth=1, ff_act=1)
+    B, T = 1, 150
+    W, x = case(cfg, B, T, True)
+    got = run(cfg, W, x, mrf.MRF_FP16)
+    check16(got, oracle_model.forward(x, cfg, W), "vocals depth 1 GEGLU")
