@@ -47,7 +47,8 @@ def test_istft_inverts_stft():
 
 
 def test_chunk_counts_follow_the_pages_formula():
-    # section "Verified inference hot path": n_chunks(d) = len(range(0, L, 317520)), L = 44100 d
+    # "Mel-Band RoFormer — ...", section "The chunking arithmetic": n_chunks(d) = len(range(0, L,
+    # 317520)), L = 44100 d
     # plus 2 * 35280 of reflect padding when 44100 d > 70560
     for d in (1.0, 1.7, 5.0, 8.0, 16.0, 60.0, 120.0):
         L = int(44100 * d)
