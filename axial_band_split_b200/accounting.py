@@ -39,8 +39,6 @@ def kernel_work(cfg, widths, B: int, T: int):
         "gemm_band_split": ("flop", 2 * BT * D * n_feat, 1),
         # stft_repr read once, normalised fp16 band features written once
         "band_gather": ("byte", B * rows * T * 2 * 4 + BT * n_feat * 2, 1),
-        # x fp32 read + write, x fp16 write, |x|^2 read + write, gain
-        "outnorm": ("byte", L2 * NT * (D * 4 * 2 + D * 2 + 8), L2),
         # per stem: mask features fp32 read once, masks fp32 written once
         "overlap_average": ("byte", S * (BT * n_feat * 4 + B * rows * T * 2 * 4), S),
     }

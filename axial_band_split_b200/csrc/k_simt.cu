@@ -391,33 +391,6 @@ __global__ void attention_tokmajor_kernel(const __half *__restrict__ qkv, int ld
   if (lane + 32 < dh) orow[lane + 32] = __float2half_rn(o1 * g);
 }
 
-// ------------------------------------------------------------------ output norm (fp16 schedule)
-// x = x / max(sqrt(ss), eps) * gain; writes x (fp32), its fp16 copy and the new sum of squares.
-__global__ void outnorm_kernel(float *__restrict__ x, float *__restrict__ ss, const float *__restrict__ gain,
-                               __half *__restrict__ xh, long long rows, int D) {
-  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const float r = 1.f / fmaxf(sqrtf(ss[row]), kNormEps);
-  float *xr = x + row * D;
-  __half *hr = xh + row * D;
-  float s = 0.f;
-  for (int j = lane * 4; j < D; j += 128) {
-    float4 a = *reinterpret_cast<float4 *>(xr + j);
-    const float4 g = *reinterpret_cast<const float4 *>(gain + j);
-    a.x *= r * g.x; a.y *= r * g.y; a.z *= r * g.z; a.w *= r * g.w;
-    *reinterpret_cast<float4 *>(xr + j) = a;
-    __half2 h0 = __floats2half2_rn(a.x, a.y), h1 = __floats2half2_rn(a.z, a.w);
-    uint2 u;
-    u.x = *reinterpret_cast<uint32_t *>(&h0);
-    u.y = *reinterpret_cast<uint32_t *>(&h1);
-    *reinterpret_cast<uint2 *>(hr + j) = u;
-    s += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
-  }
-  s = warp_sum(s);
-  if (lane == 0) ss[row] = s;
-}
-
 // ------------------------------------------------------------------ overlap average
 // masks[b, r, t, c] = wrow[r] * (m[b, t, src0] + m[b, t, src1]) written at out + b * out_bstride
 // + (r T + t) 2 + c; with `spec` (stft_repr [B, R, T, 2]) the complex product of the mask and
@@ -516,10 +489,6 @@ void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int 
   attention_tokmajor_kernel<<<grid1(rows, 8), 256, 0, st>>>(qkv, ld, o, B, T, nb, heads, dh, axis);
 }
 
-void launch_outnorm(float *x, float *ss, const float *gain, __half *xh, long long rows, int D,
-                    cudaStream_t st) {
-  outnorm_kernel<<<grid1(rows, 8), 256, 0, st>>>(x, ss, gain, xh, rows, D);
-}
 
 void launch_overlap_average(const float *m, int ldm, const int32_t *src0, const int32_t *src1,
                             const float *row_weight, float *masks, long long out_bstride, const float *spec,

@@ -75,9 +75,6 @@ void launch_attention_f32(const float *q, const float *k, const float *v, const 
 void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int T, int nb, int heads, int dh,
                                int axis, cudaStream_t st);
 
-// x = x / max(sqrt(ss), eps) * gain (D % 128 == 0); writes x, its fp16 copy and ss = |x|^2.
-void launch_outnorm(float *x, float *ss, const float *gain, __half *xh, long long rows, int D,
-                    cudaStream_t st);
 
 // masks[b, r, t, c] = row_weight[r] * sum of the (<= 2) source features of (r, c)
 // ------------------------------------------------------------------ spectral front / back end (k_signal.cu)
