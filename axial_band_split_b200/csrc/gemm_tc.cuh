@@ -31,6 +31,7 @@ enum GemmEpi : int {
 
 struct GemmParams {
   int M, K, BN, ngroups, total_n_tiles, a_mode, m_tiles;
+  int stall_test;  // test hook: CTA 0's loads never arrive, so its bounded waits expire
   const GemmGroup *groups;
   unsigned *status;
   // epilogue

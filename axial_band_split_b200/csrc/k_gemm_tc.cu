@@ -203,7 +203,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
 
   if (warp == kEpiWarps) {
     // ---------------- TMA producer
-    if (lane == 0) {
+    // (stall test: CTA 0 loads nothing, a flag nobody sets; its MMA and epilogue waits expire
+    // after their bounded limit, record the site and return)
+    if (lane == 0 && !(p.stall_test && blockIdx.x == 0)) {
       int stage = 0;
       uint32_t phase = 0;
       const uint32_t bytes = A_STAGE + p.BN * BK * 2;

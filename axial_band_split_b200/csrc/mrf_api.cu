@@ -528,7 +528,7 @@ mrf_status forward_impl(mrf_handle *h, const float *in, float *out, int B, int T
   cudaGetLastError();
   mrf_status s = MRF_OK;
   h->apply_masks = apply;
-  if (h->timing || !h->use_graph) {
+  if (h->timing || !h->use_graph || h->stall_test) {  // a stalled forward is never recorded into a graph
     h->cur_stream = st;
     run_schedule(h, in, out, B, T);
     if (!h->sched_error.empty()) return fail(h, MRF_ECUDA, h->sched_error);
@@ -665,6 +665,13 @@ mrf_status mrf_kernel_times(mrf_handle *h, mrf_kernel_time *out, int max_n, int 
   h->pending.clear();
   *n_out = (int)acc.size();
   for (int i = 0; i < (int)acc.size() && i < max_n && out; ++i) out[i] = acc[i];
+  return MRF_OK;
+}
+
+mrf_status mrf_debug_stall_next(mrf_handle *h) {
+  if (!h) return fail(nullptr, MRF_EINVAL, "null handle");
+  if (h->cfg.compute != MRF_FP16) return fail(h, MRF_EUNSUPPORTED, "the stall test runs the fp16 schedule");
+  h->stall_test = true;  // consumed by the next forward, which runs eagerly
   return MRF_OK;
 }
 

@@ -96,6 +96,7 @@ struct mrf_handle {
   // execution
   bool timing = false, use_graph = true;
   bool apply_masks = false;  // the schedule being recorded multiplies stft_repr by the masks
+  bool stall_test = false;   // test hook: the next fp16 schedule's first GEMM stalls (bounded)
   cudaStream_t cur_stream = nullptr, cap_stream = nullptr;
   std::vector<mrf::PendingTiming> pending;
   std::vector<mrf::GraphEntry> graphs;

@@ -411,6 +411,8 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   {
     GemmParams p = base_params(h, B * T, f->k_bs, kBnNarrow, f->g_bs, nb, nb * cdiv(D, kBnNarrow));
     p.bias = h->b_bs; p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ssg; p.ld = D; p.nb = nb;
+    p.stall_test = h->stall_test ? 1 : 0;
+    h->stall_test = false;
     gemm(h, "gemm_band_split", kTcBandSplit, mAbs, mWbs, p, &mXbs, &mXhbs);
   }
 

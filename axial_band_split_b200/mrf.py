@@ -26,7 +26,8 @@ STATUS = {0: "MRF_OK", -1: "MRF_EINVAL", -2: "MRF_ESHAPE", -3: "MRF_ENOMEM", -4:
 EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_separate", "mrf_stft", "mrf_istft", "mrf_separate_audio",
            "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
            "mrf_last_error", "mrf_band_tables", "mrf_set_timing", "mrf_kernel_times",
-           "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer", "mrf_forward_static"]
+           "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer", "mrf_forward_static",
+           "mrf_debug_stall_next"]
 
 
 class MrfError(RuntimeError):
@@ -94,6 +95,8 @@ def lib():
         L.mrf_kernel_times.restype = I
         L.mrf_debug_buffer.argtypes = [P, ctypes.c_char_p, P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)]
         L.mrf_debug_buffer.restype = I
+        L.mrf_debug_stall_next.argtypes = [P]
+        L.mrf_debug_stall_next.restype = I
         L.mrf_launches_per_forward.argtypes = [P, I, I]
         L.mrf_launches_per_forward.restype = I
         _lib = L
@@ -292,6 +295,10 @@ class Model:
         _check(lib().mrf_debug_buffer(self._h, name.encode(), out.ctypes.data_as(ctypes.c_void_p),
                                       out.nbytes, ctypes.byref(n)), self._h)
         return out[: n.value // 4]
+
+    def debug_stall_next(self):
+        """mrf_debug_stall_next: the next fp16 forward's first GEMM lets its bounded waits expire."""
+        _check(lib().mrf_debug_stall_next(self._h), self._h)
 
     def launches_per_forward(self, B, T):
         return lib().mrf_launches_per_forward(self._h, B, T)

@@ -58,6 +58,46 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
 
+class RankGroup:
+    """The ranks of a replicas run, one process per GPU: a barrier, the maximum of a number over
+    the ranks (the slowest rank's device time) and the teardown.  No collective touches the data
+    path.  Backend NCCL on GPUs; gloo for the CPU tests of this plumbing.  The group's timeout is
+    short, so a rank that fails or leaves ends the others' next collective with an error."""
+
+    def __init__(self, backend="nccl", timeout_s=120):
+        self.rank, self.world, self.local = dist_env()
+        self.backend = backend
+        self._dist = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+            self._dist = dist
+
+    def barrier(self):
+        if self._dist is not None:
+            self._dist.barrier()
+
+    def max(self, value):
+        if self._dist is None:
+            return float(value)
+        import torch
+        t = torch.tensor([float(value)], dtype=torch.float64, device="cuda" if self.backend == "nccl" else "cpu")
+        self._dist.all_reduce(t, op=self._dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self._dist is not None:
+            self._dist.barrier()
+            self._dist.destroy_process_group()
+            self._dist = None
+
+
+def aggregate(units_per_rank, world, ms_max):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time (ms)."""
+    return world * units_per_rank / (ms_max / 1e3)
+
+
 def workload(cfg, B, T):
     return {"workload": f"vocals core forward, B={B}, T={T} ({B * T * cfg.hop / cfg.sample_rate:.2f} s audio)",
             "dim": cfg.dim, "depth": cfg.depth, "heads": cfg.heads, "dim_head": cfg.dim_head,
@@ -220,15 +260,11 @@ def run_ours(args):
     import torch
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    ranks = RankGroup("nccl")
     from axial_band_split_b200 import accounting, build, mrf
     if rank == 0:
         build.build()
-    if world > 1:
-        dist.barrier()
+    ranks.barrier()
     import synth
     cfg = synth.VOCALS
     B, T = args.batch, args.frames
@@ -242,8 +278,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     def barrier():
-        if world > 1:
-            torch.distributed.barrier()
+        ranks.barrier()
         torch.cuda.synchronize()
 
     def timed(fn, steps):
@@ -266,6 +301,7 @@ def run_ours(args):
         model.sync_status()
         torch.cuda.synchronize()
         print(f"plain run ok: {args.warmup + args.steps} forwards, {model.launches_per_forward(B, T)} launches each")
+        ranks.close()
         model.close()
         return 0
     for _ in range(args.warmup):
@@ -274,14 +310,10 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         ms = timed(fwd, args.steps)
     model.sync_status()
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = ranks.max(ms)
     launches = model.launches_per_forward(B, T)
-    audio_total = world * args.steps * accounting.audio_seconds(cfg, B, T)
-    value = audio_total / (ms_max / 1e3)
+    audio_per_rank = args.steps * accounting.audio_seconds(cfg, B, T)
+    value = aggregate(audio_per_rank, world, ms_max)
 
     # per-kernel times: the same steps launched eagerly with an event pair around each kernel
     model.set_timing(True)
@@ -295,17 +327,12 @@ def run_ours(args):
     xout = torch.empty_like(xin).pin_memory()
     e2e_fn = lambda: model.forward_host(xin, xout, stream=stream)
     e2e_fn()
-    ms_e2e = timed(e2e_fn, args.steps)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = ranks.max(timed(e2e_fn, args.steps))
     io_bytes = int(x_host.nbytes)
 
     if rank != 0:
-        if world > 1:
-            torch.distributed.barrier()
-            torch.distributed.destroy_process_group()
+        ranks.close()
+        model.close()
         return 0
 
     peaks, peak_src = load_peaks()
@@ -358,7 +385,7 @@ def run_ours(args):
                     "frac_of_peak_burst": total_fl / (ms_max / args.steps / 1e3) / 1e12 / peaks["bf16_tflops"]},
         "kernels": per_kernel,
         "kernel_timing_ms_per_step": ktimed / args.steps,
-        "e2e": {"value": world * args.steps * accounting.audio_seconds(cfg, B, T) / (ms_e2e / 1e3), "unit": UNIT,
+        "e2e": {"value": aggregate(audio_per_rank, world, ms_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
@@ -366,9 +393,7 @@ def run_ours(args):
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, args.cpu_sample_frames, rank)
     print(json.dumps(line), flush=True)
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    ranks.close()
     model.close()
     return 0
 

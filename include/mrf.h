@@ -231,6 +231,16 @@ mrf_status mrf_kernel_times(mrf_handle *h, mrf_kernel_time *out, int max_n, int 
 mrf_status mrf_set_graph(mrf_handle *h, int enable);
 
 /*
+ * mrf_debug_stall_next - test hook of the failure path: in the next fp16 forward, CTA 0 of the
+ * first tensor-core GEMM issues no loads (a flag nothing sets), so its bounded waits expire
+ * (about 2 s), record their site in the device status word and return; the forward's other
+ * work runs on.  mrf_sync_status then returns MRF_ETIMEOUT and clears the status word, and the
+ * handle stays usable.  The stalled forward runs without a CUDA graph, so no captured graph
+ * holds the stall.  No fault, trap or hang is involved.
+ */
+mrf_status mrf_debug_stall_next(mrf_handle *h);
+
+/*
  * mrf_debug_buffer - test hook: wait for the device, then copy the start of an internal
  * buffer of the last forward to host memory.  "X": the residual stream after the last
  * transformer, float32 [B*T*num_bands, dim], token (b*T + t)*num_bands + k; "M": the mask
