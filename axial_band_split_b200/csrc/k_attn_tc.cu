@@ -268,19 +268,16 @@ __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t
     md = max3(md, sv[3 * Q + i], sv[3 * Q + i2]);
   }
   const float m_cand = fmaxf(m_run, fmaxf(fmaxf(ma, mb), fmaxf(mc, md)));
-  // P_t and O_t are free once the previous block's P*V has completed
-  if (wait_pv && !tc::mbar_wait(pv_done, pv_parity, status, 39, abort)) return false;
   const bool need = m_cand > m_run + kRescaleLog2;
-  const bool any_need = __any_sync(0xffffffffu, need);
   const float alpha = need ? ex2(m_run - m_cand) : 1.f;
   if (need) { l *= alpha; m_run = m_cand; }
-  // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU, and P into
-  // tensor memory two fp16 per column, four columns (8 keys) per store
+  // p = 2^(s - m) in place of the scores: pairs through packed f32x2 subtract, exponentials
+  // on MUFU.  This needs neither P_t nor O_t, so it runs before the wait for the previous
+  // block's P*V, which then overlaps it.
   float2 sa = make_float2(0.f, 0.f), sb = sa, sc = sa, sd = sa;  // four independent sum chains
   const float2 negm = make_float2(-m_run, -m_run);
 #pragma unroll
   for (int i = 0; i < NC; i += 8) {
-    uint32_t hh[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float2 d = add2(make_float2(sv[i + 2 * u], sv[i + 2 * u + 1]), negm);
@@ -291,16 +288,24 @@ __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t
         case 2: sc = add2(sc, pp); break;
         default: sd = add2(sd, pp); break;
       }
-      hh[u] = pack_h2(pp.x, pp.y);
+      sv[i + 2 * u] = pp.x;
+      sv[i + 2 * u + 1] = pp.y;
     }
-    tmem_st4(tP + (i >> 1), hh[0], hh[1], hh[2], hh[3]);
   }
+  // P_t and O_t are free once the previous block's P*V has completed
+  if (wait_pv && !tc::mbar_wait(pv_done, pv_parity, status, 39, abort)) return false;
+  tc::tc_fence_after();
+  const bool any_need = __any_sync(0xffffffffu, need);
+  // P into tensor memory, two fp16 per column, four columns (8 keys) per store
+#pragma unroll
+  for (int i = 0; i < NC; i += 8)
+    tmem_st4(tP + (i >> 1), pack_h2(sv[i], sv[i + 1]), pack_h2(sv[i + 2], sv[i + 3]), pack_h2(sv[i + 4], sv[i + 5]),
+             pack_h2(sv[i + 6], sv[i + 7]));
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
   const float2 s01 = add2(sa, sb), s23 = add2(sc, sd);
   const float2 s4 = add2(s01, s23);
   // O row rescaled in place when this row's max was raised
   if (any_need && wait_pv) {
-    tc::tc_fence_after();
 #pragma unroll
     for (int c = 0; c < kDh; c += 32) {
       float v[32];

@@ -24,33 +24,33 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigne
   return d;
 }
 
-// GELU of y0 = v0 * rs + b0 and y1 = v1 * rs + b1, y * (1 + erf(y / sqrt 2)) / 2, with the
-// erf of Abramowitz & Stegun 7.1.26 (|error| <= 1.5e-7), branch-free:
-// erf(z) = 1 - t (a1 + t (a2 + t (a3 + t (a4 + t a5)))) exp(-z^2), t = 1 / (1 + p z), z >= 0;
-// the polynomial and the scalings in packed pairs.
+// GELU of y0 = v0 * rs + b0 and y1 = v1 * rs + b1, y * (1 + erf(y / sqrt 2)) / 2.  The
+// complementary error function of z = |y| / sqrt 2 comes from Abramowitz & Stegun 7.1.28,
+// erfc(z) = (1 + a1 z + ... + a6 z^6)^-16 (|error| <= 3e-7), one reciprocal per value (the
+// power by four squarings; it overflows to inf for large z, whose reciprocal is 0).  Then
+// 1 + erf(y / sqrt 2) = 2 - erfc for y >= 0 and erfc for y < 0, so no cancellation on the
+// negative side.  The polynomial and the scalings run in packed pairs.
 __device__ __forceinline__ float2 gelu2(float v0, float v1, float rs, float b0, float b1) {
   const unsigned long long y = fma2(f2_pack(v0, v1), f2_pack(rs, rs), f2_pack(b0, b1));
   const float2 yy = f2_unpack(y);
   const unsigned long long z = mul2(f2_pack(fabsf(yy.x), fabsf(yy.y)), f2_pack(0.70710678118654752f, 0.70710678118654752f));
-  const unsigned long long den = fma2(z, f2_pack(0.3275911f, 0.3275911f), f2_pack(1.f, 1.f));
-  const float2 dd = f2_unpack(den);
-  float t0, t1;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t0) : "f"(dd.x));
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t1) : "f"(dd.y));
-  const unsigned long long t = f2_pack(t0, t1);
-  unsigned long long poly = fma2(t, f2_pack(1.061405429f, 1.061405429f), f2_pack(-1.453152027f, -1.453152027f));
-  poly = fma2(t, poly, f2_pack(1.421413741f, 1.421413741f));
-  poly = fma2(t, poly, f2_pack(-0.284496736f, -0.284496736f));
-  poly = fma2(t, poly, f2_pack(0.254829592f, 0.254829592f));
-  poly = mul2(poly, t);
-  const float2 ez = f2_unpack(mul2(mul2(z, z), f2_pack(-1.4426950408889634f, -1.4426950408889634f)));
-  float e0, e1;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(ez.x));
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(ez.y));
-  const float2 er = f2_unpack(fma2(poly, f2_pack(-e0, -e1), f2_pack(1.f, 1.f)));   // erf(|y| / sqrt 2)
-  const unsigned long long h = mul2(y, f2_pack(0.5f, 0.5f));
-  const float2 g = f2_unpack(fma2(h, f2_pack(copysignf(er.x, yy.x), copysignf(er.y, yy.y)), h));
-  return g;
+  unsigned long long p = fma2(z, f2_pack(0.0000430638f, 0.0000430638f), f2_pack(0.0002765672f, 0.0002765672f));
+  p = fma2(z, p, f2_pack(0.0001520143f, 0.0001520143f));
+  p = fma2(z, p, f2_pack(0.0092705272f, 0.0092705272f));
+  p = fma2(z, p, f2_pack(0.0422820123f, 0.0422820123f));
+  p = fma2(z, p, f2_pack(0.0705230784f, 0.0705230784f));
+  p = fma2(z, p, f2_pack(1.f, 1.f));
+  p = mul2(p, p);
+  p = mul2(p, p);
+  p = mul2(p, p);
+  p = mul2(p, p);
+  const float2 pp = f2_unpack(p);
+  float r0, r1;  // erfc(|y| / sqrt 2)
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(pp.x));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r1) : "f"(pp.y));
+  const float2 two_minus = f2_unpack(fma2(f2_pack(r0, r1), f2_pack(-1.f, -1.f), f2_pack(2.f, 2.f)));
+  const unsigned long long q = f2_pack(yy.x >= 0.f ? two_minus.x : r0, yy.y >= 0.f ? two_minus.y : r1);
+  return f2_unpack(mul2(mul2(y, f2_pack(0.5f, 0.5f)), q));
 }
 
 }  // namespace tcm
