@@ -284,10 +284,16 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       if (EPI == kTcQkv) {
         qr_pf = qkv_row(p, v_ ? m_ : 0, t_.g);
         ss_pf = (v_ && p.ss_in) ? p.ss_in[qr_pf.tok] : 1.f;
-        if (p.dh == 64) {
-          const float2 *rp = p.rope + (long long)qr_pf.pos * 32 + (sub & 1) * 16;
+        // rotary pairs only for q and k column blocks; 16-byte loads (a row's 16 pairs are
+        // 128 contiguous bytes at a 128-byte offset of the table's 256-byte row)
+        if (p.dh == 64 && t_.nblk * p.BN < 2 * p.A) {
+          const float4 *rp = reinterpret_cast<const float4 *>(p.rope + (long long)qr_pf.pos * 32 + (sub & 1) * 16);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) cs_pf[i] = rp[i];
+          for (int i = 0; i < 8; ++i) {
+            const float4 w = rp[i];
+            cs_pf[2 * i] = make_float2(w.x, w.y);
+            cs_pf[2 * i + 1] = make_float2(w.z, w.w);
+          }
         }
       } else if (EPI == kTcGelu || EPI == kTcGeglu) {
         ss_pf = (v_ && p.ss_in) ? p.ss_in[m_] : 1.f;
