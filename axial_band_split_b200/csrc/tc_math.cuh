@@ -24,33 +24,34 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigne
   return d;
 }
 
-// GELU of y0 = v0 * rs + b0 and y1 = v1 * rs + b1, y * (1 + erf(y / sqrt 2)) / 2.  The
-// complementary error function of z = |y| / sqrt 2 comes from Abramowitz & Stegun 7.1.28,
-// erfc(z) = (1 + a1 z + ... + a6 z^6)^-16 (|error| <= 3e-7), one reciprocal per value (the
-// power by four squarings; it overflows to inf for large z, whose reciprocal is 0).  Then
-// 1 + erf(y / sqrt 2) = 2 - erfc for y >= 0 and erfc for y < 0, so no cancellation on the
-// negative side.  The polynomial and the scalings run in packed pairs.
+// GELU of y0 = v0 * rs + b0 and y1 = v1 * rs + b1, y * (1 + erf(y / sqrt 2)) / 2, written
+// as max(y, 0) - |y| * erfc(|y| / sqrt 2) / 2 (both signs of y).  The complementary error
+// function comes from Abramowitz & Stegun 7.1.28, erfc(z) = (1 + a1 z + ... + a6 z^6)^-16
+// (|error| <= 3e-7): one reciprocal per value, the power by four squarings (it overflows to inf
+// for large z, whose reciprocal is 0).  The polynomial is evaluated in w = -|y|: coefficient k
+// is a_k 2^(-k/2) (z = |y| / sqrt 2) times (-1)^k (the sign of w^k) times 2^(1/16) (so the
+// 16th power is doubled and its reciprocal is erfc / 2).  Packed pairs throughout.  (An
+// infinite y gives NaN; finite inputs never reach inf.)
 __device__ __forceinline__ float2 gelu2(float v0, float v1, float rs, float b0, float b1) {
   const unsigned long long y = fma2(f2_pack(v0, v1), f2_pack(rs, rs), f2_pack(b0, b1));
   const float2 yy = f2_unpack(y);
-  const unsigned long long z = mul2(f2_pack(fabsf(yy.x), fabsf(yy.y)), f2_pack(0.70710678118654752f, 0.70710678118654752f));
-  unsigned long long p = fma2(z, f2_pack(0.0000430638f, 0.0000430638f), f2_pack(0.0002765672f, 0.0002765672f));
-  p = fma2(z, p, f2_pack(0.0001520143f, 0.0001520143f));
-  p = fma2(z, p, f2_pack(0.0092705272f, 0.0092705272f));
-  p = fma2(z, p, f2_pack(0.0422820123f, 0.0422820123f));
-  p = fma2(z, p, f2_pack(0.0705230784f, 0.0705230784f));
-  p = fma2(z, p, f2_pack(1.f, 1.f));
-  p = mul2(p, p);
-  p = mul2(p, p);
-  p = mul2(p, p);
-  p = mul2(p, p);
-  const float2 pp = f2_unpack(p);
-  float r0, r1;  // erfc(|y| / sqrt 2)
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(pp.x));
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r1) : "f"(pp.y));
-  const float2 two_minus = f2_unpack(fma2(f2_pack(r0, r1), f2_pack(-1.f, -1.f), f2_pack(2.f, 2.f)));
-  const unsigned long long q = f2_pack(yy.x >= 0.f ? two_minus.x : r0, yy.y >= 0.f ? two_minus.y : r1);
-  return f2_unpack(mul2(mul2(y, f2_pack(0.5f, 0.5f)), q));
+  const unsigned long long w = f2_pack(-fabsf(yy.x), -fabsf(yy.y));
+  unsigned long long q = fma2(w, f2_pack(5.62129980608006e-06f, 5.62129980608006e-06f),
+                              f2_pack(-5.105520904180594e-05f, -5.105520904180594e-05f));
+  q = fma2(w, q, f2_pack(3.9686136005911976e-05f, 3.9686136005911976e-05f));
+  q = fma2(w, q, f2_pack(-0.003422739217057824f, -0.003422739217057824f));
+  q = fma2(w, q, f2_pack(0.02207699790596962f, 0.02207699790596962f));
+  q = fma2(w, q, f2_pack(-0.052075162529945374f, -0.052075162529945374f));
+  q = fma2(w, q, f2_pack(1.0442737340927124f, 1.0442737340927124f));
+  q = mul2(q, q);
+  q = mul2(q, q);
+  q = mul2(q, q);
+  q = mul2(q, q);
+  const float2 qq = f2_unpack(q);
+  float e0, e1;  // erfc(|y| / sqrt 2) / 2
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(qq.x));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(qq.y));
+  return f2_unpack(fma2(w, f2_pack(e0, e1), f2_pack(fmaxf(yy.x, 0.f), fmaxf(yy.y, 0.f))));
 }
 
 }  // namespace tcm
