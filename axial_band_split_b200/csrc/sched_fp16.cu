@@ -405,7 +405,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   }
 
   h->begin("band_gather");
-  launch_band_gather(in, h->d_feat_row, h->d_feat_c, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, h->max_width, st);
+  launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, h->max_width, st);
   h->end();
   cudaMemsetAsync(f->ssg, 0, sizeof(float) * M, st);
   {
