@@ -72,6 +72,33 @@ float *scratch(mrf_handle *h, size_t slot, size_t bytes) {
   return static_cast<float *>(e.first);
 }
 
+// The chunk loop's geometry for a mix of L samples ("Mel-Band RoFormer — ...", section
+// "Verified inference hot path"): 8 s chunks, stride 0.9 chunk, fades of chunk / 10, the mix
+// reflect-padded by the border chunk - stride when longer than two borders, a short last chunk
+// padded by reflection when more than half a chunk remains (mode 1), by zeros otherwise (2).
+struct ChunkGeometry {
+  int chunk, stride, fade, border, Lp;
+  bool padded;
+  std::vector<int> off, n, mode;
+};
+
+ChunkGeometry chunk_geometry(int sample_rate, int L) {
+  ChunkGeometry g;
+  g.chunk = sample_rate * 8;
+  g.stride = (int)(g.chunk * 0.9);
+  g.fade = g.chunk / 10;
+  g.border = g.chunk - g.stride;
+  g.padded = L > 2 * g.border;
+  g.Lp = g.padded ? L + 2 * g.border : L;
+  for (int o = 0; o < g.Lp; o += g.stride) {
+    const int nk = std::min(g.chunk, g.Lp - o);
+    g.off.push_back(o);
+    g.n.push_back(nk);
+    g.mode.push_back(nk == g.chunk ? 0 : (nk > g.chunk / 2 ? 1 : 2));
+  }
+  return g;
+}
+
 }  // namespace
 
 extern "C" {
@@ -113,16 +140,16 @@ mrf_status mrf_separate_audio(mrf_handle *h, const float *mix, float *stems, int
   if (!mix || !stems) return sfail(h, MRF_EINVAL, "null mix or stems pointer");
   const mrf_config &c = h->cfg;
   const int C = c.audio_channels, S = c.num_stems, n = c.n_fft;
-  // the chunk loop's geometry: 8 s chunks, stride 0.9 chunk, fades of chunk / 10, border
-  const int chunk = c.sample_rate * 8, stride = (int)(chunk * 0.9), fade = chunk / 10, border = chunk - stride;
   if (hop < 1 || L < 2) return sfail(h, MRF_ESHAPE, "hop >= 1 and L >= 2 required");
+  const ChunkGeometry g = chunk_geometry(c.sample_rate, L);
+  const int chunk = g.chunk, stride = g.stride, fade = g.fade, border = g.border;
   const int T = 1 + chunk / hop;
   if (T > c.max_frames) return sfail(h, MRF_ESHAPE, "max_frames is below the frames of one 8 s chunk");
   mrf_status s = ensure_tables(h);
   if (s != MRF_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool padded = L > 2 * border;
-  const int Lp = padded ? L + 2 * border : L;
+  const bool padded = g.padded;
+  const int Lp = g.Lp;
   const int nb_max = std::min(std::min(c.max_batch, 16), (Lp + stride - 1) / stride);
   const size_t F = (size_t)n / 2 + 1;
   float *xp = scratch(h, 1, (size_t)C * Lp * 4);
@@ -144,16 +171,14 @@ mrf_status mrf_separate_audio(mrf_handle *h, const float *mix, float *stems, int
     launch_pad_reflect(mix, xp, C, L, border, st);
     src = xp;
   }
-  std::vector<int> offs;
-  for (int off = 0; off < Lp; off += stride) offs.push_back(off);
+  const std::vector<int> &offs = g.off;
   for (size_t k0 = 0; k0 < offs.size(); k0 += nb_max) {
     ChunkBatch cb{};
     cb.count = (int)std::min<size_t>(nb_max, offs.size() - k0);
     for (int k = 0; k < cb.count; ++k) {
-      const int off = offs[k0 + k], nk = std::min(chunk, Lp - off);
-      cb.off[k] = off;
-      cb.n[k] = nk;
-      cb.reflect[k] = nk < chunk && nk > chunk / 2;
+      cb.off[k] = offs[k0 + k];
+      cb.n[k] = g.n[k0 + k];
+      cb.reflect[k] = g.mode[k0 + k] == 1;
     }
     launch_gather_chunks(src, chunks, cb, C, Lp, chunk, st);
     launch_stft(chunks, spec_in, h->d_tw, h->d_win, cb.count, C, chunk, T, log2_exact(n), hop, st);
@@ -167,6 +192,22 @@ mrf_status mrf_separate_audio(mrf_handle *h, const float *mix, float *stems, int
   launch_finalize(acc, counter, stems, S, C, Lp, L, padded ? border : 0, st);
   sok(h, cudaGetLastError(), "separation launches", &s);
   return s;
+}
+
+mrf_status mrf_chunk_plan(int sample_rate, int L, int *chunk, int *border, int *padded_length, int *n_chunks,
+                          int32_t *off, int32_t *valid, int32_t *mode, int max_chunks) {
+  if (sample_rate < 1 || L < 2 || !chunk || !border || !padded_length || !n_chunks) return MRF_EINVAL;
+  const ChunkGeometry g = chunk_geometry(sample_rate, L);
+  *chunk = g.chunk;
+  *border = g.padded ? g.border : 0;
+  *padded_length = g.Lp;
+  *n_chunks = (int)g.off.size();
+  for (int i = 0; i < (int)g.off.size() && i < max_chunks; ++i) {
+    if (off) off[i] = g.off[i];
+    if (valid) valid[i] = g.n[i];
+    if (mode) mode[i] = g.mode[i];
+  }
+  return MRF_OK;
 }
 
 }  // extern "C"

@@ -27,7 +27,7 @@ EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_separate", "mrf_stft", "mrf
            "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
            "mrf_last_error", "mrf_band_tables", "mrf_set_timing", "mrf_kernel_times",
            "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer", "mrf_forward_static",
-           "mrf_debug_stall_next"]
+           "mrf_debug_stall_next", "mrf_chunk_plan"]
 
 
 class MrfError(RuntimeError):
@@ -99,6 +99,9 @@ def lib():
         L.mrf_debug_stall_next.restype = I
         L.mrf_launches_per_forward.argtypes = [P, I, I]
         L.mrf_launches_per_forward.restype = I
+        IP = ctypes.POINTER(I)
+        L.mrf_chunk_plan.argtypes = [I, I, IP, IP, IP, IP, P, P, P, I]
+        L.mrf_chunk_plan.restype = I
         _lib = L
     return _lib
 
@@ -134,6 +137,21 @@ def band_tables(cfg):
     ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
     _check(lib().mrf_band_tables(ctypes.byref(c), ptr(out["first_bin"]), ptr(out["last_bin"]),
                                  ptr(out["width"]), ptr(out["feat_row"]), ptr(out["row_weight"]), None))
+    return out
+
+
+def chunk_plan(sample_rate, length):
+    """mrf_chunk_plan: the separation loop's geometry for a mix of `length` samples: dict with
+    chunk, border, padded_length and the per-chunk arrays off, valid, mode (0 full, 1 reflect
+    tail, 2 zero tail)."""
+    vals = [ctypes.c_int(0) for _ in range(4)]
+    _check(lib().mrf_chunk_plan(sample_rate, length, *[ctypes.byref(v) for v in vals], None, None, None, 0))
+    n = vals[3].value
+    out = {k: np.zeros(n, np.int32) for k in ("off", "valid", "mode")}
+    ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _check(lib().mrf_chunk_plan(sample_rate, length, *[ctypes.byref(v) for v in vals], ptr(out["off"]),
+                                ptr(out["valid"]), ptr(out["mode"]), n))
+    out.update(chunk=vals[0].value, border=vals[1].value, padded_length=vals[2].value)
     return out
 
 

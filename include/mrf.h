@@ -219,6 +219,20 @@ const char *mrf_last_error(const mrf_handle *h);
 mrf_status mrf_band_tables(const mrf_config *cfg, int32_t *first_bin, int32_t *last_bin,
                            int32_t *width, int32_t *feat_row, float *row_weight, int32_t *n_feat);
 
+/*
+ * mrf_chunk_plan - host-only test hook: the geometry mrf_separate_audio uses for a mix of L
+ * samples at sample_rate (no device work, no handle).  *chunk = 8 * sample_rate samples, the
+ * stride 0.9 chunk (truncated), *border = chunk - stride when L > 2 * (chunk - stride) (the mix
+ * is then reflect-padded by it on both sides) else 0, *padded_length = L + 2 * border, and
+ * chunks at offsets 0, stride, 2 stride, ... below padded_length: off[i], valid[i] =
+ * min(chunk, padded_length - off[i]) samples, mode[i] = 0 (full), 1 (tail padded by
+ * reflection: more than half a chunk valid) or 2 (tail padded by zeros).  Writes at most
+ * max_chunks entries of each array (any array may be NULL); *n_chunks receives the count.
+ * MRF_EINVAL for sample_rate < 1, L < 2 or a NULL scalar output.
+ */
+mrf_status mrf_chunk_plan(int sample_rate, int L, int *chunk, int *border, int *padded_length, int *n_chunks,
+                          int32_t *off, int32_t *valid, int32_t *mode, int max_chunks);
+
 /* Kernel timing, for measurement.  When enabled, mrf_forward launches eagerly (no CUDA
  * graph) and records a CUDA event pair around every kernel on the forward's stream;
  * mrf_kernel_times waits for the events and returns, per kernel kind, the number of
