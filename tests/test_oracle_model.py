@@ -358,3 +358,142 @@ def test_geglu_parameter_count():
     g = model.param_count(dataclasses.replace(synth.VOCALS, ff_act=1), widths)
     D, FF = 384, 1536
     assert g - base == 2 * 6 * (D * FF + FF) and g == 235_299_108
+
+
+# ---------------------------------------------------------------- feed-forward and band split, by scalar loops
+def brute_feed_forward(x, w, ff_act=0):
+    """Scalar loops over the definition of the feed-forward block ("@audio/neural-separate
+    0.4.0 → 0.5.0", package/scripts/export-roformer.py, class FF: norm, Linear with bias, GELU,
+    Linear with bias): a = x / max(|x|, 1e-12) * sqrt(D) * gamma; h_i = gelu(W1[i] . a + b1[i])
+    with gelu(y) = y (1 + erf(y / sqrt 2)) / 2 (math.erf); out_j = W2[j] . h + b2[j].  The GEGLU
+    variant pairs h_i = (W1[i] . a + b1[i]) * gelu(W1[F + i] . a + b1[F + i])."""
+    n, D = x.shape
+    g, W1, b1, W2, b2 = w["net.0.gamma"], w["net.1.weight"], w["net.1.bias"], w["net.4.weight"], w["net.4.bias"]
+    F = W2.shape[1]
+    gelu = lambda y: 0.5 * y * (1.0 + math.erf(y / math.sqrt(2.0)))
+    out = np.zeros((n, D))
+    for t in range(n):
+        nrm = math.sqrt(sum(x[t, j] ** 2 for j in range(D)))
+        a = [x[t, j] / max(nrm, 1e-12) * math.sqrt(D) * g[j] for j in range(D)]
+        y = [sum(W1[i, j] * a[j] for j in range(D)) + b1[i] for i in range(W1.shape[0])]
+        h = [y[i] * gelu(y[F + i]) for i in range(F)] if ff_act == 1 else [gelu(y[i]) for i in range(F)]
+        for o in range(D):
+            out[t, o] = sum(W2[o, i] * h[i] for i in range(F)) + b2[o]
+    return out
+
+
+def _ff_weights(rng, D, F, ff_act=0):
+    F1 = 2 * F if ff_act == 1 else F
+    return {"net.0.gamma": 1 + 0.2 * rng.standard_normal(D), "net.1.weight": rng.standard_normal((F1, D)) / 2,
+            "net.1.bias": rng.standard_normal(F1), "net.4.weight": rng.standard_normal((D, F)) / 3,
+            "net.4.bias": rng.standard_normal(D)}
+
+
+@pytest.mark.parametrize("ff_act", [0, 1])
+def test_feed_forward_brute_force(ff_act):
+    rng = np.random.default_rng(11 + ff_act)
+    D, F = 6, 10
+    w = _ff_weights(rng, D, F, ff_act)
+    x = rng.standard_normal((5, D)) * 3
+    assert np.allclose(model.feed_forward(x, w, ff_act), brute_feed_forward(x, w, ff_act), rtol=0, atol=1e-11)
+
+
+def test_feed_forward_brute_force_catches_slips():
+    # each plausible slip changes the result by far more than the 1e-11 of the test above
+    rng = np.random.default_rng(13)
+    D, F = 6, 10
+    w = _ff_weights(rng, D, F)
+    x = rng.standard_normal((5, D)) * 3
+    ref = brute_feed_forward(x, w)
+    for key in ("net.1.bias", "net.4.bias"):          # a dropped bias
+        w2 = dict(w)
+        w2[key] = np.zeros_like(w[key])
+        assert np.abs(model.feed_forward(x, w2) - ref).max() > 1e-3
+    w2 = dict(w)
+    w2["net.0.gamma"] = w["net.0.gamma"] / math.sqrt(D)    # the norm's sqrt(D) left out
+    assert np.abs(model.feed_forward(x, w2) - ref).max() > 1e-3
+    # GELU after the second projection instead of the first, and no pre-norm at all
+    a = model.rms_norm(x, w["net.0.gamma"])
+    late = model.gelu((a @ w["net.1.weight"].T + w["net.1.bias"]) @ w["net.4.weight"].T + w["net.4.bias"])
+    assert np.abs(late - ref).max() > 1e-3
+    raw = model.gelu(x @ w["net.1.weight"].T + w["net.1.bias"]) @ w["net.4.weight"].T + w["net.4.bias"]
+    assert np.abs(raw - ref).max() > 1e-3
+
+
+def brute_transformer(x, w, h, dh, theta):
+    """One transformer by scalar loops: x += attention(x); x += ff(x); x = norm_out(x)."""
+    aw = {k[len("layers.0.0."):]: v for k, v in w.items() if k.startswith("layers.0.0.")}
+    fw = {k[len("layers.0.1."):]: v for k, v in w.items() if k.startswith("layers.0.1.")}
+    x = x + brute_attention_layer(x, aw, h, dh, theta)
+    x = x + brute_feed_forward(x, fw)
+    n, D = x.shape
+    out = np.zeros_like(x)
+    for t in range(n):
+        nrm = math.sqrt(sum(x[t, j] ** 2 for j in range(D)))
+        for j in range(D):
+            out[t, j] = x[t, j] / max(nrm, 1e-12) * math.sqrt(D) * w["norm.gamma"][j]
+    return out
+
+
+def test_transformer_brute_force():
+    rng = np.random.default_rng(14)
+    n, D, h, dh, F = 4, 6, 2, 4, 8
+    w = {"layers.0.0.norm.gamma": 1 + 0.1 * rng.standard_normal(D),
+         "layers.0.0.to_qkv.weight": rng.standard_normal((3 * h * dh, D)) / 2,
+         "layers.0.0.to_gates.weight": rng.standard_normal((h, D)),
+         "layers.0.0.to_gates.bias": rng.standard_normal(h),
+         "layers.0.0.to_out.0.weight": rng.standard_normal((D, h * dh)) / 2,
+         "norm.gamma": 1 + 0.1 * rng.standard_normal(D)}
+    w.update({"layers.0.1." + k: v for k, v in _ff_weights(rng, D, F).items()})
+    x = rng.standard_normal((2, n, D))
+    got = model.transformer(x, w, h, dh, 10000.0)
+    for s in range(2):
+        assert np.allclose(got[s], brute_transformer(x[s], w, h, dh, 10000.0), rtol=0, atol=1e-10)
+
+
+def brute_band_split(spec, first_bin, last_bin, channels, weights):
+    """BandSplit by scalar loops ("Mel-Band RoFormer — architecture, inference hot path & RTX 3050
+    feasibility", section "The mel-band split, exactly"): band k's features at frame t are, for
+    each bin f = first..last of the band in ascending order, each channel s and each complex part
+    c, spec[f * C + s, t, c] (feature (j * C + s) * 2 + c for the j-th bin); then
+    x / max(|x|, 1e-12) * sqrt(d_in) * gamma and Linear(d_in, D) with bias."""
+    R, T, _ = spec.shape
+    nb = len(first_bin)
+    D = weights["band_split.to_features.0.1.bias"].shape[0]
+    out = np.zeros((T, nb, D))
+    for k in range(nb):
+        p = f"band_split.to_features.{k}."
+        g, W, b = weights[p + "0.gamma"], weights[p + "1.weight"], weights[p + "1.bias"]
+        for t in range(T):
+            feats = []
+            for f in range(first_bin[k], last_bin[k] + 1):
+                for s in range(channels):
+                    for c in range(2):
+                        feats.append(spec[f * channels + s, t, c])
+            d = len(feats)
+            nrm = math.sqrt(sum(v * v for v in feats))
+            a = [feats[e] / max(nrm, 1e-12) * math.sqrt(d) * g[e] for e in range(d)]
+            for o in range(D):
+                out[t, k, o] = sum(W[o, e] * a[e] for e in range(d)) + b[o]
+    return out
+
+
+def test_band_split_brute_force():
+    rng = np.random.default_rng(15)
+    tab = tables.band_tables(44100, 256, 8)
+    D = 5
+    widths = tab["widths"]
+    W = {}
+    for k, d in enumerate(widths):
+        p = f"band_split.to_features.{k}."
+        W[p + "0.gamma"] = 1 + 0.2 * rng.standard_normal(d)
+        W[p + "1.weight"] = rng.standard_normal((D, d))
+        W[p + "1.bias"] = rng.standard_normal(D)
+    spec = rng.standard_normal((258, 3, 2))
+    spec[:, 2] = 0.0                                       # a silent frame: every band's norm clamps
+    ref = brute_band_split(spec, tab["first_bin"], tab["last_bin"], 2, W)
+    got = model.band_split(spec, tab, W)
+    assert np.allclose(got, ref, rtol=0, atol=1e-11)
+    # the silent frame gives exactly the biases (x / max(0, eps) = 0)
+    for k in range(8):
+        assert np.array_equal(got[2, k], W[f"band_split.to_features.{k}.1.bias"])
