@@ -6,9 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 #include <string>
-#include <vector>
 
 #include "mrf_handle.h"
 
@@ -21,22 +19,9 @@ constexpr size_t kStaticScratchBytes = size_t(64) << 20;  // 64 MiB on every dev
 // Zero at load; afterwards it keeps whatever the last call left in it.
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-std::mutex g_scratch_mu;
-std::vector<void *> g_scratch_addr;  // per device: device address of g_static_scratch
-
-// Device address of the array on `dev` (the current device), resolved once per device.
-cudaError_t scratch_address(int dev, void **out) {
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if ((int)g_scratch_addr.size() <= dev) g_scratch_addr.resize(dev + 1, nullptr);
-  if (!g_scratch_addr[dev]) {
-    void *p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
-  return cudaSuccess;
-}
+// Device address of the array on the current device.  Looked up on every call (the lookup
+// allocates nothing), so no address outlives the context it was taken in.
+cudaError_t scratch_address(void **out) { return cudaGetSymbolAddress(out, g_static_scratch); }
 
 }  // namespace
 }  // namespace mrf
@@ -79,7 +64,7 @@ extern "C" mrf_status mrf_forward_static(mrf_handle *h, const float *in, float *
     return MRF_EINVAL;
   }
   void *base = nullptr;
-  e = scratch_address(dev, &base);
+  e = scratch_address(&base);
   if (e != cudaSuccess) {
     cudaGetLastError();
     h->err = std::string("cudaGetSymbolAddress failed: ") + cudaGetErrorString(e);
@@ -87,18 +72,28 @@ extern "C" mrf_status mrf_forward_static(mrf_handle *h, const float *in, float *
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaGetLastError();
-  // the schedule clears its own accumulators (the row sums of squares) on every call; every
-  // other buffer is written before it is read
+  // The schedule clears the accumulators it needs at zero (the row sums of squares) on every
+  // call.  Rows of the activation buffers past this call's B*T keep what an earlier call left
+  // (possibly another handle's, in another layout): ragged GEMM tiles read them, but a GEMM
+  // row only feeds the same output row, which the epilogue drops, so they never reach a
+  // result.  The masks are written, never multiplied into stft_repr (apply_masks is a
+  // property of the handle's last mrf_forward_separate, not of this call).
   Fp16Workspace saved{};
   fp16_workspace_layout(h, base, true, &saved, nullptr, nullptr);
-  const bool timing = h->timing;
+  const bool timing = h->timing, apply = h->apply_masks;
   h->timing = false;
+  h->apply_masks = false;
   h->cur_stream = st;
   h->launch_counter = 0;
   h->sched_error.clear();
   schedule_fp16(h, in, out, B, T);
   h->timing = timing;
+  h->apply_masks = apply;
   fp16_restore_workspace(h, saved);
+  h->last_launches = h->launch_counter;
+  h->last_B = B;
+  h->last_T = T;
+  h->last_static = true;
   if (!h->sched_error.empty()) { h->err = h->sched_error; return MRF_ECUDA; }
   e = cudaGetLastError();
   if (e != cudaSuccess) { h->err = std::string("kernel launch: ") + cudaGetErrorString(e); return MRF_ECUDA; }

@@ -437,6 +437,7 @@ void run_schedule(mrf_handle *h, const float *in, float *out, int B, int T) {
   h->last_launches = h->launch_counter;
   h->last_B = B;
   h->last_T = T;
+  h->last_static = false;
 }
 
 }  // namespace
@@ -561,7 +562,7 @@ mrf_status forward_impl(mrf_handle *h, const float *in, float *out, int B, int T
     h->graphs.push_back({key, exec, h->last_launches});
   }
   for (auto &g : h->graphs)
-    if (g.key == key) { h->last_launches = g.launches; h->last_B = B; h->last_T = T; }
+    if (g.key == key) { h->last_launches = g.launches; h->last_B = B; h->last_T = T; h->last_static = false; }
   if (!cuda_ok(h, cudaGraphLaunch(exec, st), "graph launch", &s)) return s;
   return MRF_OK;
 }
@@ -678,6 +679,8 @@ mrf_status mrf_debug_stall_next(mrf_handle *h) {
 mrf_status mrf_debug_buffer(mrf_handle *h, const char *name, void *dst, size_t max_bytes, size_t *bytes_out) {
   if (!h || !name || !dst) return fail(h, MRF_EINVAL, "null argument");
   if (h->last_B < 1) return fail(h, MRF_EINVAL, "no forward has run");
+  if (h->last_static)
+    return fail(h, MRF_EINVAL, "the last forward ran in mrf_forward_static's shared scratch, which this hook does not read");
   const void *src = nullptr;
   size_t bytes = 0;
   const std::string n(name);

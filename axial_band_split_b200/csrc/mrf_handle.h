@@ -101,6 +101,7 @@ struct mrf_handle {
   std::vector<mrf::PendingTiming> pending;
   std::vector<mrf::GraphEntry> graphs;
   int launch_counter = 0, last_launches = -1, last_B = -1, last_T = -1;
+  bool last_static = false;  // the last forward ran in mrf_forward_static's shared scratch
   float *io_in = nullptr, *io_out = nullptr;
   // spectral front / back end (signal_api.cu): FFT tables of n_fft and grow-only scratch
   float2 *d_tw = nullptr;

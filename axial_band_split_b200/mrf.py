@@ -203,10 +203,27 @@ class Model:
         except Exception:
             pass
 
+    def _check_input(self, x):
+        """stft_repr must be a contiguous CUDA float32 [B, F*C, T, 2] of this model's rows."""
+        import torch
+        assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous(), "stft_repr: contiguous CUDA float32"
+        assert x.dim() == 4 and x.shape[1] == self.rows and x.shape[3] == 2, \
+            f"stft_repr must be [B, {self.rows}, T, 2], got {tuple(x.shape)}"
+
+    def _check_out(self, x, out):
+        """`out` must hold exactly B * num_stems * rows * T * 2 floats, on x's device."""
+        import torch
+        B, R, T, _ = x.shape
+        need = B * self.cfg.num_stems * R * T * 2
+        assert out.dtype == torch.float32 and out.is_contiguous(), "out: contiguous float32"
+        assert out.device == x.device and out.is_cuda == x.is_cuda, "out must be on stft_repr's device"
+        assert out.numel() == need, f"out holds {out.numel()} floats, the forward writes {need}"
+
     def _out_like(self, x, out):
         """[B, F*2, T, 2] for one stem, [B, stems, F*2, T, 2] for more."""
         import torch
         if out is not None:
+            self._check_out(x, out)
             return out
         B, R, T, two = x.shape
         stems = self.cfg.num_stems
@@ -215,8 +232,7 @@ class Model:
 
     def forward(self, stft_repr, out=None, stream=None):
         """masks for a CUDA float32 tensor [B, F*2, T, 2] (queued on `stream`)."""
-        import torch
-        assert stft_repr.is_cuda and stft_repr.dtype == torch.float32 and stft_repr.is_contiguous()
+        self._check_input(stft_repr)
         B, R, T, two = stft_repr.shape
         out = self._out_like(stft_repr, out)
         _check(lib().mrf_forward(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
@@ -226,8 +242,7 @@ class Model:
     def separate(self, stft_repr, out=None, stream=None):
         """mrf_forward_separate: the separated spectra (masks times stft_repr, complex), same
         shape as forward's masks."""
-        import torch
-        assert stft_repr.is_cuda and stft_repr.dtype == torch.float32 and stft_repr.is_contiguous()
+        self._check_input(stft_repr)
         B, R, T, two = stft_repr.shape
         out = self._out_like(stft_repr, out)
         _check(lib().mrf_forward_separate(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
@@ -273,8 +288,8 @@ class Model:
     def forward_static(self, stft_repr, out, stream=None):
         """mrf_forward_static: the same forward with the library's fixed device scratch
         instead of the handle's workspace; allocates nothing (out must be given)."""
-        import torch
-        assert stft_repr.is_cuda and stft_repr.dtype == torch.float32 and stft_repr.is_contiguous()
+        self._check_input(stft_repr)
+        self._check_out(stft_repr, out)
         B, R, T, _ = stft_repr.shape
         _check(lib().mrf_forward_static(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
                                         ctypes.c_void_p(out.data_ptr()), B, T, _stream_ptr(stream)), self._h)

@@ -185,12 +185,15 @@ mrf_status mrf_forward_host(mrf_handle *h, const float *stft_repr_host, float *m
  * (the tiny model fits at T <= ~2000; the vocals model only at a few tens of frames).
  * stft_repr and masks as for mrf_forward; the handle's device must be current.
  *
- * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- * with that device current; make that first call before any stream capture.  Every call
- * uses the same array, which keeps the last call's contents (each call clears the
- * accumulators it needs at zero and writes every other buffer before reading it): calls
- * that overlap on the GPU, from any handle or thread, race and corrupt each other's
- * results.  Serialise them (one stream, or events).
+ * Each call looks up the array's device address (cudaGetSymbolAddress, which allocates
+ * nothing) with the handle's device current; the first lookup on a device may load the
+ * library's device code there, so make the first call before any stream capture.  Every
+ * call uses the same array, which keeps the last call's contents: each call clears the
+ * accumulators it needs at zero; rows past this call's B*T may hold an earlier call's bytes,
+ * which feed only rows that are dropped.  Calls that overlap on the GPU, from any handle or
+ * thread, race and corrupt each other's results: serialise them (one stream, or events).
+ * This call always writes masks (never the separated spectra of mrf_forward_separate), and
+ * mrf_debug_buffer does not read its buffers (it returns MRF_EINVAL after it).
  */
 mrf_status mrf_forward_static(mrf_handle *h, const float *stft_repr, float *masks, int B, int T,
                               void *stream);
@@ -259,7 +262,8 @@ mrf_status mrf_debug_stall_next(mrf_handle *h);
  * buffer of the last forward to host memory.  "X": the residual stream after the last
  * transformer, float32 [B*T*num_bands, dim], token (b*T + t)*num_bands + k; "M": the mask
  * estimator output before the overlap average, float32 [B*T, sum d_in].  At most
- * max_bytes are copied; *bytes_out receives the number copied.
+ * max_bytes are copied; *bytes_out receives the number copied.  MRF_EINVAL when no forward
+ * has run, or when the last one was mrf_forward_static (its buffers are not the handle's).
  */
 mrf_status mrf_debug_buffer(mrf_handle *h, const char *name, void *host_dst, size_t max_bytes,
                             size_t *bytes_out);

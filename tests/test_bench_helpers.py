@@ -45,16 +45,23 @@ def test_clock_summary(tmp_path):
     c.proc = object()                       # as if nvidia-smi had run
     c.path = str(tmp_path / "clocks.csv")
     rows = [
-        "0, 1800, 1965, 700.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
-        "0, 1700, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
-        "0, 1750, 1965, 980.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 700.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active, 98",
+        "0, 1700, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active, 100",
+        "0, 1750, 1965, 980.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active, 97",
+        "0, 1965, 1965, 250.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active, 0",
+        "0, 1965, 1965, 250.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active, 3",
         "garbage line",
-        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active, 0",
     ]
     open(c.path, "w").write("\n".join(rows) + "\n")
     s = c.summary()
-    assert s == {"sm_mhz": 1750.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    # the median is taken over the samples under load only; idle samples still count as samples
+    assert s == {"sm_mhz": 1750.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 5,
+                 "samples_under_load": 3}
     assert not os.path.exists(c.path)
+    # no utilisation column, or nothing under load: the median of every sample
+    s = bench.summarize_clock_lines([r.rsplit(",", 1)[0] for r in rows[:4]])
+    assert s["sm_mhz"] == 1775.0 and s["samples_under_load"] == 0
 
 
 def test_aggregate_is_all_ranks_units_over_the_slowest_time():

@@ -49,3 +49,51 @@ def test_static_forward_refuses_oversized_workspace():
         m.forward_static(xin, out)
     assert e.value.status == -2 and "static scratch" in str(e.value)
     m.close()
+
+
+def test_static_forward_after_separate_writes_masks():
+    # a separate() call leaves the handle in its apply-masks state; the static entry point must
+    # still write the masks, not the separated spectra
+    from axial_band_split_b200 import mrf
+    cfg = synth.TINY
+    B, T = 1, 32
+    W, x = case(cfg, B, T, True)
+    m = mrf.Model(cfg, W, max_batch=B, max_frames=T, compute=mrf.MRF_FP16)
+    xin = torch.from_numpy(x).cuda()
+    ref = m.forward(xin).cpu().numpy()
+    m.separate(xin)
+    out = torch.full_like(xin, float("nan"))
+    m.forward_static(xin, out)
+    m.sync_status()
+    got = out.cpu().numpy()
+    assert np.abs(got - ref).max() <= 2e-2 and snr_db(got, ref) >= 40.0
+    with pytest.raises(mrf.MrfError):          # the debug hook does not read the shared scratch
+        m.debug_buffer("M", 16)
+    m.close()
+
+
+def test_static_forward_short_window_after_another_handle():
+    # B*T below the handle's maximum, after a handle of another shape filled the shared scratch:
+    # the rows past B*T hold that handle's bytes and must not reach the masks
+    from axial_band_split_b200 import mrf
+    import dataclasses
+    other = dataclasses.replace(synth.TINY, dim=128, heads=2, dim_head=64)
+    Wo, xo = case(other, 2, 40, True)
+    mo = mrf.Model(other, Wo, max_batch=2, max_frames=40, compute=mrf.MRF_FP16)
+    oo = torch.empty_like(torch.from_numpy(xo).cuda())
+    mo.forward_static(torch.from_numpy(xo).cuda(), oo)
+    mo.sync_status()
+    mo.close()
+    cfg = synth.TINY
+    B, T = 1, 21
+    W, x = case(cfg, B, T, True)
+    m = mrf.Model(cfg, W, max_batch=2, max_frames=40, compute=mrf.MRF_FP16)
+    xin = torch.from_numpy(x).cuda()
+    ref = m.forward(xin).cpu().numpy()
+    out = torch.full_like(xin, float("nan"))
+    m.forward_static(xin, out)
+    m.sync_status()
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    assert np.abs(got - ref).max() <= 2e-2 and snr_db(got, ref) >= 40.0
+    m.close()
