@@ -39,7 +39,8 @@ def kernel_work(cfg, widths, B: int, T: int):
         "gemm_band_split": ("flop", 2 * BT * D * n_feat, 1),
         # stft_repr read once, normalised fp16 band features written once
         "band_gather": ("byte", B * rows * T * 2 * 4 + BT * n_feat * 2, 1),
-        # per stem: mask features fp32 read once, masks fp32 written once
+        # fp32 debug schedule, per stem: mask features fp32 read once, masks fp32 written once (the
+        # fp16 schedule averages inside the GLU GEMM's epilogue)
         "overlap_average": ("byte", S * (BT * n_feat * 4 + B * rows * T * 2 * 4), S),
     }
     return w

@@ -24,7 +24,7 @@ enum GemmEpi : int {
   kTcResid = 1,   // X += acc (+ bias); writes X fp32, X fp16, row sum of squares
   kTcGelu = 2,    // out = gelu(acc * rowscale + bias) fp16
   kTcTanh = 3,    // out = tanh(acc + bias) fp16 (group-strided)
-  kTcGlu = 4,     // interleaved (value, gate) pairs -> value * sigmoid(gate), fp32
+  kTcGlu = 4,     // interleaved (value, gate) pairs -> value * sigmoid(gate), averaged into the masks
   kTcBandSplit = 5,  // X = acc + bias for token m*nb + group (band); X fp32, X fp16, row sum of squares
   kTcGeglu = 6,   // interleaved (value, gate) pairs of acc * rowscale + bias -> value * gelu(gate), fp16
 };
@@ -57,6 +57,15 @@ struct GemmParams {
   // kTcResid: also accumulate sum_j (out_gain[j] * x_j)^2 per row into ssg_out (null: skip)
   float *ssg_out;
   const float *out_gain;
+  // kTcGlu: the overlap average.  Feature e (global feature index) adds row_weight[feat_row[e]]
+  // times its GLU output to masks[b * mask_bstride + (feat_row[e] * T + t) * 2 + (e & 1)] (zeroed
+  // beforehand), multiplied by the complex spec[b, feat_row[e], t] when spec is not null.
+  const int32_t *feat_row;
+  const float *row_weight;
+  float *masks;
+  long long mask_bstride;
+  const float *spec;
+  int R;
 };
 
 enum TmapDtype : int { kTmF16 = 0, kTmF32 = 1 };
@@ -79,7 +88,7 @@ bool gemm_tc_init();
 // (kTcQkv: [q | k | v | gates] fp16 [M, ld] box 32x32 swizzle 64; kTcResid: X fp32 [M, ld] box 32x32 swizzle 128 and X fp16 box 32x32 swizzle 64;
 //  kTcBandSplit: the same as 3D (ld, nb, frames) boxes 32x1x32; kTcGelu: out fp16 [M, ldo]
 //  box 32x32 swizzle 64; kTcTanh: out fp16 (ldo, frames, groups) box 32x32x1 swizzle 64;
-//  kTcGlu: out fp32 [frames, ldo] box 16x32 swizzle 64; kTcGeglu: out fp16 [M, ldo] box 16x32,
+//  kTcGlu: none (atomic adds into the masks); kTcGeglu: out fp16 [M, ldo] box 16x32,
 //  no swizzle).  Unused maps may be any valid map.
 void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
                     const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st);

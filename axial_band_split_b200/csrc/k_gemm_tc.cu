@@ -527,34 +527,43 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
             tc::bulk_commit();
           }
           ++nstore;
-        } else {  // kTcGlu: interleaved (value, gate) pairs -> 16 fp32 outputs per row
+        } else {  // kTcGlu: interleaved (value, gate) pairs -> up to 16 band features of frame m
+          // The overlap average is fused here: feature e of the band adds
+          // row_weight[r] * value * sigmoid(gate) to masks[b, r, t] (component e & 1) for its
+          // stft_repr row r.  A row's (re, im) are features e, e + 1, so each pair is one
+          // 8-byte add.  An element receives one add per band covering its bin, at most two,
+          // onto the zeroed output: the sum is the same in either order (0 + a = a, a + b =
+          // b + a), so the result does not depend on the order of the adds.
           const float *bias = p.bias + gr.bias_off + c0;
+          const int nf = min(16, (gr.N - c0) >> 1);
           float o[16];
 #pragma unroll
           for (int j = 0; j < 32; j += 2) {
-            const bool ok = c0 + j + 1 < gr.N;
+            const bool ok = (j >> 1) < nf;
             const float val = v[j] + (ok ? bias[j] : 0.f);
             const float gt = v[j + 1] + (ok ? bias[j + 1] : 0.f);
             o[j >> 1] = val * sigmoidf_(gt);
           }
-          if (full_chunk) {
-            uint8_t *box = stg + (nstore & 1) * 2048;
-            if (lane == 0) tc::bulk_wait_read<1>();
-            __syncwarp();
+          if (valid) {
+            const int fe0 = gr.out_off + (c0 >> 1);
+            const int bb = m / p.T, t = m - bb * p.T;
+            float *dst0 = p.masks + bb * p.mask_bstride + 2LL * t;
+            const float *x0 = p.spec ? p.spec + ((long long)bb * p.R * p.T + t) * 2 : nullptr;
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              *reinterpret_cast<float4 *>(box + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) =
-                  make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-            tc::fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) {
-              tc::tma_store_2d(&tmC, box, gr.out_off + (c0 >> 1), m0w);
-              tc::bulk_commit();
+            for (int i = 0; i < 8; ++i) {
+              if (2 * i < nf) {
+                const int r = __ldg(p.feat_row + fe0 + 2 * i);
+                const float w = __ldg(p.row_weight + r);
+                if (w != 0.f) {
+                  float2 add = make_float2(o[2 * i] * w, o[2 * i + 1] * w);
+                  if (x0) {
+                    const float2 x = *reinterpret_cast<const float2 *>(x0 + 2LL * r * p.T);
+                    add = make_float2(add.x * x.x - add.y * x.y, add.x * x.y + add.y * x.x);
+                  }
+                  atomicAdd(reinterpret_cast<float2 *>(dst0 + 2LL * r * p.T), add);
+                }
+              }
             }
-            ++nstore;
-          } else if (valid) {
-            float *dst = p.out_f + (long long)m * p.ldo + gr.out_off + (c0 >> 1);
-            for (int j = 0; 2 * j + 1 < gr.N - c0; ++j) dst[j] = o[j];
           }
         }
       }

@@ -117,52 +117,6 @@ __global__ void __launch_bounds__(kBsThreads) band_split_kernel(
   }
 }
 
-// Gather + normalise only (fp16 schedule): per band k and frame bt, the band's features
-// divided by their L2 norm, fp16, into A[(k * frame_stride + bt) * k_stride + e] for
-// e < k_pad(k) (zeros past the band's width), the A operand of the band-split GEMM.
-__global__ void __launch_bounds__(kBsThreads) band_gather_kernel(
-    const float *__restrict__ in, const int32_t *__restrict__ feat_row, const BandDesc *__restrict__ bands, int B,
-    int T, int R, long long frame_stride, int k_stride, __half *__restrict__ A) {
-  extern __shared__ float xs[];  // [kBsFrames][width + 2]: an even row stride that is 2 mod 4 words
-  const int k = blockIdx.y;
-  const BandDesc bd = bands[k];
-  const int W = bd.width, Ws = W + 2, Wp = (W + 63) & ~63;
-  const long long frames = (long long)B * T;
-  const long long f0 = (long long)blockIdx.x * kBsFrames;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // A band's features come in (re, im) pairs of one stft_repr row (feature 2p + c is component c
-  // of row feat_row[2p]).  Consecutive threads take consecutive frames of one row, so a
-  // half-warp reads 16 frames' (re, im) pairs: 128 contiguous bytes.
-  const float2 *in2 = reinterpret_cast<const float2 *>(in);
-  for (int i = tid; i < kBsFrames * (W >> 1); i += kBsThreads) {
-    const int f = i % kBsFrames, p = i / kBsFrames;
-    const long long bt = f0 + f;
-    float2 v = make_float2(0.f, 0.f);
-    if (bt < frames) {
-      const long long b = bt / T, t = bt % T;
-      v = in2[(b * R + feat_row[bd.feat_off + 2 * p]) * T + t];
-    }
-    *reinterpret_cast<float2 *>(xs + f * Ws + 2 * p) = v;
-  }
-  __syncthreads();
-  for (int f = warp; f < kBsFrames; f += kBsThreads / 32) {
-    float s = 0.f;
-    for (int e = lane; e < W; e += 32) s += xs[f * Ws + e] * xs[f * Ws + e];
-    s = warp_sum(s);
-    const float r = 1.f / fmaxf(sqrtf(s), kNormEps);
-    for (int e = lane; e < W; e += 32) xs[f * Ws + e] *= r;
-  }
-  __syncthreads();
-  // fp16 pairs, the band's row zero-padded to a multiple of 64 features
-  for (int i = tid; i < kBsFrames * (Wp >> 1); i += kBsThreads) {
-    const int f = i / (Wp >> 1), e = 2 * (i % (Wp >> 1));
-    const long long bt = f0 + f;
-    if (bt >= frames) continue;
-    const __half2 h = e < W ? __floats2half2_rn(xs[f * Ws + e], xs[f * Ws + e + 1]) : __floats2half2_rn(0.f, 0.f);
-    *reinterpret_cast<__half2 *>(A + ((long long)k * frame_stride + bt) * k_stride + e) = h;
-  }
-}
-
 // ------------------------------------------------------------------ grouped SIMT GEMM
 constexpr int kGt = 64, kGk = 16;
 
@@ -450,14 +404,6 @@ void launch_band_split(const float *in, const int32_t *feat_row, const int32_t *
   const size_t smem = sizeof(float) * kBsFrames * max_width;
   band_split_kernel<<<grid, kBsThreads, smem, st>>>(in, feat_row, feat_c, bands, nb, w, bias, dim,
                                                    B, T, rows, X, Xh, ss);
-}
-
-void launch_band_gather(const float *in, const int32_t *feat_row, const BandDesc *bands, int nb, int B, int T,
-                        int rows, long long frame_stride, int k_stride, __half *A, int max_width, cudaStream_t st) {
-  const long long frames = (long long)B * T;
-  dim3 grid(grid1(frames, kBsFrames), nb);
-  band_gather_kernel<<<grid, kBsThreads, sizeof(float) * kBsFrames * (max_width + 2), st>>>(
-      in, feat_row, bands, B, T, rows, frame_stride, k_stride, A);
 }
 
 void launch_gemm_f32(const float *A, const float *W, const float *bias, float *C,

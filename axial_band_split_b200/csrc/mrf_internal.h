@@ -32,10 +32,10 @@ void launch_band_split(const float *in, const int32_t *feat_row, const int32_t *
                        int dim, int B, int T, int rows, float *X, __half *Xh, float *ss,
                        cudaStream_t st, int max_width);
 
-// fp16 schedule: normalised band features, fp16, [band][frame_stride][k_stride], each band's
-// row zero-padded to a multiple of 64 (the A operand of the band-split GEMM).
+// fp16 schedule (k_gather.cu): normalised band features, fp16, [band][frame_stride][k_stride],
+// each band's row zero-padded to a multiple of 64 (the A operand of the band-split GEMM).
 void launch_band_gather(const float *in, const int32_t *feat_row, const BandDesc *bands, int nb, int B, int T,
-                        int rows, long long frame_stride, int k_stride, __half *A, int max_width, cudaStream_t st);
+                        int rows, long long frame_stride, int k_stride, __half *A, cudaStream_t st);
 
 enum SimtEpi : int {
   kEpiStore = 0,      // C = acc (+ bias)

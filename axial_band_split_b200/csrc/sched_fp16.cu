@@ -9,8 +9,8 @@
 //     FF1 GEMM, GELU epilogue                  -> H fp16
 //     FF2 GEMM, residual epilogue              -> X, X fp16, |x|^2
 //     output norm                              -> X, X fp16, |x|^2
-//   mask head: per-band GEMMs (tanh, tanh, GLU) -> m fp32 [B*T, sum d_in]
-//   overlap average                            -> masks
+//   mask head: per-band GEMMs (tanh, tanh, GLU), the GLU epilogue adding each band feature
+//   into its stft_repr row of the zeroed masks (the overlap average)  -> masks
 //
 // Exact rewrites (package/scripts/export-roformer.py of "@audio/neural-separate 0.4.0 →
 // 0.5.0", class Core and its module docstring): each RMSNorm's sqrt(d)*gamma is folded
@@ -56,7 +56,7 @@ struct Fp16State {
   GemmGroup *g_m0 = nullptr, *g_mid = nullptr, *g_last = nullptr;
   int n_last_tiles = 0;
   // workspace
-  float *X = nullptr, *ss = nullptr, *Mg = nullptr;
+  float *X = nullptr, *ss = nullptr;
   // deferred output norm: |x|^2 and |g x|^2 of the last FF2 output (g = sqrt(D) gamma_out)
   float *ssx = nullptr, *ssg = nullptr;
   __half *Xh = nullptr, *QKV = nullptr, *O = nullptr, *Hh = nullptr, *H1 = nullptr, *H2 = nullptr;
@@ -260,8 +260,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->Hh = h->alloc<__half>(NT * FF);
   f->H1 = h->alloc<__half>((long long)nb * MBT * MH);
   f->H2 = h->alloc<__half>((long long)nb * MBT * MH);
-  f->Mg = h->alloc<float>(MBT * t.n_feat());
-  if (!f->X || !f->Xh || !f->ss || !f->ssx || !f->ssg || !f->QKV || !f->O || !f->Hh || !f->H1 || !f->H2 || !f->Mg)
+  if (!f->X || !f->Xh || !f->ss || !f->ssx || !f->ssg || !f->QKV || !f->O || !f->Hh || !f->H1 || !f->H2)
     return MRF_ENOMEM;
   // rows past a forward's B*T are read by ragged tiles (and discarded): keep them finite
   if (cudaMemset(f->QKV, 0, NT * f->ldq * 2) != cudaSuccess || cudaMemset(f->H1, 0, (size_t)nb * MBT * MH * 2) != cudaSuccess ||
@@ -295,8 +294,7 @@ bool debug_buffer_fp16(mrf_handle *h, const std::string &name, const void **ptr,
     *bytes = hx.size() * 4;
     return true;
   }
-  if (name == "M") { *ptr = f->Mg; *bytes = BT * h->tab.n_feat() * sizeof(float); return true; }
-  return false;
+  return false;  // the mask features ("M") are never stored: the GLU epilogue averages them into the masks
 }
 
 void destroy_fp16(mrf_handle *h) {
@@ -382,7 +380,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     ok = ok && make_tmap_f16(&wmaps[w0 + c.mask_depth], f->mw_last[s], MH, rows_last, 1, MH, rows_last * MH, kBnWide, 1);
   }
   // bulk-store output maps
-  CUtensorMap mXo, mXho, mXbs, mXhbs, mHo, mHo16, mH1o, mH2o, mMg, mQKVo;
+  CUtensorMap mXo, mXho, mXbs, mXhbs, mHo, mHo16, mH1o, mH2o, mQKVo;
   {
     const unsigned long long BT = (unsigned long long)B * T;
     const unsigned long long dx[3] = {(unsigned long long)D, (unsigned long long)nb, BT};
@@ -396,7 +394,6 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
          map2(&mHo, f->Hh, kTmF16, FF, M, FF, 32, 64) && map2(&mHo16, f->Hh, kTmF16, FF, M, FF, 16, 0) &&
          make_tmap(&mH1o, f->H1, kTmF16, 3, dh3, sh3, bh, 64) &&
          make_tmap(&mH2o, f->H2, kTmF16, 3, dh3, sh3, bh, 64) &&
-         map2(&mMg, f->Mg, kTmF32, h->tab.n_feat(), BT, h->tab.n_feat(), 16, 64) &&
          map2(&mQKVo, f->QKV, kTmF16, 3 * A + H, M, f->ldq, 32, 64);
   }
   if (!ok) {
@@ -405,7 +402,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   }
 
   h->begin("band_gather");
-  launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, h->max_width, st);
+  launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, st);
   h->end();
   cudaMemsetAsync(f->ssg, 0, sizeof(float) * M, st);
   {
@@ -460,10 +457,12 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p, &mXo, &mXho);
   }
 
-  // mask heads, one per stem, each followed by its overlap average (or, for
-  // mrf_forward_separate, the masks multiplied into stft_repr) into the stem's slice
+  // mask heads, one per stem; each GLU epilogue adds its band features into the stem's slice
+  // of the zeroed output (the overlap average; for mrf_forward_separate the features times
+  // stft_repr, so the masks are never stored)
   const int BT = B * T;
   const long long per_stem = (long long)R * T * 2;  // one stem's masks of one window
+  cudaMemsetAsync(out, 0, sizeof(float) * (size_t)B * c.num_stems * per_stem, st);
   for (int s = 0; s < c.num_stems; ++s) {
     const int w0 = wm0 + s * n_mask_maps;
     GemmParams p = base_params(h, BT, D, kBnWide, f->g_m0, nb, nb * cdiv(MH, kBnWide));
@@ -484,13 +483,12 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
       std::swap(ocur, onxt);
     }
     p = base_params(h, BT, MH, kBnWide, f->g_last, nb, f->n_last_tiles);
-    p.bias = f->mb_last[s]; p.out_f = f->Mg; p.ldo = h->tab.n_feat();
-    gemm(h, "gemm_mask_glu", kTcGlu, *mcur, wmaps[w0 + c.mask_depth], p, &mMg);
-
-    h->begin("overlap_average");
-    launch_overlap_average(f->Mg, h->tab.n_feat(), h->d_src0, h->d_src1, h->d_row_weight, out + s * per_stem,
-                           c.num_stems * per_stem, h->apply_masks ? in : nullptr, B, T, R, st);
-    h->end();
+    p.bias = f->mb_last[s];
+    p.feat_row = h->d_feat_row; p.row_weight = h->d_row_weight;
+    p.masks = out + s * per_stem; p.mask_bstride = c.num_stems * per_stem;
+    p.spec = h->apply_masks ? in : nullptr;
+    p.B = B; p.T = T; p.R = R;
+    gemm(h, "gemm_mask_glu", kTcGlu, *mcur, wmaps[w0 + c.mask_depth], p);
   }
 }
 
@@ -519,12 +517,12 @@ size_t fp16_workspace_layout(mrf_handle *h, void *base, bool apply, Fp16Workspac
                oss = take(NT * 4), ossx = take(NT * 4), ossg = take(NT * 4);
   const size_t oQ = take(NT * f->ldq * 2);
   const size_t oO = take(NT * A * 2), oHh = take(NT * FF * 2), oH1 = take((size_t)nb * MBT * MH * 2),
-               oH2 = take((size_t)nb * MBT * MH * 2), oMg = take(MBT * h->tab.n_feat() * 4);
+               oH2 = take((size_t)nb * MBT * MH * 2);
   (void)H;
   if (qkv_offset) *qkv_offset = oQ;
   if (qkv_bytes) *qkv_bytes = oO - oQ;
   if (apply && f) {
-    if (saved) *saved = {f->X, f->ss, f->Mg, f->Xh, f->QKV, f->O, f->Hh, f->H1, f->H2, f->A_bs, f->ssx, f->ssg};
+    if (saved) *saved = {f->X, f->ss, f->Xh, f->QKV, f->O, f->Hh, f->H1, f->H2, f->A_bs, f->ssx, f->ssg};
     uint8_t *b = static_cast<uint8_t *>(base);
     f->A_bs = reinterpret_cast<__half *>(b + oA);
     f->X = reinterpret_cast<float *>(b + oX);
@@ -537,14 +535,13 @@ size_t fp16_workspace_layout(mrf_handle *h, void *base, bool apply, Fp16Workspac
     f->Hh = reinterpret_cast<__half *>(b + oHh);
     f->H1 = reinterpret_cast<__half *>(b + oH1);
     f->H2 = reinterpret_cast<__half *>(b + oH2);
-    f->Mg = reinterpret_cast<float *>(b + oMg);
   }
   return off;
 }
 
 void fp16_restore_workspace(mrf_handle *h, const Fp16Workspace &s) {
   Fp16State *f = h->f16;
-  f->X = s.X; f->ss = s.ss; f->Mg = s.Mg; f->Xh = s.Xh; f->QKV = s.QKV;
+  f->X = s.X; f->ss = s.ss; f->Xh = s.Xh; f->QKV = s.QKV;
   f->O = s.O; f->Hh = s.Hh; f->H1 = s.H1; f->H2 = s.H2; f->A_bs = s.A_bs; f->ssx = s.ssx; f->ssg = s.ssg;
 }
 

@@ -260,8 +260,9 @@ mrf_status mrf_debug_stall_next(mrf_handle *h);
 /*
  * mrf_debug_buffer - test hook: wait for the device, then copy the start of an internal
  * buffer of the last forward to host memory.  "X": the residual stream after the last
- * transformer, float32 [B*T*num_bands, dim], token (b*T + t)*num_bands + k; "M": the mask
- * estimator output before the overlap average, float32 [B*T, sum d_in].  At most
+ * transformer, float32 [B*T*num_bands, dim], token (b*T + t)*num_bands + k; "M" (MRF_FP32_DEBUG
+ * only: the fp16 schedule averages the mask features into the masks without storing them): the
+ * mask estimator output before the overlap average, float32 [B*T, sum d_in].  At most
  * max_bytes are copied; *bytes_out receives the number copied.  MRF_EINVAL when no forward
  * has run, or when the last one was mrf_forward_static (its buffers are not the handle's).
  */

@@ -68,7 +68,7 @@ def test_static_forward_after_separate_writes_masks():
     got = out.cpu().numpy()
     assert np.abs(got - ref).max() <= 2e-2 and snr_db(got, ref) >= 40.0
     with pytest.raises(mrf.MrfError):          # the debug hook does not read the shared scratch
-        m.debug_buffer("M", 16)
+        m.debug_buffer("X", 16)
     m.close()
 
 
