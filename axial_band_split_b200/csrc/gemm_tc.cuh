@@ -21,11 +21,11 @@ struct GemmGroup {
 
 enum GemmEpi : int {
   kTcQkv = 0,     // row norm, RoPE on q and k, softmax scale on q, sigmoid gates; token-major fp16 rows
-  kTcResid = 1,   // X += acc (+ bias); writes X fp32, X fp16, row sum of squares
+  kTcResid = 1,   // x += acc (+ bias) on the fp16 residual stream Xh; row sums of squares
   kTcGelu = 2,    // out = gelu(acc * rowscale + bias) fp16
   kTcTanh = 3,    // out = tanh(acc + bias) fp16 (group-strided)
   kTcGlu = 4,     // interleaved (value, gate) pairs -> value * sigmoid(gate), averaged into the masks
-  kTcBandSplit = 5,  // X = acc + bias for token m*nb + group (band); X fp32, X fp16, row sum of squares
+  kTcBandSplit = 5,  // x = acc + bias for token m*nb + group (band) into Xh; row sums of squares
   kTcGeglu = 6,   // interleaved (value, gate) pairs of acc * rowscale + bias -> value * gelu(gate), fp16
 };
 
@@ -35,11 +35,15 @@ struct GemmParams {
   const GemmGroup *groups;
   unsigned *status;
   // epilogue
-  const float *ss_in;       // row sums of squares giving the row scale 1 / max(sqrt(ss), eps); null: 1
+  // Row sums of squares are written as partial sums, one slot per (column tile, epilogue warp of
+  // the row's lane quarter), ss_out_parts slots a row; a consumer adds its ss_in_parts slots in
+  // order (deterministic: no atomics).
+  const float *ss_in;       // row scale 1 / max(sqrt(sum of the row's slots), eps); null: 1
+  int ss_in_parts;
   const float *bias;
-  float *X;                 // fp32 residual [M, ld]
-  __half *Xh;               // fp16 copy of X
-  float *ss_out;            // row sums of squares (atomic partials)
+  __half *Xh;               // fp16 residual stream [M, ld] (kTcResid reads and rewrites it)
+  float *ss_out;            // row sums of squares of the output (partial slots)
+  int ss_out_parts;
   int ld;
   __half *out_h;            // fp16 output
   float *out_f;             // fp32 output
@@ -51,10 +55,11 @@ struct GemmParams {
   int B, T, nb, H, dh, A, axis;
   float q_scale;            // q is multiplied by this after RoPE (the attention's softmax scale)
   // deferred output norm of the previous transformer (kTcResid): the residual input x is
-  // scaled by res_gain[col] / max(sqrt(res_ss[row]), eps) before the add (null: no scaling)
+  // scaled by res_gain[col] / max(sqrt(res_ss[row]), eps) before the add (null: no scaling);
+  // res_ss has ss_in_parts slots a row
   const float *res_ss;
   const float *res_gain;
-  // kTcResid: also accumulate sum_j (out_gain[j] * x_j)^2 per row into ssg_out (null: skip)
+  // kTcResid: also the partial sums of (out_gain[j] * x_j)^2 into ssg_out (null: skip)
   float *ssg_out;
   const float *out_gain;
   // kTcGlu: the overlap average.  Feature e (global feature index) adds row_weight[feat_row[e]]
@@ -85,8 +90,8 @@ bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, un
 bool gemm_tc_init();
 
 // tmC / tmD: output tensor maps of the epilogues that store through bulk tensor stores
-// (kTcQkv: [q | k | v | gates] fp16 [M, ld] box 32x32 swizzle 64; kTcResid: X fp32 [M, ld] box 32x32 swizzle 128 and X fp16 box 32x32 swizzle 64;
-//  kTcBandSplit: the same as 3D (ld, nb, frames) boxes 32x1x32; kTcGelu: out fp16 [M, ldo]
+// (kTcQkv: [q | k | v | gates] fp16 [M, ld] box 32x32 swizzle 64; kTcResid: tmD = Xh fp16 [M, ld] box 32x32
+//  swizzle 64; kTcBandSplit: tmD = the same as 3D (ld, nb, frames) boxes 32x1x32; kTcGelu: out fp16 [M, ldo]
 //  box 32x32 swizzle 64; kTcTanh: out fp16 (ldo, frames, groups) box 32x32x1 swizzle 64;
 //  kTcGlu: none (atomic adds into the masks); kTcGeglu: out fp16 [M, ldo] box 16x32,
 //  no swizzle).  Unused maps may be any valid map.

@@ -50,10 +50,7 @@ __host__ __device__ constexpr int gemm_threads(int epi) { return 32 * (epi_warps
 
 // Widest B tile of an epilogue kind, and the shared memory each epilogue warp needs.
 __host__ __device__ constexpr int bn_max(int epi) { return (epi == kTcResid || epi == kTcBandSplit) ? 192 : 256; }
-__host__ __device__ constexpr int warp_stage_bytes(int epi) {
-  return (epi == kTcResid || epi == kTcBandSplit) ? 4096 + 2048          // fp32 box + fp16 box
-                                                  : 2 * 2048;            // two 2 KB boxes
-}
+__host__ __device__ constexpr int warp_stage_bytes(int epi) { return 2 * 2048; }  // two 2 KB boxes
 
 template <int EPI>
 struct SmemLayout {
@@ -131,6 +128,20 @@ __device__ __forceinline__ void box64_put_row(uint8_t *box, int row, const uint4
   for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4 *>(box + row * 64 + ((q ^ ((row >> 1) & 3)) << 4)) = d[q];
 }
 
+__device__ __forceinline__ void box64_get_row(const uint8_t *box, int row, float *v) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 a = *reinterpret_cast<const uint4 *>(box + row * 64 + ((q ^ ((row >> 1) & 3)) << 4));
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+      v[8 * q + 2 * i] = f.x;
+      v[8 * q + 2 * i + 1] = f.y;
+    }
+  }
+}
+
 // Token of row m of group g: band-major rows (a_mode 1) are frame m of band g.
 __device__ __forceinline__ long long token_of(const GemmParams &p, int m, int g) {
   return p.a_mode == 1 ? (long long)m * p.nb + g : (long long)m;
@@ -158,6 +169,15 @@ __device__ __forceinline__ void load_bias32(const float *b, float *bv) {
     const float4 x = b4[j];
     bv[4 * j] = x.x; bv[4 * j + 1] = x.y; bv[4 * j + 2] = x.z; bv[4 * j + 3] = x.w;
   }
+}
+
+// A row's sum of squares from its `parts` partial sums (one per (column tile, epilogue warp)
+// of the producing GEMM), added in a fixed order so every run gives the same value.
+__device__ __forceinline__ float row_ss(const float *s, long long row, int parts) {
+  const float *q = s + row * parts;
+  float a = 0.f;
+  for (int i = 0; i < parts; ++i) a += q[i];
+  return a;
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -283,7 +303,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       const bool v_ = m_ < p.M;
       if (EPI == kTcQkv) {
         qr_pf = qkv_row(p, v_ ? m_ : 0, t_.g);
-        ss_pf = (v_ && p.ss_in) ? p.ss_in[qr_pf.tok] : 1.f;
+        ss_pf = (v_ && p.ss_in) ? row_ss(p.ss_in, qr_pf.tok, p.ss_in_parts) : 1.f;
         // rotary pairs only for q and k column blocks; 16-byte loads (a row's 16 pairs are
         // 128 contiguous bytes at a 128-byte offset of the table's 256-byte row)
         if (p.dh == 64 && t_.nblk * p.BN < 2 * p.A) {
@@ -296,11 +316,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           }
         }
       } else if (EPI == kTcGelu || EPI == kTcGeglu) {
-        ss_pf = (v_ && p.ss_in) ? p.ss_in[m_] : 1.f;
+        ss_pf = (v_ && p.ss_in) ? row_ss(p.ss_in, m_, p.ss_in_parts) : 1.f;
       } else if (EPI == kTcTanh) {
-        ss_pf = (v_ && p.ss_in) ? p.ss_in[token_of(p, m_, t_.g)] : 1.f;
+        ss_pf = (v_ && p.ss_in) ? row_ss(p.ss_in, token_of(p, m_, t_.g), p.ss_in_parts) : 1.f;
       } else if (EPI == kTcResid) {
-        ss_pf = (v_ && p.res_ss) ? p.res_ss[m_] : 1.f;
+        ss_pf = (v_ && p.res_ss) ? row_ss(p.res_ss, m_, p.ss_in_parts) : 1.f;
       }
     };
     row_fetch(blockIdx.x);
@@ -330,15 +350,16 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       if (EPI == kTcQkv || EPI == kTcGelu || EPI == kTcGeglu || EPI == kTcTanh) rs = rsq;
       const float res_s = rsq;  // kTcResid
       row_fetch(tile + gridDim.x);
-      // residual prefetch (kTcResid): lane covers rows i*4 + lane/8, 16-byte piece lane%8
-      uint4 pre[8];
+      // residual prefetch (kTcResid, fp16 rows of 64 bytes): lane covers rows i*8 + lane/4,
+      // 16-byte piece lane%4
+      uint4 pre[4];
       int c = sub;
       if (EPI == kTcResid && c < nchunks) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = i * 4 + (lane >> 3);
+        for (int i = 0; i < 4; ++i) {
+          const int r = i * 8 + (lane >> 2);
           pre[i] = (m0w + r < p.M)
-                       ? *reinterpret_cast<const uint4 *>(p.X + (long long)(m0w + r) * p.ld + nbase + 32 * c + (lane & 7) * 4)
+                       ? *reinterpret_cast<const uint4 *>(p.Xh + (long long)(m0w + r) * p.ld + nbase + 32 * c + (lane & 3) * 8)
                        : make_uint4(0, 0, 0, 0);
         }
       }
@@ -350,20 +371,21 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         const bool full_chunk = c0 + 32 <= gr.N;
         float v[32];
         if (EPI == kTcResid || EPI == kTcBandSplit) {
-          uint8_t *xb = stg, *hb = stg + 4096;
-          // the previous boxes' stores must have read their sources
-          if (lane == 0) tc::bulk_wait_read<0>();
+          // the fp16 residual stream: x (+ bias) + acc, its row statistics in fp32, stored fp16
+          uint8_t *hb = stg + (nstore & 1) * 2048;
+          // the box's previous store (two chunks ago) must have read it
+          if (lane == 0) tc::bulk_wait_read<1>();
           __syncwarp();
           float x[32];
           if (EPI == kTcResid) {
             // residual rows: coalesced pieces -> swizzled box -> own row
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int r = i * 4 + (lane >> 3), q = lane & 7;
-              *reinterpret_cast<uint4 *>(xb + r * 128 + ((q ^ (r & 7)) << 4)) = pre[i];
+            for (int i = 0; i < 4; ++i) {
+              const int r = i * 8 + (lane >> 2), q = lane & 3;
+              *reinterpret_cast<uint4 *>(hb + r * 64 + ((q ^ ((r >> 1) & 3)) << 4)) = pre[i];
             }
             __syncwarp();
-            box128_get_row(xb, lane, x);
+            box64_get_row(hb, lane, x);
             if (p.res_ss) {
               float gv[32];
               load_bias32(p.res_gain + c0, gv);
@@ -372,10 +394,10 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
             }
             if (c + kSplit < nchunks) {
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const int r = i * 4 + (lane >> 3);
+              for (int i = 0; i < 4; ++i) {
+                const int r = i * 8 + (lane >> 2);
                 pre[i] = (m0w + r < p.M)
-                             ? *reinterpret_cast<const uint4 *>(p.X + (long long)(m0w + r) * p.ld + c0 + 32 * kSplit + (lane & 7) * 4)
+                             ? *reinterpret_cast<const uint4 *>(p.Xh + (long long)(m0w + r) * p.ld + c0 + 32 * kSplit + (lane & 3) * 8)
                              : make_uint4(0, 0, 0, 0);
               }
             }
@@ -404,22 +426,17 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
               sqg += y * y;
             }
           }
-          box128_put_row(xb, lane, x);
           uint4 d[4];
           pack16(x, d);
           box64_put_row(hb, lane, d);
           tc::fence_proxy_async();
           __syncwarp();
           if (lane == 0) {
-            if (EPI == kTcResid) {
-              tc::tma_store_2d(&tmC, xb, c0, m0w);
-              tc::tma_store_2d(&tmD, hb, c0, m0w);
-            } else {
-              tc::tma_store_3d(&tmC, xb, c0, ti.g, m0w);
-              tc::tma_store_3d(&tmD, hb, c0, ti.g, m0w);
-            }
+            if (EPI == kTcResid) tc::tma_store_2d(&tmD, hb, c0, m0w);
+            else tc::tma_store_3d(&tmD, hb, c0, ti.g, m0w);
             tc::bulk_commit();
           }
+          ++nstore;
           continue;
         }
         tc::tmem_ld32(tbase + 32 * c, v);
@@ -567,9 +584,12 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           }
         }
       }
-      if (EPI == kTcResid && valid && p.ss_out && sub < nchunks) atomicAdd(p.ss_out + m, sq);
-      if (EPI == kTcResid && valid && p.ssg_out && sub < nchunks) atomicAdd(p.ssg_out + m, sqg);
-      if (EPI == kTcBandSplit && valid && sub < nchunks) atomicAdd(p.ss_out + (long long)m * p.nb + ti.g, sq);
+      // this warp's partial row sums: one slot per (column tile, warp of the quarter), written
+      // (zero when the warp had no chunk) so the consumer adds all slots in a fixed order
+      const int slot = ti.nblk * kSplit + sub;
+      if (EPI == kTcResid && valid && p.ss_out) p.ss_out[(long long)m * p.ss_out_parts + slot] = sq;
+      if (EPI == kTcResid && valid && p.ssg_out) p.ssg_out[(long long)m * p.ss_out_parts + slot] = sqg;
+      if (EPI == kTcBandSplit && valid) p.ss_out[((long long)m * p.nb + ti.g) * p.ss_out_parts + slot] = sq;
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(tempty + acc);
@@ -600,6 +620,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int EPI>
 constexpr size_t smem_bytes() { return SmemLayout<EPI>::total + 1024; }
+static_assert(smem_bytes<kTcQkv>() <= 232448 && smem_bytes<kTcResid>() <= 232448 && smem_bytes<kTcGelu>() <= 232448 &&
+                  smem_bytes<kTcBandSplit>() <= 232448 && smem_bytes<kTcGlu>() <= 232448,
+              "shared memory per CTA over the 227 KB limit");
 
 }  // namespace
 

@@ -126,7 +126,7 @@ bool debug_buffer_fp16(mrf_handle *h, const std::string &name, const void **ptr,
 // The fp16 schedule's per-forward workspace pointers, and their layout in one
 // caller-provided region (sched_fp16.cu); used by mrf_forward_static.
 struct Fp16Workspace {
-  float *X, *ss;
+  float *ss;
   __half *Xh, *QKV, *O, *Hh, *H1, *H2, *A_bs;
   float *ssx, *ssg;
 };

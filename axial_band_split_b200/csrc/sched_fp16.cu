@@ -1,14 +1,14 @@
 // fp16 tensor-core schedule: weight packing, workspace and the per-forward launch list.
 //
 // Per forward (N_tok = B*T*bands tokens, token (b*T + t)*bands + k):
-//   band split (gather + norm + Linear)        -> X fp32, X fp16, |x|^2
+//   band split (gather + norm + Linear)        -> x (fp16 residual stream), |x|^2
 //   per transformer (time axis, then band axis, depth times):
 //     QKV+gates GEMM, RoPE epilogue            -> q, k, v fp16 in attention layout, gates
 //     attention                                -> O fp16 (times the gate)
-//     out-projection GEMM, residual epilogue   -> X, X fp16, |x|^2
+//     out-projection GEMM, residual epilogue   -> x, |x|^2
 //     FF1 GEMM, GELU epilogue                  -> H fp16
-//     FF2 GEMM, residual epilogue              -> X, X fp16, |x|^2
-//     output norm                              -> X, X fp16, |x|^2
+//     FF2 GEMM, residual epilogue              -> x, |x|^2 and |g x|^2 (the output norm, deferred
+//                                                 to the consumers' epilogues)
 //   mask head: per-band GEMMs (tanh, tanh, GLU), the GLU epilogue adding each band feature
 //   into its stft_repr row of the zeroed masks (the overlap average)  -> masks
 //
@@ -56,9 +56,11 @@ struct Fp16State {
   GemmGroup *g_m0 = nullptr, *g_mid = nullptr, *g_last = nullptr;
   int n_last_tiles = 0;
   // workspace
-  float *X = nullptr, *ss = nullptr;
-  // deferred output norm: |x|^2 and |g x|^2 of the last FF2 output (g = sqrt(D) gamma_out)
-  float *ssx = nullptr, *ssg = nullptr;
+  // Row sums of squares as partial slots (parts_* a row, added in order by the consumer): |x|^2
+  // of the out-projection output (ss), and the deferred output norm's |x|^2 and |g x|^2 of the
+  // last FF2 output (ssx, ssg; g = sqrt(D) gamma_out; ssg holds the band split's |x|^2 first)
+  float *ss = nullptr, *ssx = nullptr, *ssg = nullptr;
+  int parts_res = 0, parts_bs = 0;
   __half *Xh = nullptr, *QKV = nullptr, *O = nullptr, *Hh = nullptr, *H1 = nullptr, *H2 = nullptr;
   int ldq = 0;  // row length of QKV: [q | k | v | gates], padded to a multiple of 8
   int sms = 148;
@@ -250,17 +252,19 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   if (!f->g_qkv || !f->g_out || !f->g_ff1 || !f->g_ff2 || !f->g_m0 || !f->g_mid || !f->g_last) return MRF_ENOMEM;
   // workspace
   f->ldq = cdiv(3 * A + H, 8) * 8;
-  f->X = h->alloc<float>(NT * D);
   f->Xh = h->alloc<__half>(NT * D);
-  f->ss = h->alloc<float>(NT);
-  f->ssx = h->alloc<float>(NT);
-  f->ssg = h->alloc<float>(NT);
+  f->parts_res = cdiv(D, kBnNarrow) * 2;  // residual GEMMs: 8 epilogue warps, 2 per lane quarter
+  f->parts_bs = cdiv(D, kBnNarrow) * 4;   // band split: 16 epilogue warps, 4 per lane quarter
+  const int parts = std::max(f->parts_res, f->parts_bs);
+  f->ss = h->alloc<float>(NT * parts);
+  f->ssx = h->alloc<float>(NT * parts);
+  f->ssg = h->alloc<float>(NT * parts);
   f->QKV = h->alloc<__half>(NT * f->ldq);
   f->O = h->alloc<__half>(NT * A);
   f->Hh = h->alloc<__half>(NT * FF);
   f->H1 = h->alloc<__half>((long long)nb * MBT * MH);
   f->H2 = h->alloc<__half>((long long)nb * MBT * MH);
-  if (!f->X || !f->Xh || !f->ss || !f->ssx || !f->ssg || !f->QKV || !f->O || !f->Hh || !f->H1 || !f->H2)
+  if (!f->Xh || !f->ss || !f->ssx || !f->ssg || !f->QKV || !f->O || !f->Hh || !f->H1 || !f->H2)
     return MRF_ENOMEM;
   // rows past a forward's B*T are read by ragged tiles (and discarded): keep them finite
   if (cudaMemset(f->QKV, 0, NT * f->ldq * 2) != cudaSuccess || cudaMemset(f->H1, 0, (size_t)nb * MBT * MH * 2) != cudaSuccess ||
@@ -279,14 +283,18 @@ bool debug_buffer_fp16(mrf_handle *h, const std::string &name, const void **ptr,
     const long long rows = BT * h->cfg.num_bands;
     static thread_local std::vector<float> hx;
     hx.resize((size_t)rows * D);
-    if (cudaMemcpy(hx.data(), f->X, hx.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess) return false;
+    std::vector<__half> xh((size_t)rows * D);
+    if (cudaMemcpy(xh.data(), f->Xh, xh.size() * 2, cudaMemcpyDeviceToHost) != cudaSuccess) return false;
+    for (size_t i = 0; i < xh.size(); ++i) hx[i] = __half2float(xh[i]);
     if (h->cfg.depth > 0) {
-      std::vector<float> s2(rows), g(D);
-      if (cudaMemcpy(s2.data(), f->ssx, rows * 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
+      std::vector<float> s2((size_t)rows * f->parts_res), g(D);
+      if (cudaMemcpy(s2.data(), f->ssx, s2.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
           cudaMemcpy(g.data(), f->tr.back().gout, D * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
         return false;
       for (long long r = 0; r < rows; ++r) {
-        const float inv = 1.f / std::max(std::sqrt(s2[r]), 1e-12f);
+        float ssr = 0.f;
+        for (int q = 0; q < f->parts_res; ++q) ssr += s2[(size_t)r * f->parts_res + q];
+        const float inv = 1.f / std::max(std::sqrt(ssr), 1e-12f);
         for (int k = 0; k < D; ++k) hx[(size_t)r * D + k] *= inv * g[k];
       }
     }
@@ -380,7 +388,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     ok = ok && make_tmap_f16(&wmaps[w0 + c.mask_depth], f->mw_last[s], MH, rows_last, 1, MH, rows_last * MH, kBnWide, 1);
   }
   // bulk-store output maps
-  CUtensorMap mXo, mXho, mXbs, mXhbs, mHo, mHo16, mH1o, mH2o, mQKVo;
+  CUtensorMap mXho, mXhbs, mHo, mHo16, mH1o, mH2o, mQKVo;
   {
     const unsigned long long BT = (unsigned long long)B * T;
     const unsigned long long dx[3] = {(unsigned long long)D, (unsigned long long)nb, BT};
@@ -389,8 +397,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     const unsigned long long dh3[3] = {(unsigned long long)MH, BT, (unsigned long long)nb};
     const unsigned long long sh3[2] = {(unsigned long long)MH, (unsigned long long)MBT * MH};
     const unsigned bh[3] = {32, 32, 1};
-    ok = ok && map2(&mXo, f->X, kTmF32, D, M, D, 32, 128) && map2(&mXho, f->Xh, kTmF16, D, M, D, 32, 64) &&
-         make_tmap(&mXbs, f->X, kTmF32, 3, dx, sx, bx, 128) && make_tmap(&mXhbs, f->Xh, kTmF16, 3, dx, sx, bx, 64) &&
+    ok = ok && map2(&mXho, f->Xh, kTmF16, D, M, D, 32, 64) && make_tmap(&mXhbs, f->Xh, kTmF16, 3, dx, sx, bx, 64) &&
          map2(&mHo, f->Hh, kTmF16, FF, M, FF, 32, 64) && map2(&mHo16, f->Hh, kTmF16, FF, M, FF, 16, 0) &&
          make_tmap(&mH1o, f->H1, kTmF16, 3, dh3, sh3, bh, 64) &&
          make_tmap(&mH2o, f->H2, kTmF16, 3, dh3, sh3, bh, 64) &&
@@ -404,13 +411,12 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   h->begin("band_gather");
   launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, st);
   h->end();
-  cudaMemsetAsync(f->ssg, 0, sizeof(float) * M, st);
   {
     GemmParams p = base_params(h, B * T, f->k_bs, kBnNarrow, f->g_bs, nb, nb * cdiv(D, kBnNarrow));
-    p.bias = h->b_bs; p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ssg; p.ld = D; p.nb = nb;
+    p.bias = h->b_bs; p.Xh = f->Xh; p.ss_out = f->ssg; p.ss_out_parts = f->parts_bs; p.ld = D; p.nb = nb;
     p.stall_test = h->stall_test ? 1 : 0;
     h->stall_test = false;
-    gemm(h, "gemm_band_split", kTcBandSplit, mAbs, mWbs, p, &mXbs, &mXhbs);
+    gemm(h, "gemm_band_split", kTcBandSplit, mAbs, mWbs, p, &mXhbs, &mXhbs);
   }
 
   for (int i = 0; i < 2 * c.depth; ++i) {
@@ -421,6 +427,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     // [q | k | v | gates] per token (RoPE positions along this transformer's axis)
     GemmParams p = base_params(h, M, D, kBnWide, f->g_qkv, 1, cdiv(3 * A + H, kBnWide));
     p.ss_in = f->ssg;  // |g x|^2 of the previous output (band split: |x|^2)
+    p.ss_in_parts = i == 0 ? f->parts_bs : f->parts_res;
     p.rope = h->d_rope; p.gbias = w.bg;
     p.B = B; p.T = T; p.nb = nb; p.H = H; p.dh = dh; p.A = A; p.axis = axis;
     // the tensor-core attention takes scores in log2 units: fold log2(e) / sqrt(dh) into q
@@ -438,23 +445,22 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
       launch_attention_simt_f16(f->QKV, f->ldq, f->O, B, T, nb, H, dh, axis, st);
     h->end();
 
-    cudaMemsetAsync(f->ss, 0, sizeof(float) * M, st);
     p = base_params(h, M, A, kBnNarrow, f->g_out, 1, cdiv(D, kBnNarrow));
-    p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ss; p.ld = D;
-    if (i > 0) { p.res_ss = f->ssx; p.res_gain = f->tr[i - 1].gout; }  // the previous output norm
-    gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p, &mXo, &mXho);
+    p.Xh = f->Xh; p.ss_out = f->ss; p.ss_out_parts = f->parts_res; p.ld = D;
+    if (i > 0) {  // the previous output norm
+      p.res_ss = f->ssx; p.res_gain = f->tr[i - 1].gout; p.ss_in_parts = f->parts_res;
+    }
+    gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p, &mXho, &mXho);
 
     p = base_params(h, M, D, kBnWide, f->g_ff1, 1, cdiv(F1, kBnWide));
-    p.ss_in = f->ss; p.bias = w.b1; p.out_h = f->Hh; p.ldo = FF;
+    p.ss_in = f->ss; p.ss_in_parts = f->parts_res; p.bias = w.b1; p.out_h = f->Hh; p.ldo = FF;
     if (c.ff_act == 1) gemm(h, "gemm_ff1_geglu", kTcGeglu, mXh, mW1, p, &mHo16);
     else gemm(h, "gemm_ff1_gelu", kTcGelu, mXh, mW1, p, &mHo);
 
-    cudaMemsetAsync(f->ssx, 0, sizeof(float) * M, st);
-    cudaMemsetAsync(f->ssg, 0, sizeof(float) * M, st);
     p = base_params(h, M, FF, kBnNarrow, f->g_ff2, 1, cdiv(D, kBnNarrow));
-    p.X = f->X; p.Xh = f->Xh; p.ss_out = f->ssx; p.ld = D; p.bias = w.b2;
+    p.Xh = f->Xh; p.ss_out = f->ssx; p.ss_out_parts = f->parts_res; p.ld = D; p.bias = w.b2;
     p.ssg_out = f->ssg; p.out_gain = w.gout;  // the output norm is left to the consumers
-    gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p, &mXo, &mXho);
+    gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p, &mXho, &mXho);
   }
 
   // mask heads, one per stem; each GLU epilogue adds its band features into the stem's slice
@@ -468,6 +474,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     GemmParams p = base_params(h, BT, D, kBnWide, f->g_m0, nb, nb * cdiv(MH, kBnWide));
     p.a_mode = 1;
     p.ss_in = c.depth > 0 ? f->ssx : nullptr;  // 1 / |x| of the deferred last output norm
+    p.ss_in_parts = f->parts_res;
     p.nb = nb;
     p.bias = f->mb[s][0]; p.out_h = f->H1; p.ldo = MH; p.out_group_stride = MBT * MH;
     gemm(h, "gemm_mask_tanh", kTcTanh, mXband, wmaps[w0], p, &mH1o);
@@ -513,8 +520,9 @@ size_t fp16_workspace_layout(mrf_handle *h, void *base, bool apply, Fp16Workspac
     off += (n + 255) & ~size_t(255);
     return o;
   };
-  const size_t oA = take((size_t)nb * MBT * f->k_bs * 2), oX = take(NT * D * 4), oXh = take(NT * D * 2),
-               oss = take(NT * 4), ossx = take(NT * 4), ossg = take(NT * 4);
+  const size_t parts = (size_t)std::max(f->parts_res, f->parts_bs);
+  const size_t oA = take((size_t)nb * MBT * f->k_bs * 2), oXh = take(NT * D * 2),
+               oss = take(NT * 4 * parts), ossx = take(NT * 4 * parts), ossg = take(NT * 4 * parts);
   const size_t oQ = take(NT * f->ldq * 2);
   const size_t oO = take(NT * A * 2), oHh = take(NT * FF * 2), oH1 = take((size_t)nb * MBT * MH * 2),
                oH2 = take((size_t)nb * MBT * MH * 2);
@@ -522,10 +530,9 @@ size_t fp16_workspace_layout(mrf_handle *h, void *base, bool apply, Fp16Workspac
   if (qkv_offset) *qkv_offset = oQ;
   if (qkv_bytes) *qkv_bytes = oO - oQ;
   if (apply && f) {
-    if (saved) *saved = {f->X, f->ss, f->Xh, f->QKV, f->O, f->Hh, f->H1, f->H2, f->A_bs, f->ssx, f->ssg};
+    if (saved) *saved = {f->ss, f->Xh, f->QKV, f->O, f->Hh, f->H1, f->H2, f->A_bs, f->ssx, f->ssg};
     uint8_t *b = static_cast<uint8_t *>(base);
     f->A_bs = reinterpret_cast<__half *>(b + oA);
-    f->X = reinterpret_cast<float *>(b + oX);
     f->Xh = reinterpret_cast<__half *>(b + oXh);
     f->ss = reinterpret_cast<float *>(b + oss);
     f->ssx = reinterpret_cast<float *>(b + ossx);
@@ -541,7 +548,7 @@ size_t fp16_workspace_layout(mrf_handle *h, void *base, bool apply, Fp16Workspac
 
 void fp16_restore_workspace(mrf_handle *h, const Fp16Workspace &s) {
   Fp16State *f = h->f16;
-  f->X = s.X; f->ss = s.ss; f->Xh = s.Xh; f->QKV = s.QKV;
+  f->ss = s.ss; f->Xh = s.Xh; f->QKV = s.QKV;
   f->O = s.O; f->Hh = s.Hh; f->H1 = s.H1; f->H2 = s.H2; f->A_bs = s.A_bs; f->ssx = s.ssx; f->ssg = s.ssg;
 }
 
