@@ -41,7 +41,8 @@ struct GemmParams {
   const float *ss_in;       // row scale 1 / max(sqrt(sum of the row's slots), eps); null: 1
   int ss_in_parts;
   const float *bias;
-  __half *Xh;               // fp16 residual stream [M, ld] (kTcResid reads and rewrites it)
+  __half *Xh;               // the 16-bit residual stream [M, ld] (fp16: kTcResid reads and rewrites it)
+  float *X;                 // bf16 schedule: the fp32 master copy of the residual stream (read and rewritten)
   float *ss_out;            // row sums of squares of the output (partial slots)
   int ss_out_parts;
   int ld;
@@ -95,7 +96,10 @@ bool gemm_tc_init();
 //  box 32x32 swizzle 64; kTcTanh: out fp16 (ldo, frames, groups) box 32x32x1 swizzle 64;
 //  kTcGlu: none (atomic adds into the masks); kTcGeglu: out fp16 [M, ldo] box 16x32,
 //  no swizzle).  Unused maps may be any valid map.
-void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
+// bf16: A, W and every 16-bit output in bf16 (MRF_BF16), the residual kinds also keeping the fp32
+// master copy X (tmC: X fp32 box 32x32 swizzle 128, or the 3-D (ld, nb, frames) 32x1x32 box of the
+// band split); otherwise fp16.
+void launch_gemm_tc(int epi, bool bf16, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
                     const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st);
 
 }  // namespace mrf

@@ -28,6 +28,8 @@
 // O accumulates in tensor memory across key blocks; a row's running max is raised (and
 // its O row rescaled in place) only when a block's max exceeds it by more than 2^8, so
 // the unnormalised p stay below 256 and most blocks need no correction.
+#include <cuda_bf16.h>
+
 #include <cmath>
 
 #include "gemm_tc.cuh"
@@ -181,9 +183,22 @@ __device__ __forceinline__ void tma_store_5d(const CUtensorMap *map, const void 
                : "memory");
 }
 
+// Two floats as one pair of the schedule's 16-bit type (fp16, or bf16 with kBF).
+template <bool kBF>
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t *>(&h);
+  if constexpr (kBF) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+  }
+}
+
+template <bool kBF>
+__device__ __forceinline__ float to_float16b(unsigned short v) {
+  if constexpr (kBF) return __uint_as_float((unsigned)v << 16);
+  else return __half2float(__ushort_as_half(v));
 }
 
 struct AttnArgs {
@@ -270,7 +285,7 @@ __device__ __forceinline__ TileC tile_coords(const AttnArgs &a, int item, int t)
 // fp16, and the O row rescaled in place when its max was raised.  NC live score columns at
 // tS (columns >= hi are masked); P's matching NC / 2 columns at tP.  Returns false if a
 // wait timed out.
-template <int NC>
+template <int NC, bool kBF>
 __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t tO, int hi, float &m_run, float &l,
                                               bool wait_pv, uint64_t *pv_done, uint32_t pv_parity,
                                               uint64_t *s_free, uint64_t *p_full, int lane, unsigned *status,
@@ -303,7 +318,7 @@ __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t
   if (need) { l *= alpha; m_run = m_cand; }
   uint32_t pk[NC / 2];  // p = 2^(s - m) as fp16 pairs, the P*V MMA's A operand
   float2 s4;
-  if (kExpF16x2) {
+  if (kExpF16x2 && !kBF) {
     // Pairs (s - m) through a packed f32x2 subtract, rounded to an fp16 pair and exponentiated
     // by one MUFU instruction for both (ex2.approx.f16x2), whose fp16 result is P itself.  The
     // row sum adds the same fp16 values: neighbouring pairs first in fp16 (one rounding of a
@@ -339,7 +354,7 @@ __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t
           case 2: sc = add2(sc, pp); break;
           default: sd = add2(sd, pp); break;
         }
-        pk[(i >> 1) + u] = pack_h2(pp.x, pp.y);
+        pk[(i >> 1) + u] = pack_h2<kBF>(pp.x, pp.y);
       }
     }
     const float2 s01 = add2(sa, sb), s23 = add2(sc, sd);
@@ -371,6 +386,7 @@ __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t
   return true;
 }
 
+template <bool kBF>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                    const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
@@ -465,8 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // P*V waits behind the other tile's softmax (the tensor core queues both streams)
     const int t = warp - 9;
     if (lane == 0) {
-      const uint32_t id_s = tc::idesc_f16(kRows, kKeys);
-      const uint32_t id_pv = tc::idesc_f16(kRows, kDh, true);
+      const uint32_t id_s = tc::idesc_f16(kRows, kKeys, false, kBF);
+      const uint32_t id_pv = tc::idesc_f16(kRows, kDh, true, kBF);
       int g = 0;    // key blocks consumed so far
       int ptr = 0;  // ring tile of the next item's first block (the producer's order)
       int li = 0;
@@ -565,15 +581,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int f = it.frame0 + prob, k = r & 63;
         if (k < a.n && f < a.BT) tok = (long long)f * a.nb + k;
       }
-      const __half gate = tok >= 0 ? a.qkv[tok * a.ld + 3 * a.H * kDh + it.head] : __float2half(0.f);
+      const unsigned short gate =
+          tok >= 0 ? reinterpret_cast<const unsigned short *>(a.qkv)[tok * a.ld + 3 * a.H * kDh + it.head] : 0;
       for (int j = 0; j < a.n_blocks; ++j, ++g) {
         if (!tc::mbar_wait(s_full + t, g & 1, a.status, 38, abort)) { ok = false; break; }
         tc::tc_fence_after();
         const bool go = a.axis == 0
-                            ? softmax_block<kKeys>(tS, tP, tO, min(kKeys, a.n - j * kKeys), m_run, l, j > 0,
+                            ? softmax_block<kKeys, kBF>(tS, tP, tO, min(kKeys, a.n - j * kKeys), m_run, l, j > 0,
                                                    pv_done + t, (g - 1) & 1, s_free + t, p_full + t, lane, a.status,
                                                    abort)
-                            : softmax_block<64>(tS + 64 * prob, tP + 32 * prob, tO, a.n, m_run, l, false,
+                            : softmax_block<64, kBF>(tS + 64 * prob, tP + 32 * prob, tO, a.n, m_run, l, false,
                                                 pv_done + t, 0, s_free + t, p_full + t, lane, a.status, abort);
         if (!go) { ok = false; break; }
       }
@@ -597,7 +614,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // staged in shared memory (128-byte swizzle: 16-byte chunk c of row i at c ^ (i % 8))
       // and written by one bulk tensor store per warp; rows outside the output tensor
       // (frames past T, bands past nb) are not written
-      const float gsc = tok >= 0 ? __half2float(gate) / l : 0.f;
+      const float gsc = tok >= 0 ? to_float16b<kBF>(gate) / l : 0.f;
       uint8_t *stg = smem + AttnSmem::ostage + warp * 4096;
       if (lane == 0) tc::bulk_wait_read<0>();
       __syncwarp();
@@ -605,8 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 8; ++c) {
         const float *oc = o + 8 * c;
         *reinterpret_cast<uint4 *>(stg + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-            make_uint4(pack_h2(oc[0] * gsc, oc[1] * gsc), pack_h2(oc[2] * gsc, oc[3] * gsc),
-                       pack_h2(oc[4] * gsc, oc[5] * gsc), pack_h2(oc[6] * gsc, oc[7] * gsc));
+            make_uint4(pack_h2<kBF>(oc[0] * gsc, oc[1] * gsc), pack_h2<kBF>(oc[2] * gsc, oc[3] * gsc),
+                       pack_h2<kBF>(oc[4] * gsc, oc[5] * gsc), pack_h2<kBF>(oc[6] * gsc, oc[7] * gsc));
       }
       tc::fence_proxy_async();
       __syncwarp();
@@ -644,12 +661,15 @@ bool attention_tc_init() {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, attn_tc_kernel) != cudaSuccess || fa.numRegs < kRegsLaunch) return false;
-  return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncGetAttributes(&fa, attn_tc_kernel<false>) != cudaSuccess || fa.numRegs < kRegsLaunch) return false;
+  if (cudaFuncGetAttributes(&fa, attn_tc_kernel<true>) != cudaSuccess || fa.numRegs < kRegsLaunch) return false;
+  return cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)(AttnSmem::total + 1024)) == cudaSuccess &&
+         cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)(AttnSmem::total + 1024)) == cudaSuccess;
 }
 
-bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int axis,
+bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int axis, bool bf16,
                          unsigned *status, cudaStream_t st) {
   AttnArgs a;
   a.qkv = qkv;
@@ -697,7 +717,8 @@ bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int
     return false;
   const size_t smem = AttnSmem::total + 1024;
   const int grid = (int)std::min<long long>(a.items, g_num_sms > 0 ? g_num_sms : 148);
-  attn_tc_kernel<<<grid, kThreads, smem, st>>>(tq, tk, tv, to, a);
+  if (bf16) attn_tc_kernel<true><<<grid, kThreads, smem, st>>>(tq, tk, tv, to, a);
+  else attn_tc_kernel<false><<<grid, kThreads, smem, st>>>(tq, tk, tv, to, a);
   return true;
 }
 

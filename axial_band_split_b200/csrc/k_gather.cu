@@ -1,5 +1,6 @@
-// Mel-band gather and BandSplit norm of the fp16 schedule: per (band, frame) the band's
-// features divided by their L2 norm, fp16, laid out as the A operand of the band-split GEMM.
+// Mel-band gather and BandSplit norm of the tensor-core schedule: per (band, frame) the band's
+// features divided by their L2 norm, in the schedule's 16-bit type (fp16 or bf16), laid out as
+// the A operand of the band-split GEMM.
 //
 // "Mel-Band RoFormer — architecture, inference hot path & RTX 3050 feasibility", section "The
 // mel-band split, exactly": band k's features at frame t are the (re, im) pairs of the
@@ -20,6 +21,7 @@
 //           shared memory; rows up to the band's width rounded up to 64 features store zeros.
 // Keeping the registers and shared memory small lets many CTAs share an SM, which hides the
 // loads' latency; the widest bands (40 times the narrowest's data) are scheduled first.
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "mrf_internal.h"
@@ -50,7 +52,19 @@ __device__ __forceinline__ float4 load_pair(const float *p, int t, int T) {
   return v;
 }
 
-template <bool kEvenT>
+// Two floats as one pair of the schedule's 16-bit type (fp16, or bf16 with kBF).
+template <bool kBF>
+__device__ __forceinline__ uint32_t pack2(float a, float b) {
+  if constexpr (kBF) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+  }
+}
+
+template <bool kEvenT, bool kBF>
 __global__ void __launch_bounds__(kThreads) band_gather_kernel(const float *__restrict__ in,
                                                                    const int32_t *__restrict__ feat_row,
                                                                    const BandDesc *__restrict__ bands, int nb,
@@ -95,23 +109,27 @@ __global__ void __launch_bounds__(kThreads) band_gather_kernel(const float *__re
   for (int r = rl; r < prow; r += 16) {
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r < nrows) v = load_pair<kEvenT>(base + (long long)r * T * 2, t, T);
-    if (st0) *reinterpret_cast<__half2 *>(out0 + 2 * r) = __floats2half2_rn(v.x * sc0, v.y * sc0);
-    if (st1) *reinterpret_cast<__half2 *>(out1 + 2 * r) = __floats2half2_rn(v.z * sc1, v.w * sc1);
+    if (st0) *reinterpret_cast<uint32_t *>(out0 + 2 * r) = pack2<kBF>(v.x * sc0, v.y * sc0);
+    if (st1) *reinterpret_cast<uint32_t *>(out1 + 2 * r) = pack2<kBF>(v.z * sc1, v.w * sc1);
   }
 }
 
 }  // namespace
 
 void launch_band_gather(const float *in, const int32_t *feat_row, const BandDesc *bands, int nb, int B, int T,
-                        int rows, long long frame_stride, int k_stride, __half *A, cudaStream_t st) {
+                        int rows, long long frame_stride, int k_stride, __half *A, bool bf16, cudaStream_t st) {
   const int tiles = (T + kFrames - 1) / kFrames;
   const unsigned grid = (unsigned)(nb * B * tiles);
-  if (T % 2 == 0)
-    band_gather_kernel<true><<<grid, kThreads, 0, st>>>(in, feat_row, bands, nb, B, T, rows, tiles, frame_stride,
-                                                           k_stride, A);
-  else
-    band_gather_kernel<false><<<grid, kThreads, 0, st>>>(in, feat_row, bands, nb, B, T, rows, tiles,
-                                                            frame_stride, k_stride, A);
+#define MRF_GATHER(E, BF) \
+  band_gather_kernel<E, BF><<<grid, kThreads, 0, st>>>(in, feat_row, bands, nb, B, T, rows, tiles, frame_stride, k_stride, A)
+  if (T % 2 == 0) {
+    if (bf16) MRF_GATHER(true, true);
+    else MRF_GATHER(true, false);
+  } else {
+    if (bf16) MRF_GATHER(false, true);
+    else MRF_GATHER(false, false);
+  }
+#undef MRF_GATHER
 }
 
 }  // namespace mrf

@@ -22,6 +22,7 @@
 // tensor map's swizzled layout and one lane issues a bulk tensor store (cp.async.bulk.tensor),
 // so global writes leave the SM as whole lines; rows past M are clipped by the tensor map.
 #include <cudaTypedefs.h>
+#include <cuda_bf16.h>
 
 #include <cmath>
 #include <cstdio>
@@ -50,23 +51,35 @@ __host__ __device__ constexpr int gemm_threads(int epi) { return 32 * (epi_warps
 
 // Widest B tile of an epilogue kind, and the shared memory each epilogue warp needs.
 __host__ __device__ constexpr int bn_max(int epi) { return (epi == kTcResid || epi == kTcBandSplit) ? 192 : 256; }
-__host__ __device__ constexpr int warp_stage_bytes(int epi) { return 2 * 2048; }  // two 2 KB boxes
+// Per epilogue warp: two 2 KB boxes; the bf16 schedule's residual kinds keep an fp32 master
+// copy of the residual stream and stage a 4 KB fp32 box and a 2 KB bf16 box instead.
+__host__ __device__ constexpr int warp_stage_bytes(int epi, bool bf) {
+  return (bf && (epi == kTcResid || epi == kTcBandSplit)) ? 4096 + 2048 : 2 * 2048;
+}
 
-template <int EPI>
+template <int EPI, bool kBF>
 struct SmemLayout {
   static constexpr int b_stage = bn_max(EPI) * BK * 2;
   static constexpr int a_off = 0;
   static constexpr int b_off = gemm_stages(EPI) * A_STAGE;
   static constexpr int stg_off = b_off + gemm_stages(EPI) * b_stage;        // 1024-aligned
-  static constexpr int bar_off = stg_off + epi_warps(EPI) * warp_stage_bytes(EPI);
+  static constexpr int bar_off = stg_off + epi_warps(EPI) * warp_stage_bytes(EPI, kBF);
   static constexpr int total = bar_off + 256;
 };
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
 
+// Two floats as one 32-bit pair of the schedule's 16-bit type (fp16, or bf16 with kBF), rounded
+// to nearest even.
+template <bool kBF>
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t *>(&h);
+  if constexpr (kBF) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+  } else {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t *>(&h);
+  }
 }
 
 __device__ __forceinline__ int find_group(const GemmGroup *g, int n, int tile, int m_tiles) {
@@ -97,12 +110,13 @@ __device__ __forceinline__ TileInfo decode_tile(const GemmParams &p, int tile) {
 
 
 
+template <bool kBF>
 __device__ __forceinline__ void pack16(const float *v, uint4 (&d)[4]) {
-  // 32 floats -> 32 fp16 (64 bytes)
+  // 32 floats -> 32 16-bit values (64 bytes)
 #pragma unroll
   for (int q = 0; q < 4; ++q)
-    d[q] = make_uint4(pack_h2(v[8 * q], v[8 * q + 1]), pack_h2(v[8 * q + 2], v[8 * q + 3]),
-                      pack_h2(v[8 * q + 4], v[8 * q + 5]), pack_h2(v[8 * q + 6], v[8 * q + 7]));
+    d[q] = make_uint4(pack_h2<kBF>(v[8 * q], v[8 * q + 1]), pack_h2<kBF>(v[8 * q + 2], v[8 * q + 3]),
+                      pack_h2<kBF>(v[8 * q + 4], v[8 * q + 5]), pack_h2<kBF>(v[8 * q + 6], v[8 * q + 7]));
 }
 
 // Box rows in shared memory, in the layouts the tensor maps' swizzle modes define:
@@ -181,12 +195,12 @@ __device__ __forceinline__ float row_ss(const float *s, long long row, int parts
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int EPI>
+template <int EPI, bool kBF>
 __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                    const GemmParams p) {
-  using L = SmemLayout<EPI>;
+  using L = SmemLayout<EPI, kBF>;
   constexpr int kEpiWarps = epi_warps(EPI), kSplit = kEpiWarps / 4, kGemmStages = gemm_stages(EPI);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -259,7 +273,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         const uint32_t aphase = (local >> 1) & 1;
         int n_eff = min(p.BN, gr.N - ti.nblk * p.BN);
         n_eff = (n_eff + 15) & ~15;
-        const uint32_t idesc = tc::idesc_f16(BM, n_eff);
+        const uint32_t idesc = tc::idesc_f16(BM, n_eff, false, kBF);
         const uint32_t d_tmem = tmem_base + acc * 256;
         const int kblocks = gr.kblocks ? gr.kblocks : p.K / BK;
         if (!tc::mbar_wait(tempty + acc, aphase ^ 1, p.status, 11, abort)) break;
@@ -287,7 +301,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   } else {
     // ---------------- epilogue warps 0-7
     const int quarter = warp & 3, sub = warp >> 2;  // rows 32 quarter.., chunks sub, sub + kSplit, ...
-    uint8_t *stg = smem + L::stg_off + warp * warp_stage_bytes(EPI);
+    uint8_t *stg = smem + L::stg_off + warp * warp_stage_bytes(EPI, kBF);
     int nstore = 0;  // boxes this warp has stored (double-buffer parity)
     int local = 0;
     // The row's deferred-norm sum of squares (and, for QKV, its rotary (cos, sin) pairs),
@@ -350,19 +364,25 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       if (EPI == kTcQkv || EPI == kTcGelu || EPI == kTcGeglu || EPI == kTcTanh) rs = rsq;
       const float res_s = rsq;  // kTcResid
       row_fetch(tile + gridDim.x);
-      // residual prefetch (kTcResid, fp16 rows of 64 bytes): lane covers rows i*8 + lane/4,
-      // 16-byte piece lane%4
-      uint4 pre[4];
+      // residual prefetch (kTcResid): fp16 rows of 64 bytes, lane covering rows i*8 + lane/4 and
+      // 16-byte piece lane%4; with kBF the fp32 master rows of 128 bytes, rows i*4 + lane/8, piece lane%8
+      constexpr int kPieces = kBF ? 8 : 4;
+      uint4 pre[kPieces];
       int c = sub;
-      if (EPI == kTcResid && c < nchunks) {
+      auto residual_fetch = [&](int col) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = i * 8 + (lane >> 2);
-          pre[i] = (m0w + r < p.M)
-                       ? *reinterpret_cast<const uint4 *>(p.Xh + (long long)(m0w + r) * p.ld + nbase + 32 * c + (lane & 3) * 8)
-                       : make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < kPieces; ++i) {
+          const int r = kBF ? i * 4 + (lane >> 3) : i * 8 + (lane >> 2);
+          const bool ok = m0w + r < p.M;
+          if constexpr (kBF)
+            pre[i] = ok ? *reinterpret_cast<const uint4 *>(p.X + (long long)(m0w + r) * p.ld + col + (lane & 7) * 4)
+                        : make_uint4(0, 0, 0, 0);
+          else
+            pre[i] = ok ? *reinterpret_cast<const uint4 *>(p.Xh + (long long)(m0w + r) * p.ld + col + (lane & 3) * 8)
+                        : make_uint4(0, 0, 0, 0);
         }
-      }
+      };
+      if (EPI == kTcResid && c < nchunks) residual_fetch(nbase + 32 * c);
       if (!tc::mbar_wait(tfull + acc, aphase, p.status, 14, abort)) break;
       tc::tc_fence_after();
       float sq = 0.f, sqg = 0.f;
@@ -371,36 +391,43 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         const bool full_chunk = c0 + 32 <= gr.N;
         float v[32];
         if (EPI == kTcResid || EPI == kTcBandSplit) {
-          // the fp16 residual stream: x (+ bias) + acc, its row statistics in fp32, stored fp16
-          uint8_t *hb = stg + (nstore & 1) * 2048;
-          // the box's previous store (two chunks ago) must have read it
-          if (lane == 0) tc::bulk_wait_read<1>();
+          // x (+ bias) + acc with its row statistics in fp32.  fp16: the residual stream is the
+          // fp16 buffer itself.  bf16: an fp32 master copy X, and the bf16 copy the GEMMs read.
+          uint8_t *hb = kBF ? stg + 4096 : stg + (nstore & 1) * 2048;
+          uint8_t *xb = stg;  // kBF: the fp32 box
+          // the boxes' previous stores must have read them (fp16: the store two chunks ago)
+          if (lane == 0) {
+            if (kBF) tc::bulk_wait_read<0>();
+            else tc::bulk_wait_read<1>();
+          }
           __syncwarp();
           float x[32];
           if (EPI == kTcResid) {
             // residual rows: coalesced pieces -> swizzled box -> own row
+            if constexpr (kBF) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int r = i * 8 + (lane >> 2), q = lane & 3;
-              *reinterpret_cast<uint4 *>(hb + r * 64 + ((q ^ ((r >> 1) & 3)) << 4)) = pre[i];
+              for (int i = 0; i < 8; ++i) {
+                const int r = i * 4 + (lane >> 3), q = lane & 7;
+                *reinterpret_cast<uint4 *>(xb + r * 128 + ((q ^ (r & 7)) << 4)) = pre[i];
+              }
+              __syncwarp();
+              box128_get_row(xb, lane, x);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int r = i * 8 + (lane >> 2), q = lane & 3;
+                *reinterpret_cast<uint4 *>(hb + r * 64 + ((q ^ ((r >> 1) & 3)) << 4)) = pre[i];
+              }
+              __syncwarp();
+              box64_get_row(hb, lane, x);
             }
-            __syncwarp();
-            box64_get_row(hb, lane, x);
             if (p.res_ss) {
               float gv[32];
               load_bias32(p.res_gain + c0, gv);
 #pragma unroll
               for (int j = 0; j < 32; ++j) x[j] *= res_s * gv[j];
             }
-            if (c + kSplit < nchunks) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int r = i * 8 + (lane >> 2);
-                pre[i] = (m0w + r < p.M)
-                             ? *reinterpret_cast<const uint4 *>(p.Xh + (long long)(m0w + r) * p.ld + c0 + 32 * kSplit + (lane & 3) * 8)
-                             : make_uint4(0, 0, 0, 0);
-              }
-            }
+            if (c + kSplit < nchunks) residual_fetch(c0 + 32 * kSplit);
             if (p.bias) {
               float bv[32];
               load_bias32(p.bias + c0, bv);
@@ -426,14 +453,20 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
               sqg += y * y;
             }
           }
+          if (kBF) box128_put_row(xb, lane, x);
           uint4 d[4];
-          pack16(x, d);
+          pack16<kBF>(x, d);
           box64_put_row(hb, lane, d);
           tc::fence_proxy_async();
           __syncwarp();
           if (lane == 0) {
-            if (EPI == kTcResid) tc::tma_store_2d(&tmD, hb, c0, m0w);
-            else tc::tma_store_3d(&tmD, hb, c0, ti.g, m0w);
+            if (EPI == kTcResid) {
+              if (kBF) tc::tma_store_2d(&tmC, xb, c0, m0w);
+              tc::tma_store_2d(&tmD, hb, c0, m0w);
+            } else {
+              if (kBF) tc::tma_store_3d(&tmC, xb, c0, ti.g, m0w);
+              tc::tma_store_3d(&tmD, hb, c0, ti.g, m0w);
+            }
             tc::bulk_commit();
           }
           ++nstore;
@@ -480,7 +513,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           if (lane == 0) tc::bulk_wait_read<1>();
           __syncwarp();
           uint4 d[4];
-          pack16(v, d);
+          pack16<kBF>(v, d);
           box64_put_row(box, lane, d);
           tc::fence_proxy_async();
           __syncwarp();
@@ -508,7 +541,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
             for (int j = 0; j < 32; ++j) v[j] = tanhf(fmaf(v[j], rs, bv[j]));
           }
           uint4 d[4];
-          pack16(v, d);
+          pack16<kBF>(v, d);
           box64_put_row(box, lane, d);
           tc::fence_proxy_async();
           __syncwarp();
@@ -534,9 +567,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
             o[(j >> 1) + 1] = fmaf(v[j + 2], rs, bv[j + 2]) * g.y;
           }
           *reinterpret_cast<uint4 *>(box + lane * 32) =
-              make_uint4(pack_h2(o[0], o[1]), pack_h2(o[2], o[3]), pack_h2(o[4], o[5]), pack_h2(o[6], o[7]));
+              make_uint4(pack_h2<kBF>(o[0], o[1]), pack_h2<kBF>(o[2], o[3]), pack_h2<kBF>(o[4], o[5]),
+                         pack_h2<kBF>(o[6], o[7]));
           *reinterpret_cast<uint4 *>(box + lane * 32 + 16) =
-              make_uint4(pack_h2(o[8], o[9]), pack_h2(o[10], o[11]), pack_h2(o[12], o[13]), pack_h2(o[14], o[15]));
+              make_uint4(pack_h2<kBF>(o[8], o[9]), pack_h2<kBF>(o[10], o[11]), pack_h2<kBF>(o[12], o[13]),
+                         pack_h2<kBF>(o[14], o[15]));
           tc::fence_proxy_async();
           __syncwarp();
           if (lane == 0) {
@@ -618,10 +653,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int EPI>
-constexpr size_t smem_bytes() { return SmemLayout<EPI>::total + 1024; }
-static_assert(smem_bytes<kTcQkv>() <= 232448 && smem_bytes<kTcResid>() <= 232448 && smem_bytes<kTcGelu>() <= 232448 &&
-                  smem_bytes<kTcBandSplit>() <= 232448 && smem_bytes<kTcGlu>() <= 232448,
+template <int EPI, bool kBF>
+constexpr size_t smem_bytes() { return SmemLayout<EPI, kBF>::total + 1024; }
+constexpr size_t kSmemLimit = 232448;  // 227 KB per CTA
+static_assert(smem_bytes<kTcQkv, true>() <= kSmemLimit && smem_bytes<kTcResid, true>() <= kSmemLimit &&
+                  smem_bytes<kTcGelu, true>() <= kSmemLimit && smem_bytes<kTcBandSplit, true>() <= kSmemLimit &&
+                  smem_bytes<kTcGlu, true>() <= kSmemLimit && smem_bytes<kTcTanh, true>() <= kSmemLimit &&
+                  smem_bytes<kTcGeglu, true>() <= kSmemLimit,
               "shared memory per CTA over the 227 KB limit");
 
 }  // namespace
@@ -656,9 +694,12 @@ bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, un
 
 bool gemm_tc_init() {
   bool ok = encode_fn() != nullptr;
-#define MRF_GEMM_ATTR(E)                                                                                       \
-  ok = ok && cudaFuncSetAttribute(gemm_tc_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,              \
-                                  (int)smem_bytes<E>()) == cudaSuccess;
+#define MRF_GEMM_ATTR(E)                                                                                    \
+  ok = ok &&                                                                                                \
+       cudaFuncSetAttribute(gemm_tc_kernel<E, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,          \
+                            (int)smem_bytes<E, false>()) == cudaSuccess &&                                  \
+       cudaFuncSetAttribute(gemm_tc_kernel<E, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,           \
+                            (int)smem_bytes<E, true>()) == cudaSuccess;
   MRF_GEMM_ATTR(kTcQkv)
   MRF_GEMM_ATTR(kTcResid)
   MRF_GEMM_ATTR(kTcGelu)
@@ -670,12 +711,15 @@ bool gemm_tc_init() {
   return ok;
 }
 
-void launch_gemm_tc(int epi, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
+void launch_gemm_tc(int epi, bool bf16, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
                     const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st) {
   switch (epi) {
-#define MRF_GEMM_CASE(E)                                                                  \
-  case E:                                                                                 \
-    gemm_tc_kernel<E><<<grid, gemm_threads(E), smem_bytes<E>(), st>>>(tmA, tmB, tmC, tmD, p); \
+#define MRF_GEMM_CASE(E)                                                                                      \
+  case E:                                                                                                     \
+    if (bf16)                                                                                                 \
+      gemm_tc_kernel<E, true><<<grid, gemm_threads(E), smem_bytes<E, true>(), st>>>(tmA, tmB, tmC, tmD, p);   \
+    else                                                                                                      \
+      gemm_tc_kernel<E, false><<<grid, gemm_threads(E), smem_bytes<E, false>(), st>>>(tmA, tmB, tmC, tmD, p); \
     break;
     MRF_GEMM_CASE(kTcQkv)
     MRF_GEMM_CASE(kTcResid)

@@ -7,6 +7,7 @@
 // shape"; "@audio/neural-separate 0.4.0 → 0.5.0", package/scripts/export-roformer.py,
 // class Core (gamma*sqrt(d) folded into the next Linear; masks averaged from at most two
 // sources with a per-row weight).
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <cmath>
@@ -297,9 +298,19 @@ __global__ void attention_simt_kernel(const TI *__restrict__ q, const TI *__rest
   if (lane + 32 < dh) st_f(orow + lane + 32, o1 * g);
 }
 
-// Same on the fp16 schedule's token-major projection rows qkv[tok][ld] = [q | k | v | gates]
+__device__ __forceinline__ float to_f(__half v) { return __half2float(v); }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <class T16>
+__device__ __forceinline__ T16 from_f(float v);
+template <>
+__device__ __forceinline__ __half from_f<__half>(float v) { return __float2half_rn(v); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// Same on the tensor-core schedule's token-major projection rows (fp16, or bf16) qkv[tok][ld] = [q | k | v | gates]
 // (gates already squashed by the sigmoid), for head widths the tensor-core kernel does not take.
-__global__ void attention_tokmajor_kernel(const __half *__restrict__ qkv, int ld, __half *__restrict__ o, int B,
+template <class T16>
+__global__ void attention_tokmajor_kernel(const T16 *__restrict__ qkv, int ld, T16 *__restrict__ o, int B,
                                           int T, int nb, int H, int dh, int axis) {
   __shared__ float qs[8][64];
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
@@ -319,16 +330,16 @@ __global__ void attention_tokmajor_kernel(const __half *__restrict__ qkv, int ld
   };
   const long long tq = tok_of(pos);
   const float scale = rsqrtf((float)dh);
-  for (int d = lane; d < dh; d += 32) qs[warp][d] = __half2float(qkv[tq * ld + head * dh + d]) * scale;
+  for (int d = lane; d < dh; d += 32) qs[warp][d] = to_f(qkv[tq * ld + head * dh + d]) * scale;
   __syncwarp();
   float m = -INFINITY, l = 0.f, o0 = 0.f, o1 = 0.f;
   for (int j0 = 0; j0 < n; j0 += 32) {
     const int j = j0 + lane;
     float s = -INFINITY;
     if (j < n) {
-      const __half *kr = qkv + tok_of(j) * ld + A + head * dh;
+      const T16 *kr = qkv + tok_of(j) * ld + A + head * dh;
       s = 0.f;
-      for (int d = 0; d < dh; ++d) s = fmaf(qs[warp][d], __half2float(kr[d]), s);
+      for (int d = 0; d < dh; ++d) s = fmaf(qs[warp][d], to_f(kr[d]), s);
     }
     const float mn = fmaxf(m, warp_max(s));
     const float p = (j < n) ? expf(s - mn) : 0.f;
@@ -338,16 +349,16 @@ __global__ void attention_tokmajor_kernel(const __half *__restrict__ qkv, int ld
     const int cnt = min(32, n - j0);
     for (int jj = 0; jj < cnt; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
-      const __half *vr = qkv + tok_of(j0 + jj) * ld + 2 * A + head * dh;
-      if (lane < dh) o0 = fmaf(pj, __half2float(vr[lane]), o0);
-      if (lane + 32 < dh) o1 = fmaf(pj, __half2float(vr[lane + 32]), o1);
+      const T16 *vr = qkv + tok_of(j0 + jj) * ld + 2 * A + head * dh;
+      if (lane < dh) o0 = fmaf(pj, to_f(vr[lane]), o0);
+      if (lane + 32 < dh) o1 = fmaf(pj, to_f(vr[lane + 32]), o1);
     }
     m = mn;
   }
-  const float g = __half2float(qkv[tq * ld + 3 * A + head]) / l;
-  __half *orow = o + tq * (long long)A + head * dh;
-  if (lane < dh) orow[lane] = __float2half_rn(o0 * g);
-  if (lane + 32 < dh) orow[lane + 32] = __float2half_rn(o1 * g);
+  const float g = to_f(qkv[tq * ld + 3 * A + head]) / l;
+  T16 *orow = o + tq * (long long)A + head * dh;
+  if (lane < dh) orow[lane] = from_f<T16>(o0 * g);
+  if (lane + 32 < dh) orow[lane + 32] = from_f<T16>(o1 * g);
 }
 
 // ------------------------------------------------------------------ overlap average
@@ -434,9 +445,14 @@ void launch_attention_f32(const float *q, const float *k, const float *v, const 
 }
 
 void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int T, int nb, int heads, int dh,
-                               int axis, cudaStream_t st) {
+                               int axis, bool bf16, cudaStream_t st) {
   const long long rows = (long long)B * T * nb * heads;
-  attention_tokmajor_kernel<<<grid1(rows, 8), 256, 0, st>>>(qkv, ld, o, B, T, nb, heads, dh, axis);
+  if (bf16)
+    attention_tokmajor_kernel<__nv_bfloat16><<<grid1(rows, 8), 256, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(qkv), ld, reinterpret_cast<__nv_bfloat16 *>(o), B, T, nb, heads, dh,
+        axis);
+  else
+    attention_tokmajor_kernel<__half><<<grid1(rows, 8), 256, 0, st>>>(qkv, ld, o, B, T, nb, heads, dh, axis);
 }
 
 

@@ -51,7 +51,7 @@ std::string validate_config(const mrf_config &c) {
   if (c.max_batch < 1 || c.max_frames < 1) return "max_batch and max_frames must be >= 1";
   if ((long long)c.max_batch * c.max_frames > (1LL << 22)) return "max_batch * max_frames too large";
   if (!(c.rope_theta > 1.f)) return "rope_theta must be > 1";
-  if (c.compute != MRF_FP16 && c.compute != MRF_FP32_DEBUG) return "compute mode not implemented";
+  if (c.compute != MRF_FP16 && c.compute != MRF_BF16 && c.compute != MRF_FP32_DEBUG) return "compute mode not implemented";
   return "";
 }
 
@@ -474,7 +474,7 @@ mrf_status mrf_create(const mrf_config *cfg, const mrf_tensor *w, int n_w, mrf_h
   const std::string te = build_band_tables(cfg->sample_rate, cfg->n_fft, cfg->num_bands,
                                            cfg->audio_channels, cfg->zero_dc != 0, &tab);
   if (!te.empty()) return fail(nullptr, MRF_EINVAL, te);
-  if (cfg->compute == MRF_FP16) {
+  if (cfg->compute != MRF_FP32_DEBUG) {
     const std::string fe = fp16_supported(*cfg, tab);
     if (!fe.empty()) return fail(nullptr, MRF_EUNSUPPORTED, fe);
   }

@@ -32,10 +32,11 @@ void launch_band_split(const float *in, const int32_t *feat_row, const int32_t *
                        int dim, int B, int T, int rows, float *X, __half *Xh, float *ss,
                        cudaStream_t st, int max_width);
 
-// fp16 schedule (k_gather.cu): normalised band features, fp16, [band][frame_stride][k_stride],
+// tensor-core schedule (k_gather.cu): normalised band features, fp16 (bf16 with bf16; the buffer
+// type is the 16-bit container of either), [band][frame_stride][k_stride],
 // each band's row zero-padded to a multiple of 64 (the A operand of the band-split GEMM).
 void launch_band_gather(const float *in, const int32_t *feat_row, const BandDesc *bands, int nb, int B, int T,
-                        int rows, long long frame_stride, int k_stride, __half *A, cudaStream_t st);
+                        int rows, long long frame_stride, int k_stride, __half *A, bool bf16, cudaStream_t st);
 
 enum SimtEpi : int {
   kEpiStore = 0,      // C = acc (+ bias)
@@ -70,9 +71,10 @@ void launch_attention_f32(const float *q, const float *k, const float *v, const 
                           float *o, int B, int T, int nb, int heads, int dh, int axis,
                           cudaStream_t st);
 
-// Same on the fp16 schedule's token-major rows qkv[tok][ld] = [q | k | v | sigmoid gates]; fp16 output.
+// Same on the tensor-core schedule's token-major rows qkv[tok][ld] = [q | k | v | sigmoid gates];
+// 16-bit input and output (fp16, or bf16 with bf16).
 void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int T, int nb, int heads, int dh,
-                               int axis, cudaStream_t st);
+                               int axis, bool bf16, cudaStream_t st);
 
 
 // masks[b, r, t, c] = row_weight[r] * sum of the (<= 2) source features of (r, c)

@@ -18,6 +18,7 @@
 // epilogue scale; the gates' projection is appended to q, k, v; the mask head's bands
 // are batched as groups of one GEMM; its last layer's value and gate rows are interleaved
 // so that a GLU pair is two adjacent accumulator columns.
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -29,7 +30,7 @@
 
 namespace mrf {
 
-bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int axis,
+bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int axis, bool bf16,
                          unsigned *status, cudaStream_t st);
 bool attention_tc_supported(int dh);
 bool attention_tc_init();
@@ -65,15 +66,28 @@ struct Fp16State {
   int ldq = 0;  // row length of QKV: [q | k | v | gates], padded to a multiple of 8
   int sms = 148;
   bool tc_attention = true;
+  // MRF_BF16: every 16-bit buffer and weight holds bf16 (the __half pointers are 16-bit
+  // containers), and the residual stream also keeps an fp32 master copy X (rounding the residual
+  // adds of twelve transformers to bf16's 8-bit significand would cost too much precision)
+  bool bf16 = false;
+  float *X = nullptr;
 };
 
 namespace {
 
 constexpr int kBnWide = 256, kBnNarrow = 192;
 
-std::vector<__half> to_half(const std::vector<float> &v) {
+// Weights rounded once (to nearest even) to the schedule's 16-bit type, in 16-bit containers.
+std::vector<__half> to16(const std::vector<float> &v, bool bf16) {
   std::vector<__half> o(v.size());
-  for (size_t i = 0; i < v.size(); ++i) o[i] = __float2half_rn(v[i]);
+  if (bf16) {
+    for (size_t i = 0; i < v.size(); ++i) {
+      const __nv_bfloat16 b = __float2bfloat16_rn(v[i]);
+      memcpy(&o[i], &b, 2);
+    }
+  } else {
+    for (size_t i = 0; i < v.size(); ++i) o[i] = __float2half_rn(v[i]);
+  }
   return o;
 }
 
@@ -120,6 +134,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   h->f16 = f;
   cudaDeviceGetAttribute(&f->sms, cudaDevAttrMultiProcessorCount, h->device);
   f->tc_attention = attention_tc_supported(dh);
+  f->bf16 = c.compute == MRF_BF16;
   if (!gemm_tc_init() || (f->tc_attention && !attention_tc_init())) {
     h->err = "tcgen05 kernel initialisation failed (tensor-map encoder or shared-memory limit)";
     return MRF_ECUDA;
@@ -138,7 +153,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
         for (int e = 0; e < wd; ++e)
           wb[((size_t)k * D + n) * f->k_bs + e] = (float)((double)w[(size_t)n * wd + e] * g[e] * sc);
     }
-    f->w_bs = up(h, to_half(wb));
+    f->w_bs = up(h, to16(wb, f->bf16));
     std::vector<GemmGroup> gb(nb);
     for (int k = 0; k < nb; ++k)
       gb[k] = {D, cdiv(D, kBnNarrow), k * cdiv(D, kBnNarrow), (int)(k * MBT), k * D, k, k * D, cdiv(t.width[k], 64)};
@@ -165,18 +180,18 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
         for (int n = 0; n < 3 * A + H; ++n)
           for (int k = 0; k < D; ++k) qkvg[(size_t)n * D + k] = (float)((double)qkvg[(size_t)n * D + k] * gp[k] * sd);
       }
-      x.wqkvg = up(h, to_half(qkvg));
+      x.wqkvg = up(h, to16(qkvg, f->bf16));
       x.bg = up(h, W[p + "layers.0.0.to_gates.bias"].v);
-      x.wo = up(h, to_half(W[p + "layers.0.0.to_out.0.weight"].v));
+      x.wo = up(h, to16(W[p + "layers.0.0.to_out.0.weight"].v, f->bf16));
       if (c.ff_act == 1) {  // GEGLU: (value, gate) rows paired for the epilogue
-        x.w1 = up(h, to_half(fold_cols(interleave_halves(W[p + "layers.0.1.net.1.weight"].v, FF, D),
-                                       W[p + "layers.0.1.net.0.gamma"].v, 2 * FF, D)));
+        x.w1 = up(h, to16(fold_cols(interleave_halves(W[p + "layers.0.1.net.1.weight"].v, FF, D),
+                                       W[p + "layers.0.1.net.0.gamma"].v, 2 * FF, D), f->bf16));
         x.b1 = up(h, interleave_halves(W[p + "layers.0.1.net.1.bias"].v, FF, 1));
       } else {
-        x.w1 = up(h, to_half(fold_cols(W[p + "layers.0.1.net.1.weight"].v, W[p + "layers.0.1.net.0.gamma"].v, FF, D)));
+        x.w1 = up(h, to16(fold_cols(W[p + "layers.0.1.net.1.weight"].v, W[p + "layers.0.1.net.0.gamma"].v, FF, D), f->bf16));
         x.b1 = up(h, W[p + "layers.0.1.net.1.bias"].v);
       }
-      x.w2 = up(h, to_half(W[p + "layers.0.1.net.4.weight"].v));
+      x.w2 = up(h, to16(W[p + "layers.0.1.net.4.weight"].v, f->bf16));
       x.b2 = up(h, W[p + "layers.0.1.net.4.bias"].v);
       std::vector<float> go(W[p + "norm.gamma"].v);
       for (auto &v : go) v = (float)(v * std::sqrt((double)D));
@@ -218,11 +233,11 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->mw.emplace_back();
   f->mb.emplace_back();
   for (int i = 0; i < c.mask_depth; ++i) {
-    f->mw.back().push_back(up(h, to_half(mw[i])));
+    f->mw.back().push_back(up(h, to16(mw[i], f->bf16)));
     f->mb.back().push_back(up(h, mb[i]));
     if (!f->mw.back().back() || !f->mb.back().back()) return MRF_ENOMEM;
   }
-  f->mw_last.push_back(up(h, to_half(wl)));
+  f->mw_last.push_back(up(h, to16(wl, f->bf16)));
   f->mb_last.push_back(up(h, bl));
   if (!f->mw_last.back() || !f->mb_last.back()) return MRF_ENOMEM;
   }
@@ -264,6 +279,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->Hh = h->alloc<__half>(NT * FF);
   f->H1 = h->alloc<__half>((long long)nb * MBT * MH);
   f->H2 = h->alloc<__half>((long long)nb * MBT * MH);
+  if (f->bf16 && !(f->X = h->alloc<float>(NT * D))) return MRF_ENOMEM;
   if (!f->Xh || !f->ss || !f->ssx || !f->ssg || !f->QKV || !f->O || !f->Hh || !f->H1 || !f->H2)
     return MRF_ENOMEM;
   // rows past a forward's B*T are read by ragged tiles (and discarded): keep them finite
@@ -283,9 +299,13 @@ bool debug_buffer_fp16(mrf_handle *h, const std::string &name, const void **ptr,
     const long long rows = BT * h->cfg.num_bands;
     static thread_local std::vector<float> hx;
     hx.resize((size_t)rows * D);
-    std::vector<__half> xh((size_t)rows * D);
-    if (cudaMemcpy(xh.data(), f->Xh, xh.size() * 2, cudaMemcpyDeviceToHost) != cudaSuccess) return false;
-    for (size_t i = 0; i < xh.size(); ++i) hx[i] = __half2float(xh[i]);
+    if (f->bf16) {
+      if (cudaMemcpy(hx.data(), f->X, hx.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess) return false;
+    } else {
+      std::vector<__half> xh((size_t)rows * D);
+      if (cudaMemcpy(xh.data(), f->Xh, xh.size() * 2, cudaMemcpyDeviceToHost) != cudaSuccess) return false;
+      for (size_t i = 0; i < xh.size(); ++i) hx[i] = __half2float(xh[i]);
+    }
     if (h->cfg.depth > 0) {
       std::vector<float> s2((size_t)rows * f->parts_res), g(D);
       if (cudaMemcpy(s2.data(), f->ssx, s2.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
@@ -332,7 +352,7 @@ void gemm(mrf_handle *h, const char *name, int epi, const CUtensorMap &a, const 
   const int tiles = p.m_tiles * p.total_n_tiles;
   const int grid = std::min(tiles, h->f16->sms);
   h->begin(name);
-  launch_gemm_tc(epi, a, b, c ? *c : a, d ? *d : a, p, grid, h->cur_stream);
+  launch_gemm_tc(epi, h->f16->bf16, a, b, c ? *c : a, d ? *d : a, p, grid, h->cur_stream);
   h->end();
 }
 
@@ -389,6 +409,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   }
   // bulk-store output maps
   CUtensorMap mXho, mXhbs, mHo, mHo16, mH1o, mH2o, mQKVo;
+  CUtensorMap mXo, mXbs;  // MRF_BF16: the fp32 master copy of the residual stream
   {
     const unsigned long long BT = (unsigned long long)B * T;
     const unsigned long long dx[3] = {(unsigned long long)D, (unsigned long long)nb, BT};
@@ -398,6 +419,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     const unsigned long long sh3[2] = {(unsigned long long)MH, (unsigned long long)MBT * MH};
     const unsigned bh[3] = {32, 32, 1};
     ok = ok && map2(&mXho, f->Xh, kTmF16, D, M, D, 32, 64) && make_tmap(&mXhbs, f->Xh, kTmF16, 3, dx, sx, bx, 64) &&
+         (!f->bf16 || (map2(&mXo, f->X, kTmF32, D, M, D, 32, 128) && make_tmap(&mXbs, f->X, kTmF32, 3, dx, sx, bx, 128))) &&
          map2(&mHo, f->Hh, kTmF16, FF, M, FF, 32, 64) && map2(&mHo16, f->Hh, kTmF16, FF, M, FF, 16, 0) &&
          make_tmap(&mH1o, f->H1, kTmF16, 3, dh3, sh3, bh, 64) &&
          make_tmap(&mH2o, f->H2, kTmF16, 3, dh3, sh3, bh, 64) &&
@@ -409,14 +431,14 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   }
 
   h->begin("band_gather");
-  launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, st);
+  launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, f->bf16, st);
   h->end();
   {
     GemmParams p = base_params(h, B * T, f->k_bs, kBnNarrow, f->g_bs, nb, nb * cdiv(D, kBnNarrow));
-    p.bias = h->b_bs; p.Xh = f->Xh; p.ss_out = f->ssg; p.ss_out_parts = f->parts_bs; p.ld = D; p.nb = nb;
+    p.bias = h->b_bs; p.Xh = f->Xh; p.X = f->X; p.ss_out = f->ssg; p.ss_out_parts = f->parts_bs; p.ld = D; p.nb = nb;
     p.stall_test = h->stall_test ? 1 : 0;
     h->stall_test = false;
-    gemm(h, "gemm_band_split", kTcBandSplit, mAbs, mWbs, p, &mXhbs, &mXhbs);
+    gemm(h, "gemm_band_split", kTcBandSplit, mAbs, mWbs, p, f->bf16 ? &mXbs : &mXhbs, &mXhbs);
   }
 
   for (int i = 0; i < 2 * c.depth; ++i) {
@@ -436,21 +458,21 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
 
     h->begin(f->tc_attention ? (axis == 0 ? "attn_time_tc" : "attn_band_tc") : "attn_simt_f16");
     if (f->tc_attention) {
-      if (!launch_attention_tc(f->QKV, f->ldq, f->O, B, T, nb, H, axis, h->status, st)) {
+      if (!launch_attention_tc(f->QKV, f->ldq, f->O, B, T, nb, H, axis, f->bf16, h->status, st)) {
         h->end();
         h->sched_error = "tensor-map encoding failed (attention)";
         return;
       }
     } else
-      launch_attention_simt_f16(f->QKV, f->ldq, f->O, B, T, nb, H, dh, axis, st);
+      launch_attention_simt_f16(f->QKV, f->ldq, f->O, B, T, nb, H, dh, axis, f->bf16, st);
     h->end();
 
     p = base_params(h, M, A, kBnNarrow, f->g_out, 1, cdiv(D, kBnNarrow));
-    p.Xh = f->Xh; p.ss_out = f->ss; p.ss_out_parts = f->parts_res; p.ld = D;
+    p.Xh = f->Xh; p.X = f->X; p.ss_out = f->ss; p.ss_out_parts = f->parts_res; p.ld = D;
     if (i > 0) {  // the previous output norm
       p.res_ss = f->ssx; p.res_gain = f->tr[i - 1].gout; p.ss_in_parts = f->parts_res;
     }
-    gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p, &mXho, &mXho);
+    gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p, f->bf16 ? &mXo : &mXho, &mXho);
 
     p = base_params(h, M, D, kBnWide, f->g_ff1, 1, cdiv(F1, kBnWide));
     p.ss_in = f->ss; p.ss_in_parts = f->parts_res; p.bias = w.b1; p.out_h = f->Hh; p.ldo = FF;
@@ -458,9 +480,9 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     else gemm(h, "gemm_ff1_gelu", kTcGelu, mXh, mW1, p, &mHo);
 
     p = base_params(h, M, FF, kBnNarrow, f->g_ff2, 1, cdiv(D, kBnNarrow));
-    p.Xh = f->Xh; p.ss_out = f->ssx; p.ss_out_parts = f->parts_res; p.ld = D; p.bias = w.b2;
+    p.Xh = f->Xh; p.X = f->X; p.ss_out = f->ssx; p.ss_out_parts = f->parts_res; p.ld = D; p.bias = w.b2;
     p.ssg_out = f->ssg; p.out_gain = w.gout;  // the output norm is left to the consumers
-    gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p, &mXho, &mXho);
+    gemm(h, "gemm_ff2_resid", kTcResid, mHh, mW2, p, f->bf16 ? &mXo : &mXho, &mXho);
   }
 
   // mask heads, one per stem; each GLU epilogue adds its band features into the stem's slice

@@ -218,10 +218,11 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t smem_addr) {
   return d;
 }
 
-// Instruction descriptor: f16 x f16 -> f32, A and B K-major (or B MN-major), M x N.
-__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major = false) {
+// Instruction descriptor of kind::f16: f16 x f16 (or, with bf16, bf16 x bf16) -> f32, A and B
+// K-major (or B MN-major), M x N.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major = false, bool bf16 = false) {
   return (1u << 4)                                   // D format f32
-         | (0u << 7) | (0u << 10)                    // A, B format f16
+         | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10)  // A, B format: 0 f16, 1 bf16
          | ((b_mn_major ? 1u : 0u) << 16)            // B major
          | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }

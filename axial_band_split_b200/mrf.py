@@ -18,6 +18,7 @@ import numpy as np
 _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmrf.so")
 
 MRF_FP16 = 0
+MRF_BF16 = 1
 MRF_FP32_DEBUG = 2
 STATUS = {0: "MRF_OK", -1: "MRF_EINVAL", -2: "MRF_ESHAPE", -3: "MRF_ENOMEM", -4: "MRF_ECUDA",
           -5: "MRF_EUNSUPPORTED", -6: "MRF_ETIMEOUT", -7: "MRF_EWEIGHTS"}

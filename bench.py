@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--ref-frames", type=int, default=32, help="window of one reference-arm step")
     ap.add_argument("--cpu-sample-frames", type=int, default=1100, help="window of the oracle CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bf16", action="store_true", help="skip the bf16-mode timing beside the fp16 line")
     ap.add_argument("--plain", action="store_true",
                     help="profiling run: warmup + steps eager forwards only, no timing or report")
     return ap.parse_args()
@@ -361,6 +362,22 @@ def run_ours(args):
     e2e_fn()
     ms_e2e = ranks.max(timed(e2e_fn, args.steps))
     io_bytes = int(x_host.nbytes)
+
+    # the same workload in the bf16 compute mode (weights rounded to bf16), device-timed like `value`
+    bf_line = None
+    if not args.no_bf16:
+        Wb = {k: v for k, v in synth.make_weights(cfg, widths, bf16=True).items()}
+        mb = mrf.Model(cfg, Wb, max_batch=B, max_frames=T, compute=mrf.MRF_BF16)
+        outb = torch.empty_like(x)
+        fwd_b = lambda: mb.forward(x, outb)
+        for _ in range(args.warmup):
+            fwd_b()
+        mb.sync_status()
+        ms_b = ranks.max(timed(fwd_b, args.steps))
+        mb.sync_status()
+        mb.close()
+        bf_line = {"value": aggregate(audio_per_rank, world, ms_b), "unit": UNIT, "ms_per_step": ms_b / args.steps,
+                   "dtype": "bf16", "note": "same workload, MRF_BF16 (bf16 operands, fp32 residual master copy)"}
     clk.__exit__()
 
     if rank != 0:
@@ -422,6 +439,7 @@ def run_ours(args):
         "kernel_timing_ms_per_step": ktimed / args.steps,
         "e2e": {"value": aggregate(audio_per_rank, world, ms_e2e), "unit": UNIT,
                 "h2d_bytes_per_step": io_bytes, "d2h_bytes_per_step": io_bytes},
+        "bf16": bf_line,
         "gpu_launches": launches * args.steps,
         "clocks": clk.summary(),
     }

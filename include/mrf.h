@@ -42,7 +42,11 @@ typedef enum {
 } mrf_status;
 
 typedef enum {
-  MRF_FP16 = 0,           /* fp16 operands, fp32 accumulation on tcgen05 tensor cores */
+  MRF_FP16 = 0,           /* fp16 operands, fp32 accumulation on tcgen05 tensor cores; the residual
+                             stream between the GEMMs is stored in fp16 */
+  MRF_BF16 = 1,           /* the same schedule with bf16 operands and activations (weights rounded
+                             to bf16 once), fp32 accumulation; the residual stream also keeps an
+                             fp32 master copy */
   MRF_FP32_DEBUG = 2      /* fp32 CUDA-core schedule, unfused, for debugging and tight parity */
 } mrf_compute;
 

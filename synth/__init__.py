@@ -27,7 +27,7 @@ import math
 import numpy as np
 
 __all__ = [
-    "ModelConfig", "preset", "PRESETS", "weight_shapes", "make_weights",
+    "ModelConfig", "preset", "PRESETS", "weight_shapes", "make_weights", "round_bf16",
     "synth_audio", "stft_stereo", "make_stft_repr", "clip_chunks",
 ]
 
@@ -130,11 +130,19 @@ def weight_shapes(cfg: ModelConfig, widths):
     return out
 
 
-def make_weights(cfg: ModelConfig, widths, seed: int = 0, fp16: bool = True, std: float = 0.02):
+def round_bf16(a):
+    """float32 values rounded to bfloat16 (round to nearest, ties to even), returned as float32."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32)
+
+
+def make_weights(cfg: ModelConfig, widths, seed: int = 0, fp16: bool = True, std: float = 0.02,
+                 bf16: bool = False):
     """Random-init weights: every Linear weight and bias ~ N(0, std); every norm gamma
-    1 + N(0, std).  With ``fp16`` each tensor is rounded to float16 once (round to
-    nearest even) and returned as float32 holding exactly those values, so both sides
-    of a comparison use the same rounded weights."""
+    1 + N(0, std).  With ``fp16`` (or ``bf16``) each tensor is rounded to float16 (bfloat16)
+    once (round to nearest even) and returned as float32 holding exactly those values, so both
+    sides of a comparison use the same rounded weights."""
     rng = np.random.Generator(np.random.PCG64(seed))
     out = {}
     for name, shape in weight_shapes(cfg, widths):
@@ -142,7 +150,9 @@ def make_weights(cfg: ModelConfig, widths, seed: int = 0, fp16: bool = True, std
         if name.endswith("gamma"):
             a = a + 1.0
         a = a.astype(np.float32)
-        if fp16:
+        if bf16:
+            a = round_bf16(a)
+        elif fp16:
             a = a.astype(np.float16).astype(np.float32)
         out[name] = a
     return out
