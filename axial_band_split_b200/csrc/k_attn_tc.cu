@@ -33,9 +33,6 @@
 #include <cmath>
 
 #include "gemm_tc.cuh"
-#ifndef MRF_ATTN_EXP_F16X2
-#define MRF_ATTN_EXP_F16X2 1
-#endif
 #include "mrf_internal.h"
 #include "tc_ptx.cuh"
 
@@ -60,10 +57,6 @@ constexpr int kThreads = 384;
 constexpr int kRegsLaunch = 168, kRegsSoftmax = 208, kRegsIo = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * kRegsLaunch, "register split over budget");
 constexpr float kRescaleLog2 = 8.f;
-// Exponentials of the softmax as fp16 pairs (ex2.approx.f16x2, two values per MUFU instruction)
-// rather than one fp32 value per instruction: the MUFU's exponential rate bounds this kernel at
-// dim_head 64 (one exponential per 256 MMA flops), and P is fp16 either way.
-constexpr bool kExpF16x2 = MRF_ATTN_EXP_F16X2;
 
 struct AttnSmem {
   static constexpr int q = 0;                              // [2 tiles]
@@ -97,29 +90,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
       : "=f"(r.x), "=f"(r.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return r;
-}
-
-// Exponentials as fp16 pairs: one MUFU instruction for two values.
-__device__ __forceinline__ uint32_t cvt_h2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-__device__ __forceinline__ uint32_t ex2_h2(uint32_t x) {
-  uint32_t r;
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(x));
-  return r;
-}
-__device__ __forceinline__ uint32_t hadd2_u(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-// acc + (fp16 value in the low 16 bits of h), rounded once in fp32
-__device__ __forceinline__ float addf_h(float acc, uint32_t h) {
-  const unsigned short x = (unsigned short)h;
-  asm("add.rn.f32.f16 %0, %1, %0;" : "+f"(acc) : "h"(x));
-  return acc;
 }
 
 // Consecutive fp32 columns of this thread's TMEM lane.  The wait takes the destination
@@ -316,50 +286,29 @@ __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t
   const bool need = m_cand > m_run + kRescaleLog2;
   const float alpha = need ? ex2(m_run - m_cand) : 1.f;
   if (need) { l *= alpha; m_run = m_cand; }
-  uint32_t pk[NC / 2];  // p = 2^(s - m) as fp16 pairs, the P*V MMA's A operand
-  float2 s4;
-  if (kExpF16x2 && !kBF) {
-    // Pairs (s - m) through a packed f32x2 subtract, rounded to an fp16 pair and exponentiated
-    // by one MUFU instruction for both (ex2.approx.f16x2), whose fp16 result is P itself.  The
-    // row sum adds the same fp16 values: neighbouring pairs first in fp16 (one rounding of a
-    // sum of two), then each half into fp32.  None of this needs P_t or O_t, so it runs before
-    // the wait for the previous block's P*V, which then overlaps it.
-    const float2 negm = make_float2(-m_run, -m_run);
-    float la = 0.f, lb = 0.f, lc = 0.f, ld = 0.f;
+  // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU, packed to 16-bit
+  // pairs.  This needs neither P_t nor O_t, so it runs before the wait for the previous block's
+  // P*V, which then overlaps it.
+  uint32_t pk[NC / 2];  // the P*V MMA's A operand, two values per 32-bit column
+  float2 sa = make_float2(0.f, 0.f), sb = sa, sc = sa, sd = sa;  // four independent sum chains
+  const float2 negm = make_float2(-m_run, -m_run);
 #pragma unroll
-    for (int i = 0; i < NC; i += 4) {
-      const float2 d0 = add2(make_float2(sv[i], sv[i + 1]), negm);
-      const float2 d1 = add2(make_float2(sv[i + 2], sv[i + 3]), negm);
-      const uint32_t e0 = ex2_h2(cvt_h2(d0.x, d0.y)), e1 = ex2_h2(cvt_h2(d1.x, d1.y));
-      pk[i >> 1] = e0;
-      pk[(i >> 1) + 1] = e1;
-      const uint32_t s01 = hadd2_u(e0, e1);
-      if ((i >> 2) & 1) { la = addf_h(la, s01 & 0xffffu); lb = addf_h(lb, s01 >> 16); }
-      else { lc = addf_h(lc, s01 & 0xffffu); ld = addf_h(ld, s01 >> 16); }
-    }
-    s4 = make_float2(la + lc, lb + ld);
-  } else {
-    // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU, packed to fp16
-    float2 sa = make_float2(0.f, 0.f), sb = sa, sc = sa, sd = sa;  // four independent sum chains
-    const float2 negm = make_float2(-m_run, -m_run);
+  for (int i = 0; i < NC; i += 8) {
 #pragma unroll
-    for (int i = 0; i < NC; i += 8) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 d = add2(make_float2(sv[i + 2 * u], sv[i + 2 * u + 1]), negm);
-        const float2 pp = make_float2(ex2(d.x), ex2(d.y));
-        switch (u) {
-          case 0: sa = add2(sa, pp); break;
-          case 1: sb = add2(sb, pp); break;
-          case 2: sc = add2(sc, pp); break;
-          default: sd = add2(sd, pp); break;
-        }
-        pk[(i >> 1) + u] = pack_h2<kBF>(pp.x, pp.y);
+    for (int u = 0; u < 4; ++u) {
+      const float2 d = add2(make_float2(sv[i + 2 * u], sv[i + 2 * u + 1]), negm);
+      const float2 pp = make_float2(ex2(d.x), ex2(d.y));
+      switch (u) {
+        case 0: sa = add2(sa, pp); break;
+        case 1: sb = add2(sb, pp); break;
+        case 2: sc = add2(sc, pp); break;
+        default: sd = add2(sd, pp); break;
       }
+      pk[(i >> 1) + u] = pack_h2<kBF>(pp.x, pp.y);
     }
-    const float2 s01 = add2(sa, sb), s23 = add2(sc, sd);
-    s4 = add2(s01, s23);
   }
+  const float2 s01 = add2(sa, sb), s23 = add2(sc, sd);
+  const float2 s4 = add2(s01, s23);
   // P_t and O_t are free once the previous block's P*V has completed
   if (wait_pv && !tc::mbar_wait(pv_done, pv_parity, status, 39, abort)) return false;
   tc::tc_fence_after();

@@ -10,11 +10,13 @@
 //
 // The gather is a transpose: stft_repr is [row][frame][re, im] (frames contiguous) and the
 // GEMM wants [frame][feature] (features contiguous, feature 2 * (row - first row) + c).  A CTA
-// takes one band and 32 frames of one window; a warp covers 16 rows x 4 frames per step, two
-// lanes per row, each lane one 16-byte load of two frames' (re, im) (two 8-byte loads when T is
-// odd, where a row's frame pairs are not 16-byte aligned): 32 contiguous bytes per row.
-//   pass 1  loads, per-frame sums of squares (shuffle-xor over the lanes holding the same
-//           frames, one shared-memory add per warp);
+// takes one band and 32 frames of one window with 16 warps: warp w covers frames 4 (w % 8) ..
+// 4 (w % 8) + 3 and every second 16-row step (from step w / 8), two lanes per row, each lane one
+// 16-byte load of two frames' (re, im) (two 8-byte loads when T is odd, where a row's frame pairs
+// are not 16-byte aligned): 32 contiguous bytes per row.
+//   pass 1  loads (eight in flight per thread), per-frame sums of squares (shuffle-xor over the
+//           lanes holding the same frames, then the two warps sharing the frames through shared
+//           memory);
 //   pass 2  the same loads again (the CTA's tile, at most 133 KB, is still in L2), scaled by
 //           1 / max(|x|, 1e-12) and stored as fp16 pairs: each store instruction of a warp
 //           writes 64 contiguous bytes of two frames' feature rows, so nothing is staged in
@@ -31,7 +33,7 @@ namespace mrf {
 namespace {
 
 constexpr int kFrames = 32;    // frames per CTA
-constexpr int kThreads = 256;  // 8 warps: warp w covers frames 4w .. 4w + 3
+constexpr int kThreads = 512;  // 16 warps: warp w covers frames 4 (w % 8) .. 4 (w % 8) + 3
 constexpr float kNormEps = 1e-12f;
 
 template <bool kEvenT>
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(kThreads) band_gather_kernel(const float *__re
                                                                    int B, int T, int R, int tiles,
                                                                    long long frame_stride, int k_stride,
                                                                    __half *__restrict__ A) {
-  __shared__ float ss[kFrames];
+  __shared__ float ss[2][kFrames];
   const int per_band = B * tiles;
   const int k = nb - 1 - (int)(blockIdx.x / per_band);   // widest bands first
   const int rem = (int)(blockIdx.x % per_band);
@@ -80,13 +82,13 @@ __global__ void __launch_bounds__(kThreads) band_gather_kernel(const float *__re
   const int nrows = bd.width >> 1, prow = ((bd.width + 63) & ~63) >> 1;  // rows, rows incl. zero padding
   const int row0 = feat_row[bd.feat_off];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int f0 = 4 * warp + 2 * (lane & 1);  // this lane's two frames of the tile
+  const int f0 = 4 * (warp & 7) + 2 * (lane & 1);  // this lane's two frames of the tile
   const int t = t0 + f0;
-  const int rl = lane >> 1;                  // row within a 16-row step
+  const int rl = (warp >> 3) * 16 + (lane >> 1);   // first row; rows step by 32
   const float *base = in + (((long long)b * R + row0) * T + t) * 2;
   float s0 = 0.f, s1 = 0.f;
-#pragma unroll 4
-  for (int r = rl; r < nrows; r += 16) {
+#pragma unroll 8
+  for (int r = rl; r < nrows; r += 32) {
     const float4 v = load_pair<kEvenT>(base + (long long)r * T * 2, t, T);
     s0 = fmaf(v.x, v.x, fmaf(v.y, v.y, s0));
     s1 = fmaf(v.z, v.z, fmaf(v.w, v.w, s1));
@@ -96,17 +98,18 @@ __global__ void __launch_bounds__(kThreads) band_gather_kernel(const float *__re
     s0 += __shfl_xor_sync(0xffffffffu, s0, o);
     s1 += __shfl_xor_sync(0xffffffffu, s1, o);
   }
-  if (lane < 2) {  // every frame of the tile is written by exactly one lane
-    ss[f0] = s0;
-    ss[f0 + 1] = s1;
+  if (lane < 2) {  // every frame of the tile is written by exactly one lane of each row group
+    ss[warp >> 3][f0] = s0;
+    ss[warp >> 3][f0 + 1] = s1;
   }
   __syncthreads();
-  const float sc0 = 1.f / fmaxf(sqrtf(ss[f0]), kNormEps), sc1 = 1.f / fmaxf(sqrtf(ss[f0 + 1]), kNormEps);
+  const float sc0 = 1.f / fmaxf(sqrtf(ss[0][f0] + ss[1][f0]), kNormEps);
+  const float sc1 = 1.f / fmaxf(sqrtf(ss[0][f0 + 1] + ss[1][f0 + 1]), kNormEps);
   const bool st0 = t < T, st1 = t + 1 < T;
   __half *out0 = A + ((long long)k * frame_stride + (long long)b * T + t) * k_stride;
   __half *out1 = out0 + k_stride;
 #pragma unroll 4
-  for (int r = rl; r < prow; r += 16) {
+  for (int r = rl; r < prow; r += 32) {
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r < nrows) v = load_pair<kEvenT>(base + (long long)r * T * 2, t, T);
     if (st0) *reinterpret_cast<uint32_t *>(out0 + 2 * r) = pack2<kBF>(v.x * sc0, v.y * sc0);
