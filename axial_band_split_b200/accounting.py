@@ -14,7 +14,9 @@ from __future__ import annotations
 def kernel_work(cfg, widths, B: int, T: int):
     """{kernel name: (kind, total per forward, launches per forward)}; kind is "flop" or "byte"."""
     D, H, dh = cfg.dim, cfg.heads, cfg.dim_head
-    A = H * dh
+    dv = getattr(cfg, "dim_head_v", 0) or dh   # v per head (q and k are dh deep)
+    A = H * dv                                  # attention output width
+    QKV = H * (2 * dh + dv)
     FF = D * cfg.ff_mult
     F1 = FF * (2 if getattr(cfg, "ff_act", 0) == 1 else 1)  # GEGLU: value and gate halves
     MH = D * cfg.mask_hidden_mult
@@ -26,9 +28,9 @@ def kernel_work(cfg, widths, B: int, T: int):
     rows = (cfg.n_fft // 2 + 1) * cfg.audio_channels
     S = cfg.num_stems  # one mask estimator (and overlap average) per stem
     w = {
-        "gemm_qkv": ("flop", L2 * 2 * NT * D * (3 * A + H), L2),
-        "attn_time_tc": ("flop", cfg.depth * 4 * (B * nb * H) * T * T * dh, cfg.depth),
-        "attn_band_tc": ("flop", cfg.depth * 4 * (BT * H) * nb * nb * dh, cfg.depth),
+        "gemm_qkv": ("flop", L2 * 2 * NT * D * (QKV + H), L2),
+        "attn_time_tc": ("flop", cfg.depth * 2 * (B * nb * H) * T * T * (dh + dv), cfg.depth),
+        "attn_band_tc": ("flop", cfg.depth * 2 * (BT * H) * nb * nb * (dh + dv), cfg.depth),
         "gemm_out_resid": ("flop", L2 * 2 * NT * A * D, L2),
         "gemm_ff1_gelu": ("flop", L2 * 2 * NT * D * F1, L2),
         "gemm_ff1_geglu": ("flop", L2 * 2 * NT * D * F1, L2),   # the GEGLU variant's launch name

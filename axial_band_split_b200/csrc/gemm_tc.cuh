@@ -54,6 +54,7 @@ struct GemmParams {
   const float2 *rope;
   const float *gbias;
   int B, T, nb, H, dh, A, axis;
+  int Av;                   // kTcQkv: v width (heads x dim_head_v); the row is [q (A) | k (A) | v (Av) | gates]
   float q_scale;            // q is multiplied by this after RoPE (the attention's softmax scale)
   // deferred output norm of the previous transformer (kTcResid): the residual input x is
   // scaled by res_gain[col] / max(sqrt(res_ss[row]), eps) before the add (null: no scaling);

@@ -46,7 +46,7 @@ constexpr int kDh = 64, kRows = 128, kKeys = 128;
 // a K and a V tile per query tile otherwise (band axis; time-axis items that pair the odd
 // last tiles of two sequences).  At most kMaxStages blocks are in flight, each with its own
 // full/empty barrier pair.
-constexpr int kRingTiles = 10, kMaxStages = 5;
+constexpr int kMaxStages = 5;
 static_assert(kKeys == 128, "the softmax reads a score row as two 64-column halves");
 constexpr int kTile = kRows * kDh * 2;  // 16 KB: one 128 x 64 fp16 tile
 constexpr int kThreads = 384;
@@ -58,10 +58,15 @@ constexpr int kRegsLaunch = 168, kRegsSoftmax = 208, kRegsIo = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * kRegsLaunch, "register split over budget");
 constexpr float kRescaleLog2 = 8.f;
 
+// q and k are kQA 64-wide atoms deep (dim_head 64 or 128; v is 64 wide either way): each query
+// tile takes kQA 16 KB tiles, a key block kQA K tiles and one V tile.  The ring shrinks to 8 tiles
+// when q and k are 128 deep, so that the doubled q buffer fits.
+template <int kQA>
 struct AttnSmem {
-  static constexpr int q = 0;                              // [2 tiles]
-  static constexpr int kv = q + 2 * kTile;                 // [stage][tile][K, V]
-  static constexpr int ostage = kv + kRingTiles * kTile;  // [8 warps] 32 rows x 128 B of output
+  static constexpr int ring = kQA == 1 ? 10 : 8;          // K/V ring tiles
+  static constexpr int q = 0;                              // [2 query tiles][kQA atoms]
+  static constexpr int kv = q + 2 * kQA * kTile;           // ring of 16 KB tiles
+  static constexpr int ostage = kv + ring * kTile;         // [8 warps] 32 rows x 128 B of output
   static constexpr int bar = ostage + 8 * 4096;
   static constexpr int total = bar + 256;
 };
@@ -176,6 +181,7 @@ struct AttnArgs {
   __half *o;
   unsigned *status;
   int B, T, nb, H, axis, ld, n, q_tiles, pairs, items, n_blocks, BT;
+  int gate_col;  // column of head 0's gate in a projection row (after q, k and v)
   int S;  // time axis: sequences (b, band, head)
 };
 
@@ -335,14 +341,14 @@ __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t
   return true;
 }
 
-template <bool kBF>
+template <bool kBF, int kQA>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                    const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
                    const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + AttnSmem::bar);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + AttnSmem<kQA>::bar);
   uint64_t *q_full = bars + 0, *q_empty = bars + 1;
   uint64_t *kv_full = bars + 2;     // [kMaxStages]
   uint64_t *kv_empty = bars + 8;    // [kMaxStages]
@@ -394,13 +400,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileC c0 = tile_coords(a, item, 0), c1 = tile_coords(a, item, 1);
         const bool mixed = item_mixed(a, item);
         if (!tc::mbar_wait(q_empty, (li & 1) ^ 1, a.status, 30, abort)) break;
-        tc::mbar_arrive_expect_tx(q_full, 2 * kTile);
-        tc::tma_load_4d(smem + AttnSmem::q, &tq, q_full, 0, c0.head, c0.band, c0.frame0);
-        tc::tma_load_4d(smem + AttnSmem::q + kTile, &tq, q_full, 0, c1.head, c1.band, c1.frame0);
-        const int need = mixed ? 4 : 2;
+        tc::mbar_arrive_expect_tx(q_full, 2 * kQA * kTile);
+#pragma unroll
+        for (int qa = 0; qa < kQA; ++qa) {
+          tc::tma_load_4d(smem + AttnSmem<kQA>::q + qa * kTile, &tq, q_full, 64 * qa, c0.head, c0.band, c0.frame0);
+          tc::tma_load_4d(smem + AttnSmem<kQA>::q + (kQA + qa) * kTile, &tq, q_full, 64 * qa, c1.head, c1.band,
+                          c1.frame0);
+        }
+        const int need = (kQA + 1) * (mixed ? 2 : 1);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
           // a free slot and `need` free ring tiles: release the oldest blocks in order
-          while (ok && (g - oldest >= kMaxStages || used + need > kRingTiles)) {
+          while (ok && (g - oldest >= kMaxStages || used + need > AttnSmem<kQA>::ring)) {
             const int so = oldest % kMaxStages;
             if (!tc::mbar_wait(kv_empty + so, (oldest / kMaxStages) & 1, a.status, 31, abort)) ok = false;
             used -= held[so];
@@ -415,12 +425,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (t == 1 && !mixed) break;
             const TileC &c = t == 0 ? c0 : c1;
             const int f = c.kv0 + j * kKeys;
-            tc::tma_load_4d(smem + AttnSmem::kv + ((ptr + 2 * t) % kRingTiles) * kTile, &tk, kv_full + s, 0,
-                            c.head, c.band, f);
-            tc::tma_load_4d(smem + AttnSmem::kv + ((ptr + 2 * t + 1) % kRingTiles) * kTile, &tv, kv_full + s, 0,
+            const int b0 = ptr + (kQA + 1) * t;  // this tile's K atoms, then its V
+#pragma unroll
+            for (int qa = 0; qa < kQA; ++qa)
+              tc::tma_load_4d(smem + AttnSmem<kQA>::kv + ((b0 + qa) % AttnSmem<kQA>::ring) * kTile, &tk, kv_full + s,
+                              64 * qa, c.head, c.band, f);
+            tc::tma_load_4d(smem + AttnSmem<kQA>::kv + ((b0 + kQA) % AttnSmem<kQA>::ring) * kTile, &tv, kv_full + s, 0,
                             c.head, c.band, f);
           }
-          ptr = (ptr + need) % kRingTiles;
+          ptr = (ptr + need) % AttnSmem<kQA>::ring;
           used += need;
         }
       }
@@ -437,22 +450,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       int li = 0;
       bool ok = true;
       bool mixed = false;
-      // block at ring tile `base`: tile t's K at base (+ 2 t when the tiles have separate
-      // keys), its V one tile further
+      // block at ring tile `base`: tile t's K atoms at base (+ (kQA + 1) t when the tiles have
+      // separate keys), its V after them
       auto kv_tile = [&](int base, int t, int which) {
-        return smem + AttnSmem::kv + ((base + (mixed ? 2 * t : 0) + which) % kRingTiles) * kTile;
+        return smem + AttnSmem<kQA>::kv + ((base + (mixed ? (kQA + 1) * t : 0) + which) % AttnSmem<kQA>::ring) * kTile;
       };
       auto issue_s = [&](int t, int base) {
-        const uint32_t q_addr = tc::smem_u32(smem + AttnSmem::q + t * kTile);
-        const uint32_t k_addr = tc::smem_u32(kv_tile(base, t, 0));
 #pragma unroll
-        for (int kk = 0; kk < kDh / 16; ++kk)
-          tc::mma_f16(tmem + 128 * t, tc::sw128_kmajor_desc(q_addr + kk * 32), tc::sw128_kmajor_desc(k_addr + kk * 32),
-                      id_s, kk != 0);
+        for (int kk = 0; kk < 4 * kQA; ++kk) {
+          const uint32_t q_addr = tc::smem_u32(smem + AttnSmem<kQA>::q + (t * kQA + kk / 4) * kTile);
+          const uint32_t k_addr = tc::smem_u32(kv_tile(base, t, kk / 4));
+          tc::mma_f16(tmem + 128 * t, tc::sw128_kmajor_desc(q_addr + (kk % 4) * 32),
+                      tc::sw128_kmajor_desc(k_addr + (kk % 4) * 32), id_s, kk != 0);
+        }
         tc::mma_commit(s_full + t);
       };
       auto issue_pv = [&](int t, int base, bool acc) {
-        const uint32_t v_addr = tc::smem_u32(kv_tile(base, t, 1));
+        const uint32_t v_addr = tc::smem_u32(kv_tile(base, t, kQA));
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
           mma_f16_ts(tmem + 256 + 64 * t, tmem + 384 + 64 * t + 8 * kk, tc::sw128_mnmajor_desc(v_addr + kk * 2048),
@@ -465,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // buffer are released when both issuers have committed their last read of them.
       for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
         mixed = item_mixed(a, item);
-        const int need = mixed ? 4 : 2;
+        const int need = (kQA + 1) * (mixed ? 2 : 1);
         if (!tc::mbar_wait(q_full, li & 1, a.status, 32, abort)) break;
         if (!tc::mbar_wait(kv_full + g % kMaxStages, (g / kMaxStages) & 1, a.status, 33, abort)) break;
         if (g > 0 && !tc::mbar_wait(s_free + t, (g - 1) & 1, a.status, 41, abort)) break;
@@ -473,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(t, ptr);
         if (a.n_blocks == 1) tc::mma_commit(q_empty);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
-          const int base = (ptr + j * need) % kRingTiles;
+          const int base = (ptr + j * need) % AttnSmem<kQA>::ring;
           if (j + 1 < a.n_blocks) {
             if (!tc::mbar_wait(kv_full + (g + 1) % kMaxStages, ((g + 1) / kMaxStages) & 1, a.status, 36, abort) ||
                 !tc::mbar_wait(s_free + t, g & 1, a.status, 41, abort)) {
@@ -481,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc::tc_fence_after();
-            issue_s(t, (base + need) % kRingTiles);
+            issue_s(t, (base + need) % AttnSmem<kQA>::ring);
             if (j + 2 == a.n_blocks) tc::mma_commit(q_empty);
           }
           if (!tc::mbar_wait(p_full + t, g & 1, a.status, 34, abort) ||
@@ -493,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_pv(t, base, j != 0);
           tc::mma_commit(kv_empty + g % kMaxStages);
         }
-        ptr = (ptr + a.n_blocks * need) % kRingTiles;
+        ptr = (ptr + a.n_blocks * need) % AttnSmem<kQA>::ring;
       }
       tc::mma_commit(done);
       tc::mbar_wait(done, 0, a.status, 37, abort);
@@ -531,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (k < a.n && f < a.BT) tok = (long long)f * a.nb + k;
       }
       const unsigned short gate =
-          tok >= 0 ? reinterpret_cast<const unsigned short *>(a.qkv)[tok * a.ld + 3 * a.H * kDh + it.head] : 0;
+          tok >= 0 ? reinterpret_cast<const unsigned short *>(a.qkv)[tok * a.ld + a.gate_col + it.head] : 0;
       for (int j = 0; j < a.n_blocks; ++j, ++g) {
         if (!tc::mbar_wait(s_full + t, g & 1, a.status, 38, abort)) { ok = false; break; }
         tc::tc_fence_after();
@@ -564,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // and written by one bulk tensor store per warp; rows outside the output tensor
       // (frames past T, bands past nb) are not written
       const float gsc = tok >= 0 ? to_float16b<kBF>(gate) / l : 0.f;
-      uint8_t *stg = smem + AttnSmem::ostage + warp * 4096;
+      uint8_t *stg = smem + AttnSmem<kQA>::ostage + warp * 4096;
       if (lane == 0) tc::bulk_wait_read<0>();
       __syncwarp();
 #pragma unroll
@@ -603,23 +617,30 @@ int g_num_sms = 0;
 
 }  // namespace
 
-bool attention_tc_supported(int dh) { return dh == kDh; }
+// The tensor-core kernel takes q and k of 64 or 128 per head and v of 64.
+bool attention_tc_supported(int dqk, int dv) { return dv == kDh && (dqk == 64 || dqk == 128); }
+
+namespace {
+template <bool kBF, int kQA>
+bool attn_prepare() {
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, attn_tc_kernel<kBF, kQA>) != cudaSuccess || fa.numRegs < kRegsLaunch) return false;
+  return cudaFuncSetAttribute(attn_tc_kernel<kBF, kQA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)(AttnSmem<kQA>::total + 1024)) == cudaSuccess;
+}
+static_assert(AttnSmem<1>::total + 1024 <= 232448 && AttnSmem<2>::total + 1024 <= 232448,
+              "attention shared memory over the 227 KB limit");
+}  // namespace
 
 bool attention_tc_init() {
   int dev = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, attn_tc_kernel<false>) != cudaSuccess || fa.numRegs < kRegsLaunch) return false;
-  if (cudaFuncGetAttributes(&fa, attn_tc_kernel<true>) != cudaSuccess || fa.numRegs < kRegsLaunch) return false;
-  return cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)(AttnSmem::total + 1024)) == cudaSuccess &&
-         cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)(AttnSmem::total + 1024)) == cudaSuccess;
+  return attn_prepare<false, 1>() && attn_prepare<true, 1>() && attn_prepare<false, 2>() && attn_prepare<true, 2>();
 }
 
-bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int axis, bool bf16,
-                         unsigned *status, cudaStream_t st) {
+bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int dqk, int axis,
+                         bool bf16, unsigned *status, cudaStream_t st) {
   AttnArgs a;
   a.qkv = qkv;
   a.o = o;
@@ -628,6 +649,8 @@ bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int
   a.BT = B * T;
   a.n = axis == 0 ? T : nb;
   a.q_tiles = (a.n + kRows - 1) / kRows;
+  const size_t Aqk = (size_t)H * dqk, A = (size_t)H * kDh;  // q (and k) width, v width
+  a.gate_col = (int)(2 * Aqk + A);
   unsigned box[4];
   if (axis == 0) {
     // pairs of consecutive tiles of one sequence; an odd last tile pairs with the next
@@ -636,21 +659,23 @@ bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int
     a.pairs = a.q_tiles / 2;
     a.items = a.S * a.pairs + ((a.q_tiles & 1) ? (a.S + 1) / 2 : 0);
     a.n_blocks = (a.n + kKeys - 1) / kKeys;
-    box[0] = kDh; box[1] = 1; box[2] = 1; box[3] = kRows;      // 128 frames of one (band, head)
+    box[0] = 64; box[1] = 1; box[2] = 1; box[3] = kRows;       // 128 frames of one (band, head)
   } else {
     if (nb > 64) return false;
     a.pairs = 0;
     a.S = 0;
     a.items = H * ((a.BT + 3) / 4);
     a.n_blocks = 1;
-    box[0] = kDh; box[1] = 1; box[2] = 64; box[3] = 2;         // bands 0..63 of two frames
+    box[0] = 64; box[1] = 1; box[2] = 64; box[3] = 2;          // bands 0..63 of two frames
   }
-  // (d, head, band, frame) over the token-major buffer; q, k, v differ by their column offset
-  const unsigned long long dims[4] = {(unsigned long long)kDh, (unsigned long long)H, (unsigned long long)nb,
-                                      (unsigned long long)a.BT};
-  const unsigned long long str[3] = {(unsigned long long)kDh, (unsigned long long)ld,
-                                     (unsigned long long)nb * ld};
-  const size_t A = (size_t)H * kDh;
+  // (d, head, band, frame) over the token-major buffer; q, k, v differ by their column offset,
+  // q and k by their depth (a 64-wide box of them per load)
+  const unsigned long long dqk_dims[4] = {(unsigned long long)dqk, (unsigned long long)H, (unsigned long long)nb,
+                                          (unsigned long long)a.BT};
+  const unsigned long long dqk_str[3] = {(unsigned long long)dqk, (unsigned long long)ld, (unsigned long long)nb * ld};
+  const unsigned long long dv_dims[4] = {(unsigned long long)kDh, (unsigned long long)H, (unsigned long long)nb,
+                                         (unsigned long long)a.BT};
+  const unsigned long long dv_str[3] = {(unsigned long long)kDh, (unsigned long long)ld, (unsigned long long)nb * ld};
   // output [token][head][d] as (d, head, band, frame within the window, batch); a warp
   // stores 32 rows: 32 frames of one band (time axis) or 32 bands of one frame (band axis)
   const unsigned long long odims[5] = {(unsigned long long)kDh, (unsigned long long)H, (unsigned long long)nb,
@@ -659,15 +684,21 @@ bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int
                                       (unsigned long long)T * nb * A};
   const unsigned obox[5] = {(unsigned)kDh, 1u, axis == 0 ? 1u : 32u, axis == 0 ? 32u : 1u, 1u};
   CUtensorMap tq, tk, tv, to;
-  if (!make_tmap(&tq, qkv, kTmF16, 4, dims, str, box, 128) ||
-      !make_tmap(&tk, qkv + A, kTmF16, 4, dims, str, box, 128) ||
-      !make_tmap(&tv, qkv + 2 * A, kTmF16, 4, dims, str, box, 128) ||
+  if (!make_tmap(&tq, qkv, kTmF16, 4, dqk_dims, dqk_str, box, 128) ||
+      !make_tmap(&tk, qkv + Aqk, kTmF16, 4, dqk_dims, dqk_str, box, 128) ||
+      !make_tmap(&tv, qkv + 2 * Aqk, kTmF16, 4, dv_dims, dv_str, box, 128) ||
       !make_tmap(&to, o, kTmF16, 5, odims, ostr, obox, 128))
     return false;
-  const size_t smem = AttnSmem::total + 1024;
   const int grid = (int)std::min<long long>(a.items, g_num_sms > 0 ? g_num_sms : 148);
-  if (bf16) attn_tc_kernel<true><<<grid, kThreads, smem, st>>>(tq, tk, tv, to, a);
-  else attn_tc_kernel<false><<<grid, kThreads, smem, st>>>(tq, tk, tv, to, a);
+#define MRF_ATTN(BF, QA) attn_tc_kernel<BF, QA><<<grid, kThreads, AttnSmem<QA>::total + 1024, st>>>(tq, tk, tv, to, a)
+  if (dqk == 128) {
+    if (bf16) MRF_ATTN(true, 2);
+    else MRF_ATTN(false, 2);
+  } else {
+    if (bf16) MRF_ATTN(true, 1);
+    else MRF_ATTN(false, 1);
+  }
+#undef MRF_ATTN
   return true;
 }
 

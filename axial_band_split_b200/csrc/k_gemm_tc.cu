@@ -476,7 +476,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         if (EPI == kTcQkv) {
           // one token-major row [q | k | v | gates]: scale by the row's norm, rotate q and k,
           // fold the softmax scale into q, squash the gates
-          const int A3 = 3 * p.A;
+          const int A3 = 2 * p.A + p.Av;  // the gates' first column
           if (c0 >= A3) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {

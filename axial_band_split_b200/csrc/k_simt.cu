@@ -205,35 +205,37 @@ __global__ void rownorm_kernel(const float *__restrict__ x, const float *__restr
 }
 
 // ------------------------------------------------------------------ RoPE split
+// One thread per (token, feature pair) of the projection row [q | k | v] (q and k heads x dqk,
+// v heads x dv, each (head, d)); pairs of q and k are rotated by their position.
 __global__ void rope_split_kernel(const float *__restrict__ qkv, const float2 *__restrict__ rope,
                                   float *__restrict__ q, float *__restrict__ k,
-                                  float *__restrict__ v, int B, int T, int nb, int H, int dh,
+                                  float *__restrict__ v, int B, int T, int nb, int H, int dqk, int dv,
                                   int axis) {
   const long long ntok = (long long)B * T * nb;
-  const int A = H * dh, half = dh / 2;
+  const int Aqk = H * dqk, W = 2 * Aqk + H * dv, halfw = W / 2;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= ntok * 3 * H * half) return;
-  const int p = i % half;
-  const long long r = i / half;
-  const int head = r % H;
-  const int which = (r / H) % 3;
-  const long long tok = r / (3 * H);
+  if (i >= ntok * halfw) return;
+  const int c = 2 * (int)(i % halfw);           // feature of the pair's first value
+  const long long tok = i / halfw;
+  const int which = c < Aqk ? 0 : c < 2 * Aqk ? 1 : 2;
+  const int width = which < 2 ? dqk : dv;
+  const int rel = c - which * Aqk;
+  const int head = rel / width, d = rel % width;
   const int band = tok % nb;
   const long long bt = tok / nb;
   const long long b = bt / T, t = bt % T;
   long long seq; int pos, n;
   if (axis == 0) { seq = b * nb + band; pos = (int)t; n = T; }
   else { seq = bt; pos = band; n = nb; }
-  const float x0 = qkv[tok * 3 * A + which * A + head * dh + 2 * p];
-  const float x1 = qkv[tok * 3 * A + which * A + head * dh + 2 * p + 1];
+  const float x0 = qkv[tok * W + c], x1 = qkv[tok * W + c + 1];
   float y0 = x0, y1 = x1;
   if (which < 2) {
-    const float2 cs = rope[(long long)pos * half + p];
+    const float2 cs = rope[(long long)pos * (dqk / 2) + d / 2];
     y0 = x0 * cs.x - x1 * cs.y;
     y1 = x1 * cs.x + x0 * cs.y;
   }
   float *dst = which == 0 ? q : which == 1 ? k : v;
-  const long long o = ((seq * H + head) * n + pos) * dh + 2 * p;
+  const long long o = ((seq * H + head) * n + pos) * width + d;
   dst[o] = y0;
   dst[o + 1] = y1;
 }
@@ -250,8 +252,8 @@ template <class TI, class TO>
 __global__ void attention_simt_kernel(const TI *__restrict__ q, const TI *__restrict__ k,
                                       const TI *__restrict__ v, const float *__restrict__ gate,
                                       TO *__restrict__ o, int B, int T, int nb, int H, int dh,
-                                      int axis, int n_pad) {
-  __shared__ float qs[8][64];
+                                      int dv, int axis, int n_pad) {
+  __shared__ float qs[8][128];
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const long long nseq = axis == 0 ? (long long)B * nb : (long long)B * T;
   const int n = axis == 0 ? T : nb;
@@ -266,7 +268,7 @@ __global__ void attention_simt_kernel(const TI *__restrict__ q, const TI *__rest
   for (int d = lane; d < dh; d += 32) qs[warp][d] = ld_f(qr + d) * scale;
   __syncwarp();
   const TI *kb = k + sh * n_pad * dh;
-  const TI *vb = v + sh * n_pad * dh;
+  const TI *vb = v + sh * n_pad * dv;
   float m = -INFINITY, l = 0.f, o0 = 0.f, o1 = 0.f;
   for (int j0 = 0; j0 < n; j0 += 32) {
     const int j = j0 + lane;
@@ -283,9 +285,9 @@ __global__ void attention_simt_kernel(const TI *__restrict__ q, const TI *__rest
     const int cnt = min(32, n - j0);
     for (int jj = 0; jj < cnt; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
-      const TI *vr = vb + (long long)(j0 + jj) * dh;
-      if (lane < dh) o0 = fmaf(pj, ld_f(vr + lane), o0);
-      if (lane + 32 < dh) o1 = fmaf(pj, ld_f(vr + lane + 32), o1);
+      const TI *vr = vb + (long long)(j0 + jj) * dv;
+      if (lane < dv) o0 = fmaf(pj, ld_f(vr + lane), o0);
+      if (lane + 32 < dv) o1 = fmaf(pj, ld_f(vr + lane + 32), o1);
     }
     m = mn;
   }
@@ -293,9 +295,9 @@ __global__ void attention_simt_kernel(const TI *__restrict__ q, const TI *__rest
   if (axis == 0) { const long long b = seq / nb, band = seq % nb; tok = (b * T + pos) * nb + band; }
   else tok = seq * nb + pos;
   const float g = gate[tok * H + head] / l;
-  TO *orow = o + tok * (long long)H * dh + head * dh;
-  if (lane < dh) st_f(orow + lane, o0 * g);
-  if (lane + 32 < dh) st_f(orow + lane + 32, o1 * g);
+  TO *orow = o + tok * (long long)H * dv + head * dv;
+  if (lane < dv) st_f(orow + lane, o0 * g);
+  if (lane + 32 < dv) st_f(orow + lane + 32, o1 * g);
 }
 
 __device__ __forceinline__ float to_f(__half v) { return __half2float(v); }
@@ -311,14 +313,14 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return
 // (gates already squashed by the sigmoid), for head widths the tensor-core kernel does not take.
 template <class T16>
 __global__ void attention_tokmajor_kernel(const T16 *__restrict__ qkv, int ld, T16 *__restrict__ o, int B,
-                                          int T, int nb, int H, int dh, int axis) {
-  __shared__ float qs[8][64];
+                                          int T, int nb, int H, int dh, int dv, int axis) {
+  __shared__ float qs[8][128];
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const long long nseq = axis == 0 ? (long long)B * nb : (long long)B * T;
   const int n = axis == 0 ? T : nb;
   const long long qi = (long long)blockIdx.x * 8 + warp;
   if (qi >= nseq * H * n) return;
-  const int A = H * dh;
+  const int A = H * dh, Av = H * dv;  // q (and k) width, v width
   const int pos = qi % n;
   const long long sh = qi / n;
   const int head = sh % H;
@@ -349,16 +351,16 @@ __global__ void attention_tokmajor_kernel(const T16 *__restrict__ qkv, int ld, T
     const int cnt = min(32, n - j0);
     for (int jj = 0; jj < cnt; ++jj) {
       const float pj = __shfl_sync(0xffffffffu, p, jj);
-      const T16 *vr = qkv + tok_of(j0 + jj) * ld + 2 * A + head * dh;
-      if (lane < dh) o0 = fmaf(pj, to_f(vr[lane]), o0);
-      if (lane + 32 < dh) o1 = fmaf(pj, to_f(vr[lane + 32]), o1);
+      const T16 *vr = qkv + tok_of(j0 + jj) * ld + 2 * A + head * dv;
+      if (lane < dv) o0 = fmaf(pj, to_f(vr[lane]), o0);
+      if (lane + 32 < dv) o1 = fmaf(pj, to_f(vr[lane + 32]), o1);
     }
     m = mn;
   }
-  const float g = to_f(qkv[tq * ld + 3 * A + head]) / l;
-  T16 *orow = o + tq * (long long)A + head * dh;
-  if (lane < dh) orow[lane] = from_f<T16>(o0 * g);
-  if (lane + 32 < dh) orow[lane + 32] = from_f<T16>(o1 * g);
+  const float g = to_f(qkv[tq * ld + 2 * A + Av + head]) / l;
+  T16 *orow = o + tq * (long long)Av + head * dv;
+  if (lane < dv) orow[lane] = from_f<T16>(o0 * g);
+  if (lane + 32 < dv) orow[lane + 32] = from_f<T16>(o1 * g);
 }
 
 // ------------------------------------------------------------------ overlap average
@@ -430,29 +432,29 @@ void launch_rownorm_f32(const float *x, const float *gain, float *y, long long r
 }
 
 void launch_rope_split_f32(const float *qkv, const float2 *rope, float *q, float *k, float *v,
-                           int B, int T, int nb, int heads, int dh, int axis, cudaStream_t st) {
-  const long long n = (long long)B * T * nb * 3 * heads * (dh / 2);
-  rope_split_kernel<<<grid1(n, 256), 256, 0, st>>>(qkv, rope, q, k, v, B, T, nb, heads, dh, axis);
+                           int B, int T, int nb, int heads, int dqk, int dv, int axis, cudaStream_t st) {
+  const long long n = (long long)B * T * nb * heads * (2 * dqk + dv) / 2;
+  rope_split_kernel<<<grid1(n, 256), 256, 0, st>>>(qkv, rope, q, k, v, B, T, nb, heads, dqk, dv, axis);
 }
 
 void launch_attention_f32(const float *q, const float *k, const float *v, const float *gate,
-                          float *o, int B, int T, int nb, int heads, int dh, int axis,
+                          float *o, int B, int T, int nb, int heads, int dqk, int dv, int axis,
                           cudaStream_t st) {
   const long long rows = (long long)B * T * nb * heads;
   const int n = axis == 0 ? T : nb;
-  attention_simt_kernel<float, float><<<grid1(rows, 8), 256, 0, st>>>(q, k, v, gate, o, B, T, nb, heads, dh,
-                                                                      axis, n);
+  attention_simt_kernel<float, float><<<grid1(rows, 8), 256, 0, st>>>(q, k, v, gate, o, B, T, nb, heads, dqk,
+                                                                      dv, axis, n);
 }
 
-void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int T, int nb, int heads, int dh,
-                               int axis, bool bf16, cudaStream_t st) {
+void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int T, int nb, int heads, int dqk,
+                               int dv, int axis, bool bf16, cudaStream_t st) {
   const long long rows = (long long)B * T * nb * heads;
   if (bf16)
     attention_tokmajor_kernel<__nv_bfloat16><<<grid1(rows, 8), 256, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16 *>(qkv), ld, reinterpret_cast<__nv_bfloat16 *>(o), B, T, nb, heads, dh,
-        axis);
+        reinterpret_cast<const __nv_bfloat16 *>(qkv), ld, reinterpret_cast<__nv_bfloat16 *>(o), B, T, nb, heads, dqk,
+        dv, axis);
   else
-    attention_tokmajor_kernel<__half><<<grid1(rows, 8), 256, 0, st>>>(qkv, ld, o, B, T, nb, heads, dh, axis);
+    attention_tokmajor_kernel<__half><<<grid1(rows, 8), 256, 0, st>>>(qkv, ld, o, B, T, nb, heads, dqk, dv, axis);
 }
 
 

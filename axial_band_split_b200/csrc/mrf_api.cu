@@ -42,7 +42,9 @@ std::string validate_config(const mrf_config &c) {
   if (c.dim < 16 || c.dim > 1024 || c.dim % 16) return "dim must be a multiple of 16 in [16, 1024]";
   if (c.depth < 0 || c.depth > 64) return "depth out of range";
   if (c.heads < 1 || c.heads > 32) return "heads out of range";
-  if (c.dim_head < 2 || c.dim_head > 64 || (c.dim_head & 1)) return "dim_head must be even and <= 64";
+  if (c.dim_head < 2 || c.dim_head > 128 || (c.dim_head & 1)) return "dim_head must be even and <= 128";
+  if (c.dim_head_v < 0 || c.dim_head_v > c.dim_head || (c.dim_head_v & 1) || head_v(c) > 64)
+    return "dim_head_v must be 0 or even, at most dim_head and at most 64";
   if (c.ff_mult < 1 || c.ff_mult > 8) return "ff_mult out of range";
   if (c.mask_hidden < 16 || c.mask_hidden > 8192) return "mask_hidden out of range";
   if (c.mask_depth < 1 || c.mask_depth > 4) return "mask_depth out of range";
@@ -58,7 +60,7 @@ std::string validate_config(const mrf_config &c) {
 // Expected weight names and shapes from the configuration and the band tables.
 std::map<std::string, std::vector<int64_t>> expected_weights(const mrf_config &c, const BandTables &t) {
   std::map<std::string, std::vector<int64_t>> e;
-  const int64_t D = c.dim, A = (int64_t)c.heads * c.dim_head, H = c.heads, FF = (int64_t)c.ff_mult * c.dim,
+  const int64_t D = c.dim, A = attn_out_width(c), QKV = qkv_width(c), H = c.heads, FF = (int64_t)c.ff_mult * c.dim,
                 MH = c.mask_hidden;
   for (int k = 0; k < c.num_bands; ++k) {
     const std::string p = "band_split.to_features." + std::to_string(k) + ".";
@@ -70,7 +72,7 @@ std::map<std::string, std::vector<int64_t>> expected_weights(const mrf_config &c
     for (int a = 0; a < 2; ++a) {
       const std::string p = "layers." + std::to_string(l) + "." + std::to_string(a) + ".";
       e[p + "layers.0.0.norm.gamma"] = {D};
-      e[p + "layers.0.0.to_qkv.weight"] = {3 * A, D};
+      e[p + "layers.0.0.to_qkv.weight"] = {QKV, D};
       e[p + "layers.0.0.to_gates.weight"] = {H, D};
       e[p + "layers.0.0.to_gates.bias"] = {H};
       e[p + "layers.0.0.to_out.0.weight"] = {D, A};
@@ -344,9 +346,9 @@ mrf_status pack_f32(mrf_handle *h, std::map<std::string, HostW> &W) {
       !h->upload(h->mf.g_last, g2.data(), nb * sizeof(SimtGroup)))
     return fail(h, MRF_ECUDA, "upload failed");
   // trunk groups (one group each)
-  const int A = c.heads * c.dim_head, H = c.heads, FF = c.ff_mult * D;
+  const int A = attn_out_width(c), QKVW = qkv_width(c), H = c.heads, FF = c.ff_mult * D;
   SimtGroup tg[5] = {
-      {0, 0, 0, 0, D, 3 * A, 3 * A, 0},  // qkv
+      {0, 0, 0, 0, D, QKVW, QKVW, 0},    // qkv
       {0, 0, 0, 0, D, H, H, 0},          // gates
       {0, 0, 0, 0, A, D, D, 0},          // out
       {0, 0, 0, 0, D, FF, c.ff_act == 1 ? 2 * FF : FF, 0},  // ff1 (GEGLU: 2 FF paired columns, FF outputs)
@@ -358,10 +360,10 @@ mrf_status pack_f32(mrf_handle *h, std::map<std::string, HostW> &W) {
   const long long NT = MBT * nb;
   h->ws.X = h->alloc<float>(NT * D);
   h->ws.Xa = h->alloc<float>(NT * D);
-  h->ws.QKV = h->alloc<float>(NT * 3 * A);
+  h->ws.QKV = h->alloc<float>(NT * QKVW);
   h->ws.G = h->alloc<float>(NT * H);
-  h->ws.Q = h->alloc<float>(NT * A);
-  h->ws.K = h->alloc<float>(NT * A);
+  h->ws.Q = h->alloc<float>(NT * H * c.dim_head);
+  h->ws.K = h->alloc<float>(NT * H * c.dim_head);
   h->ws.V = h->alloc<float>(NT * A);
   h->ws.O = h->alloc<float>(NT * A);
   h->ws.Hf = h->alloc<float>(NT * FF);
@@ -377,7 +379,8 @@ mrf_status pack_f32(mrf_handle *h, std::map<std::string, HostW> &W) {
 // ------------------------------------------------------------------ fp32 debug schedule
 void schedule_f32(mrf_handle *h, const float *in, float *out, int B, int T) {
   const mrf_config &c = h->cfg;
-  const int nb = c.num_bands, D = c.dim, H = c.heads, dh = c.dim_head, A = H * dh, FF = c.ff_mult * D;
+  const int nb = c.num_bands, D = c.dim, H = c.heads, dh = c.dim_head, dv = head_v(c), A = attn_out_width(c),
+            QKVW = qkv_width(c), FF = c.ff_mult * D;
   const long long NT = (long long)B * T * nb;
   const int R = h->tab.n_freqs * h->tab.channels;
   cudaStream_t st = h->cur_stream;
@@ -391,10 +394,10 @@ void schedule_f32(mrf_handle *h, const float *in, float *out, int B, int T) {
     const TrF32 &x = h->trf[i];
     const int axis = i & 1;
     h->begin("rownorm_f32"); launch_rownorm_f32(w.X, x.g_attn, w.Xa, NT, D, st); h->end();
-    h->begin("gemm_f32"); launch_gemm_f32(w.Xa, x.wqkv, nullptr, w.QKV, tg + 0, 1, (int)NT, D, 3 * A, kEpiStore, st); h->end();
+    h->begin("gemm_f32"); launch_gemm_f32(w.Xa, x.wqkv, nullptr, w.QKV, tg + 0, 1, (int)NT, D, QKVW, kEpiStore, st); h->end();
     h->begin("gemm_f32"); launch_gemm_f32(w.Xa, x.wg, x.bg, w.G, tg + 1, 1, (int)NT, D, H, kEpiSigmoid, st); h->end();
-    h->begin("rope_split_f32"); launch_rope_split_f32(w.QKV, h->d_rope, w.Q, w.K, w.V, B, T, nb, H, dh, axis, st); h->end();
-    h->begin("attention_f32"); launch_attention_f32(w.Q, w.K, w.V, w.G, w.O, B, T, nb, H, dh, axis, st); h->end();
+    h->begin("rope_split_f32"); launch_rope_split_f32(w.QKV, h->d_rope, w.Q, w.K, w.V, B, T, nb, H, dh, dv, axis, st); h->end();
+    h->begin("attention_f32"); launch_attention_f32(w.Q, w.K, w.V, w.G, w.O, B, T, nb, H, dh, dv, axis, st); h->end();
     h->begin("gemm_f32"); launch_gemm_f32(w.O, x.wo, nullptr, w.X, tg + 2, 1, (int)NT, A, D, kEpiResidual, st); h->end();
     h->begin("rownorm_f32"); launch_rownorm_f32(w.X, x.g_ff, w.Xa, NT, D, st); h->end();
     if (c.ff_act == 1) {

@@ -12,6 +12,13 @@
 
 namespace mrf {
 
+// ------------------------------------------------------------------ attention widths
+// v per head (dim_head_v, or dim_head when 0); the projection row [q | k | v] and the attention
+// output (the output projection's input).
+inline int head_v(const mrf_config &c) { return c.dim_head_v > 0 ? c.dim_head_v : c.dim_head; }
+inline int qkv_width(const mrf_config &c) { return c.heads * (2 * c.dim_head + head_v(c)); }
+inline int attn_out_width(const mrf_config &c) { return c.heads * head_v(c); }
+
 // ------------------------------------------------------------------ device status word
 // Kernels with bounded waits write a nonzero code here instead of hanging or trapping.
 enum DeviceStatus : unsigned { kStatusOk = 0, kStatusTimeout = 1 };
@@ -61,20 +68,21 @@ void launch_gemm_f32(const float *A, const float *W, const float *bias, float *C
 void launch_rownorm_f32(const float *x, const float *gain, float *y, long long rows, int D,
                         cudaStream_t st);
 
-// qkv [tok, 3*A] fp32 -> q, k, v [seq*heads, n, dh] with RoPE on q and k.
+// qkv [tok, heads*(2 dqk + dv)] fp32 (q, k, v blocks, each (head, d)) -> q, k [seq*heads, n, dqk],
+// v [seq*heads, n, dv], with RoPE on q and k.
 // axis 0: sequences over time (seq = b*nb + band, pos = t); axis 1: over bands.
 void launch_rope_split_f32(const float *qkv, const float2 *rope, float *q, float *k, float *v,
-                           int B, int T, int nb, int heads, int dh, int axis, cudaStream_t st);
+                           int B, int T, int nb, int heads, int dqk, int dv, int axis, cudaStream_t st);
 
-// o[tok, head*dh + d] = gate[tok, head] * softmax(q k^T / sqrt(dh)) v
+// o[tok, head*dv + d] = gate[tok, head] * softmax(q k^T / sqrt(dqk)) v  (dqk <= 128, dv <= 64)
 void launch_attention_f32(const float *q, const float *k, const float *v, const float *gate,
-                          float *o, int B, int T, int nb, int heads, int dh, int axis,
+                          float *o, int B, int T, int nb, int heads, int dqk, int dv, int axis,
                           cudaStream_t st);
 
 // Same on the tensor-core schedule's token-major rows qkv[tok][ld] = [q | k | v | sigmoid gates];
 // 16-bit input and output (fp16, or bf16 with bf16).
-void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int T, int nb, int heads, int dh,
-                               int axis, bool bf16, cudaStream_t st);
+void launch_attention_simt_f16(const __half *qkv, int ld, __half *o, int B, int T, int nb, int heads, int dqk,
+                               int dv, int axis, bool bf16, cudaStream_t st);
 
 
 // masks[b, r, t, c] = row_weight[r] * sum of the (<= 2) source features of (r, c)

@@ -30,9 +30,9 @@
 
 namespace mrf {
 
-bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int axis, bool bf16,
-                         unsigned *status, cudaStream_t st);
-bool attention_tc_supported(int dh);
+bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int dqk, int axis,
+                         bool bf16, unsigned *status, cudaStream_t st);
+bool attention_tc_supported(int dqk, int dv);
 bool attention_tc_init();
 
 struct TrF16 {
@@ -115,10 +115,10 @@ GemmGroup *upload_groups(mrf_handle *h, const std::vector<GemmGroup> &g) { retur
 
 std::string fp16_supported(const mrf_config &c, const BandTables &t) {
   (void)t;
-  const int A = c.heads * c.dim_head;
+  const int Aqk = c.heads * c.dim_head, A = attn_out_width(c);
   if (c.dim % 64) return "fp16 schedule needs dim % 64 == 0";
-  if (A % 64) return "fp16 schedule needs heads*dim_head % 64 == 0";
-  if (c.dim_head % 16) return "fp16 schedule needs dim_head % 16 == 0";
+  if (Aqk % 64 || A % 64) return "fp16 schedule needs heads*dim_head and heads*dim_head_v multiples of 64";
+  if (c.dim_head % 16 || head_v(c) % 16) return "fp16 schedule needs dim_head and dim_head_v multiples of 16";
   if (c.mask_hidden % 64) return "fp16 schedule needs mask_hidden % 64 == 0";
   return "";
 }
@@ -126,14 +126,14 @@ std::string fp16_supported(const mrf_config &c, const BandTables &t) {
 mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   const mrf_config &c = h->cfg;
   const BandTables &t = h->tab;
-  const int nb = c.num_bands, D = c.dim, H = c.heads, dh = c.dim_head, A = H * dh, FF = c.ff_mult * D,
-            MH = c.mask_hidden;
+  const int nb = c.num_bands, D = c.dim, H = c.heads, dh = c.dim_head, A = attn_out_width(c), QKVW = qkv_width(c),
+            FF = c.ff_mult * D, MH = c.mask_hidden;
   const long long MBT = (long long)c.max_batch * c.max_frames, NT = MBT * nb;
   Fp16State *f = new (std::nothrow) Fp16State();
   if (!f) return MRF_ENOMEM;
   h->f16 = f;
   cudaDeviceGetAttribute(&f->sms, cudaDevAttrMultiProcessorCount, h->device);
-  f->tc_attention = attention_tc_supported(dh);
+  f->tc_attention = attention_tc_supported(dh, head_v(c));
   f->bf16 = c.compute == MRF_BF16;
   if (!gemm_tc_init() || (f->tc_attention && !attention_tc_init())) {
     h->err = "tcgen05 kernel initialisation failed (tensor-map encoder or shared-memory limit)";
@@ -168,7 +168,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
       const std::string p = "layers." + std::to_string(l) + "." + std::to_string(a) + ".";
       TrF16 &x = f->tr[2 * l + a];
       const auto &ga = W[p + "layers.0.0.norm.gamma"].v;
-      std::vector<float> qkvg = fold_cols(W[p + "layers.0.0.to_qkv.weight"].v, ga, 3 * A, D);
+      std::vector<float> qkvg = fold_cols(W[p + "layers.0.0.to_qkv.weight"].v, ga, QKVW, D);
       std::vector<float> wg = fold_cols(W[p + "layers.0.0.to_gates.weight"].v, ga, H, D);
       qkvg.insert(qkvg.end(), wg.begin(), wg.end());
       if (2 * l + a > 0) {
@@ -177,7 +177,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
         const int pl = a == 1 ? l : l - 1, pa = a == 1 ? 0 : 1;
         const auto &gp = W["layers." + std::to_string(pl) + "." + std::to_string(pa) + ".norm.gamma"].v;
         const double sd = std::sqrt((double)D);
-        for (int n = 0; n < 3 * A + H; ++n)
+        for (int n = 0; n < QKVW + H; ++n)
           for (int k = 0; k < D; ++k) qkvg[(size_t)n * D + k] = (float)((double)qkvg[(size_t)n * D + k] * gp[k] * sd);
       }
       x.wqkvg = up(h, to16(qkvg, f->bf16));
@@ -246,7 +246,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
     GemmGroup g{N, cdiv(N, BN), 0, 0, 0, 0, 0, 0};
     return upload_groups(h, {g});
   };
-  f->g_qkv = single(3 * A + H, kBnWide);
+  f->g_qkv = single(QKVW + H, kBnWide);
   f->g_out = single(D, kBnNarrow);
   const int F1 = c.ff_act == 1 ? 2 * FF : FF;  // first feed-forward projection's outputs
   f->g_ff1 = single(F1, kBnWide);
@@ -266,7 +266,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->g_last = upload_groups(h, g2);
   if (!f->g_qkv || !f->g_out || !f->g_ff1 || !f->g_ff2 || !f->g_m0 || !f->g_mid || !f->g_last) return MRF_ENOMEM;
   // workspace
-  f->ldq = cdiv(3 * A + H, 8) * 8;
+  f->ldq = cdiv(QKVW + H, 8) * 8;
   f->Xh = h->alloc<__half>(NT * D);
   f->parts_res = cdiv(D, kBnNarrow) * 2;  // residual GEMMs: 8 epilogue warps, 2 per lane quarter
   f->parts_bs = cdiv(D, kBnNarrow) * 4;   // band split: 16 epilogue warps, 4 per lane quarter
@@ -369,8 +369,8 @@ bool map2(CUtensorMap *m, const void *base, int dtype, unsigned long long cols, 
 void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   const mrf_config &c = h->cfg;
   Fp16State *f = h->f16;
-  const int nb = c.num_bands, D = c.dim, H = c.heads, dh = c.dim_head, A = H * dh, FF = c.ff_mult * D,
-            MH = c.mask_hidden;
+  const int nb = c.num_bands, D = c.dim, H = c.heads, dh = c.dim_head, A = attn_out_width(c), QKVW = qkv_width(c),
+            FF = c.ff_mult * D, MH = c.mask_hidden;
   const long long MBT = (long long)c.max_batch * c.max_frames, NT = MBT * nb;
   const int F1 = c.ff_act == 1 ? 2 * FF : FF;  // first feed-forward projection's outputs
   const int M = B * T * nb;
@@ -392,7 +392,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   std::vector<CUtensorMap> wmaps(4 * 2 * c.depth + c.num_stems * n_mask_maps);
   for (int i = 0; ok && i < 2 * c.depth; ++i) {
     const TrF16 &w = f->tr[i];
-    ok = make_tmap_f16(&wmaps[4 * i + 0], w.wqkvg, D, 3 * A + H, 1, D, (3LL * A + H) * D, kBnWide, 1) &&
+    ok = make_tmap_f16(&wmaps[4 * i + 0], w.wqkvg, D, QKVW + H, 1, D, ((long long)QKVW + H) * D, kBnWide, 1) &&
          make_tmap_f16(&wmaps[4 * i + 1], w.wo, A, D, 1, A, (long long)D * A, kBnNarrow, 1) &&
          make_tmap_f16(&wmaps[4 * i + 2], w.w1, D, F1, 1, D, (long long)F1 * D, kBnWide, 1) &&
          make_tmap_f16(&wmaps[4 * i + 3], w.w2, FF, D, 1, FF, (long long)D * FF, kBnNarrow, 1);
@@ -423,7 +423,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
          map2(&mHo, f->Hh, kTmF16, FF, M, FF, 32, 64) && map2(&mHo16, f->Hh, kTmF16, FF, M, FF, 16, 0) &&
          make_tmap(&mH1o, f->H1, kTmF16, 3, dh3, sh3, bh, 64) &&
          make_tmap(&mH2o, f->H2, kTmF16, 3, dh3, sh3, bh, 64) &&
-         map2(&mQKVo, f->QKV, kTmF16, 3 * A + H, M, f->ldq, 32, 64);
+         map2(&mQKVo, f->QKV, kTmF16, QKVW + H, M, f->ldq, 32, 64);
   }
   if (!ok) {
     h->sched_error = "tensor-map encoding failed";
@@ -447,24 +447,24 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     const CUtensorMap &mWqkv = wmaps[4 * i + 0], &mWo = wmaps[4 * i + 1], &mW1 = wmaps[4 * i + 2],
                       &mW2 = wmaps[4 * i + 3];
     // [q | k | v | gates] per token (RoPE positions along this transformer's axis)
-    GemmParams p = base_params(h, M, D, kBnWide, f->g_qkv, 1, cdiv(3 * A + H, kBnWide));
+    GemmParams p = base_params(h, M, D, kBnWide, f->g_qkv, 1, cdiv(QKVW + H, kBnWide));
     p.ss_in = f->ssg;  // |g x|^2 of the previous output (band split: |x|^2)
     p.ss_in_parts = i == 0 ? f->parts_bs : f->parts_res;
     p.rope = h->d_rope; p.gbias = w.bg;
-    p.B = B; p.T = T; p.nb = nb; p.H = H; p.dh = dh; p.A = A; p.axis = axis;
+    p.B = B; p.T = T; p.nb = nb; p.H = H; p.dh = dh; p.A = H * dh; p.Av = A; p.axis = axis;
     // the tensor-core attention takes scores in log2 units: fold log2(e) / sqrt(dh) into q
     p.q_scale = f->tc_attention ? (float)(1.4426950408889634 / std::sqrt((double)dh)) : 1.f;
     gemm(h, "gemm_qkv", kTcQkv, mXh, mWqkv, p, &mQKVo);
 
     h->begin(f->tc_attention ? (axis == 0 ? "attn_time_tc" : "attn_band_tc") : "attn_simt_f16");
     if (f->tc_attention) {
-      if (!launch_attention_tc(f->QKV, f->ldq, f->O, B, T, nb, H, axis, f->bf16, h->status, st)) {
+      if (!launch_attention_tc(f->QKV, f->ldq, f->O, B, T, nb, H, dh, axis, f->bf16, h->status, st)) {
         h->end();
         h->sched_error = "tensor-map encoding failed (attention)";
         return;
       }
     } else
-      launch_attention_simt_f16(f->QKV, f->ldq, f->O, B, T, nb, H, dh, axis, f->bf16, st);
+      launch_attention_simt_f16(f->QKV, f->ldq, f->O, B, T, nb, H, dh, head_v(c), axis, f->bf16, st);
     h->end();
 
     p = base_params(h, M, A, kBnNarrow, f->g_out, 1, cdiv(D, kBnNarrow));
@@ -534,7 +534,7 @@ size_t fp16_workspace_layout(mrf_handle *h, void *base, bool apply, Fp16Workspac
                              size_t *qkv_offset, size_t *qkv_bytes) {
   Fp16State *f = h->f16;
   const mrf_config &c = h->cfg;
-  const int nb = c.num_bands, D = c.dim, H = c.heads, A = H * c.dim_head, FF = c.ff_mult * D, MH = c.mask_hidden;
+  const int nb = c.num_bands, D = c.dim, H = c.heads, A = attn_out_width(c), FF = c.ff_mult * D, MH = c.mask_hidden;
   const long long MBT = (long long)c.max_batch * c.max_frames, NT = MBT * nb;
   size_t off = 0;
   auto take = [&](size_t n) {

@@ -41,7 +41,8 @@ class mrf_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "sample_rate", "n_fft", "audio_channels", "num_bands", "dim", "depth", "heads", "dim_head",
         "ff_mult", "mask_hidden", "mask_depth", "num_stems", "zero_dc", "max_batch", "max_frames")] + \
-        [("rope_theta", ctypes.c_float), ("compute", ctypes.c_int), ("ff_act", ctypes.c_int)]
+        [("rope_theta", ctypes.c_float), ("compute", ctypes.c_int), ("ff_act", ctypes.c_int),
+         ("dim_head_v", ctypes.c_int)]
 
 
 class mrf_tensor(ctypes.Structure):
@@ -122,6 +123,7 @@ def make_config(cfg, max_batch=1, max_frames=1100, compute=MRF_FP16):
     c.max_batch, c.max_frames = max_batch, max_frames
     c.rope_theta, c.compute = cfg.rope_theta, compute
     c.ff_act = getattr(cfg, "ff_act", 0)
+    c.dim_head_v = getattr(cfg, "dim_head_v", 0)
     return c
 
 

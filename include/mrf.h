@@ -61,7 +61,7 @@ typedef struct {
   int dim;               /* 384 */
   int depth;             /* 6 axial blocks, each a time and a band transformer */
   int heads;             /* 8 */
-  int dim_head;          /* 64 */
+  int dim_head;          /* 64: depth of q and k per head (and of v unless dim_head_v is set) */
   int ff_mult;           /* 4: feed-forward inner width ff_mult*dim */
   int mask_hidden;       /* 4*dim: hidden width of the mask MLP */
   int mask_depth;        /* 2: tanh layers of the mask MLP before its GLU layer */
@@ -74,6 +74,13 @@ typedef struct {
   int ff_act;            /* feed-forward activation: 0 GELU (the pages' models); 1 GEGLU, a variant
                             whose first projection is [2*ff, dim] with halves (value, gate) and
                             whose hidden is value * gelu(gate) */
+  int dim_head_v;        /* width of v per head; 0: dim_head.  A value below dim_head gives the
+                            attention whose q and k are deeper than v ("stemd evaluation.md",
+                            section "BS PolarFormer: the same quality for a quarter of the
+                            arithmetic": q and k 128 deep against v 64; rotary positions on q and
+                            k): to_qkv is then [heads*(2*dim_head + dim_head_v), dim] with
+                            features q (head, d), k (head, d), v (head, d), and to_out is
+                            [dim, heads*dim_head_v].  The softmax scale stays dim_head^-1/2. */
 } mrf_config;
 
 /* One named weight, PyTorch [out, in] layout, contiguous, in host memory. */
@@ -97,9 +104,9 @@ typedef struct mrf_handle mrf_handle;
  * Weight names (n_w entries, any order): for each band k,
  *   band_split.to_features.{k}.0.gamma [d_in_k], .1.weight [dim, d_in_k], .1.bias [dim];
  * for each block l and axis a (0 = time, 1 = band), under layers.{l}.{a}.:
- *   layers.0.0.norm.gamma [dim], layers.0.0.to_qkv.weight [3*heads*dim_head, dim],
+ *   layers.0.0.norm.gamma [dim], layers.0.0.to_qkv.weight [heads*(2*dim_head + dv), dim],
  *   layers.0.0.to_gates.weight [heads, dim], layers.0.0.to_gates.bias [heads],
- *   layers.0.0.to_out.0.weight [dim, heads*dim_head],
+ *   layers.0.0.to_out.0.weight [dim, heads*dv] (dv = dim_head_v, or dim_head when 0),
  *   layers.0.1.net.0.gamma [dim], layers.0.1.net.1.weight [ff, dim], .net.1.bias [ff],
  *   layers.0.1.net.4.weight [dim, ff], .net.4.bias [dim], norm.gamma [dim];
  * for each stem s and band k: mask_estimators.{s}.to_freqs.{k}.0.{0,2,4}.{weight,bias}.

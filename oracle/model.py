@@ -85,21 +85,27 @@ def attend(q, k, v):
     return np.matmul(softmax(s), v)
 
 
-def attention(x, w, heads: int, dim_head: int, theta: float):
+def attention(x, w, heads: int, dim_head: int, theta: float, dim_head_v: int = 0):
     """Pre-norm gated multi-head attention over x (S sequences, n, D) -> (S, n, D).
 
     a = norm(x); [q; k; v] = a W_qkv^T with features ordered (which, head, d); q, k
     rotated; o_h = attend(q_h, k_h, v_h) * sigmoid(a W_g^T + b_g)_h; out = concat_h o_h W_o^T.
+    With dim_head_v (v narrower than q and k, as in the PolarFormer attention of "stemd
+    evaluation.md", section "BS PolarFormer: the same quality for a quarter of the arithmetic")
+    the projection's features are q (heads x dim_head), k (heads x dim_head), v (heads x
+    dim_head_v), each ordered (head, d); the softmax scale stays dim_head^-0.5 (the q.k width).
     """
     S, n, D = x.shape
-    A = heads * dim_head
+    dv = dim_head_v or dim_head
+    A = heads * dv
+    Aqk = heads * dim_head
     out = np.empty_like(x)
     for i in range(S):
         a = rms_norm(x[i], w["norm.gamma"])                          # (n, D)
-        qkv = (a @ w["to_qkv.weight"].T).reshape(n, 3, heads, dim_head)
-        q = rope(np.transpose(qkv[:, 0], (1, 0, 2)), theta)          # (h, n, dh)
-        k = rope(np.transpose(qkv[:, 1], (1, 0, 2)), theta)
-        v = np.transpose(qkv[:, 2], (1, 0, 2))
+        qkv = a @ w["to_qkv.weight"].T                                # (n, 2 Aqk + A)
+        q = rope(np.transpose(qkv[:, :Aqk].reshape(n, heads, dim_head), (1, 0, 2)), theta)   # (h, n, dh)
+        k = rope(np.transpose(qkv[:, Aqk:2 * Aqk].reshape(n, heads, dim_head), (1, 0, 2)), theta)
+        v = np.transpose(qkv[:, 2 * Aqk:].reshape(n, heads, dv), (1, 0, 2))
         o = attend(q, k, v)                                          # (h, n, dh)
         g = sigmoid(a @ w["to_gates.weight"].T + w["to_gates.bias"])  # (n, h)
         o = o * np.transpose(g)[:, :, None]
@@ -122,11 +128,11 @@ def feed_forward(x, w, ff_act: int = 0):
     return h @ w["net.4.weight"].T + w["net.4.bias"]
 
 
-def transformer(x, w, heads, dim_head, theta, ff_act: int = 0):
+def transformer(x, w, heads, dim_head, theta, ff_act: int = 0, dim_head_v: int = 0):
     """x += attn(x); x += ff(x); return norm_out(x).  x (S, n, D)."""
     aw = {k[len("layers.0.0."):]: v for k, v in w.items() if k.startswith("layers.0.0.")}
     fw = {k[len("layers.0.1."):]: v for k, v in w.items() if k.startswith("layers.0.1.")}
-    x = attention(x, aw, heads, dim_head, theta) + x
+    x = attention(x, aw, heads, dim_head, theta, dim_head_v) + x
     x = feed_forward(x, fw, ff_act) + x
     return rms_norm(x, w["norm.gamma"])
 
@@ -207,10 +213,11 @@ def forward(stft_repr, cfg, weights, dtype=np.float64, return_stages: bool = Fal
             tw = _sub(W, f"layers.{l}.0.")
             bw = _sub(W, f"layers.{l}.1.")
             ff_act = getattr(cfg, "ff_act", 0)
+            dv = getattr(cfg, "dim_head_v", 0)
             X = np.transpose(transformer(np.transpose(X, (1, 0, 2)), tw, cfg.heads,
-                                         cfg.dim_head, cfg.rope_theta, ff_act), (1, 0, 2))
+                                         cfg.dim_head, cfg.rope_theta, ff_act, dv), (1, 0, 2))
             st[f"layer{l}.time"] = X.copy()
-            X = transformer(X, bw, cfg.heads, cfg.dim_head, cfg.rope_theta, ff_act)
+            X = transformer(X, bw, cfg.heads, cfg.dim_head, cfg.rope_theta, ff_act, dv)
             st[f"layer{l}.band"] = X.copy()
         per_stem = []
         for s in range(cfg.num_stems):
@@ -227,12 +234,14 @@ def param_count(cfg, widths):
     """Number of parameters of the core (weights, biases, norm gammas; the rotary
     embedding's fixed frequencies are not parameters)."""
     D, H, dh = cfg.dim, cfg.heads, cfg.dim_head
-    A = H * dh
+    dv = getattr(cfg, "dim_head_v", 0) or dh
+    A = H * dv                      # attention output width (v)
+    QKV = H * (2 * dh + dv)
     FF = D * cfg.ff_mult
     MH = D * cfg.mask_hidden_mult
     n = sum(w + D * w + D for w in widths)
     F1 = 2 * FF if getattr(cfg, "ff_act", 0) == 1 else FF   # GEGLU: value and gate halves
-    per_tr = (D + 3 * A * D + H * D + H + D * A) + (D + F1 * D + F1 + D * FF + D) + D
+    per_tr = (D + QKV * D + H * D + H + D * A) + (D + F1 * D + F1 + D * FF + D) + D
     n += 2 * cfg.depth * per_tr
     for _ in range(cfg.num_stems):
         for w in widths:
@@ -245,21 +254,22 @@ def mac_count(cfg, widths, B: int, T: int):
     """Multiply-accumulates of one forward, by term (the FLOP accounting of the pages'
     section "FLOP shares"; FLOPs = 2 * MACs)."""
     D, H, dh = cfg.dim, cfg.heads, cfg.dim_head
-    A = H * dh
+    dv = getattr(cfg, "dim_head_v", 0) or dh
+    A = H * dv                      # attention output width (v)
     FF = D * cfg.ff_mult
     MH = D * cfg.mask_hidden_mult
     nb = len(widths)
     tok = B * T * nb
     L = cfg.depth
     per_axis = {
-        "qkv": L * tok * D * 3 * A,
+        "qkv": L * tok * D * H * (2 * dh + dv),
         "gates": L * tok * D * H,
         "out": L * tok * A * D,
         "ff1": L * tok * D * FF * (2 if getattr(cfg, "ff_act", 0) == 1 else 1),
         "ff2": L * tok * FF * D,
     }
-    attn_time = L * (B * nb * H) * 2 * T * T * dh
-    attn_band = L * (B * T * H) * 2 * nb * nb * dh
+    attn_time = L * (B * nb * H) * T * T * (dh + dv)   # q k^T over dh, p v over dv
+    attn_band = L * (B * T * H) * nb * nb * (dh + dv)
     band_split_m = B * T * D * sum(widths)
     mask = cfg.num_stems * B * T * sum(D * MH + (cfg.mask_depth - 1) * MH * MH + MH * 2 * w
                                        for w in widths)

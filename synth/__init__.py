@@ -44,6 +44,7 @@ class ModelConfig:
     depth: int = 6
     heads: int = 8
     dim_head: int = 64
+    dim_head_v: int = 0        # width of v per head; 0: dim_head (q, k and v equally wide)
     ff_mult: int = 4
     ff_act: int = 0            # feed-forward activation: 0 GELU (the pages), 1 GEGLU (variant)
     mask_hidden_mult: int = 4
@@ -69,13 +70,23 @@ class ModelConfig:
         return self.dim * self.mask_hidden_mult
 
     @property
+    def head_v(self) -> int:
+        return self.dim_head_v or self.dim_head
+
+    @property
     def attn_inner(self) -> int:
-        return self.heads * self.dim_head
+        """Width of the attention output (heads x v width): the output projection's input."""
+        return self.heads * self.head_v
 
 
 # Workload presets: model, batch, frames.  "tiny" is the small correctness model;
 # "vocals" is the dim-384 / depth-6 / 60-band vocals checkpoint shape.
 TINY = ModelConfig(n_fft=256, num_bands=8, dim=64, depth=1, heads=4, dim_head=16)
+# An attention whose q and k are twice as wide as v (the shape of the BS PolarFormer attention of
+# "stemd evaluation.md", section "BS PolarFormer: the same quality for a quarter of the
+# arithmetic": 8 heads, q and k of 128 against v of 64), on the vocals band split, with rotary
+# positions on q and k.
+WIDE_QK = ModelConfig(dim=256, depth=1, heads=8, dim_head=128, dim_head_v=64)
 VOCALS = ModelConfig()
 DEUX = ModelConfig(dim=256, depth=12, num_stems=2)
 
@@ -104,6 +115,7 @@ def weight_shapes(cfg: ModelConfig, widths):
     ``widths`` are the per-band input widths d_in = 2 * bins * channels.
     """
     D, A, H, FF, MH = cfg.dim, cfg.attn_inner, cfg.heads, cfg.ff_inner, cfg.mask_hidden
+    QKV = H * (2 * cfg.dim_head + cfg.head_v)  # q and k of dim_head, v of head_v per head
     out = []
     for k, w in enumerate(widths):
         p = f"band_split.to_features.{k}."
@@ -112,7 +124,7 @@ def weight_shapes(cfg: ModelConfig, widths):
         for a in range(2):
             p = f"layers.{l}.{a}."
             q = p + "layers.0.0."
-            out += [(q + "norm.gamma", (D,)), (q + "to_qkv.weight", (3 * A, D)),
+            out += [(q + "norm.gamma", (D,)), (q + "to_qkv.weight", (QKV, D)),
                     (q + "to_gates.weight", (H, D)), (q + "to_gates.bias", (H,)),
                     (q + "to_out.0.weight", (D, A))]
             f = p + "layers.0.1.net."

@@ -497,3 +497,69 @@ def test_band_split_brute_force():
     # the silent frame gives exactly the biases (x / max(0, eps) = 0)
     for k in range(8):
         assert np.array_equal(got[2, k], W[f"band_split.to_features.{k}.1.bias"])
+
+
+# ---------------------------------------------------------------- v narrower than q and k
+def brute_attention_layer_wide_qk(x, w, h, dh, dv, theta):
+    """Scalar loops for the attention whose q and k (dh per head) are wider than v (dv per head)
+    ("stemd evaluation.md", section "BS PolarFormer: the same quality for a quarter of the
+    arithmetic"): projection features q (head, d < dh), then k (head, d < dh), then v (head, d <
+    dv); softmax scale dh^-1/2; heads concatenated head-major (h * dv wide)."""
+    n, D = x.shape
+    g = w["norm.gamma"]
+    a = []
+    for t in range(n):
+        nrm = math.sqrt(sum(x[t, j] ** 2 for j in range(D)))
+        a.append([x[t, j] / max(nrm, 1e-12) * math.sqrt(D) * g[j] for j in range(D)])
+    Wq = w["to_qkv.weight"]
+    def feat(row, t):
+        return sum(Wq[row, j] * a[t][j] for j in range(D))
+    def rot(vec, p):
+        out = list(vec)
+        for i in range(len(vec) // 2):
+            z = complex(vec[2 * i], vec[2 * i + 1]) * cmath.exp(1j * p * theta ** (-2 * i / len(vec)))
+            out[2 * i], out[2 * i + 1] = z.real, z.imag
+        return out
+    cat = [[0.0] * (h * dv) for _ in range(n)]
+    for head in range(h):
+        q = [rot([feat(head * dh + d, t) for d in range(dh)], t) for t in range(n)]
+        k = [rot([feat(h * dh + head * dh + d, t) for d in range(dh)], t) for t in range(n)]
+        v = [[feat(2 * h * dh + head * dv + d, t) for d in range(dv)] for t in range(n)]
+        o = brute_attend(q, k, v)
+        for t in range(n):
+            gate = sum(w["to_gates.weight"][head, j] * a[t][j] for j in range(D)) + w["to_gates.bias"][head]
+            sg = 1 / (1 + math.exp(-gate))
+            for d in range(dv):
+                cat[t][head * dv + d] = o[t][d] * sg
+    Wo = w["to_out.0.weight"]
+    return np.array([[sum(Wo[i, j] * cat[t][j] for j in range(h * dv)) for i in range(D)] for t in range(n)])
+
+
+def test_attention_layer_wide_qk_brute_force():
+    rng = np.random.default_rng(16)
+    n, D, h, dh, dv = 5, 6, 2, 8, 4
+    w = {"norm.gamma": 1 + 0.1 * rng.standard_normal(D),
+         "to_qkv.weight": rng.standard_normal((h * (2 * dh + dv), D)) / 2,
+         "to_gates.weight": rng.standard_normal((h, D)), "to_gates.bias": rng.standard_normal(h),
+         "to_out.0.weight": rng.standard_normal((D, h * dv))}
+    x = rng.standard_normal((1, n, D))
+    got = model.attention(x, w, h, dh, 10000.0, dim_head_v=dv)[0]
+    assert np.allclose(got, brute_attention_layer_wide_qk(x[0], w, h, dh, dv, 10000.0), rtol=0, atol=1e-11)
+    # with dv = dh the general layout is the (which, head, d) layout of the equal-width layer
+    w2 = dict(w, **{"to_qkv.weight": rng.standard_normal((3 * h * dh, D)) / 2,
+                    "to_out.0.weight": rng.standard_normal((D, h * dh))})
+    assert np.allclose(model.attention(x, w2, h, dh, 10000.0, dim_head_v=dh),
+                       model.attention(x, w2, h, dh, 10000.0), rtol=0, atol=0)
+
+
+def test_wide_qk_parameter_and_mac_counts():
+    # to_qkv is h (2 dh + dv) x D and to_out D x h dv; attention MACs per score are dh + dv
+    import dataclasses
+    w = widths60()
+    base = dataclasses.replace(synth.WIDE_QK, dim_head_v=0, dim_head=64)
+    D, H = 256, 8
+    extra_qkv = H * (2 * 128 + 64) * D - 3 * H * 64 * D
+    assert model.param_count(synth.WIDE_QK, w) - model.param_count(base, w) == 2 * (extra_qkv)
+    m = model.mac_count(synth.WIDE_QK, w, 1, 100)
+    assert m["attn_time"] == 1 * (60 * H) * 100 * 100 * (128 + 64)
+    assert m["per_axis"]["qkv"] == 1 * 100 * 60 * D * H * (2 * 128 + 64)
