@@ -73,7 +73,7 @@ float *scratch(mrf_handle *h, size_t slot, size_t bytes) {
 }
 
 // The chunk loop's geometry for a mix of L samples ("Mel-Band RoFormer — ...", section
-// "Verified inference hot path"): 8 s chunks, stride 0.9 chunk, fades of chunk / 10, the mix
+// "Verified inference hot path"): 8 s chunks (or chunk_samples), stride 0.9 chunk, fades of chunk / 10, the mix
 // reflect-padded by the border chunk - stride when longer than two borders, a short last chunk
 // padded by reflection when more than half a chunk remains (mode 1), by zeros otherwise (2).
 struct ChunkGeometry {
@@ -82,9 +82,9 @@ struct ChunkGeometry {
   std::vector<int> off, n, mode;
 };
 
-ChunkGeometry chunk_geometry(int sample_rate, int L) {
+ChunkGeometry chunk_geometry(int sample_rate, int chunk_samples, int L) {
   ChunkGeometry g;
-  g.chunk = sample_rate * 8;
+  g.chunk = chunk_samples > 0 ? chunk_samples : sample_rate * 8;
   g.stride = (int)(g.chunk * 0.9);
   g.fade = g.chunk / 10;
   g.border = g.chunk - g.stride;
@@ -136,15 +136,22 @@ mrf_status mrf_istft(mrf_handle *h, const float *spec, float *audio, int S, int 
 }
 
 mrf_status mrf_separate_audio(mrf_handle *h, const float *mix, float *stems, int L, int hop, void *stream) {
+  return mrf_separate_audio_chunked(h, mix, stems, L, hop, 0, stream);
+}
+
+mrf_status mrf_separate_audio_chunked(mrf_handle *h, const float *mix, float *stems, int L, int hop,
+                                      int chunk_samples, void *stream) {
   if (!h) return MRF_EINVAL;
   if (!mix || !stems) return sfail(h, MRF_EINVAL, "null mix or stems pointer");
   const mrf_config &c = h->cfg;
   const int C = c.audio_channels, S = c.num_stems, n = c.n_fft;
   if (hop < 1 || L < 2) return sfail(h, MRF_ESHAPE, "hop >= 1 and L >= 2 required");
-  const ChunkGeometry g = chunk_geometry(c.sample_rate, L);
+  if (chunk_samples != 0 && (chunk_samples < 10 || chunk_samples <= n / 2))
+    return sfail(h, MRF_EINVAL, "chunk_samples must be 0 (8 s) or at least 10 and above n_fft / 2");
+  const ChunkGeometry g = chunk_geometry(c.sample_rate, chunk_samples, L);
   const int chunk = g.chunk, stride = g.stride, fade = g.fade, border = g.border;
   const int T = 1 + chunk / hop;
-  if (T > c.max_frames) return sfail(h, MRF_ESHAPE, "max_frames is below the frames of one 8 s chunk");
+  if (T > c.max_frames) return sfail(h, MRF_ESHAPE, "max_frames is below the frames of one chunk");
   mrf_status s = ensure_tables(h);
   if (s != MRF_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -194,10 +201,12 @@ mrf_status mrf_separate_audio(mrf_handle *h, const float *mix, float *stems, int
   return s;
 }
 
-mrf_status mrf_chunk_plan(int sample_rate, int L, int *chunk, int *border, int *padded_length, int *n_chunks,
-                          int32_t *off, int32_t *valid, int32_t *mode, int max_chunks) {
-  if (sample_rate < 1 || L < 2 || !chunk || !border || !padded_length || !n_chunks) return MRF_EINVAL;
-  const ChunkGeometry g = chunk_geometry(sample_rate, L);
+mrf_status mrf_chunk_plan(int sample_rate, int chunk_samples, int L, int *chunk, int *border, int *padded_length,
+                          int *n_chunks, int32_t *off, int32_t *valid, int32_t *mode, int max_chunks) {
+  if (sample_rate < 1 || L < 2 || chunk_samples < 0 || (chunk_samples > 0 && chunk_samples < 10) || !chunk ||
+      !border || !padded_length || !n_chunks)
+    return MRF_EINVAL;
+  const ChunkGeometry g = chunk_geometry(sample_rate, chunk_samples, L);
   *chunk = g.chunk;
   *border = g.padded ? g.border : 0;
   *padded_length = g.Lp;

@@ -28,7 +28,7 @@ EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_separate", "mrf_stft", "mrf
            "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
            "mrf_last_error", "mrf_band_tables", "mrf_set_timing", "mrf_kernel_times",
            "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer", "mrf_forward_static",
-           "mrf_debug_stall_next", "mrf_chunk_plan"]
+           "mrf_debug_stall_next", "mrf_chunk_plan", "mrf_separate_audio_chunked"]
 
 
 class MrfError(RuntimeError):
@@ -77,6 +77,8 @@ def lib():
         L.mrf_istft.restype = I
         L.mrf_separate_audio.argtypes = [P, P, P, I, I, P]
         L.mrf_separate_audio.restype = I
+        L.mrf_separate_audio_chunked.argtypes = [P, P, P, I, I, I, P]
+        L.mrf_separate_audio_chunked.restype = I
         L.mrf_forward_static.argtypes = [P, P, P, I, I, P]
         L.mrf_forward_static.restype = I
         L.mrf_forward_host.argtypes = [P, P, P, I, I, P]
@@ -102,7 +104,7 @@ def lib():
         L.mrf_launches_per_forward.argtypes = [P, I, I]
         L.mrf_launches_per_forward.restype = I
         IP = ctypes.POINTER(I)
-        L.mrf_chunk_plan.argtypes = [I, I, IP, IP, IP, IP, P, P, P, I]
+        L.mrf_chunk_plan.argtypes = [I, I, I, IP, IP, IP, IP, P, P, P, I]
         L.mrf_chunk_plan.restype = I
         _lib = L
     return _lib
@@ -143,17 +145,18 @@ def band_tables(cfg):
     return out
 
 
-def chunk_plan(sample_rate, length):
-    """mrf_chunk_plan: the separation loop's geometry for a mix of `length` samples: dict with
-    chunk, border, padded_length and the per-chunk arrays off, valid, mode (0 full, 1 reflect
-    tail, 2 zero tail)."""
+def chunk_plan(sample_rate, length, chunk_samples=0):
+    """mrf_chunk_plan: the separation loop's geometry for a mix of `length` samples (chunks of
+    chunk_samples, 0: 8 s): dict with chunk, border, padded_length and the per-chunk arrays off,
+    valid, mode (0 full, 1 reflect tail, 2 zero tail)."""
     vals = [ctypes.c_int(0) for _ in range(4)]
-    _check(lib().mrf_chunk_plan(sample_rate, length, *[ctypes.byref(v) for v in vals], None, None, None, 0))
+    _check(lib().mrf_chunk_plan(sample_rate, chunk_samples, length, *[ctypes.byref(v) for v in vals], None, None,
+                                None, 0))
     n = vals[3].value
     out = {k: np.zeros(n, np.int32) for k in ("off", "valid", "mode")}
     ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
-    _check(lib().mrf_chunk_plan(sample_rate, length, *[ctypes.byref(v) for v in vals], ptr(out["off"]),
-                                ptr(out["valid"]), ptr(out["mode"]), n))
+    _check(lib().mrf_chunk_plan(sample_rate, chunk_samples, length, *[ctypes.byref(v) for v in vals],
+                                ptr(out["off"]), ptr(out["valid"]), ptr(out["mode"]), n))
     out.update(chunk=vals[0].value, border=vals[1].value, padded_length=vals[2].value)
     return out
 
@@ -277,15 +280,19 @@ class Model:
                                hop, length, _stream_ptr(stream)), self._h)
         return out
 
-    def separate_audio(self, mix, hop, out=None, stream=None):
-        """mrf_separate_audio: CUDA float32 mix [C, L] -> stems [num_stems, C, L]."""
+    def separate_audio(self, mix, hop, out=None, stream=None, chunk_samples=0):
+        """mrf_separate_audio(_chunked): CUDA float32 mix [C, L] -> stems [num_stems, C, L], in chunks
+        of chunk_samples samples (0: 8 s)."""
         import torch
         assert mix.is_cuda and mix.dtype == torch.float32 and mix.is_contiguous()
         C, L = mix.shape
         if out is None:
             out = torch.empty((self.cfg.num_stems, C, L), dtype=mix.dtype, device=mix.device)
-        _check(lib().mrf_separate_audio(self._h, ctypes.c_void_p(mix.data_ptr()), ctypes.c_void_p(out.data_ptr()),
-                                        L, hop, _stream_ptr(stream)), self._h)
+        assert out.is_cuda and out.dtype == torch.float32 and out.is_contiguous() and \
+            out.numel() == self.cfg.num_stems * C * L
+        _check(lib().mrf_separate_audio_chunked(self._h, ctypes.c_void_p(mix.data_ptr()),
+                                                ctypes.c_void_p(out.data_ptr()), L, hop, chunk_samples,
+                                                _stream_ptr(stream)), self._h)
         return out
 
     def forward_static(self, stft_repr, out, stream=None):

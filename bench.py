@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--cpu-sample-frames", type=int, default=1100, help="window of the oracle CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bf16", action="store_true", help="skip the bf16-mode timing beside the fp16 line")
+    ap.add_argument("--chunk-sweep", type=str, default=None, metavar="SECONDS,...",
+                    help="instead of the core forward: time mrf_separate_audio_chunked on a 60 s mix for each "
+                         "chunk length (seconds), one JSON line each")
     ap.add_argument("--plain", action="store_true",
                     help="profiling run: warmup + steps eager forwards only, no timing or report")
     return ap.parse_args()
@@ -451,10 +454,55 @@ def run_ours(args):
     return 0
 
 
+def run_chunk_sweep(args):
+    """The chunk-length question the pages leave open: the full separation of one 60 s stereo mix
+    (STFT, core forward with mask application, iSTFT, fades, overlap-add) per chunk length, up to 16
+    chunks per forward, device-timed (CUDA events, L2 flushed before each timed call)."""
+    import numpy as np
+    import torch
+    from axial_band_split_b200 import build, mrf
+    import synth
+    build.build()
+    cfg = synth.VOCALS
+    widths = mrf.band_tables(cfg)["width"]
+    W = {k: v.astype(np.float16) for k, v in synth.make_weights(cfg, widths, fp16=True).items()}
+    L = 60 * cfg.sample_rate
+    mix = torch.from_numpy(synth.synth_audio(L, seed=7, clicks=True).astype(np.float32)).cuda()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for sec in [float(v) for v in args.chunk_sweep.split(",")]:
+        chunk = int(round(sec * cfg.sample_rate))
+        T = 1 + chunk // cfg.hop
+        plan = mrf.chunk_plan(cfg.sample_rate, L, chunk)
+        m = mrf.Model(cfg, W, max_batch=16, max_frames=T)
+        out = torch.empty((1, 2, L), dtype=torch.float32, device="cuda")
+        for _ in range(max(args.warmup, 1)):
+            m.separate_audio(mix, cfg.hop, out, chunk_samples=chunk)
+        m.sync_status()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record()
+            m.separate_audio(mix, cfg.hop, out, chunk_samples=chunk)
+            e1.record()
+        torch.cuda.synchronize()
+        m.sync_status()
+        ms = sorted(a.elapsed_time(b) for a, b in ev)[len(ev) // 2]
+        m.close()
+        n = len(plan["off"])
+        print(json.dumps({"chunk_s": sec, "chunk_samples": chunk, "frames_per_chunk": T, "chunks": n,
+                          "forwards": -(-n // 16), "ms_per_60s": ms, "real_time_factor": ms / 1e3 / 60.0,
+                          "audio_s_per_s": 60.0 / (ms / 1e3), "steps": args.steps,
+                          "model": "vocals (dim 384, depth 6, 60 bands), fp16, random-init",
+                          "mix": "60 s synthetic stereo (tones, pink noise, clicks)"}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.chunk_sweep:
+        return run_chunk_sweep(args)
     return run_ours(args)
 
 

@@ -173,6 +173,17 @@ mrf_status mrf_istft(mrf_handle *h, const float *spec, float *audio, int S, int 
 mrf_status mrf_separate_audio(mrf_handle *h, const float *mix, float *stems, int L, int hop, void *stream);
 
 /*
+ * mrf_separate_audio_chunked - mrf_separate_audio with a chunk of chunk_samples samples instead of
+ * 8 s (0: 8 s), the stride, border and fades scaling with it (stride 0.9 chunk, fades chunk / 10).
+ * The pages fix the 8 s chunk of their checkpoints and leave the chunk length open ("Mel-Band
+ * RoFormer — ...", section "Gaps and open questions"); this entry point serves that sweep.
+ * max_frames must hold 1 + chunk_samples / hop frames.  MRF_EINVAL for chunk_samples below 10 or
+ * not above n_fft / 2; otherwise as mrf_separate_audio.
+ */
+mrf_status mrf_separate_audio_chunked(mrf_handle *h, const float *mix, float *stems, int L, int hop,
+                                      int chunk_samples, void *stream);
+
+/*
  * mrf_forward_host - the same forward from and to HOST memory: copies stft_repr to the
  * device, runs mrf_forward, copies the masks back ([B, num_stems, F*C, T, 2] floats), and
  * waits for the stream.  For the
@@ -234,18 +245,19 @@ mrf_status mrf_band_tables(const mrf_config *cfg, int32_t *first_bin, int32_t *l
                            int32_t *width, int32_t *feat_row, float *row_weight, int32_t *n_feat);
 
 /*
- * mrf_chunk_plan - host-only test hook: the geometry mrf_separate_audio uses for a mix of L
- * samples at sample_rate (no device work, no handle).  *chunk = 8 * sample_rate samples, the
- * stride 0.9 chunk (truncated), *border = chunk - stride when L > 2 * (chunk - stride) (the mix
- * is then reflect-padded by it on both sides) else 0, *padded_length = L + 2 * border, and
- * chunks at offsets 0, stride, 2 stride, ... below padded_length: off[i], valid[i] =
- * min(chunk, padded_length - off[i]) samples, mode[i] = 0 (full), 1 (tail padded by
- * reflection: more than half a chunk valid) or 2 (tail padded by zeros).  Writes at most
- * max_chunks entries of each array (any array may be NULL); *n_chunks receives the count.
- * MRF_EINVAL for sample_rate < 1, L < 2 or a NULL scalar output.
+ * mrf_chunk_plan - host-only test hook: the geometry mrf_separate_audio_chunked uses for a mix of L
+ * samples at sample_rate with chunks of chunk_samples samples (0: 8 s; no device work, no
+ * handle).  *chunk = chunk_samples (or 8 * sample_rate), the stride 0.9 chunk (truncated), *border
+ * = chunk - stride when L > 2 * (chunk - stride) (the mix is then reflect-padded by it on both
+ * sides) else 0, *padded_length = L + 2 * border, and chunks at offsets 0, stride, 2 stride, ...
+ * below padded_length: off[i], valid[i] = min(chunk, padded_length - off[i]) samples, mode[i] = 0
+ * (full), 1 (tail padded by reflection: more than half a chunk valid) or 2 (tail padded by zeros).
+ * Writes at most max_chunks entries of each array (any array may be NULL); *n_chunks receives the
+ * count.  MRF_EINVAL for sample_rate < 1, L < 2, chunk_samples < 0 or in 1..9, or a NULL scalar
+ * output.
  */
-mrf_status mrf_chunk_plan(int sample_rate, int L, int *chunk, int *border, int *padded_length, int *n_chunks,
-                          int32_t *off, int32_t *valid, int32_t *mode, int max_chunks);
+mrf_status mrf_chunk_plan(int sample_rate, int chunk_samples, int L, int *chunk, int *border, int *padded_length,
+                          int *n_chunks, int32_t *off, int32_t *valid, int32_t *mode, int max_chunks);
 
 /* Kernel timing, for measurement.  When enabled, mrf_forward launches eagerly (no CUDA
  * graph) and records a CUDA event pair around every kernel on the forward's stream;

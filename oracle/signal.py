@@ -77,11 +77,11 @@ def istft(spec, channels: int, length: int, n_fft: int = 2048, hop: int = 441) -
     return keep
 
 
-def chunk_plan(length: int, sample_rate: int = 44100):
+def chunk_plan(length: int, sample_rate: int = 44100, chunk: int = 0):
     """The chunk loop's geometry for a mix of `length` samples: (chunk, border or 0 when the mix
     is not padded, padded length, [(offset, valid samples, tail padding mode or None)],
-    fade window of the chunk)."""
-    chunk = int(sample_rate * 8)
+    fade window of the chunk).  `chunk` samples per chunk, 0 for the page's 8 s."""
+    chunk = int(chunk) if chunk else int(sample_rate * 8)
     stride = int(chunk * 0.9)
     fade = chunk // 10
     border = chunk - stride
@@ -98,12 +98,12 @@ def chunk_plan(length: int, sample_rate: int = 44100):
     return chunk, (border if padded else 0), Lp, chunks, window
 
 
-def separate(mix, estimate, sample_rate: int = 44100):
+def separate(mix, estimate, sample_rate: int = 44100, chunk: int = 0):
     """The chunk loop: mix (C, L) -> stems (S, C, L), with estimate(chunk (C, chunk)) ->
-    (S, C, chunk) the model run on one chunk."""
+    (S, C, chunk) the model run on one chunk; chunks of `chunk` samples (0: 8 s)."""
     mix = np.asarray(mix, dtype=np.float64)
     C, L = mix.shape
-    chunk, border, Lp, chunks, window = chunk_plan(L, sample_rate)
+    chunk, border, Lp, chunks, window = chunk_plan(L, sample_rate, chunk)
     x = np.pad(mix, ((0, 0), (border, border)), mode="reflect") if border else mix
     out, counter = None, np.zeros(Lp)
     fade = chunk // 10

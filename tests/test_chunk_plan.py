@@ -41,3 +41,23 @@ def test_chunk_plan_rejects_bad_arguments():
         mrf.chunk_plan(0, 1000)
     with pytest.raises(mrf.MrfError):
         mrf.chunk_plan(SR, 1)
+
+
+@pytest.mark.parametrize("seconds", [2.0, 4.0, 11.0, 16.0, 13.35])
+@pytest.mark.parametrize("L", [5 * SR, 60 * SR, 61 * SR + 12345])
+def test_chunk_plan_other_chunk_lengths_match_the_oracle(seconds, L):
+    # the chunk-length sweep's geometry: every quantity scales with the chunk
+    from axial_band_split_b200 import mrf
+    c = int(seconds * SR)
+    got = mrf.chunk_plan(SR, L, c)
+    chunk, border, Lp, chunks, _ = signal.chunk_plan(L, SR, c)
+    assert got["chunk"] == chunk == c and got["border"] == border and got["padded_length"] == Lp
+    modes = {None: 0, "reflect": 1, "zeros": 2}
+    assert [(int(o), int(n), int(m)) for o, n, m in zip(got["off"], got["valid"], got["mode"])] == \
+        [(off, n, modes[mode]) for off, n, mode in chunks]
+
+
+def test_chunk_plan_rejects_tiny_chunks():
+    from axial_band_split_b200 import mrf
+    with pytest.raises(mrf.MrfError):
+        mrf.chunk_plan(SR, 1000, 5)

@@ -106,3 +106,26 @@ def test_separation_matches_the_oracle():
     snr = snr_db(got, ref)
     print(f"separated audio: max|diff|/max|mix| = {err:.2e}, snr = {snr:.1f} dB")
     assert err <= 2e-2 and snr >= 40.0
+
+
+def test_separation_with_short_chunks_matches_the_oracle():
+    # chunks of 2 s instead of 8 s on a 5 s mix (padded, three chunks): the chunk-length
+    # parameter of the separation loop against the oracle's loop with the same chunk
+    cfg = dataclasses.replace(synth.VOCALS, depth=1)
+    W = weights(cfg)
+    L, chunk = 5 * 44100, 2 * 44100
+    mix = synth.synth_audio(L, seed=5).astype(np.float32)
+    m = make_model(cfg, W, max_batch=4)
+    got = m.separate_audio(torch.from_numpy(mix).cuda(), HOP, chunk_samples=chunk).cpu().numpy()
+    m.close()
+
+    def estimate(part):
+        x = signal.stft(part[None])
+        spec = oracle_model.apply_masks(x, oracle_model.forward(x, cfg, W))
+        return signal.istft(spec[0][None], channels=2, length=part.shape[-1])
+
+    ref = signal.separate(mix.astype(np.float64), estimate, chunk=chunk)
+    err = float(np.abs(got - ref).max()) / float(np.abs(mix).max())
+    snr = snr_db(got, ref)
+    print(f"2 s chunks: max|diff|/max|mix| = {err:.2e}, snr = {snr:.1f} dB")
+    assert err <= 2e-2 and snr >= 40.0
