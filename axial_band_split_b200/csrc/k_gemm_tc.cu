@@ -186,12 +186,33 @@ __device__ __forceinline__ void load_bias32(const float *b, float *bv) {
 }
 
 // A row's sum of squares from its `parts` partial sums (one per (column tile, epilogue warp)
-// of the producing GEMM), added in a fixed order so every run gives the same value.
-__device__ __forceinline__ float row_ss(const float *s, long long row, int parts) {
+// of the producing GEMM), added in a fixed order so every run gives the same value.  The first
+// kPf slots are only loaded here (independent loads whose latency hides under the current tile,
+// summed by row_ss_sum when the next tile needs them); slots beyond kPf (more than three column
+// tiles of the producer) are added at once.
+constexpr int kPf = 8;
+struct RowSS {
+  float v[kPf];
+  float extra;
+};
+__device__ __forceinline__ void row_ss_fetch(RowSS &r, const float *s, long long row, int parts) {
   const float *q = s + row * parts;
+#pragma unroll
+  for (int i = 0; i < kPf; ++i) r.v[i] = i < parts ? q[i] : 0.f;
+  r.extra = 0.f;
+  for (int i = kPf; i < parts; ++i) r.extra += q[i];
+}
+__device__ __forceinline__ float row_ss_sum(const RowSS &r) {
   float a = 0.f;
-  for (int i = 0; i < parts; ++i) a += q[i];
-  return a;
+#pragma unroll
+  for (int i = 0; i < kPf; ++i) a += r.v[i];
+  return a + r.extra;
+}
+__device__ __forceinline__ void row_ss_one(RowSS &r) {
+#pragma unroll
+  for (int i = 0; i < kPf; ++i) r.v[i] = 0.f;
+  r.v[0] = 1.f;
+  r.extra = 0.f;
 }
 
 // ------------------------------------------------------------------ the kernel
@@ -307,7 +328,8 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     // The row's deferred-norm sum of squares (and, for QKV, its rotary (cos, sin) pairs),
     // fetched one tile ahead so the loads' latency hides under the previous tile's
     // epilogue: nothing reads them before the next tile.
-    float ss_pf = 1.f;
+    RowSS ss_pf;
+    row_ss_one(ss_pf);
     QkvRow qr_pf{0, 0};
     float2 cs_pf[16];
     auto row_fetch = [&](int tile_) {
@@ -317,7 +339,8 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       const bool v_ = m_ < p.M;
       if (EPI == kTcQkv) {
         qr_pf = qkv_row(p, v_ ? m_ : 0, t_.g);
-        ss_pf = (v_ && p.ss_in) ? row_ss(p.ss_in, qr_pf.tok, p.ss_in_parts) : 1.f;
+        if (v_ && p.ss_in) row_ss_fetch(ss_pf, p.ss_in, qr_pf.tok, p.ss_in_parts);
+        else row_ss_one(ss_pf);
         // rotary pairs only for q and k column blocks; 16-byte loads (a row's 16 pairs are
         // 128 contiguous bytes at a 128-byte offset of the table's 256-byte row)
         if (p.dh == 64 && t_.nblk * p.BN < 2 * p.A) {
@@ -330,11 +353,14 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           }
         }
       } else if (EPI == kTcGelu || EPI == kTcGeglu) {
-        ss_pf = (v_ && p.ss_in) ? row_ss(p.ss_in, m_, p.ss_in_parts) : 1.f;
+        if (v_ && p.ss_in) row_ss_fetch(ss_pf, p.ss_in, m_, p.ss_in_parts);
+        else row_ss_one(ss_pf);
       } else if (EPI == kTcTanh) {
-        ss_pf = (v_ && p.ss_in) ? row_ss(p.ss_in, token_of(p, m_, t_.g), p.ss_in_parts) : 1.f;
+        if (v_ && p.ss_in) row_ss_fetch(ss_pf, p.ss_in, token_of(p, m_, t_.g), p.ss_in_parts);
+        else row_ss_one(ss_pf);
       } else if (EPI == kTcResid) {
-        ss_pf = (v_ && p.res_ss) ? row_ss(p.res_ss, m_, p.ss_in_parts) : 1.f;
+        if (v_ && p.res_ss) row_ss_fetch(ss_pf, p.res_ss, m_, p.ss_in_parts);
+        else row_ss_one(ss_pf);
       }
     };
     row_fetch(blockIdx.x);
@@ -355,7 +381,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       QkvRow qr{0, 0};
       float2 cs[16];
       // 1 / |x| of the row (deferred norm: of the GEMM input, or of the residual for kTcResid)
-      const float rsq = 1.f / fmaxf(sqrtf(ss_pf), kEps);
+      const float rsq = 1.f / fmaxf(sqrtf(row_ss_sum(ss_pf)), kEps);
       if (EPI == kTcQkv) {
         qr = qr_pf;
 #pragma unroll
