@@ -75,7 +75,7 @@ typedef struct {
                             whose first projection is [2*ff, dim] with halves (value, gate) and
                             whose hidden is value * gelu(gate) */
   int dim_head_v;        /* width of v per head; 0: dim_head.  A value below dim_head gives the
-                            attention whose q and k are deeper than v ("stemd evaluation.md",
+                            attention whose q and k are deeper than v ("evaluation.md",
                             section "BS PolarFormer: the same quality for a quarter of the
                             arithmetic": q and k 128 deep against v 64; rotary positions on q and
                             k): to_qkv is then [heads*(2*dim_head + dim_head_v), dim] with

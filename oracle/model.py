@@ -90,8 +90,8 @@ def attention(x, w, heads: int, dim_head: int, theta: float, dim_head_v: int = 0
 
     a = norm(x); [q; k; v] = a W_qkv^T with features ordered (which, head, d); q, k
     rotated; o_h = attend(q_h, k_h, v_h) * sigmoid(a W_g^T + b_g)_h; out = concat_h o_h W_o^T.
-    With dim_head_v (v narrower than q and k, as in the PolarFormer attention of "stemd
-    evaluation.md", section "BS PolarFormer: the same quality for a quarter of the arithmetic")
+    With dim_head_v (v narrower than q and k, as in the PolarFormer attention of
+    "evaluation.md", section "BS PolarFormer: the same quality for a quarter of the arithmetic")
     the projection's features are q (heads x dim_head), k (heads x dim_head), v (heads x
     dim_head_v), each ordered (head, d); the softmax scale stays dim_head^-0.5 (the q.k width).
     """

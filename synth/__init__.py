@@ -83,7 +83,7 @@ class ModelConfig:
 # "vocals" is the dim-384 / depth-6 / 60-band vocals checkpoint shape.
 TINY = ModelConfig(n_fft=256, num_bands=8, dim=64, depth=1, heads=4, dim_head=16)
 # An attention whose q and k are twice as wide as v (the shape of the BS PolarFormer attention of
-# "stemd evaluation.md", section "BS PolarFormer: the same quality for a quarter of the
+# "evaluation.md", section "BS PolarFormer: the same quality for a quarter of the
 # arithmetic": 8 heads, q and k of 128 against v of 64), on the vocals band split, with rotary
 # positions on q and k.
 WIDE_QK = ModelConfig(dim=256, depth=1, heads=8, dim_head=128, dim_head_v=64)

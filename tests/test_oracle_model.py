@@ -502,7 +502,7 @@ def test_band_split_brute_force():
 # ---------------------------------------------------------------- v narrower than q and k
 def brute_attention_layer_wide_qk(x, w, h, dh, dv, theta):
     """Scalar loops for the attention whose q and k (dh per head) are wider than v (dv per head)
-    ("stemd evaluation.md", section "BS PolarFormer: the same quality for a quarter of the
+    ("evaluation.md", section "BS PolarFormer: the same quality for a quarter of the
     arithmetic"): projection features q (head, d < dh), then k (head, d < dh), then v (head, d <
     dv); softmax scale dh^-1/2; heads concatenated head-major (h * dv wide)."""
     n, D = x.shape

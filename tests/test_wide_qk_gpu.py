@@ -1,6 +1,6 @@
 """Attention whose q and k are deeper than v, through the C ABI (GPU), against the oracle.
 
-"stemd evaluation.md", section "BS PolarFormer: the same quality for a quarter of the
+"evaluation.md", section "BS PolarFormer: the same quality for a quarter of the
 arithmetic": that model's positional encoding doubles the depth of q and k (128) and leaves v at
 64, and the fix it names is "a fused attention that tolerates v being narrower than q".  The
 pages define neither PoPE nor that model's 62-band table, so the shape is built on this model's
