@@ -34,7 +34,6 @@
 
 #include "gemm_tc.cuh"
 #include "mrf_internal.h"
-#include "tc_math.cuh"
 #include "tc_ptx.cuh"
 
 namespace mrf {
@@ -58,21 +57,7 @@ constexpr int kThreads = 384;
 constexpr int kRegsLaunch = 168, kRegsSoftmax = 208, kRegsIo = 72;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsIo <= kThreads * kRegsLaunch, "register split over budget");
 constexpr float kRescaleLog2 = 8.f;
-#ifndef MRF_ATTN_POLY_EVERY
-#define MRF_ATTN_POLY_EVERY 4
-#endif
-// Every kPolyEvery-th pair of softmax exponentials on the FMA pipe (0: all on the MUFU).
-constexpr int kPolyEvery = MRF_ATTN_POLY_EVERY;
-#ifndef MRF_ATTN_SPEC
-#define MRF_ATTN_SPEC 0
-#endif
-#ifndef MRF_ATTN_MAXTREE
-#define MRF_ATTN_MAXTREE 0
-#endif
-// Later blocks exponentiate against the running max with the block max computed alongside
-// (rows whose max rose by more than 2^8 recompute), rather than taking the block max first.
-constexpr bool kSpeculativeMax = MRF_ATTN_SPEC;
-constexpr bool kMaxTree = MRF_ATTN_MAXTREE;
+
 
 // q and k are kQA 64-wide atoms deep (dim_head 64 or 128; v is 64 wide either way): each query
 // tile takes kQA 16 KB tiles, a key block kQA K tiles and one V tile.  The ring shrinks to 8 tiles
@@ -198,6 +183,10 @@ struct AttnArgs {
   unsigned *status;
   int B, T, nb, H, axis, ld, n, q_tiles, pairs, items, n_blocks, BT;
   int gate_col;  // column of head 0's gate in a projection row (after q, k and v)
+  // odd last query tiles run alone (one per item, the item's second tile idle) instead of paired
+  // across two sequences: with 128-deep q and k a block with separate keys would fill 6 of the
+  // 8 ring tiles, and the MMA issuer needs the next block before it releases the current one
+  int split_odd;
   int S;  // time axis: sequences (b, band, head)
 };
 
@@ -218,17 +207,22 @@ struct TileC {
 // count) the item of their two last tiles, so all items reading a sequence's keys run close
 // together and find them in L2.  With an odd sequence count the last group has one sequence.
 struct ItemPos {
-  int seq, pair;  // shared: sequence and pair index; mixed: first sequence, pair = -1
+  int seq, pair;  // shared: sequence and pair index; mixed: first sequence, pair = -1;
+                  // a lone odd last tile (split_odd): its sequence, pair = -2
 };
 
 __device__ __forceinline__ ItemPos item_pos(const AttnArgs &a, int item) {
-  const int gs = 2 * a.pairs + (a.q_tiles & 1);
+  const int odd_items = (a.q_tiles & 1) ? (a.split_odd ? 2 : 1) : 0;
+  const int gs = 2 * a.pairs + odd_items;
   const int grp = item / gs, r = item - grp * gs;
   const int n_seq = 2 * grp + 1 < a.S ? 2 : 1;
   ItemPos ip;
   if (r < n_seq * a.pairs) {
     ip.seq = 2 * grp + r / a.pairs;
     ip.pair = r % a.pairs;
+  } else if (a.split_odd) {
+    ip.seq = 2 * grp + (r - n_seq * a.pairs);
+    ip.pair = -2;
   } else {
     ip.seq = 2 * grp;
     ip.pair = -1;
@@ -237,7 +231,7 @@ __device__ __forceinline__ ItemPos item_pos(const AttnArgs &a, int item) {
 }
 
 __device__ __forceinline__ bool item_mixed(const AttnArgs &a, int item) {
-  return a.axis != 0 || item_pos(a, item).pair < 0;
+  return a.axis != 0 || item_pos(a, item).pair == -1;
 }
 
 __device__ __forceinline__ TileC tile_coords(const AttnArgs &a, int item, int t) {
@@ -249,6 +243,10 @@ __device__ __forceinline__ TileC tile_coords(const AttnArgs &a, int item, int t)
     if (ip.pair >= 0) {
       seq = ip.seq;
       qt = 2 * ip.pair + t;
+    } else if (ip.pair == -2) {
+      seq = ip.seq;  // a lone odd last tile: tile 1 repeats it on the same keys and stores nothing
+      qt = a.q_tiles - 1;
+      c.valid = t == 0;
     } else {
       seq = ip.seq + t;
       if (seq >= a.S) { seq = a.S - 1; c.valid = false; }
@@ -272,27 +270,9 @@ __device__ __forceinline__ TileC tile_coords(const AttnArgs &a, int item, int t)
   return c;
 }
 
-// Max of a score row: four max3 chains (kMaxTree: a tree of max3, depth 5 for 128 values).
+// Max of a score row: four independent max3 chains, joined at the end.
 template <int NC>
 __device__ __forceinline__ float row_max(const float (&sv)[NC]) {
-  if (kMaxTree) {
-    float a[(NC + 2) / 3];
-#pragma unroll
-    for (int i = 0; i < NC / 3; ++i) a[i] = max3(sv[3 * i], sv[3 * i + 1], sv[3 * i + 2]);
-    int n = NC / 3;
-    if (NC % 3 == 1) a[n++] = sv[NC - 1];
-    if (NC % 3 == 2) a[n++] = fmaxf(sv[NC - 2], sv[NC - 1]);
-#pragma unroll
-    for (int len = (NC + 2) / 3; len > 1; len = (len + 2) / 3) {
-#pragma unroll
-      for (int i = 0; i < (len + 2) / 3; ++i) {
-        const float x = a[3 * i], y = 3 * i + 1 < len ? a[3 * i + 1] : x, z = 3 * i + 2 < len ? a[3 * i + 2] : x;
-        a[i] = max3(x, y, z);
-      }
-    }
-    (void)n;
-    return a[0];
-  }
   constexpr int Q = NC / 4;
   float ma = sv[0], mb = sv[Q], mc = sv[2 * Q], md = sv[3 * Q];
 #pragma unroll
@@ -306,39 +286,12 @@ __device__ __forceinline__ float row_max(const float (&sv)[NC]) {
   return fmaxf(fmaxf(ma, mb), fmaxf(mc, md));
 }
 
-// 2^x for a pair on the FMA pipe, relieving the MUFU (16 exponentials per clock per SM, this
-// kernel's bound at 64-wide heads): x = n + f with n = rint(x) (the 1.5 * 2^23 rounding trick), f
-// in [-1/2, 1/2]; 2^f by a degree-3 polynomial, the minimax fit of the relative error on that
-// interval (Remez exchange: max relative error 7.5e-5, below the fp16 rounding of P); 2^n added
-// to the exponent field as an integer.  x is clamped at -125 so the exponent stays normal (the
-// result then rounds to 0 in fp16, as the MUFU's 2^-inf does).
-__device__ __forceinline__ float2 exp2_poly2(float2 d) {
-  const unsigned long long x = tcm::f2_pack(fmaxf(d.x, -125.f), fmaxf(d.y, -125.f));
-  const unsigned long long magic = tcm::f2_pack(12582912.f, 12582912.f);
-  unsigned long long t, n, f;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(magic));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(n) : "l"(t), "l"(magic));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(n));
-  unsigned long long p = tcm::fma2(f, tcm::f2_pack(0.05517166905792616f, 0.05517166905792616f),
-                                   tcm::f2_pack(0.2426111221932161f, 0.2426111221932161f));
-  p = tcm::fma2(f, p, tcm::f2_pack(0.6932609854606553f, 0.6932609854606553f));
-  p = tcm::fma2(f, p, tcm::f2_pack(0.9999280735394012f, 0.9999280735394012f));
-  const unsigned lo = (unsigned)p + ((unsigned)t << 23), hi = (unsigned)(p >> 32) + ((unsigned)(t >> 32) << 23);
-  return make_float2(__uint_as_float(lo), __uint_as_float(hi));
-}
-
 // One key block of one query row: scores from tensor memory (log2 units: q was scaled by
 // log2(e) / sqrt(dh) in its projection), the running max and sum, p = 2^(s - m) into P as
 // 16-bit pairs, and the O row rescaled in place when its max was raised.  NC live score columns
 // at tS (columns >= hi are masked); P's matching NC / 2 columns at tP.  Returns false if a
 // wait timed out.
 //
-// The first block of an item takes its row max first.  Later blocks compute their
-// exponentials against the running max straight away, with the block's max alongside (its
-// instructions fill the issue slots between the MUFU's); only a row whose block max exceeds the
-// running max by more than 2^8 recomputes its p from the scores, which stay in registers.
-// Every kPolyEvery-th pair of exponentials is evaluated on the FMA pipe (exp2_poly2) instead of
-// the MUFU.
 template <int NC, bool kBF>
 __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t tO, int hi, float &m_run, float &l,
                                               bool wait_pv, uint64_t *pv_done, uint32_t pv_parity,
@@ -355,64 +308,43 @@ __device__ __forceinline__ bool softmax_block(uint32_t tS, uint32_t tP, uint32_t
     for (int i = 0; i < NC; ++i)
       if (i >= hi) sv[i] = -INFINITY;
   }
+  // the block's max; for the item's first block it is the running max (l is still 0)
   const bool first = !wait_pv;
+  const float bm = row_max<NC>(sv);
   bool need = false;
   float alpha = 1.f;
-  if (first || !kSpeculativeMax) {
-    // the block's max first (for the item's first block it is the running max: l is still 0)
-    const float bm = row_max<NC>(sv);
-    if (first) {
-      m_run = bm;
-    } else {
-      need = bm > m_run + kRescaleLog2;
-      if (need) {
-        alpha = ex2(m_run - bm);
-        l *= alpha;
-        m_run = bm;
-      }
-    }
-  }
-  // p = 2^(s - m) in 16-bit pairs (the P*V MMA's A operand), the row sum in four f32x2 chains,
-  // and (later blocks) the block max in four max3 chains.  None of this needs P_t or O_t, so it
-  // runs before the wait for the previous block's P*V, which then overlaps it.
-  uint32_t pk[NC / 2];
-  float2 s4;
-  float bmax = -INFINITY;
-  auto exp_pass = [&](float m, bool with_max) {
-    float2 sa = make_float2(0.f, 0.f), sb = sa, sc = sa, sd = sa;
-    float ma = -INFINITY, mb = ma, mc = ma, md = ma;
-    const float2 negm = make_float2(-m, -m);
-#pragma unroll
-    for (int i = 0; i < NC; i += 8) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float s0 = sv[i + 2 * u], s1 = sv[i + 2 * u + 1];
-        const float2 d = add2(make_float2(s0, s1), negm);
-        const int pair = (i >> 1) + u;
-        const float2 pp = (kPolyEvery > 0 && pair % kPolyEvery == kPolyEvery - 1) ? exp2_poly2(d)
-                                                                                  : make_float2(ex2(d.x), ex2(d.y));
-        switch (u) {
-          case 0: sa = add2(sa, pp); if (with_max) ma = max3(ma, s0, s1); break;
-          case 1: sb = add2(sb, pp); if (with_max) mb = max3(mb, s0, s1); break;
-          case 2: sc = add2(sc, pp); if (with_max) mc = max3(mc, s0, s1); break;
-          default: sd = add2(sd, pp); if (with_max) md = max3(md, s0, s1); break;
-        }
-        pk[pair] = pack_h2<kBF>(pp.x, pp.y);
-      }
-    }
-    s4 = add2(add2(sa, sb), add2(sc, sd));
-    if (with_max) bmax = fmaxf(fmaxf(ma, mb), fmaxf(mc, md));
-  };
-  exp_pass(m_run, !first && kSpeculativeMax);
-  if (!first && kSpeculativeMax) {
-    need = bmax > m_run + kRescaleLog2;
-    if (__any_sync(0xffffffffu, need) && need) {
-      alpha = ex2(m_run - bmax);
+  if (first) {
+    m_run = bm;
+  } else {
+    need = bm > m_run + kRescaleLog2;
+    if (need) {
+      alpha = ex2(m_run - bm);
       l *= alpha;
-      m_run = bmax;
-      exp_pass(m_run, false);
+      m_run = bm;
     }
   }
+  // p = 2^(s - m): pairs through packed f32x2 subtract, exponentials on MUFU, packed to 16-bit
+  // pairs (the P*V MMA's A operand), the row sum in four f32x2 chains.  This needs neither P_t
+  // nor O_t, so it runs before the wait for the previous block's P*V, which then overlaps it.
+  uint32_t pk[NC / 2];
+  float2 sa = make_float2(0.f, 0.f), sb = sa, sc = sa, sd = sa;
+  const float2 negm = make_float2(-m_run, -m_run);
+#pragma unroll
+  for (int i = 0; i < NC; i += 8) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 d = add2(make_float2(sv[i + 2 * u], sv[i + 2 * u + 1]), negm);
+      const float2 pp = make_float2(ex2(d.x), ex2(d.y));
+      switch (u) {
+        case 0: sa = add2(sa, pp); break;
+        case 1: sb = add2(sb, pp); break;
+        case 2: sc = add2(sc, pp); break;
+        default: sd = add2(sd, pp); break;
+      }
+      pk[(i >> 1) + u] = pack_h2<kBF>(pp.x, pp.y);
+    }
+  }
+  const float2 s4 = add2(add2(sa, sb), add2(sc, sd));
   // P_t and O_t are free once the previous block's P*V has completed
   if (wait_pv && !tc::mbar_wait(pv_done, pv_parity, status, 39, abort)) return false;
   tc::tc_fence_after();
@@ -755,11 +687,13 @@ bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int
     // sequence's (separate keys)
     a.S = B * nb * H;
     a.pairs = a.q_tiles / 2;
-    a.items = a.S * a.pairs + ((a.q_tiles & 1) ? (a.S + 1) / 2 : 0);
+    a.split_odd = dqk == 128;
+    a.items = a.S * a.pairs + ((a.q_tiles & 1) ? (a.split_odd ? a.S : (a.S + 1) / 2) : 0);
     a.n_blocks = (a.n + kKeys - 1) / kKeys;
     box[0] = 64; box[1] = 1; box[2] = 1; box[3] = kRows;       // 128 frames of one (band, head)
   } else {
     if (nb > 64) return false;
+    a.split_odd = 0;
     a.pairs = 0;
     a.S = 0;
     a.items = H * ((a.BT + 3) / 4);
