@@ -99,8 +99,11 @@ bool gemm_tc_init();
 //  no swizzle).  Unused maps may be any valid map.
 // bf16: A, W and every 16-bit output in bf16 (MRF_BF16), the residual kinds also keeping the fp32
 // master copy X (tmC: X fp32 box 32x32 swizzle 128, or the 3-D (ld, nb, frames) 32x1x32 box of the
-// band split); otherwise fp16.
-void launch_gemm_tc(int epi, bool bf16, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
-                    const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st);
+// band split); otherwise fp16.  pair (for the kinds gemm_tc_pair_kind accepts): clusters of two
+// CTAs, each cluster an M = 256 tile (p.m_tiles counted in 256-row tiles), grid even, and tmB's box
+// BN / 2 rows; otherwise one CTA per M = 128 tile with tmB's box BN rows.
+void launch_gemm_tc(int epi, bool bf16, bool pair, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                    const CUtensorMap &tmC, const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st);
+bool gemm_tc_pair_kind(int epi);
 
 }  // namespace mrf

@@ -46,7 +46,9 @@ constexpr float kEps = 1e-12f;
 // main loop wants four pipeline stages and the epilogue the 168 registers of a 10-warp
 // CTA.  Pipeline stages fill what shared memory the epilogue staging leaves.
 __host__ __device__ constexpr int epi_warps(int epi) { return (epi == kTcGelu || epi == kTcBandSplit) ? 16 : 8; }
-__host__ __device__ constexpr int gemm_stages(int epi) { return epi_warps(epi) == 8 ? 4 : 3; }
+__host__ __device__ constexpr int gemm_stages(int epi, bool pair = false) {
+  return pair ? (epi_warps(epi) == 8 ? 6 : 5) : (epi_warps(epi) == 8 ? 4 : 3);
+}
 __host__ __device__ constexpr int gemm_threads(int epi) { return 32 * (epi_warps(epi) + 2); }
 
 // Widest B tile of an epilogue kind, and the shared memory each epilogue warp needs.
@@ -57,12 +59,14 @@ __host__ __device__ constexpr int warp_stage_bytes(int epi, bool bf) {
   return (bf && (epi == kTcResid || epi == kTcBandSplit)) ? 4096 + 2048 : 2 * 2048;
 }
 
-template <int EPI, bool kBF>
+// kPair: a CTA of a pair holds half of the B tile's rows per stage (and has room for more stages).
+template <int EPI, bool kBF, bool kPair = false>
 struct SmemLayout {
-  static constexpr int b_stage = bn_max(EPI) * BK * 2;
+  static constexpr int stages = gemm_stages(EPI, kPair);
+  static constexpr int b_stage = (kPair ? bn_max(EPI) / 2 : bn_max(EPI)) * BK * 2;
   static constexpr int a_off = 0;
-  static constexpr int b_off = gemm_stages(EPI) * A_STAGE;
-  static constexpr int stg_off = b_off + gemm_stages(EPI) * b_stage;        // 1024-aligned
+  static constexpr int b_off = stages * A_STAGE;
+  static constexpr int stg_off = b_off + stages * b_stage;        // 1024-aligned
   static constexpr int bar_off = stg_off + epi_warps(EPI) * warp_stage_bytes(EPI, kBF);
   static constexpr int total = bar_off + 256;
 };
@@ -216,13 +220,20 @@ __device__ __forceinline__ void row_ss_one(RowSS &r) {
 }
 
 // ------------------------------------------------------------------ the kernel
-template <int EPI, bool kBF>
+// kPair: the kernel runs as clusters of two CTAs on two SMs, each cluster one M = 256 tile at a
+// time (cta_group::2 MMAs issued by the leader, rank 0): CTA r loads rows 128 r .. 128 r + 127 of
+// the tile's A and rows n_mma r / 2 .. of its B (n_mma the tile's MMA width), both CTAs' loads
+// complete on the leader's full barrier, the leader's commits arrive on both CTAs' empty and tfull
+// barriers, and both CTAs' epilogue warps release the accumulator on the leader's tempty barrier.
+// Each SM then streams half of every weight tile, halving the shared-memory traffic per MMA flop.
+template <int EPI, bool kBF, bool kPair>
 __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                    const GemmParams p) {
-  using L = SmemLayout<EPI, kBF>;
-  constexpr int kEpiWarps = epi_warps(EPI), kSplit = kEpiWarps / 4, kGemmStages = gemm_stages(EPI);
+  using L = SmemLayout<EPI, kBF, kPair>;
+  constexpr int kEpiWarps = epi_warps(EPI), kSplit = kEpiWarps / 4, kGemmStages = L::stages;
+  constexpr int kTileM = kPair ? 2 * BM : BM;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem + L::a_off;
@@ -237,20 +248,28 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = kPair ? tc::cluster_ctarank() : 0;       // rank within the CTA pair
+  const int first_tile = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tile_step = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < kGemmStages; ++s) { tc::mbar_init(full + s, 1); tc::mbar_init(empty + s, 1); }
-    for (int s = 0; s < 2; ++s) { tc::mbar_init(tfull + s, 1); tc::mbar_init(tempty + s, kEpiWarps); }
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(tfull + s, 1);
+      tc::mbar_init(tempty + s, kPair ? 2 * kEpiWarps : kEpiWarps);  // pair: both CTAs' epilogue warps
+    }
     tc::mbar_init(done, 1);
     tc::fence_barrier_init();
   }
   if (warp == kEpiWarps) {
     if (lane == 0) { tc::tma_prefetch(&tmA); tc::tma_prefetch(&tmB); }
     __syncwarp();
-    tc::tmem_alloc(tmem_slot, TMEM_COLS);
+    if (kPair) tc::tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    else tc::tmem_alloc(tmem_slot, TMEM_COLS);
   }
   tc::tc_fence_before();
   __syncthreads();
+  if (kPair) tc::cluster_sync();  // the peer's barriers are initialised before any remote arrive
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   volatile int *abort = &abort_flag;
@@ -260,22 +279,36 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     // ---------------- TMA producer
     // (stall test: CTA 0 loads nothing, a flag nobody sets; its MMA and epilogue waits expire
     // after their bounded limit, record the site and return)
-    if (lane == 0 && !(p.stall_test && blockIdx.x == 0)) {
+    if (lane == 0 && !(p.stall_test && first_tile == 0)) {
       int stage = 0;
       uint32_t phase = 0;
-      const uint32_t bytes = A_STAGE + p.BN * BK * 2;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      // bytes completing on this CTA's full barrier (pair: both CTAs' loads on the leader's)
+      const uint32_t bytes = kPair ? 2 * (A_STAGE + (p.BN / 2) * BK * 2) : A_STAGE + p.BN * BK * 2;
+      for (int tile = first_tile; tile < total; tile += tile_step) {
         const TileInfo ti = decode_tile(p, tile);
         const GemmGroup &gr = p.groups[ti.g];
-        const int m0 = ti.mb * BM, n0 = gr.b_row_off + ti.nblk * p.BN;
+        const int m0 = ti.mb * kTileM + (int)rank * BM;
+        int n0 = gr.b_row_off + ti.nblk * p.BN;
+        if (kPair) {  // this CTA's half of the tile's MMA width
+          const int n_mma = (min(p.BN, gr.N - ti.nblk * p.BN) + 15) & ~15;
+          n0 += (int)rank * (n_mma >> 1);
+        }
         const int kblocks = gr.kblocks ? gr.kblocks : p.K / BK;
         bool ok = true;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!tc::mbar_wait(empty + stage, phase ^ 1, p.status, 10, abort)) { ok = false; break; }
-          tc::mbar_arrive_expect_tx(full + stage, bytes);
-          if (p.a_mode == 0) tc::tma_load_3d(sA + stage * A_STAGE, &tmA, full + stage, kb * BK, gr.a_off + m0, 0);
-          else tc::tma_load_3d(sA + stage * A_STAGE, &tmA, full + stage, kb * BK, gr.a_off, m0);
-          tc::tma_load_3d(sB + stage * L::b_stage, &tmB, full + stage, kb * BK, n0, 0);
+          if (kPair) {
+            if (rank == 0) tc::mbar_arrive_expect_tx(full + stage, bytes);
+            const uint32_t lb = tc::leader_addr(full + stage);
+            if (p.a_mode == 0) tc::tma_load_3d_pair(sA + stage * A_STAGE, &tmA, lb, kb * BK, gr.a_off + m0, 0);
+            else tc::tma_load_3d_pair(sA + stage * A_STAGE, &tmA, lb, kb * BK, gr.a_off, m0);
+            tc::tma_load_3d_pair(sB + stage * L::b_stage, &tmB, lb, kb * BK, n0, 0);
+          } else {
+            tc::mbar_arrive_expect_tx(full + stage, bytes);
+            if (p.a_mode == 0) tc::tma_load_3d(sA + stage * A_STAGE, &tmA, full + stage, kb * BK, gr.a_off + m0, 0);
+            else tc::tma_load_3d(sA + stage * A_STAGE, &tmA, full + stage, kb * BK, gr.a_off, m0);
+            tc::tma_load_3d(sB + stage * L::b_stage, &tmB, full + stage, kb * BK, n0, 0);
+          }
           if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
@@ -283,18 +316,18 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     }
   } else if (warp == kEpiWarps + 1) {
     // ---------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {  // pair: the leader issues the pair's MMAs
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+      for (int tile = first_tile; tile < total; tile += tile_step, ++local) {
         const TileInfo ti = decode_tile(p, tile);
         const GemmGroup &gr = p.groups[ti.g];
         const int acc = local & 1;
         const uint32_t aphase = (local >> 1) & 1;
         int n_eff = min(p.BN, gr.N - ti.nblk * p.BN);
         n_eff = (n_eff + 15) & ~15;
-        const uint32_t idesc = tc::idesc_f16(BM, n_eff, false, kBF);
+        const uint32_t idesc = tc::idesc_f16(kTileM, n_eff, false, kBF);
         const uint32_t d_tmem = tmem_base + acc * 256;
         const int kblocks = gr.kblocks ? gr.kblocks : p.K / BK;
         if (!tc::mbar_wait(tempty + acc, aphase ^ 1, p.status, 11, abort)) break;
@@ -307,16 +340,23 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           const uint32_t b_addr = tc::smem_u32(sB + stage * L::b_stage);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            tc::mma_f16(d_tmem, tc::sw128_kmajor_desc(a_addr + kk * 32), tc::sw128_kmajor_desc(b_addr + kk * 32),
-                        idesc, (kb | kk) != 0);
+            if (kPair)
+              tc::mma_f16_pair(d_tmem, tc::sw128_kmajor_desc(a_addr + kk * 32),
+                               tc::sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0);
+            else
+              tc::mma_f16(d_tmem, tc::sw128_kmajor_desc(a_addr + kk * 32), tc::sw128_kmajor_desc(b_addr + kk * 32),
+                          idesc, (kb | kk) != 0);
           }
-          tc::mma_commit(empty + stage);
+          if (kPair) tc::mma_commit_pair(empty + stage, 0x3);
+          else tc::mma_commit(empty + stage);
           if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc::mma_commit(tfull + acc);
+        if (kPair) tc::mma_commit_pair(tfull + acc, 0x3);
+        else tc::mma_commit(tfull + acc);
       }
-      tc::mma_commit(done);
+      if (kPair) tc::mma_commit_pair(done, 0x1);
+      else tc::mma_commit(done);
       tc::mbar_wait(done, 0, p.status, 13, abort);
     }
   } else {
@@ -335,7 +375,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     auto row_fetch = [&](int tile_) {
       if (tile_ >= total) return;
       const TileInfo t_ = decode_tile(p, tile_);
-      const int m_ = t_.mb * BM + quarter * 32 + lane;
+      const int m_ = t_.mb * kTileM + (int)rank * BM + quarter * 32 + lane;
       const bool v_ = m_ < p.M;
       if (EPI == kTcQkv) {
         qr_pf = qkv_row(p, v_ ? m_ : 0, t_.g);
@@ -363,13 +403,13 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         else row_ss_one(ss_pf);
       }
     };
-    row_fetch(blockIdx.x);
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+    row_fetch(first_tile);
+    for (int tile = first_tile; tile < total; tile += tile_step, ++local) {
       const TileInfo ti = decode_tile(p, tile);
       const GemmGroup &gr = p.groups[ti.g];
       const int acc = local & 1;
       const uint32_t aphase = (local >> 1) & 1;
-      const int m0w = ti.mb * BM + quarter * 32;  // first row of this warp's 32
+      const int m0w = ti.mb * kTileM + (int)rank * BM + quarter * 32;  // first row of this warp's 32
       const int m = m0w + lane;
       const bool valid = m < p.M;
       const int nbase = ti.nblk * p.BN;
@@ -389,7 +429,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       }
       if (EPI == kTcQkv || EPI == kTcGelu || EPI == kTcGeglu || EPI == kTcTanh) rs = rsq;
       const float res_s = rsq;  // kTcResid
-      row_fetch(tile + gridDim.x);
+      row_fetch(tile + tile_step);
       // residual prefetch (kTcResid): fp16 rows of 64 bytes, lane covering rows i*8 + lane/4 and
       // 16-byte piece lane%4; with kBF the fp32 master rows of 128 bytes, rows i*4 + lane/8, piece lane%8
       constexpr int kPieces = kBF ? 8 : 4;
@@ -653,7 +693,10 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       if (EPI == kTcBandSplit && valid) p.ss_out[((long long)m * p.nb + ti.g) * p.ss_out_parts + slot] = sq;
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(tempty + acc);
+      if (lane == 0) {
+        if (kPair && rank != 0) tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(tempty + acc), 0));
+        else tc::mbar_arrive(tempty + acc);
+      }
     }
     // outstanding bulk stores must finish reading shared memory before the CTA exits
     if (lane == 0) tc::bulk_wait_all();
@@ -661,9 +704,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   }
   tc::tc_fence_before();
   __syncthreads();
+  if (kPair) tc::cluster_sync();  // no remote arrive or MMA of the pair is outstanding past here
   if (warp == kEpiWarps) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem_base, TMEM_COLS);
+    if (kPair) tc::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tc::tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -679,14 +724,51 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-template <int EPI, bool kBF>
-constexpr size_t smem_bytes() { return SmemLayout<EPI, kBF>::total + 1024; }
+template <int EPI, bool kBF, bool kPair = false>
+constexpr size_t smem_bytes() { return SmemLayout<EPI, kBF, kPair>::total + 1024; }
 constexpr size_t kSmemLimit = 232448;  // 227 KB per CTA
-static_assert(smem_bytes<kTcQkv, true>() <= kSmemLimit && smem_bytes<kTcResid, true>() <= kSmemLimit &&
-                  smem_bytes<kTcGelu, true>() <= kSmemLimit && smem_bytes<kTcBandSplit, true>() <= kSmemLimit &&
-                  smem_bytes<kTcGlu, true>() <= kSmemLimit && smem_bytes<kTcTanh, true>() <= kSmemLimit &&
-                  smem_bytes<kTcGeglu, true>() <= kSmemLimit,
+// The epilogue kinds that run as CTA pairs (the trunk's four GEMMs); the grouped mask-head and
+// band-split GEMMs run one CTA per tile.
+__host__ __device__ constexpr bool pair_kind(int epi) {
+  return epi == kTcQkv || epi == kTcResid || epi == kTcGelu || epi == kTcGeglu;
+}
+template <int EPI>
+constexpr bool smem_fits() {
+  return smem_bytes<EPI, false, false>() <= kSmemLimit && smem_bytes<EPI, true, false>() <= kSmemLimit &&
+         (!pair_kind(EPI) || (smem_bytes<EPI, false, true>() <= kSmemLimit && smem_bytes<EPI, true, true>() <= kSmemLimit));
+}
+static_assert(smem_fits<kTcQkv>() && smem_fits<kTcResid>() && smem_fits<kTcGelu>() && smem_fits<kTcBandSplit>() &&
+                  smem_fits<kTcGlu>() && smem_fits<kTcTanh>() && smem_fits<kTcGeglu>(),
               "shared memory per CTA over the 227 KB limit");
+
+template <int EPI, bool kBF, bool kPair>
+bool set_smem_attr() {
+  return cudaFuncSetAttribute(gemm_tc_kernel<EPI, kBF, kPair>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)smem_bytes<EPI, kBF, kPair>()) == cudaSuccess;
+}
+
+template <int EPI, bool kBF, bool kPair>
+void launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC, const CUtensorMap &tmD,
+                const GemmParams &p, int grid, cudaStream_t st) {
+  if constexpr (kPair) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(gemm_threads(EPI), 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes<EPI, kBF, true>();
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI, kBF, true>, tmA, tmB, tmC, tmD, p);
+  } else {
+    gemm_tc_kernel<EPI, kBF, false><<<grid, gemm_threads(EPI), smem_bytes<EPI, kBF, false>(), st>>>(tmA, tmB, tmC,
+                                                                                                    tmD, p);
+  }
+}
 
 }  // namespace
 
@@ -720,12 +802,9 @@ bool make_tmap_f16(CUtensorMap *map, const void *base, unsigned long long d0, un
 
 bool gemm_tc_init() {
   bool ok = encode_fn() != nullptr;
-#define MRF_GEMM_ATTR(E)                                                                                    \
-  ok = ok &&                                                                                                \
-       cudaFuncSetAttribute(gemm_tc_kernel<E, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,          \
-                            (int)smem_bytes<E, false>()) == cudaSuccess &&                                  \
-       cudaFuncSetAttribute(gemm_tc_kernel<E, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,           \
-                            (int)smem_bytes<E, true>()) == cudaSuccess;
+#define MRF_GEMM_ATTR(E)                                                                      \
+  ok = ok && set_smem_attr<E, false, false>() && set_smem_attr<E, true, false>();             \
+  if (pair_kind(E)) ok = ok && set_smem_attr<E, false, pair_kind(E)>() && set_smem_attr<E, true, pair_kind(E)>();
   MRF_GEMM_ATTR(kTcQkv)
   MRF_GEMM_ATTR(kTcResid)
   MRF_GEMM_ATTR(kTcGelu)
@@ -737,15 +816,20 @@ bool gemm_tc_init() {
   return ok;
 }
 
-void launch_gemm_tc(int epi, bool bf16, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
-                    const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st) {
+bool gemm_tc_pair_kind(int epi) { return pair_kind(epi); }
+
+void launch_gemm_tc(int epi, bool bf16, bool pair, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                    const CUtensorMap &tmC, const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st) {
   switch (epi) {
-#define MRF_GEMM_CASE(E)                                                                                      \
-  case E:                                                                                                     \
-    if (bf16)                                                                                                 \
-      gemm_tc_kernel<E, true><<<grid, gemm_threads(E), smem_bytes<E, true>(), st>>>(tmA, tmB, tmC, tmD, p);   \
-    else                                                                                                      \
-      gemm_tc_kernel<E, false><<<grid, gemm_threads(E), smem_bytes<E, false>(), st>>>(tmA, tmB, tmC, tmD, p); \
+#define MRF_GEMM_CASE(E)                                                                          \
+  case E:                                                                                         \
+    if (pair && pair_kind(E)) {                                                                   \
+      if (bf16) launch_one<E, true, pair_kind(E)>(tmA, tmB, tmC, tmD, p, grid, st);               \
+      else launch_one<E, false, pair_kind(E)>(tmA, tmB, tmC, tmD, p, grid, st);                   \
+    } else {                                                                                      \
+      if (bf16) launch_one<E, true, false>(tmA, tmB, tmC, tmD, p, grid, st);                      \
+      else launch_one<E, false, false>(tmA, tmB, tmC, tmD, p, grid, st);                          \
+    }                                                                                             \
     break;
     MRF_GEMM_CASE(kTcQkv)
     MRF_GEMM_CASE(kTcResid)
