@@ -59,7 +59,15 @@ __host__ __device__ constexpr int warp_stage_bytes(int epi, bool bf) {
   return (bf && (epi == kTcResid || epi == kTcBandSplit)) ? 4096 + 2048 : 2 * 2048;
 }
 
+// The grouped epilogue kinds (one group per band; at most kMaxGroups groups) and the trunk's
+// single-group kinds.
+constexpr int kMaxGroups = 128;
+__host__ __device__ constexpr bool grouped_kind(int epi) {
+  return epi == kTcTanh || epi == kTcGlu || epi == kTcBandSplit;
+}
+
 // kPair: a CTA of a pair holds half of the B tile's rows per stage (and has room for more stages).
+// Grouped kinds end with the groups' (first tile, column blocks) table.
 template <int EPI, bool kBF, bool kPair = false>
 struct SmemLayout {
   static constexpr int stages = gemm_stages(EPI, kPair);
@@ -68,7 +76,8 @@ struct SmemLayout {
   static constexpr int b_off = stages * A_STAGE;
   static constexpr int stg_off = b_off + stages * b_stage;        // 1024-aligned
   static constexpr int bar_off = stg_off + epi_warps(EPI) * warp_stage_bytes(EPI, kBF);
-  static constexpr int total = bar_off + 256;
+  static constexpr int gtab_off = bar_off + 256;
+  static constexpr int total = gtab_off + (grouped_kind(EPI) ? kMaxGroups * 8 : 0);
 };
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
@@ -86,28 +95,40 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   }
 }
 
-__device__ __forceinline__ int find_group(const GemmGroup *g, int n, int tile, int m_tiles) {
-  int lo = 0, hi = n - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (g[mid].n_tile_start * m_tiles <= tile) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
-struct TileInfo {
+// A tile's group g, its row block mb and column block nblk (tiles run group by group, and
+// within a group row block by row block), and the group's record.  Nothing here waits on
+// memory: the trunk GEMMs have one group, read into registers once per CTA; the grouped GEMMs
+// (mask head, band split: one group per band) search a shared-memory table of the groups'
+// (first tile, column blocks) and load the group's record from global memory, a load the
+// callers issue one tile before they use it.
+struct TileDec {
   int g, mb, nblk;
+  GemmGroup gr;
 };
 
-__device__ __forceinline__ TileInfo decode_tile(const GemmParams &p, int tile) {
-  TileInfo ti;
-  ti.g = p.ngroups == 1 ? 0 : find_group(p.groups, p.ngroups, tile, p.m_tiles);
-  const GemmGroup &gr = p.groups[ti.g];
-  const int r = tile - gr.n_tile_start * p.m_tiles;
-  ti.mb = r / gr.n_tiles;
-  ti.nblk = r % gr.n_tiles;
-  return ti;
+template <bool kGrouped>
+__device__ __forceinline__ TileDec tile_dec(const GemmParams &p, const GemmGroup &g0, const int2 *gtab, int tile) {
+  TileDec d;
+  if constexpr (!kGrouped) {
+    d.g = 0;
+    d.gr = g0;
+    d.mb = tile / g0.n_tiles;
+    d.nblk = tile - d.mb * g0.n_tiles;
+  } else {
+    int lo = 0, hi = p.ngroups - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (gtab[mid].x * p.m_tiles <= tile) lo = mid;
+      else hi = mid - 1;
+    }
+    const int2 e = gtab[lo];
+    const int r = tile - e.x * p.m_tiles;
+    d.g = lo;
+    d.mb = r / e.y;
+    d.nblk = r - d.mb * e.y;
+    d.gr = p.groups[lo];
+  }
+  return d;
 }
 
 // ------------------------------------------------------------------ epilogue helpers
@@ -245,6 +266,8 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   uint64_t *tempty = tfull + 2;                // [2]
   uint64_t *done = tempty + 2;                 // [1]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  int2 *gtab = reinterpret_cast<int2 *>(smem + L::gtab_off);
+  constexpr bool kGrouped = grouped_kind(EPI);
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -261,6 +284,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     tc::mbar_init(done, 1);
     tc::fence_barrier_init();
   }
+  if (kGrouped)
+    for (int i = threadIdx.x; i < p.ngroups; i += blockDim.x)
+      gtab[i] = make_int2(p.groups[i].n_tile_start, p.groups[i].n_tiles);
   if (warp == kEpiWarps) {
     if (lane == 0) { tc::tma_prefetch(&tmA); tc::tma_prefetch(&tmB); }
     __syncwarp();
@@ -274,6 +300,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   const uint32_t tmem_base = *tmem_slot;
   volatile int *abort = &abort_flag;
   const int total = p.m_tiles * p.total_n_tiles;
+  GemmGroup g0{};  // the single group of a trunk GEMM
+  if (!kGrouped) g0 = p.groups[0];
+  auto dec = [&](int tile_) { return tile_dec<kGrouped>(p, g0, gtab, tile_ < total ? tile_ : total - 1); };
 
   if (warp == kEpiWarps) {
     // ---------------- TMA producer
@@ -284,9 +313,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       uint32_t phase = 0;
       // bytes completing on this CTA's full barrier (pair: both CTAs' loads on the leader's)
       const uint32_t bytes = kPair ? 2 * (A_STAGE + (p.BN / 2) * BK * 2) : A_STAGE + p.BN * BK * 2;
+      TileDec nx = dec(first_tile);
       for (int tile = first_tile; tile < total; tile += tile_step) {
-        const TileInfo ti = decode_tile(p, tile);
-        const GemmGroup &gr = p.groups[ti.g];
+        const TileDec ti = nx;
+        nx = dec(tile + tile_step);
+        const GemmGroup &gr = ti.gr;
         const int m0 = ti.mb * kTileM + (int)rank * BM;
         int n0 = gr.b_row_off + ti.nblk * p.BN;
         if (kPair) {  // this CTA's half of the tile's MMA width
@@ -320,9 +351,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
+      TileDec nx = dec(first_tile);
       for (int tile = first_tile; tile < total; tile += tile_step, ++local) {
-        const TileInfo ti = decode_tile(p, tile);
-        const GemmGroup &gr = p.groups[ti.g];
+        const TileDec ti = nx;
+        nx = dec(tile + tile_step);
+        const GemmGroup &gr = ti.gr;
         const int acc = local & 1;
         const uint32_t aphase = (local >> 1) & 1;
         int n_eff = min(p.BN, gr.N - ti.nblk * p.BN);
@@ -372,9 +405,8 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     row_ss_one(ss_pf);
     QkvRow qr_pf{0, 0};
     float2 cs_pf[16];
-    auto row_fetch = [&](int tile_) {
+    auto row_fetch = [&](int tile_, const TileDec &t_) {
       if (tile_ >= total) return;
-      const TileInfo t_ = decode_tile(p, tile_);
       const int m_ = t_.mb * kTileM + (int)rank * BM + quarter * 32 + lane;
       const bool v_ = m_ < p.M;
       if (EPI == kTcQkv) {
@@ -403,10 +435,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         else row_ss_one(ss_pf);
       }
     };
-    row_fetch(first_tile);
+    TileDec nx = dec(first_tile);
+    row_fetch(first_tile, nx);
     for (int tile = first_tile; tile < total; tile += tile_step, ++local) {
-      const TileInfo ti = decode_tile(p, tile);
-      const GemmGroup &gr = p.groups[ti.g];
+      const TileDec ti = nx;
+      const GemmGroup &gr = ti.gr;
       const int acc = local & 1;
       const uint32_t aphase = (local >> 1) & 1;
       const int m0w = ti.mb * kTileM + (int)rank * BM + quarter * 32;  // first row of this warp's 32
@@ -429,7 +462,22 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       }
       if (EPI == kTcQkv || EPI == kTcGelu || EPI == kTcGeglu || EPI == kTcTanh) rs = rsq;
       const float res_s = rsq;  // kTcResid
-      row_fetch(tile + tile_step);
+      // QKV: which of q (0), k (1), v or the gates (2) the tile's columns belong to, when all
+      // of them belong to one; then the row's scale (1 / |x|, times the softmax scale for q) is
+      // folded into the rotary (cos, sin) pairs once per tile
+      int tile_which = -1;
+      if (EPI == kTcQkv) {
+        const int last = nbase + n_eff - 1;
+        const int w0 = nbase < p.A ? 0 : (nbase < 2 * p.A ? 1 : 2), w1 = last < p.A ? 0 : (last < 2 * p.A ? 1 : 2);
+        if (w0 == w1 && w0 < 2 && p.dh == 64) {
+          tile_which = w0;
+          const float k = w0 == 0 ? rs * p.q_scale : rs;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) cs[i] = make_float2(cs[i].x * k, cs[i].y * k);
+        }
+      }
+      nx = dec(tile + tile_step);
+      row_fetch(tile + tile_step, nx);
       // residual prefetch (kTcResid): fp16 rows of 64 bytes, lane covering rows i*8 + lane/4 and
       // 16-byte piece lane%4; with kBF the fp32 master rows of 128 bytes, rows i*4 + lane/8, piece lane%8
       constexpr int kPieces = kBF ? 8 : 4;
@@ -549,18 +597,24 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
               const int h = c0 + j - A3;
               v[j] = h < p.H ? sigmoidf_(v[j] * rs + p.gbias[h]) : 0.f;
             }
-          } else {
+          } else if (tile_which >= 0) {
+            // q or k with the row scale in the (cos, sin) pairs: (x0 c - x1 s, x1 c + x0 s)
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= rs;
-            const int which = c0 / p.A;
+            for (int i = 0; i < 16; ++i) {
+              const float x0 = v[2 * i], x1 = v[2 * i + 1];
+              v[2 * i] = fmaf(x0, cs[i].x, -x1 * cs[i].y);
+              v[2 * i + 1] = fmaf(x1, cs[i].x, x0 * cs[i].y);
+            }
+          } else {
+            const int which = c0 < p.A ? 0 : (c0 < 2 * p.A ? 1 : 2);
+            const float k = which == 0 ? rs * p.q_scale : rs;
             if (which < 2) {
-              const float sc = which == 0 ? p.q_scale : 1.f;
               if (p.dh == 64) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                  const float x0 = v[2 * i], x1 = v[2 * i + 1];
-                  v[2 * i] = (x0 * cs[i].x - x1 * cs[i].y) * sc;
-                  v[2 * i + 1] = (x1 * cs[i].x + x0 * cs[i].y) * sc;
+                  const float c = cs[i].x * k, sn = cs[i].y * k, x0 = v[2 * i], x1 = v[2 * i + 1];
+                  v[2 * i] = fmaf(x0, c, -x1 * sn);
+                  v[2 * i + 1] = fmaf(x1, c, x0 * sn);
                 }
               } else {
                 const int half_dh = p.dh >> 1;
@@ -568,11 +622,14 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
                 for (int i = 0; i < 16; ++i) {
                   const int dd = (c0 - which * p.A + 2 * i) % p.dh;
                   const float2 cc = p.rope[(long long)qr.pos * half_dh + (dd >> 1)];
-                  const float x0 = v[2 * i], x1 = v[2 * i + 1];
-                  v[2 * i] = (x0 * cc.x - x1 * cc.y) * sc;
-                  v[2 * i + 1] = (x1 * cc.x + x0 * cc.y) * sc;
+                  const float c = cc.x * k, sn = cc.y * k, x0 = v[2 * i], x1 = v[2 * i + 1];
+                  v[2 * i] = fmaf(x0, c, -x1 * sn);
+                  v[2 * i + 1] = fmaf(x1, c, x0 * sn);
                 }
               }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] *= k;
             }
           }
           uint8_t *box = stg + (nstore & 1) * 2048;

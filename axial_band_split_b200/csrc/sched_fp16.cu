@@ -72,9 +72,9 @@ struct Fp16State {
   // adds of twelve transformers to bf16's 8-bit significand would cost too much precision)
   bool bf16 = false;
   float *X = nullptr;
-  // the trunk GEMMs as CTA pairs (cta_group::2); MRF_GEMM_PAIR=0 in the environment at create
-  // selects one CTA per tile
-  bool pair = true;
+  // which trunk GEMMs run as CTA pairs (cta_group::2), from MRF_GEMM_PAIR in the environment at
+  // create: 0 none, 1 those with K >= kPairMinK (the default), 2 all four
+  int pair = 1;
 };
 
 namespace {
@@ -139,7 +139,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   cudaDeviceGetAttribute(&f->sms, cudaDevAttrMultiProcessorCount, h->device);
   f->tc_attention = attention_tc_supported(dh, head_v(c));
   f->bf16 = c.compute == MRF_BF16;
-  if (const char *e = getenv("MRF_GEMM_PAIR")) f->pair = atoi(e) != 0;
+  if (const char *e = getenv("MRF_GEMM_PAIR")) f->pair = std::min(std::max(atoi(e), 0), 2);
   if (!gemm_tc_init() || (f->tc_attention && !attention_tc_init())) {
     h->err = "tcgen05 kernel initialisation failed (tensor-map encoder or shared-memory limit)";
     return MRF_ECUDA;
@@ -352,14 +352,21 @@ GemmParams base_params(mrf_handle *h, int M, int K, int BN, const GemmGroup *gro
   return p;
 }
 
-// The trunk's GEMMs run as CTA pairs (M = 256 tiles, B maps with half-height boxes); the
-// grouped ones one CTA per M = 128 tile.
-bool use_pair(const mrf_handle *h, int epi) { return h->f16->pair && gemm_tc_pair_kind(epi); }
+// A trunk GEMM may run as CTA pairs (M = 256 tiles, B maps with half-height boxes): each CTA
+// then stages half of every B tile, which halves the shared-memory traffic of the main loop.
+// That pays where the main loop is long (FF2, K = 4 D) and costs where the epilogue dominates
+// (the QKV, out-projection and FF1 GEMMs, K <= 512, run about 10 % slower as pairs on B200), so
+// by default only GEMMs with K >= kPairMinK pair.  The grouped GEMMs run one CTA per M = 128 tile.
+constexpr int kPairMinK = 1024;
+bool use_pair(const mrf_handle *h, int epi, int K) {
+  const int mode = h->f16->pair;
+  return gemm_tc_pair_kind(epi) && (mode == 2 || (mode == 1 && K >= kPairMinK));
+}
 
 void gemm(mrf_handle *h, const char *name, int epi, const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p0,
           const CUtensorMap *c = nullptr, const CUtensorMap *d = nullptr) {
   GemmParams p = p0;
-  const bool pair = use_pair(h, epi);
+  const bool pair = use_pair(h, epi, p.K);
   if (pair) p.m_tiles = cdiv(p.M, 256);
   const int tiles = p.m_tiles * p.total_n_tiles;
   const int grid = pair ? 2 * std::min(tiles, h->f16->sms / 2) : std::min(tiles, h->f16->sms);
@@ -405,12 +412,14 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   for (int i = 0; ok && i < 2 * c.depth; ++i) {
     const TrF16 &w = f->tr[i];
     // weight boxes: BN rows, or BN / 2 for the CTA pairs (each CTA loads half of a B tile)
-    const unsigned bw = use_pair(h, kTcQkv) ? kBnWide / 2 : kBnWide, bn = use_pair(h, kTcResid) ? kBnNarrow / 2 : kBnNarrow;
-    const unsigned bw1 = use_pair(h, kTcGelu) ? kBnWide / 2 : kBnWide;
-    ok = make_tmap_f16(&wmaps[4 * i + 0], w.wqkvg, D, QKVW + H, 1, D, ((long long)QKVW + H) * D, bw, 1) &&
-         make_tmap_f16(&wmaps[4 * i + 1], w.wo, A, D, 1, A, (long long)D * A, bn, 1) &&
-         make_tmap_f16(&wmaps[4 * i + 2], w.w1, D, F1, 1, D, (long long)F1 * D, bw1, 1) &&
-         make_tmap_f16(&wmaps[4 * i + 3], w.w2, FF, D, 1, FF, (long long)D * FF, bn, 1);
+    const unsigned bq = use_pair(h, kTcQkv, D) ? kBnWide / 2 : kBnWide;
+    const unsigned bo = use_pair(h, kTcResid, A) ? kBnNarrow / 2 : kBnNarrow;
+    const unsigned b1 = use_pair(h, kTcGelu, D) ? kBnWide / 2 : kBnWide;
+    const unsigned b2 = use_pair(h, kTcResid, FF) ? kBnNarrow / 2 : kBnNarrow;
+    ok = make_tmap_f16(&wmaps[4 * i + 0], w.wqkvg, D, QKVW + H, 1, D, ((long long)QKVW + H) * D, bq, 1) &&
+         make_tmap_f16(&wmaps[4 * i + 1], w.wo, A, D, 1, A, (long long)D * A, bo, 1) &&
+         make_tmap_f16(&wmaps[4 * i + 2], w.w1, D, F1, 1, D, (long long)F1 * D, b1, 1) &&
+         make_tmap_f16(&wmaps[4 * i + 3], w.w2, FF, D, 1, FF, (long long)D * FF, b2, 1);
   }
   const int wm0 = 8 * c.depth;
   const long long rows_last = 2LL * h->tab.n_feat();
