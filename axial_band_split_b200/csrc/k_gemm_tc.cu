@@ -66,21 +66,32 @@ __host__ __device__ constexpr bool grouped_kind(int epi) {
   return epi == kTcTanh || epi == kTcGlu || epi == kTcBandSplit;
 }
 
+// The residual kinds' per-column vectors (bias, the gain of the deferred norm applied to the
+// residual, the gain of the output norm), copied to shared memory once per CTA: the epilogue
+// streams the residual through L1, which would evict them from it.  Columns up to kMaxDim.
+constexpr int kMaxDim = 1024;
+__host__ __device__ constexpr int vec_bytes(int epi) { return epi == kTcResid ? 3 * kMaxDim * 4 : 0; }
+constexpr int kSmemLimit = 232448;  // 227 KB per CTA
+
 // kPair: a CTA of a pair holds half of the B tile's rows per stage (and has room for more stages).
-// Grouped kinds end with the groups' (first tile, column blocks) table.
+// Grouped kinds end with the groups' (first tile, column blocks) table, residual kinds with the
+// column vectors.  A configuration whose stages would not fit the limit drops one stage.
 template <int EPI, bool kBF, bool kPair = false>
 struct SmemLayout {
-  static constexpr int stages = gemm_stages(EPI, kPair);
   static constexpr int b_stage = (kPair ? bn_max(EPI) / 2 : bn_max(EPI)) * BK * 2;
+  static constexpr int fixed = epi_warps(EPI) * warp_stage_bytes(EPI, kBF) + 256 +
+                               (grouped_kind(EPI) ? kMaxGroups * 8 : 0) + vec_bytes(EPI) + 1024;
+  static constexpr int stages = gemm_stages(EPI, kPair) * (A_STAGE + b_stage) + fixed <= kSmemLimit
+                                    ? gemm_stages(EPI, kPair) : gemm_stages(EPI, kPair) - 1;
   static constexpr int a_off = 0;
   static constexpr int b_off = stages * A_STAGE;
   static constexpr int stg_off = b_off + stages * b_stage;        // 1024-aligned
   static constexpr int bar_off = stg_off + epi_warps(EPI) * warp_stage_bytes(EPI, kBF);
   static constexpr int gtab_off = bar_off + 256;
-  static constexpr int total = gtab_off + (grouped_kind(EPI) ? kMaxGroups * 8 : 0);
+  static constexpr int vec_off = gtab_off + (grouped_kind(EPI) ? kMaxGroups * 8 : 0);
+  static constexpr int total = vec_off + vec_bytes(EPI);
 };
 
-__device__ __forceinline__ float sigmoidf_(float x) { return 1.f / (1.f + __expf(-x)); }
 
 // Two floats as one 32-bit pair of the schedule's 16-bit type (fp16, or bf16 with kBF), rounded
 // to nearest even.
@@ -287,6 +298,14 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   if (kGrouped)
     for (int i = threadIdx.x; i < p.ngroups; i += blockDim.x)
       gtab[i] = make_int2(p.groups[i].n_tile_start, p.groups[i].n_tiles);
+  // [bias | res_gain | out_gain] of a residual GEMM (its N, the model dim, is at most kMaxDim)
+  float *svec = reinterpret_cast<float *>(smem + L::vec_off);
+  if (EPI == kTcResid)
+    for (int i = threadIdx.x; i < min(p.groups[0].N, kMaxDim); i += blockDim.x) {
+      if (p.bias) svec[i] = p.bias[i];
+      if (p.res_gain) svec[kMaxDim + i] = p.res_gain[i];
+      if (p.out_gain) svec[2 * kMaxDim + i] = p.out_gain[i];
+    }
   if (warp == kEpiWarps) {
     if (lane == 0) { tc::tma_prefetch(&tmA); tc::tma_prefetch(&tmB); }
     __syncwarp();
@@ -502,7 +521,6 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       float sq = 0.f, sqg = 0.f;
       for (; c < nchunks; c += kSplit) {
         const int c0 = nbase + 32 * c;
-        const bool full_chunk = c0 + 32 <= gr.N;
         float v[32];
         if (EPI == kTcResid || EPI == kTcBandSplit) {
           // x (+ bias) + acc with its row statistics in fp32.  fp16: the residual stream is the
@@ -537,14 +555,14 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
             }
             if (p.res_ss) {
               float gv[32];
-              load_bias32(p.res_gain + c0, gv);
+              load_bias32(svec + kMaxDim + c0, gv);
 #pragma unroll
               for (int j = 0; j < 32; ++j) x[j] *= res_s * gv[j];
             }
             if (c + kSplit < nchunks) residual_fetch(c0 + 32 * kSplit);
             if (p.bias) {
               float bv[32];
-              load_bias32(p.bias + c0, bv);
+              load_bias32(svec + c0, bv);
 #pragma unroll
               for (int j = 0; j < 32; ++j) x[j] += bv[j];
             }
@@ -560,7 +578,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           }
           if (EPI == kTcResid && p.ssg_out) {
             float gv[32];
-            load_bias32(p.out_gain + c0, gv);
+            load_bias32(svec + 2 * kMaxDim + c0, gv);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const float y = gv[j] * x[j];
@@ -595,7 +613,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int h = c0 + j - A3;
-              v[j] = h < p.H ? sigmoidf_(v[j] * rs + p.gbias[h]) : 0.f;
+              v[j] = h < p.H ? tcm::sigmoid_mufu(v[j] * rs + p.gbias[h]) : 0.f;
             }
           } else if (tile_which >= 0) {
             // q or k with the row scale in the (cos, sin) pairs: (x0 c - x1 s, x1 c + x0 s)
@@ -661,7 +679,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = tanhf(fmaf(v[j], rs, bv[j]));
+            for (int j = 0; j < 32; ++j) v[j] = tcm::tanh_mufu(fmaf(v[j], rs, bv[j]));
           }
           uint4 d[4];
           pack16<kBF>(v, d);
@@ -717,7 +735,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
             const bool ok = (j >> 1) < nf;
             const float val = v[j] + (ok ? bias[j] : 0.f);
             const float gt = v[j + 1] + (ok ? bias[j + 1] : 0.f);
-            o[j >> 1] = val * sigmoidf_(gt);
+            o[j >> 1] = val * tcm::sigmoid_mufu(gt);
           }
           if (valid) {
             const int fe0 = gr.out_off + (c0 >> 1);
@@ -783,7 +801,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int EPI, bool kBF, bool kPair = false>
 constexpr size_t smem_bytes() { return SmemLayout<EPI, kBF, kPair>::total + 1024; }
-constexpr size_t kSmemLimit = 232448;  // 227 KB per CTA
 // The epilogue kinds that run as CTA pairs (the trunk's four GEMMs); the grouped mask-head and
 // band-split GEMMs run one CTA per tile.
 __host__ __device__ constexpr bool pair_kind(int epi) {
