@@ -498,24 +498,27 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       nx = dec(tile + tile_step);
       row_fetch(tile + tile_step, nx);
       // residual prefetch (kTcResid): fp16 rows of 64 bytes, lane covering rows i*8 + lane/4 and
-      // 16-byte piece lane%4; with kBF the fp32 master rows of 128 bytes, rows i*4 + lane/8, piece lane%8
+      // 16-byte piece lane%4; with kBF the fp32 master rows of 128 bytes, rows i*4 + lane/8, piece lane%8.
+      // fp16 fetches two chunks ahead (pre: this warp's next chunk, pre2: the one after), which
+      // hides a DRAM round trip; the bf16 pieces are twice as many and fetch one chunk ahead.
       constexpr int kPieces = kBF ? 8 : 4;
-      uint4 pre[kPieces];
+      uint4 pre[kPieces], pre2[kPieces];
       int c = sub;
-      auto residual_fetch = [&](int col) {
+      auto residual_fetch = [&](int col, uint4 (&dst)[kPieces]) {
 #pragma unroll
         for (int i = 0; i < kPieces; ++i) {
           const int r = kBF ? i * 4 + (lane >> 3) : i * 8 + (lane >> 2);
           const bool ok = m0w + r < p.M;
           if constexpr (kBF)
-            pre[i] = ok ? *reinterpret_cast<const uint4 *>(p.X + (long long)(m0w + r) * p.ld + col + (lane & 7) * 4)
+            dst[i] = ok ? *reinterpret_cast<const uint4 *>(p.X + (long long)(m0w + r) * p.ld + col + (lane & 7) * 4)
                         : make_uint4(0, 0, 0, 0);
           else
-            pre[i] = ok ? *reinterpret_cast<const uint4 *>(p.Xh + (long long)(m0w + r) * p.ld + col + (lane & 3) * 8)
+            dst[i] = ok ? *reinterpret_cast<const uint4 *>(p.Xh + (long long)(m0w + r) * p.ld + col + (lane & 3) * 8)
                         : make_uint4(0, 0, 0, 0);
         }
       };
-      if (EPI == kTcResid && c < nchunks) residual_fetch(nbase + 32 * c);
+      if (EPI == kTcResid && c < nchunks) residual_fetch(nbase + 32 * c, pre);
+      if (EPI == kTcResid && !kBF && c + kSplit < nchunks) residual_fetch(nbase + 32 * (c + kSplit), pre2);
       if (!tc::mbar_wait(tfull + acc, aphase, p.status, 14, abort)) break;
       tc::tc_fence_after();
       float sq = 0.f, sqg = 0.f;
@@ -559,7 +562,13 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
 #pragma unroll
               for (int j = 0; j < 32; ++j) x[j] *= res_s * gv[j];
             }
-            if (c + kSplit < nchunks) residual_fetch(c0 + 32 * kSplit);
+            if constexpr (kBF) {
+              if (c + kSplit < nchunks) residual_fetch(c0 + 32 * kSplit, pre);
+            } else {
+#pragma unroll
+              for (int i = 0; i < kPieces; ++i) pre[i] = pre2[i];
+              if (c + 2 * kSplit < nchunks) residual_fetch(c0 + 64 * kSplit, pre2);
+            }
             if (p.bias) {
               float bv[32];
               load_bias32(svec + c0, bv);
