@@ -103,7 +103,8 @@ bool gemm_tc_init();
 // CTAs, each cluster an M = 256 tile (p.m_tiles counted in 256-row tiles), grid even, and tmB's box
 // BN / 2 rows; otherwise one CTA per M = 128 tile with tmB's box BN rows.
 void launch_gemm_tc(int epi, bool bf16, bool pair, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                    const CUtensorMap &tmC, const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st);
+                    const CUtensorMap &tmC, const CUtensorMap &tmD, const GemmParams &p, int grid, bool pdl,
+                    cudaStream_t st);
 bool gemm_tc_pair_kind(int epi);
 
 }  // namespace mrf

@@ -414,6 +414,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int *abort = &abort_flag;
+  // the prologue overlaps the previous kernel's tail; q, k, v and the gates are its output
+  tc::griddep_wait();
+  tc::griddep_launch_dependents();
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsIo));
   if (warp == 8) {
@@ -669,7 +672,7 @@ bool attention_tc_init() {
   return attn_prepare<false, 1>() && attn_prepare<true, 1>() && attn_prepare<false, 2>() && attn_prepare<true, 2>();
 }
 
-bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int dqk, int axis,
+bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int dqk, int axis, bool pdl,
                          bool bf16, unsigned *status, cudaStream_t st) {
   AttnArgs a;
   a.qkv = qkv;
@@ -722,7 +725,20 @@ bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int
       !make_tmap(&to, o, kTmF16, 5, odims, ostr, obox, 128))
     return false;
   const int grid = (int)std::min<long long>(a.items, g_num_sms > 0 ? g_num_sms : 148);
-#define MRF_ATTN(BF, QA) attn_tc_kernel<BF, QA><<<grid, kThreads, AttnSmem<QA>::total + 1024, st>>>(tq, tk, tv, to, a)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+#define MRF_ATTN(BF, QA)                                       \
+  do {                                                         \
+    cfg.dynamicSmemBytes = AttnSmem<QA>::total + 1024;         \
+    cudaLaunchKernelEx(&cfg, attn_tc_kernel<BF, QA>, tq, tk, tv, to, a); \
+  } while (0)
   if (dqk == 128) {
     if (bf16) MRF_ATTN(true, 2);
     else MRF_ATTN(false, 2);

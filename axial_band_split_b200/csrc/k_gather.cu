@@ -74,6 +74,9 @@ __global__ void __launch_bounds__(kThreads) band_gather_kernel(const float *__re
                                                                    long long frame_stride, int k_stride,
                                                                    __half *__restrict__ A) {
   __shared__ float ss[2][kFrames];
+  // programmatic dependent launch: the input may be an earlier kernel's output
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int per_band = B * tiles;
   const int k = nb - 1 - (int)(blockIdx.x / per_band);   // widest bands first
   const int rem = (int)(blockIdx.x % per_band);
@@ -120,11 +123,20 @@ __global__ void __launch_bounds__(kThreads) band_gather_kernel(const float *__re
 }  // namespace
 
 void launch_band_gather(const float *in, const int32_t *feat_row, const BandDesc *bands, int nb, int B, int T,
-                        int rows, long long frame_stride, int k_stride, __half *A, bool bf16, cudaStream_t st) {
+                        int rows, long long frame_stride, int k_stride, __half *A, bool bf16, bool pdl,
+                        cudaStream_t st) {
   const int tiles = (T + kFrames - 1) / kFrames;
-  const unsigned grid = (unsigned)(nb * B * tiles);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nb * B * tiles), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
 #define MRF_GATHER(E, BF) \
-  band_gather_kernel<E, BF><<<grid, kThreads, 0, st>>>(in, feat_row, bands, nb, B, T, rows, tiles, frame_stride, k_stride, A)
+  cudaLaunchKernelEx(&cfg, band_gather_kernel<E, BF>, in, feat_row, bands, nb, B, T, rows, tiles, frame_stride, k_stride, A)
   if (T % 2 == 0) {
     if (bf16) MRF_GATHER(true, true);
     else MRF_GATHER(true, false);

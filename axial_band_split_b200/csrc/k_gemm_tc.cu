@@ -319,6 +319,10 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   const uint32_t tmem_base = *tmem_slot;
   volatile int *abort = &abort_flag;
   const int total = p.m_tiles * p.total_n_tiles;
+  // the prologue above (barriers, TMEM, group table, column vectors: none of it produced by an
+  // earlier kernel) overlaps the previous kernel's last tiles; its outputs are read from here on
+  tc::griddep_wait();
+  tc::griddep_launch_dependents();
   GemmGroup g0{};  // the single group of a trunk GEMM
   if (!kGrouped) g0 = p.groups[0];
   auto dec = [&](int tile_) { return tile_dec<kGrouped>(p, g0, gtab, tile_ < total ? tile_ : total - 1); };
@@ -830,27 +834,33 @@ bool set_smem_attr() {
                               (int)smem_bytes<EPI, kBF, kPair>()) == cudaSuccess;
 }
 
+// pdl: launched with programmatic stream serialisation (the kernel waits for its inputs in
+// griddep_wait after its prologue).
 template <int EPI, bool kBF, bool kPair>
 void launch_one(const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC, const CUtensorMap &tmD,
-                const GemmParams &p, int grid, cudaStream_t st) {
-  if constexpr (kPair) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(gemm_threads(EPI), 1, 1);
-    cfg.dynamicSmemBytes = smem_bytes<EPI, kBF, true>();
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI, kBF, true>, tmA, tmB, tmC, tmD, p);
-  } else {
-    gemm_tc_kernel<EPI, kBF, false><<<grid, gemm_threads(EPI), smem_bytes<EPI, kBF, false>(), st>>>(tmA, tmB, tmC,
-                                                                                                    tmD, p);
+                const GemmParams &p, int grid, bool pdl, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(gemm_threads(EPI), 1, 1);
+  cfg.dynamicSmemBytes = smem_bytes<EPI, kBF, kPair>();
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (kPair) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 2;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
   }
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI, kBF, kPair>, tmA, tmB, tmC, tmD, p);
 }
 
 }  // namespace
@@ -902,16 +912,17 @@ bool gemm_tc_init() {
 bool gemm_tc_pair_kind(int epi) { return pair_kind(epi); }
 
 void launch_gemm_tc(int epi, bool bf16, bool pair, const CUtensorMap &tmA, const CUtensorMap &tmB,
-                    const CUtensorMap &tmC, const CUtensorMap &tmD, const GemmParams &p, int grid, cudaStream_t st) {
+                    const CUtensorMap &tmC, const CUtensorMap &tmD, const GemmParams &p, int grid, bool pdl,
+                    cudaStream_t st) {
   switch (epi) {
 #define MRF_GEMM_CASE(E)                                                                          \
   case E:                                                                                         \
     if (pair && pair_kind(E)) {                                                                   \
-      if (bf16) launch_one<E, true, pair_kind(E)>(tmA, tmB, tmC, tmD, p, grid, st);               \
-      else launch_one<E, false, pair_kind(E)>(tmA, tmB, tmC, tmD, p, grid, st);                   \
+      if (bf16) launch_one<E, true, pair_kind(E)>(tmA, tmB, tmC, tmD, p, grid, pdl, st);               \
+      else launch_one<E, false, pair_kind(E)>(tmA, tmB, tmC, tmD, p, grid, pdl, st);                   \
     } else {                                                                                      \
-      if (bf16) launch_one<E, true, false>(tmA, tmB, tmC, tmD, p, grid, st);                      \
-      else launch_one<E, false, false>(tmA, tmB, tmC, tmD, p, grid, st);                          \
+      if (bf16) launch_one<E, true, false>(tmA, tmB, tmC, tmD, p, grid, pdl, st);                      \
+      else launch_one<E, false, false>(tmA, tmB, tmC, tmD, p, grid, pdl, st);                          \
     }                                                                                             \
     break;
     MRF_GEMM_CASE(kTcQkv)

@@ -32,7 +32,7 @@
 namespace mrf {
 
 bool launch_attention_tc(const __half *qkv, int ld, __half *o, int B, int T, int nb, int H, int dqk, int axis,
-                         bool bf16, unsigned *status, cudaStream_t st);
+                         bool pdl, bool bf16, unsigned *status, cudaStream_t st);
 bool attention_tc_supported(int dqk, int dv);
 bool attention_tc_init();
 
@@ -75,6 +75,10 @@ struct Fp16State {
   // which trunk GEMMs run as CTA pairs (cta_group::2), from MRF_GEMM_PAIR in the environment at
   // create: 0 none, 1 those with K >= kPairMinK (the default), 2 all four
   int pair = 1;
+  // the tensor-core kernels launched with programmatic stream serialisation (each waits for its
+  // inputs after its prologue, which then overlaps the previous kernel's tail); MRF_PDL=0 in the
+  // environment at create turns it off
+  bool pdl = true;
 };
 
 namespace {
@@ -140,6 +144,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->tc_attention = attention_tc_supported(dh, head_v(c));
   f->bf16 = c.compute == MRF_BF16;
   if (const char *e = getenv("MRF_GEMM_PAIR")) f->pair = std::min(std::max(atoi(e), 0), 2);
+  if (const char *e = getenv("MRF_PDL")) f->pdl = atoi(e) != 0;
   if (!gemm_tc_init() || (f->tc_attention && !attention_tc_init())) {
     h->err = "tcgen05 kernel initialisation failed (tensor-map encoder or shared-memory limit)";
     return MRF_ECUDA;
@@ -358,6 +363,10 @@ GemmParams base_params(mrf_handle *h, int M, int K, int BN, const GemmGroup *gro
 // (the QKV, out-projection and FF1 GEMMs, K <= 512, run about 10 % slower as pairs on B200), so
 // by default only GEMMs with K >= kPairMinK pair.  The grouped GEMMs run one CTA per M = 128 tile.
 constexpr int kPairMinK = 1024;
+// Per-kernel timing records an event pair around each launch, which a kernel started ahead of
+// its predecessor's end would blur: timing runs launch without the programmatic attribute.
+bool use_pdl(const mrf_handle *h) { return h->f16->pdl && !h->timing; }
+
 bool use_pair(const mrf_handle *h, int epi, int K) {
   const int mode = h->f16->pair;
   return gemm_tc_pair_kind(epi) && (mode == 2 || (mode == 1 && K >= kPairMinK));
@@ -371,7 +380,7 @@ void gemm(mrf_handle *h, const char *name, int epi, const CUtensorMap &a, const 
   const int tiles = p.m_tiles * p.total_n_tiles;
   const int grid = pair ? 2 * std::min(tiles, h->f16->sms / 2) : std::min(tiles, h->f16->sms);
   h->begin(name);
-  launch_gemm_tc(epi, h->f16->bf16, pair, a, b, c ? *c : a, d ? *d : a, p, grid, h->cur_stream);
+  launch_gemm_tc(epi, h->f16->bf16, pair, a, b, c ? *c : a, d ? *d : a, p, grid, use_pdl(h), h->cur_stream);
   h->end();
 }
 
@@ -455,7 +464,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   }
 
   h->begin("band_gather");
-  launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, f->bf16, st);
+  launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, f->bf16, use_pdl(h), st);
   h->end();
   {
     GemmParams p = base_params(h, B * T, f->k_bs, kBnNarrow, f->g_bs, nb, nb * cdiv(D, kBnNarrow));
@@ -482,7 +491,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
 
     h->begin(f->tc_attention ? (axis == 0 ? "attn_time_tc" : "attn_band_tc") : "attn_simt_f16");
     if (f->tc_attention) {
-      if (!launch_attention_tc(f->QKV, f->ldq, f->O, B, T, nb, H, dh, axis, f->bf16, h->status, st)) {
+      if (!launch_attention_tc(f->QKV, f->ldq, f->O, B, T, nb, H, dh, axis, use_pdl(h), f->bf16, h->status, st)) {
         h->end();
         h->sched_error = "tensor-map encoding failed (attention)";
         return;

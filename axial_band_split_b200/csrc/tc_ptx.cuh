@@ -75,6 +75,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
 }
 
 // ------------------------------------------------------------------ TMA
+// Programmatic dependent launch.  griddep_wait: block until the grids this one depends on
+// have completed and their writes are visible (returns at once for a launch without the
+// programmatic attribute).  griddep_launch_dependents: let the next grid in the stream be
+// scheduled; its CTAs take SMs as this grid's exit, run their prologue and wait in their own
+// griddep_wait.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap *map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
