@@ -41,7 +41,7 @@ namespace mrf {
 namespace {
 
 constexpr int kDh = 64, kRows = 128, kKeys = 128;
-// K/V ring: 10 tiles of 16 KB, filled block by block in order.  A key block takes one K and
+// K/V ring: 8 tiles of 16 KB, filled block by block in order.  A key block takes one K and
 // one V tile when both query tiles share the keys (two tiles of one time-axis sequence) and
 // a K and a V tile per query tile otherwise (band axis; time-axis items that pair the odd
 // last tiles of two sequences).  At most kMaxStages blocks are in flight, each with its own
@@ -60,13 +60,16 @@ constexpr float kRescaleLog2 = 8.f;
 
 
 // q and k are kQA 64-wide atoms deep (dim_head 64 or 128; v is 64 wide either way): each query
-// tile takes kQA 16 KB tiles, a key block kQA K tiles and one V tile.  The ring shrinks to 8 tiles
-// when q and k are 128 deep, so that the doubled q buffer fits.
+// tile takes kQA 16 KB tiles, a key block kQA K tiles and one V tile.  With 64-deep q there are
+// two q buffers (items alternate between them, so the next item's queries load while this item
+// runs: on the band axis an item is a single key block and would otherwise wait for them); with
+// 128-deep q one, as the doubled tiles leave no room for a second.
 template <int kQA>
 struct AttnSmem {
-  static constexpr int ring = kQA == 1 ? 10 : 8;          // K/V ring tiles
-  static constexpr int q = 0;                              // [2 query tiles][kQA atoms]
-  static constexpr int kv = q + 2 * kQA * kTile;           // ring of 16 KB tiles
+  static constexpr int qbufs = kQA == 1 ? 2 : 1;           // q buffers
+  static constexpr int ring = 8;                           // K/V ring tiles
+  static constexpr int q = 0;                              // [qbufs][2 query tiles][kQA atoms]
+  static constexpr int kv = q + qbufs * 2 * kQA * kTile;   // ring of 16 KB tiles
   static constexpr int ostage = kv + ring * kTile;         // [8 warps] 32 rows x 128 B of output
   static constexpr int bar = ostage + 8 * 4096;
   static constexpr int total = bar + 256;
@@ -379,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + AttnSmem<kQA>::bar);
-  uint64_t *q_full = bars + 0, *q_empty = bars + 1;
+  uint64_t *q_full = bars + 26, *q_empty = bars + 28;  // [qbufs] each
   uint64_t *kv_full = bars + 2;     // [kMaxStages]
   uint64_t *kv_empty = bars + 8;    // [kMaxStages]
   uint64_t *s_full = bars + 14;     // [2]
@@ -388,15 +391,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *o_free = bars + 20;     // [2]
   uint64_t *s_free = bars + 22;     // [2]
   uint64_t *done = bars + 24;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 25);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 30);
+  constexpr int kQBufs = AttnSmem<kQA>::qbufs;
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    tc::mbar_init(q_full, 1);
-    tc::mbar_init(q_empty, 2);  // released by both tiles' MMA issuers
+    for (int b = 0; b < kQBufs; ++b) {
+      tc::mbar_init(q_full + b, 1);
+      tc::mbar_init(q_empty + b, 2);  // released by both tiles' MMA issuers
+    }
     for (int s = 0; s < kMaxStages; ++s) { tc::mbar_init(kv_full + s, 1); tc::mbar_init(kv_empty + s, 2); }
     for (int t = 0; t < 2; ++t) {
       tc::mbar_init(s_full + t, 1);
@@ -432,12 +438,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
         const TileC c0 = tile_coords(a, item, 0), c1 = tile_coords(a, item, 1);
         const bool mixed = item_mixed(a, item);
-        if (!tc::mbar_wait(q_empty, (li & 1) ^ 1, a.status, 30, abort)) break;
-        tc::mbar_arrive_expect_tx(q_full, 2 * kQA * kTile);
+        // item li's queries go to buffer li % kQBufs (its (li / kQBufs)-th use)
+        const int qb = li % kQBufs;
+        uint8_t *qbuf = smem + AttnSmem<kQA>::q + qb * 2 * kQA * kTile;
+        if (!tc::mbar_wait(q_empty + qb, ((li / kQBufs) & 1) ^ 1, a.status, 30, abort)) break;
+        tc::mbar_arrive_expect_tx(q_full + qb, 2 * kQA * kTile);
 #pragma unroll
         for (int qa = 0; qa < kQA; ++qa) {
-          tc::tma_load_4d(smem + AttnSmem<kQA>::q + qa * kTile, &tq, q_full, 64 * qa, c0.head, c0.band, c0.frame0);
-          tc::tma_load_4d(smem + AttnSmem<kQA>::q + (kQA + qa) * kTile, &tq, q_full, 64 * qa, c1.head, c1.band,
+          tc::tma_load_4d(qbuf + qa * kTile, &tq, q_full + qb, 64 * qa, c0.head, c0.band, c0.frame0);
+          tc::tma_load_4d(qbuf + (kQA + qa) * kTile, &tq, q_full + qb, 64 * qa, c1.head, c1.band,
                           c1.frame0);
         }
         const int need = (kQA + 1) * (mixed ? 2 : 1);
@@ -483,6 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int li = 0;
       bool ok = true;
       bool mixed = false;
+      int qb = 0;  // the item's q buffer
       // block at ring tile `base`: tile t's K atoms at base (+ (kQA + 1) t when the tiles have
       // separate keys), its V after them
       auto kv_tile = [&](int base, int t, int which) {
@@ -491,7 +501,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_s = [&](int t, int base) {
 #pragma unroll
         for (int kk = 0; kk < 4 * kQA; ++kk) {
-          const uint32_t q_addr = tc::smem_u32(smem + AttnSmem<kQA>::q + (t * kQA + kk / 4) * kTile);
+          const uint32_t q_addr =
+              tc::smem_u32(smem + AttnSmem<kQA>::q + ((qb * 2 + t) * kQA + kk / 4) * kTile);
           const uint32_t k_addr = tc::smem_u32(kv_tile(base, t, kk / 4));
           tc::mma_f16(tmem + 128 * t, tc::sw128_kmajor_desc(q_addr + (kk % 4) * 32),
                       tc::sw128_kmajor_desc(k_addr + (kk % 4) * 32), id_s, kk != 0);
@@ -513,12 +524,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int item = blockIdx.x; ok && item < a.items; item += gridDim.x, ++li) {
         mixed = item_mixed(a, item);
         const int need = (kQA + 1) * (mixed ? 2 : 1);
-        if (!tc::mbar_wait(q_full, li & 1, a.status, 32, abort)) break;
+        qb = li % kQBufs;
+        if (!tc::mbar_wait(q_full + qb, (li / kQBufs) & 1, a.status, 32, abort)) break;
         if (!tc::mbar_wait(kv_full + g % kMaxStages, (g / kMaxStages) & 1, a.status, 33, abort)) break;
         if (g > 0 && !tc::mbar_wait(s_free + t, (g - 1) & 1, a.status, 41, abort)) break;
         tc::tc_fence_after();
         issue_s(t, ptr);
-        if (a.n_blocks == 1) tc::mma_commit(q_empty);
+        if (a.n_blocks == 1) tc::mma_commit(q_empty + qb);
         for (int j = 0; j < a.n_blocks; ++j, ++g) {
           const int base = (ptr + j * need) % AttnSmem<kQA>::ring;
           if (j + 1 < a.n_blocks) {
@@ -529,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc::tc_fence_after();
             issue_s(t, (base + need) % AttnSmem<kQA>::ring);
-            if (j + 2 == a.n_blocks) tc::mma_commit(q_empty);
+            if (j + 2 == a.n_blocks) tc::mma_commit(q_empty + qb);
           }
           if (!tc::mbar_wait(p_full + t, g & 1, a.status, 34, abort) ||
               (j == 0 && !tc::mbar_wait(o_free + t, (li & 1) ^ 1, a.status, 35, abort))) {
