@@ -103,3 +103,13 @@ def test_time_axis_odd_sequence_count():
     W, x = case(cfg, B, T, True)
     got, _ = run(cfg, B, T, W, x)
     check(got, oracle_masks(cfg, B, T, True), "masks")
+
+
+@pytest.mark.parametrize("n_fft,num_bands,B,T", [(512, 3, 1, 33), (1024, 2, 2, 20)])
+def test_wide_bands(n_fft, num_bands, B, T):
+    # bands wider than 640 features (896, 1920) take the two-pass gather; the narrower ones of the
+    # same forward and every other test take the single-pass shared-memory gather
+    cfg = dataclasses.replace(synth.TINY, n_fft=n_fft, num_bands=num_bands)
+    W, x = case(cfg, B, T, True)
+    got, _ = run(cfg, B, T, W, x)
+    check(got, oracle_model.forward(x, cfg, W), f"n_fft {n_fft}, {num_bands} bands")
