@@ -107,8 +107,8 @@ def test_time_axis_odd_sequence_count():
 
 @pytest.mark.parametrize("n_fft,num_bands,B,T", [(512, 3, 1, 33), (1024, 2, 2, 20)])
 def test_wide_bands(n_fft, num_bands, B, T):
-    # bands wider than 640 features (896, 1920) take the two-pass gather; the narrower ones of the
-    # same forward and every other test take the single-pass shared-memory gather
+    # a band wider than 640 features (896, 1920) sends the whole gather to the two-pass kernel;
+    # every other test's bands fit the single-pass shared-memory gather
     cfg = dataclasses.replace(synth.TINY, n_fft=n_fft, num_bands=num_bands)
     W, x = case(cfg, B, T, True)
     got, _ = run(cfg, B, T, W, x)
