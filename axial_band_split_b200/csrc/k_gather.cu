@@ -9,20 +9,20 @@
 // sqrt(d_in) * gamma is folded into the GEMM's weight).
 //
 // The gather is a transpose: stft_repr is [row][frame][re, im] (frames contiguous) and the
-// GEMM wants [frame][feature] (features contiguous, feature 2 * (row - first row) + c).
-//
-// band_tile_kernel (bands of up to kTileRows rows): a CTA takes one band and 32 frames of one
-// window through shared memory, one pass over DRAM:
-//   load   each thread moves 16-byte pieces (two frames' (re, im) of one row; two 8-byte loads
-//          when T is odd) into a swizzled [row][16 pieces] tile, 16 threads per row so a
-//          half-warp reads 256 contiguous bytes, and adds the squares into its two frames' sums;
-//   reduce the per-frame sums of the 16 row groups, added in a fixed order, give
-//          1 / max(|x|, 1e-12) per frame;
-//   store  warp w takes frame pairs, lane l row quads l, l + 32, ...: four 16-byte shared reads
-//          (conflict-free: piece slot = piece ^ ((row / 4) % 16)) give 4 rows x 2 frames, written
-//          as one 16-byte store per frame, 32 lanes on 512 contiguous bytes of a feature row; rows
-//          up to the band's width rounded up to 64 features store zeros.
-// band_gather_kernel (wider bands): two passes over the band's rows, the second from L2.
+// GEMM wants [frame][feature] (features contiguous, feature 2 * (row - first row) + c).  A CTA
+// takes one band and 32 frames of one window with 16 warps: warp w covers frames 4 (w % 8) ..
+// 4 (w % 8) + 3 and every second 16-row step (from step w / 8), two lanes per row, each lane one
+// 16-byte load of two frames' (re, im) (two 8-byte loads when T is odd, where a row's frame pairs
+// are not 16-byte aligned): 32 contiguous bytes per row.
+//   pass 1  loads (eight in flight per thread), per-frame sums of squares (shuffle-xor over the
+//           lanes holding the same frames, then the two warps sharing the frames through shared
+//           memory);
+//   pass 2  the same loads again (the CTA's tile, at most 133 KB, is still in L2), scaled by
+//           1 / max(|x|, 1e-12) and stored as fp16 pairs: each store instruction of a warp
+//           writes 64 contiguous bytes of two frames' feature rows, so nothing is staged in
+//           shared memory; rows up to the band's width rounded up to 64 features store zeros.
+// Keeping the registers and shared memory small lets many CTAs share an SM, which hides the
+// loads' latency; the widest bands (40 times the narrowest's data) are scheduled first.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -120,122 +120,21 @@ __global__ void __launch_bounds__(kThreads) band_gather_kernel(const float *__re
   }
 }
 
-constexpr int kTileThreads = 256;
-constexpr int kTileRows = 320;  // rows per band handled through shared memory (80 KB of tile)
-
-// 16-byte piece q (frames 2q, 2q + 1) of tile row r: its slot in the row's 256 bytes
-__device__ __forceinline__ int piece_slot(int r, int q) { return q ^ ((r >> 2) & 15); }
-
-template <bool kEvenT, bool kBF>
-__global__ void __launch_bounds__(kTileThreads) band_tile_kernel(const float *__restrict__ in,
-                                                                 const int32_t *__restrict__ feat_row,
-                                                                 const BandDesc *__restrict__ bands, int nb,
-                                                                 int B, int T, int R, int tiles,
-                                                                 long long frame_stride, int k_stride,
-                                                                 __half *__restrict__ A) {
-  extern __shared__ uint8_t tile_raw[];
-  float4 *tile = reinterpret_cast<float4 *>(tile_raw);  // [row][16 slots]
-  __shared__ float red[16][kFrames];
-  __shared__ float scale[kFrames];
-  // programmatic dependent launch: the input may be an earlier kernel's output
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int per_band = B * tiles;
-  const int k = nb - 1 - (int)(blockIdx.x / per_band);  // widest bands first
-  const int rem = (int)(blockIdx.x % per_band);
-  const int b = rem / tiles, t0 = (rem % tiles) * kFrames;
-  const BandDesc bd = bands[k];
-  const int nrows = bd.width >> 1, prow = ((bd.width + 63) & ~63) >> 1;
-  const int row0 = feat_row[bd.feat_off];
-  const int tid = threadIdx.x, q = tid & 15;
-  const int t = t0 + 2 * q;
-  const float *base = in + (((long long)b * R + row0) * T + t) * 2;
-  // load: rows tid / 16, tid / 16 + 16, ... of piece q
-  float s0 = 0.f, s1 = 0.f;
-#pragma unroll 4
-  for (int r = tid >> 4; r < nrows; r += kTileThreads / 16) {
-    const float4 v = load_pair<kEvenT>(base + (long long)r * T * 2, t, T);
-    tile[r * 16 + piece_slot(r, q)] = v;
-    s0 = fmaf(v.x, v.x, fmaf(v.y, v.y, s0));
-    s1 = fmaf(v.z, v.z, fmaf(v.w, v.w, s1));
-  }
-  red[tid >> 4][2 * q] = s0;
-  red[tid >> 4][2 * q + 1] = s1;
-  __syncthreads();
-  if (tid < kFrames) {
-    float ss = 0.f;
-#pragma unroll
-    for (int g = 0; g < 16; ++g) ss += red[g][tid];
-    scale[tid] = 1.f / fmaxf(sqrtf(ss), kNormEps);
-  }
-  __syncthreads();
-  // store: warp w, frame pairs w, w + 8; lane l, row quads l, l + 32, ...
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int fp = warp; fp < kFrames / 2; fp += kTileThreads / 32) {
-    const int f0 = t0 + 2 * fp;
-    const float c0 = scale[2 * fp], c1 = scale[2 * fp + 1];
-    __half *out0 = A + ((long long)k * frame_stride + (long long)b * T + f0) * k_stride;
-    __half *out1 = out0 + k_stride;
-    for (int rq = lane; rq < prow / 4; rq += 32) {
-      uint32_t w0[4], w1[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = 4 * rq + i;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (r < nrows) v = tile[r * 16 + piece_slot(r, fp)];
-        w0[i] = pack2<kBF>(v.x * c0, v.y * c0);
-        w1[i] = pack2<kBF>(v.z * c1, v.w * c1);
-      }
-      if (f0 < T) *reinterpret_cast<uint4 *>(out0 + 8 * rq) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-      if (f0 + 1 < T) *reinterpret_cast<uint4 *>(out1 + 8 * rq) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-    }
-  }
-}
-
 }  // namespace
 
-bool band_tile_fits(int max_width) { return (max_width >> 1) <= kTileRows; }
-
-bool band_tile_init() {
-  const int bytes = kTileRows * 256;
-  return cudaFuncSetAttribute(band_tile_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-             cudaSuccess &&
-         cudaFuncSetAttribute(band_tile_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-             cudaSuccess &&
-         cudaFuncSetAttribute(band_tile_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-             cudaSuccess &&
-         cudaFuncSetAttribute(band_tile_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-             cudaSuccess;
-}
-
 void launch_band_gather(const float *in, const int32_t *feat_row, const BandDesc *bands, int nb, int B, int T,
-                        int rows, long long frame_stride, int k_stride, __half *A, int max_width, bool bf16,
-                        bool pdl, cudaStream_t st) {
+                        int rows, long long frame_stride, int k_stride, __half *A, bool bf16, bool pdl,
+                        cudaStream_t st) {
   const int tiles = (T + kFrames - 1) / kFrames;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(nb * B * tiles), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  if (band_tile_fits(max_width)) {
-    cfg.blockDim = dim3(kTileThreads, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)(max_width >> 1) * 256;
-#define MRF_TILE(E, BF) \
-  cudaLaunchKernelEx(&cfg, band_tile_kernel<E, BF>, in, feat_row, bands, nb, B, T, rows, tiles, frame_stride, k_stride, A)
-    if (T % 2 == 0) {
-      if (bf16) MRF_TILE(true, true);
-      else MRF_TILE(true, false);
-    } else {
-      if (bf16) MRF_TILE(false, true);
-      else MRF_TILE(false, false);
-    }
-#undef MRF_TILE
-    return;
-  }
-  cfg.blockDim = dim3(kThreads, 1, 1);
 #define MRF_GATHER(E, BF) \
   cudaLaunchKernelEx(&cfg, band_gather_kernel<E, BF>, in, feat_row, bands, nb, B, T, rows, tiles, frame_stride, k_stride, A)
   if (T % 2 == 0) {

@@ -43,11 +43,8 @@ void launch_band_split(const float *in, const int32_t *feat_row, const int32_t *
 // type is the 16-bit container of either), [band][frame_stride][k_stride],
 // each band's row zero-padded to a multiple of 64 (the A operand of the band-split GEMM).
 void launch_band_gather(const float *in, const int32_t *feat_row, const BandDesc *bands, int nb, int B, int T,
-                        int rows, long long frame_stride, int k_stride, __half *A, int max_width, bool bf16,
-                        bool pdl, cudaStream_t st);
-// the single-pass shared-memory gather serves bands of up to 640 features; its attribute setup
-bool band_tile_fits(int max_width);
-bool band_tile_init();
+                        int rows, long long frame_stride, int k_stride, __half *A, bool bf16, bool pdl,
+                        cudaStream_t st);
 
 enum SimtEpi : int {
   kEpiStore = 0,      // C = acc (+ bias)

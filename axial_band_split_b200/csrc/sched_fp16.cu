@@ -145,7 +145,7 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->bf16 = c.compute == MRF_BF16;
   if (const char *e = getenv("MRF_GEMM_PAIR")) f->pair = std::min(std::max(atoi(e), 0), 2);
   if (const char *e = getenv("MRF_PDL")) f->pdl = atoi(e) != 0;
-  if (!gemm_tc_init() || !band_tile_init() || (f->tc_attention && !attention_tc_init())) {
+  if (!gemm_tc_init() || (f->tc_attention && !attention_tc_init())) {
     h->err = "tcgen05 kernel initialisation failed (tensor-map encoder or shared-memory limit)";
     return MRF_ECUDA;
   }
@@ -464,7 +464,7 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
   }
 
   h->begin("band_gather");
-  launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, h->max_width, f->bf16, use_pdl(h), st);
+  launch_band_gather(in, h->d_feat_row, h->d_bands, nb, B, T, R, MBT, f->k_bs, f->A_bs, f->bf16, use_pdl(h), st);
   h->end();
   {
     GemmParams p = base_params(h, B * T, f->k_bs, kBnNarrow, f->g_bs, nb, nb * cdiv(D, kBnNarrow));

@@ -107,8 +107,8 @@ def test_time_axis_odd_sequence_count():
 
 @pytest.mark.parametrize("n_fft,num_bands,B,T", [(512, 3, 1, 33), (1024, 2, 2, 20)])
 def test_wide_bands(n_fft, num_bands, B, T):
-    # a band wider than 640 features (896, 1920) sends the whole gather to the two-pass kernel;
-    # every other test's bands fit the single-pass shared-memory gather
+    # bands of 896 and 1920 features: the gather's row loop runs several passes per CTA and the
+    # band-split GEMM's per-band K reaches 1920
     cfg = dataclasses.replace(synth.TINY, n_fft=n_fft, num_bands=num_bands)
     W, x = case(cfg, B, T, True)
     got, _ = run(cfg, B, T, W, x)
