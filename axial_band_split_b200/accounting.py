@@ -35,6 +35,8 @@ def kernel_work(cfg, widths, B: int, T: int):
         "gemm_ff1_gelu": ("flop", L2 * 2 * NT * D * F1, L2),
         "gemm_ff1_geglu": ("flop", L2 * 2 * NT * D * F1, L2),   # the GEGLU variant's launch name
         "gemm_ff2_resid": ("flop", L2 * 2 * NT * FF * D, L2),
+        # the fused feed-forward (both projections in one launch per transformer)
+        "gemm_ff_fused": ("flop", L2 * 2 * NT * D * F1 + L2 * 2 * NT * FF * D, L2),
         "gemm_mask_tanh": ("flop", S * 2 * BT * nb * (D * MH + (cfg.mask_depth - 1) * MH * MH), S * cfg.mask_depth),
         "gemm_mask_glu": ("flop", S * 2 * BT * MH * 2 * n_feat, S),
         "band_split": ("flop", 2 * BT * D * n_feat, 1),
@@ -48,8 +50,9 @@ def kernel_work(cfg, widths, B: int, T: int):
     return w
 
 
-# entries that restate others' work (the SIMT band split; FF1 under its GEGLU launch name)
-_ALIASES = ("band_split", "gemm_ff1_geglu")
+# entries that restate others' work (the SIMT band split; FF1 under its GEGLU launch name; FF1 and
+# FF2 together in the fused feed-forward launch)
+_ALIASES = ("band_split", "gemm_ff1_geglu", "gemm_ff_fused")
 
 
 def total_flops(cfg, widths, B: int, T: int) -> int:

@@ -107,4 +107,22 @@ void launch_gemm_tc(int epi, bool bf16, bool pair, const CUtensorMap &tmA, const
                     cudaStream_t st);
 bool gemm_tc_pair_kind(int epi);
 
+// Fused feed-forward (k_ff_tc.cu): x <- x + W2 gelu(rs W1 x + b1) + b2 on the fp16 residual stream,
+// rs the row scale of the ss_in partial slots; the new rows' sums of squares (and of out_gain * x)
+// into ss_out / ssg_out, four slots a row.  tmX: Xh [M, D] fp16 box 64 x 128 (swizzle 128);
+// tmW1: W1 [hidden, D] box 64 x 64; tmW2: W2 [D, hidden] box 64 x (D / 2, or D / 4 when D > 256);
+// tmO: Xh box 32 x 32 (swizzle 64).  Runs as CTA pairs.
+struct FfParams {
+  int M, D, hidden, ld, ss_in_parts, ss_out_parts;
+  unsigned *status;
+  const float *ss_in;
+  const float *b1, *b2, *out_gain;
+  __half *Xh;
+  float *ss_out, *ssg_out;
+};
+bool ff_tc_supported(int D, int hidden);
+bool ff_tc_init();
+void launch_ff_tc(const CUtensorMap &tmX, const CUtensorMap &tmW1, const CUtensorMap &tmW2, const CUtensorMap &tmO,
+                  const FfParams &p, int sms, bool pdl, cudaStream_t st);
+
 }  // namespace mrf

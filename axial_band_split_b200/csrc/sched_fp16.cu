@@ -79,6 +79,11 @@ struct Fp16State {
   // inputs after its prologue, which then overlaps the previous kernel's tail); MRF_PDL=0 in the
   // environment at create turns it off
   bool pdl = true;
+  // the feed-forward as one kernel on CTA pairs (fp16, GELU, D <= 384, hidden <= 1536, four
+  // row-statistic slots) when MRF_FF_FUSED=1 at create; by default the FF1 and FF2 GEMMs, which
+  // measured faster (the fused kernel's 128-wide hidden chunks re-read x from shared memory for
+  // every chunk: its MMAs run at about half the tensor rate)
+  bool ff_fused = false;
 };
 
 namespace {
@@ -145,6 +150,13 @@ mrf_status pack_fp16(mrf_handle *h, WeightMap &W) {
   f->bf16 = c.compute == MRF_BF16;
   if (const char *e = getenv("MRF_GEMM_PAIR")) f->pair = std::min(std::max(atoi(e), 0), 2);
   if (const char *e = getenv("MRF_PDL")) f->pdl = atoi(e) != 0;
+  const char *ffe = getenv("MRF_FF_FUSED");
+  f->ff_fused = ffe && atoi(ffe) != 0 && !f->bf16 && c.ff_act == 0 && ff_tc_supported(c.dim, c.ff_mult * c.dim) &&
+                cdiv(c.dim, kBnNarrow) * 2 == 4;
+  if (f->ff_fused && !ff_tc_init()) {
+    h->err = "fused feed-forward initialisation failed (shared-memory limit)";
+    return MRF_ECUDA;
+  }
   if (!gemm_tc_init() || (f->tc_attention && !attention_tc_init())) {
     h->err = "tcgen05 kernel initialisation failed (tensor-map encoder or shared-memory limit)";
     return MRF_ECUDA;
@@ -418,6 +430,15 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
        make_tmap_f16(&mWbs, f->w_bs, f->k_bs, (long long)nb * D, 1, f->k_bs, (long long)nb * D * f->k_bs, kBnNarrow, 1);
   const int n_mask_maps = c.mask_depth + 1;  // per stem
   std::vector<CUtensorMap> wmaps(4 * 2 * c.depth + c.num_stems * n_mask_maps);
+  // the fused feed-forward's weight maps: W1 in 64-row boxes (half of a 128-unit chunk), W2 in
+  // boxes of half an MMA piece (D / 2 rows, D / 4 when D > 256)
+  std::vector<CUtensorMap> ffmaps(f->ff_fused ? 2 * 2 * c.depth : 0);
+  for (int i = 0; ok && f->ff_fused && i < 2 * c.depth; ++i) {
+    const TrF16 &w = f->tr[i];
+    const unsigned w2box = D > 256 ? D / 4 : D / 2;
+    ok = make_tmap_f16(&ffmaps[2 * i], w.w1, D, FF, 1, D, (long long)FF * D, 64, 1) &&
+         make_tmap_f16(&ffmaps[2 * i + 1], w.w2, FF, D, 1, FF, (long long)D * FF, w2box, 1);
+  }
   for (int i = 0; ok && i < 2 * c.depth; ++i) {
     const TrF16 &w = f->tr[i];
     // weight boxes: BN rows, or BN / 2 for the CTA pairs (each CTA loads half of a B tile)
@@ -507,6 +528,16 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     }
     gemm(h, "gemm_out_resid", kTcResid, mO, mWo, p, f->bf16 ? &mXo : &mXho, &mXho);
 
+    if (f->ff_fused) {
+      FfParams q{};
+      q.M = M; q.D = D; q.hidden = FF; q.ld = D; q.ss_in_parts = f->parts_res; q.ss_out_parts = f->parts_res;
+      q.status = h->status; q.ss_in = f->ss; q.b1 = w.b1; q.b2 = w.b2; q.out_gain = w.gout; q.Xh = f->Xh;
+      q.ss_out = f->ssx; q.ssg_out = f->ssg;
+      h->begin("gemm_ff_fused");
+      launch_ff_tc(mXh, ffmaps[2 * i], ffmaps[2 * i + 1], mXho, q, f->sms, use_pdl(h), st);
+      h->end();
+      continue;
+    }
     p = base_params(h, M, D, kBnWide, f->g_ff1, 1, cdiv(F1, kBnWide));
     p.ss_in = f->ss; p.ss_in_parts = f->parts_res; p.bias = w.b1; p.out_h = f->Hh; p.ldo = FF;
     if (c.ff_act == 1) gemm(h, "gemm_ff1_geglu", kTcGeglu, mXh, mW1, p, &mHo16);
