@@ -85,9 +85,9 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
   uint64_t *w1_full = bars + 2, *w1_empty = bars + 2 + kW1Stages;                     // [kW1Stages]
   uint64_t *w2_full = bars + 2 + 2 * kW1Stages, *w2_empty = w2_full + kW2Stages;     // [kW2Stages]
   uint64_t *hacc_full = w2_empty + kW2Stages, *hacc_empty = hacc_full + 1;
-  uint64_t *hsm_full = hacc_full + 2, *hsm_empty = hacc_full + 3;
-  uint64_t *o_full = hacc_full + 4, *o_empty = hacc_full + 5;
-  uint64_t *stg_free = hacc_full + 6, *done = hacc_full + 7;
+  uint64_t *hsm_full = hacc_full + 2, *hsm_empty = hacc_full + 4;  // [2]: per 64-wide K block of H
+  uint64_t *o_full = hacc_full + 6, *o_empty = hacc_full + 7;
+  uint64_t *stg_free = hacc_full + 8, *done = hacc_full + 9;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
   __shared__ int abort_flag;
 
@@ -107,8 +107,10 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
     for (int s = 0; s < kW2Stages; ++s) { tc::mbar_init(w2_full + s, 1); tc::mbar_init(w2_empty + s, 1); }
     tc::mbar_init(hacc_full, 1);
     tc::mbar_init(hacc_empty, 2 * kEpiWarps);  // both CTAs' epilogue warps
-    tc::mbar_init(hsm_full, 2 * kEpiWarps);
-    tc::mbar_init(hsm_empty, 1);
+    for (int kb = 0; kb < 2; ++kb) {
+      tc::mbar_init(hsm_full + kb, kEpiWarps);  // the 8 warps of both CTAs that write the K block
+      tc::mbar_init(hsm_empty + kb, 1);
+    }
     tc::mbar_init(o_full, 1);
     tc::mbar_init(o_empty, 2 * kEpiWarps);
     tc::mbar_init(stg_free, kEpiWarps);        // this CTA's epilogue warps
@@ -185,12 +187,11 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
       int lt = 0;
       bool ok = true;
       auto mma2 = [&](int chunk, int gch) {
-        // H(chunk) written by the epilogue (its gch-th H), and O_acc released by the previous
-        // tile's final epilogue before the tile's first accumulation
-        if (!tc::mbar_wait(hsm_full, gch & 1, p.status, 55, abort)) { ok = false; return; }
+        // O_acc released by the previous tile's final epilogue before the tile's first accumulation
         if (chunk == 0 && !tc::mbar_wait(o_empty, (lt & 1) ^ 1, p.status, 56, abort)) { ok = false; return; }
-        tc::tc_fence_after();
         for (int kb = 0; kb < kChunk / 64; ++kb) {
+          // K block kb of H(chunk) written by the epilogue (its gch-th H)
+          if (!tc::mbar_wait(hsm_full + kb, gch & 1, p.status, 55, abort)) { ok = false; return; }
           if (!tc::mbar_wait(w2_full + s2, ph2, p.status, 57, abort)) { ok = false; return; }
           tc::tc_fence_after();
           const uint32_t a = tc::smem_u32(sh + kb * kXBlock), b = tc::smem_u32(sw2 + s2 * kW2StageMax);
@@ -201,9 +202,9 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
                                tc::sw128_kmajor_desc(b + pc * (np / 2) * 128 + kk * 32), id2,
                                (chunk | kb | kk) != 0);
           tc::mma_commit_pair(w2_empty + s2, 0x3);
+          tc::mma_commit_pair(hsm_empty + kb, 0x3);  // this K block of H may be rewritten
           if (++s2 == kW2Stages) { s2 = 0; ph2 ^= 1; }
         }
-        tc::mma_commit_pair(hsm_empty, 0x3);  // H may be rewritten
       };
       for (int tile = first_tile; ok && tile < tiles; tile += tile_step, ++lt) {
         if (!tc::mbar_wait(x_full, lt & 1, p.status, 53, abort)) break;
@@ -268,9 +269,9 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
           const float2 g = tcm::gelu2(v[j], v[j + 1], rs, bv[j], bv[j + 1]);
           hw[j >> 1] = pack_f16(g.x, g.y);
         }
-        // H is free once the previous MMA2 has read it (and, for a tile's first chunk, once the
-        // previous tile's output staging has been read by its bulk stores)
-        if (!tc::mbar_wait(hsm_empty, (ch & 1) ^ 1, p.status, 61, abort)) { ok = false; break; }
+        // this warp's K block of H is free once the previous MMA2 has read it (and, for a tile's
+        // first chunk, once the previous tile's output staging has been read by its bulk stores)
+        if (!tc::mbar_wait(hsm_empty + (sub >> 1), (ch & 1) ^ 1, p.status, 61, abort)) { ok = false; break; }
         if (c == 0 && lt > 0 && !tc::mbar_wait(stg_free, (lt - 1) & 1, p.status, 62, abort)) { ok = false; break; }
         // row r's 32 hidden values at columns 32 sub .. of the chunk: K block sub / 2, 16-byte
         // pieces 4 (sub % 2) .. 4 (sub % 2) + 3 of the row's 128 bytes, 128-byte swizzle
@@ -283,7 +284,7 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
         }
         tc::fence_proxy_async();  // the tensor core reads H through the async proxy
         __syncwarp();
-        if (lane == 0) arrive_leader(hsm_full, rank);
+        if (lane == 0) arrive_leader(hsm_full + (sub >> 1), rank);
       }
       if (!ok) break;
       // ---- final epilogue: x + O_acc + b2, row statistics, bulk stores through the staging box

@@ -1,28 +1,10 @@
-// Elementwise epilogue math shared by the tensor-core kernels: packed f32x2 helpers and
-// the GELU of the feed-forward layers.
+// Elementwise epilogue math shared by the tensor-core kernels: the GELU of the feed-forward
+// layers (packed f32x2 pairs) and tanh and the sigmoid on the MUFU.
 #pragma once
 #include <cuda_fp16.h>
 
 namespace mrf {
 namespace tcm {
-
-// Packed pairs (one f32x2 instruction for two lanes of math).
-__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
-  return (static_cast<unsigned long long>(__float_as_uint(b)) << 32) | __float_as_uint(a);
-}
-__device__ __forceinline__ float2 f2_unpack(unsigned long long v) {
-  return make_float2(__uint_as_float(static_cast<unsigned>(v)), __uint_as_float(static_cast<unsigned>(v >> 32)));
-}
-__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b, unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 
 // GELU of y0 = v0 * rs + b0 and y1 = v1 * rs + b1, y * (1 + erf(y / sqrt 2)) / 2, written
 // as max(y, 0) - |y| * erfc(|y| / sqrt 2) / 2 (both signs of y).  The complementary error
@@ -33,25 +15,24 @@ __device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigne
 // 16th power is doubled and its reciprocal is erfc / 2).  Packed pairs throughout.  (An
 // infinite y gives NaN; finite inputs never reach inf.)
 __device__ __forceinline__ float2 gelu2(float v0, float v1, float rs, float b0, float b1) {
-  const unsigned long long y = fma2(f2_pack(v0, v1), f2_pack(rs, rs), f2_pack(b0, b1));
-  const float2 yy = f2_unpack(y);
-  const unsigned long long w = f2_pack(-fabsf(yy.x), -fabsf(yy.y));
-  unsigned long long q = fma2(w, f2_pack(5.62129980608006e-06f, 5.62129980608006e-06f),
-                              f2_pack(-5.105520904180594e-05f, -5.105520904180594e-05f));
-  q = fma2(w, q, f2_pack(3.9686136005911976e-05f, 3.9686136005911976e-05f));
-  q = fma2(w, q, f2_pack(-0.003422739217057824f, -0.003422739217057824f));
-  q = fma2(w, q, f2_pack(0.02207699790596962f, 0.02207699790596962f));
-  q = fma2(w, q, f2_pack(-0.052075162529945374f, -0.052075162529945374f));
-  q = fma2(w, q, f2_pack(1.0442737340927124f, 1.0442737340927124f));
-  q = mul2(q, q);
-  q = mul2(q, q);
-  q = mul2(q, q);
-  q = mul2(q, q);
-  const float2 qq = f2_unpack(q);
+  // packed pairs through the compiler's f32x2 builtins (one fma.rn.f32x2 / mul.rn.f32x2 each)
+  const float2 y = __ffma2_rn(make_float2(v0, v1), make_float2(rs, rs), make_float2(b0, b1));
+  const float2 w = make_float2(-fabsf(y.x), -fabsf(y.y));
+  float2 q = __ffma2_rn(w, make_float2(5.62129980608006e-06f, 5.62129980608006e-06f),
+                        make_float2(-5.105520904180594e-05f, -5.105520904180594e-05f));
+  q = __ffma2_rn(w, q, make_float2(3.9686136005911976e-05f, 3.9686136005911976e-05f));
+  q = __ffma2_rn(w, q, make_float2(-0.003422739217057824f, -0.003422739217057824f));
+  q = __ffma2_rn(w, q, make_float2(0.02207699790596962f, 0.02207699790596962f));
+  q = __ffma2_rn(w, q, make_float2(-0.052075162529945374f, -0.052075162529945374f));
+  q = __ffma2_rn(w, q, make_float2(1.0442737340927124f, 1.0442737340927124f));
+  q = __fmul2_rn(q, q);
+  q = __fmul2_rn(q, q);
+  q = __fmul2_rn(q, q);
+  q = __fmul2_rn(q, q);
   float e0, e1;  // erfc(|y| / sqrt 2) / 2
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(qq.x));
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(qq.y));
-  return f2_unpack(fma2(w, f2_pack(e0, e1), f2_pack(fmaxf(yy.x, 0.f), fmaxf(yy.y, 0.f))));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(q.x));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(q.y));
+  return __ffma2_rn(w, make_float2(e0, e1), make_float2(fmaxf(y.x, 0.f), fmaxf(y.y, 0.f)));
 }
 
 // tanh and the logistic sigmoid on the MUFU, from the identities tanh y = 1 - 2 / (1 + e^(2y))

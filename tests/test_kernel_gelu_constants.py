@@ -24,7 +24,7 @@ def kernel_coefficients():
     src = open(os.path.join(ROOT, "axial_band_split_b200", "csrc", "tc_math.cuh")).read()
     body = src[src.index("float2 gelu2("):]
     body = body[:body.index("\n}\n")]
-    pairs = re.findall(r"f2_pack\(([-+0-9.e]+)f, ([-+0-9.e]+)f\)", body)
+    pairs = re.findall(r"make_float2\(([-+0-9.e]+)f, ([-+0-9.e]+)f\)", body)
     vals = [float(a) for a, b in pairs if a == b]
     # Horner order in the source: the degree-6 and degree-5 coefficients first, then 4 .. 0
     return vals[:7]
