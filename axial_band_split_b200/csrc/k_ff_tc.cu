@@ -24,8 +24,11 @@
 // Tensor memory: O_acc in columns 0 .. D - 1 (D <= 384), H_acc in columns 384 .. 511.
 // Warps 0-15: epilogue (warp w: TMEM lane quarter w % 4, hidden columns 32 (w / 4) .. of a chunk;
 // output columns 32 (w / 4 + 4 j) of the final epilogue); warp 16: TMA producer; warp 17: TMEM
-// allocation and, in the leader CTA, the MMA issuer.  Every wait is bounded (the error path of
-// tc::mbar_wait).
+// allocation and, in the leader CTA, the MMA issuer.  The epilogue warps release H_acc, hand over
+// H and release O_acc on their own CTA's barriers; in the peer CTA, four lanes of warp 17 forward
+// each completed phase to the leader's barrier with one cluster-scope arrive (an arrive with
+// cluster release semantics from every epilogue warp cost each of them ~1,900 clk a chunk).  Every
+// wait is bounded (the error path of tc::mbar_wait).
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -66,10 +69,9 @@ __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Arrive on the leader CTA's copy of a barrier (the peer through the cluster address).
-__device__ __forceinline__ void arrive_leader(uint64_t *bar, uint32_t rank) {
-  if (rank == 0) tc::mbar_arrive(bar);
-  else tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(bar), 0));
+// Arrive on the leader CTA's copy of a barrier from the peer (through the cluster address).
+__device__ __forceinline__ void arrive_remote_leader(uint64_t *bar) {
+  tc::mbar_arrive_cluster(tc::mapa_shared(tc::smem_u32(bar), 0));
 }
 
 __global__ void __launch_bounds__(kThreadsFf, 1)
@@ -105,14 +107,16 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
     tc::mbar_init(x_empty, 1);
     for (int s = 0; s < kW1Stages; ++s) { tc::mbar_init(w1_full + s, 1); tc::mbar_init(w1_empty + s, 1); }
     for (int s = 0; s < kW2Stages; ++s) { tc::mbar_init(w2_full + s, 1); tc::mbar_init(w2_empty + s, 1); }
+    // released by this CTA's epilogue warps, and in the leader also by the peer's forwarding lane
+    const uint32_t fwd = rank == 0 ? 1 : 0;
     tc::mbar_init(hacc_full, 1);
-    tc::mbar_init(hacc_empty, 2 * kEpiWarps);  // both CTAs' epilogue warps
+    tc::mbar_init(hacc_empty, kEpiWarps + fwd);
     for (int kb = 0; kb < 2; ++kb) {
-      tc::mbar_init(hsm_full + kb, kEpiWarps);  // the 8 warps of both CTAs that write the K block
+      tc::mbar_init(hsm_full + kb, kEpiWarps / 2 + fwd);  // the 8 warps that write the K block
       tc::mbar_init(hsm_empty + kb, 1);
     }
     tc::mbar_init(o_full, 1);
-    tc::mbar_init(o_empty, 2 * kEpiWarps);
+    tc::mbar_init(o_empty, kEpiWarps + fwd);
     tc::mbar_init(stg_free, kEpiWarps);        // this CTA's epilogue warps
     tc::mbar_init(done, 1);
     tc::fence_barrier_init();
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
         if (chunk == 0 && !tc::mbar_wait(o_empty, (lt & 1) ^ 1, p.status, 56, abort)) { ok = false; return; }
         for (int kb = 0; kb < kChunk / 64; ++kb) {
           // K block kb of H(chunk) written by the epilogue (its gch-th H)
-          if (!tc::mbar_wait(hsm_full + kb, gch & 1, p.status, 55, abort)) { ok = false; return; }
+          if (!tc::mbar_wait<true>(hsm_full + kb, gch & 1, p.status, 55, abort)) { ok = false; return; }
           if (!tc::mbar_wait(w2_full + s2, ph2, p.status, 57, abort)) { ok = false; return; }
           tc::tc_fence_after();
           const uint32_t a = tc::smem_u32(sh + kb * kXBlock), b = tc::smem_u32(sw2 + s2 * kW2StageMax);
@@ -236,6 +240,19 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
       }
       tc::mma_commit_pair(done, 0x1);
       tc::mbar_wait(done, 0, p.status, 59, abort);
+    } else if (rank == 1 && lane < 4) {
+      // the peer's forwarding lanes: lane 0 H_acc released, lanes 1 and 2 H's K blocks written,
+      // lane 3 O_acc released; each waits for its local barrier's phases in order and arrives once
+      // on the leader's copy (a local phase runs at most one ahead: the next needs the leader's
+      // MMA, which needs this forward)
+      uint64_t *bar = lane == 0 ? hacc_empty : (lane == 3 ? o_empty : hsm_full + (lane - 1));
+      const int per_tile = lane == 3 ? 1 : nchunks;
+      int n = 0;
+      for (int tile = first_tile; tile < tiles; tile += tile_step)
+        for (int i = 0; i < per_tile; ++i, ++n) {
+          if (!tc::mbar_wait(bar, n & 1, p.status, 64, abort)) { tile = tiles; break; }
+          arrive_remote_leader(bar);
+        }
     }
   } else {
     // ---------------- epilogue warps 0-15
@@ -261,7 +278,7 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
         tc::tmem_ld32(tmem_base + lane_off + kMaxD + 32 * sub, v);
         tc::tc_fence_before();
         __syncwarp();
-        if (lane == 0) arrive_leader(hacc_empty, rank);  // MMA1 of the next chunk may overwrite H_acc
+        if (lane == 0) tc::mbar_arrive(hacc_empty);  // MMA1 of the next chunk may overwrite H_acc
         const float *bv = sb1 + c * kChunk + 32 * sub;
         uint32_t hw[16];
 #pragma unroll
@@ -282,9 +299,9 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
           *reinterpret_cast<uint4 *>(hrow + ((piece ^ (r & 7)) << 4)) =
               make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
         }
-        tc::fence_proxy_async();  // the tensor core reads H through the async proxy
+        tc::fence_proxy_async_all();  // the pair's tensor core reads H through the async proxy
         __syncwarp();
-        if (lane == 0) arrive_leader(hsm_full + (sub >> 1), rank);
+        if (lane == 0) tc::mbar_arrive(hsm_full + (sub >> 1));
       }
       if (!ok) break;
       // ---- final epilogue: x + O_acc + b2, row statistics, bulk stores through the staging box
@@ -347,7 +364,7 @@ __global__ void __launch_bounds__(kThreadsFf, 1)
       // O_acc read: the next tile's MMA2 may overwrite it
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) arrive_leader(o_empty, rank);
+      if (lane == 0) tc::mbar_arrive(o_empty);
       if (valid) {
         p.ss_out[(long long)m * p.ss_out_parts + sub] = sq;
         p.ssg_out[(long long)m * p.ss_out_parts + sub] = sqg;
