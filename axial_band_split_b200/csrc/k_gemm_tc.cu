@@ -814,10 +814,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 template <int EPI, bool kBF, bool kPair = false>
 constexpr size_t smem_bytes() { return SmemLayout<EPI, kBF, kPair>::total + 1024; }
-// The epilogue kinds that run as CTA pairs (the trunk's four GEMMs); the grouped mask-head and
-// band-split GEMMs run one CTA per tile.
+// The epilogue kinds that can run as CTA pairs (the trunk's four GEMMs and the mask MLP's tanh
+// layers); the band split and the mask GLU layer run one CTA per tile.
 __host__ __device__ constexpr bool pair_kind(int epi) {
-  return epi == kTcQkv || epi == kTcResid || epi == kTcGelu || epi == kTcGeglu;
+  return epi == kTcQkv || epi == kTcResid || epi == kTcGelu || epi == kTcGeglu || epi == kTcTanh;
 }
 template <int EPI>
 constexpr bool smem_fits() {

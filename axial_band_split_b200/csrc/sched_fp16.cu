@@ -72,8 +72,9 @@ struct Fp16State {
   // adds of twelve transformers to bf16's 8-bit significand would cost too much precision)
   bool bf16 = false;
   float *X = nullptr;
-  // which trunk GEMMs run as CTA pairs (cta_group::2), from MRF_GEMM_PAIR in the environment at
-  // create: 0 none, 1 those with K >= kPairMinK (the default), 2 all four
+  // which GEMMs run as CTA pairs (cta_group::2), from MRF_GEMM_PAIR in the environment at
+  // create: 0 none, 1 those with K >= kPairMinK (the default), 2 every pair-capable one (the four
+  // trunk GEMMs and the mask MLP's tanh layers)
   int pair = 1;
   // the tensor-core kernels launched with programmatic stream serialisation (each waits for its
   // inputs after its prologue, which then overlaps the previous kernel's tail); MRF_PDL=0 in the
@@ -369,11 +370,12 @@ GemmParams base_params(mrf_handle *h, int M, int K, int BN, const GemmGroup *gro
   return p;
 }
 
-// A trunk GEMM may run as CTA pairs (M = 256 tiles, B maps with half-height boxes): each CTA
-// then stages half of every B tile, which halves the shared-memory traffic of the main loop.
-// That pays where the main loop is long (FF2, K = 4 D) and costs where the epilogue dominates
-// (the QKV, out-projection and FF1 GEMMs, K <= 512, run about 10 % slower as pairs on B200), so
-// by default only GEMMs with K >= kPairMinK pair.  The grouped GEMMs run one CTA per M = 128 tile.
+// A trunk GEMM or a mask tanh layer may run as CTA pairs (M = 256 tiles, B maps with half-height
+// boxes): each CTA then stages half of every B tile, which halves the shared-memory traffic of the
+// main loop.  That pays where the main loop is long (FF2, K = 4 D; the mask MLP's hidden layers,
+// K = 1536) and costs where the epilogue dominates (the QKV, out-projection and FF1 GEMMs,
+// K <= 512, run about 10 % slower as pairs on B200), so by default only GEMMs with
+// K >= kPairMinK pair.  The band split and the GLU layer run one CTA per M = 128 tile.
 constexpr int kPairMinK = 1024;
 // Per-kernel timing records an event pair around each launch, which a kernel started ahead of
 // its predecessor's end would blur: timing runs launch without the programmatic attribute.
@@ -457,7 +459,8 @@ void schedule_fp16(mrf_handle *h, const float *in, float *out, int B, int T) {
     const int w0 = wm0 + s * n_mask_maps;
     for (int i = 0; ok && i < c.mask_depth; ++i) {
       const int K = i == 0 ? D : MH;
-      ok = make_tmap_f16(&wmaps[w0 + i], f->mw[s][i], K, (long long)nb * MH, 1, K, (long long)nb * MH * K, kBnWide, 1);
+      const unsigned bb = use_pair(h, kTcTanh, K) ? kBnWide / 2 : kBnWide;
+      ok = make_tmap_f16(&wmaps[w0 + i], f->mw[s][i], K, (long long)nb * MH, 1, K, (long long)nb * MH * K, bb, 1);
     }
     ok = ok && make_tmap_f16(&wmaps[w0 + c.mask_depth], f->mw_last[s], MH, rows_last, 1, MH, rows_last * MH, kBnWide, 1);
   }
