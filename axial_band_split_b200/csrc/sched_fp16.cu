@@ -372,10 +372,11 @@ GemmParams base_params(mrf_handle *h, int M, int K, int BN, const GemmGroup *gro
 
 // A trunk GEMM or a mask tanh layer may run as CTA pairs (M = 256 tiles, B maps with half-height
 // boxes): each CTA then stages half of every B tile, which halves the shared-memory traffic of the
-// main loop.  That pays where the main loop is long (FF2, K = 4 D; the mask MLP's hidden layers,
-// K = 1536) and costs where the epilogue dominates (the QKV, out-projection and FF1 GEMMs,
-// K <= 512, run about 10 % slower as pairs on B200), so by default only GEMMs with
-// K >= kPairMinK pair.  The band split and the GLU layer run one CTA per M = 128 tile.
+// main loop.  That pays where the main loop is long (FF2, K = 4 D: 1.14 -> 1.06 ms per forward)
+// and costs where the epilogue dominates (the QKV, out-projection and FF1 GEMMs, K <= 512, run
+// about 10 % slower as pairs on B200) or the rows are short (a band's T rows of the mask MLP fill
+// 256-row tiles worse than 128-row ones: its K = 1536 layer ran 7 % slower), so by default only
+// trunk GEMMs with K >= kPairMinK pair.  The band split and the GLU layer run one CTA per tile.
 constexpr int kPairMinK = 1024;
 // Per-kernel timing records an event pair around each launch, which a kernel started ahead of
 // its predecessor's end would blur: timing runs launch without the programmatic attribute.
@@ -383,7 +384,7 @@ bool use_pdl(const mrf_handle *h) { return h->f16->pdl && !h->timing; }
 
 bool use_pair(const mrf_handle *h, int epi, int K) {
   const int mode = h->f16->pair;
-  return gemm_tc_pair_kind(epi) && (mode == 2 || (mode == 1 && K >= kPairMinK));
+  return gemm_tc_pair_kind(epi) && (mode == 2 || (mode == 1 && epi != kTcTanh && K >= kPairMinK));
 }
 
 void gemm(mrf_handle *h, const char *name, int epi, const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p0,

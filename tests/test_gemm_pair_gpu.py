@@ -1,8 +1,8 @@
 """CTA-pair GEMMs (cta_group::2, M = 256 tiles) against one CTA per M = 128 tile (GPU).
 
-MRF_GEMM_PAIR, read when a model is created, selects which GEMMs pair: 0 none, 1 those with
-K >= 1024 (FF2 of a D >= 256 model and the mask MLP's hidden tanh layers, grouped by band; the
-default), 2 every trunk GEMM and every tanh layer.  A pair computes every
+MRF_GEMM_PAIR, read when a model is created, selects which GEMMs pair: 0 none, 1 the trunk GEMMs
+with K >= 1024 (FF2 of a D >= 256 model; the default), 2 every trunk GEMM and the mask MLP's tanh
+layers (grouped by band).  A pair computes every
 output element with the same K-ordered fp32 accumulation and the same epilogue arithmetic as a
 single CTA, so the three modes give the same bits; each is also held to the fp16 parity bar
 against the float64 oracle.  Shapes: a ragged row count (B T nb not a multiple of 256, so the
