@@ -582,27 +582,86 @@ mrf_status mrf_forward_separate(mrf_handle *h, const float *in, float *out, int 
   return forward_impl(h, in, out, B, T, stream, true);
 }
 
-mrf_status mrf_forward_host(mrf_handle *h, const float *in_host, float *out_host, int B, int T,
-                            void *stream) {
+}  // extern "C"
+
+namespace {
+
+// The host-buffer pipeline's one-time setup: two device slots of the largest input and output,
+// the two copy streams and the ordering events, made on the current device at the first call.
+mrf_status host_pipe_init(mrf_handle *h) {
+  if (h->io_in[1]) return MRF_OK;
+  const size_t maxb = (size_t)h->cfg.max_batch * h->tab.n_freqs * h->tab.channels * h->cfg.max_frames * 2 * sizeof(float);
+  for (int s = 0; s < 2; ++s) {
+    if (!h->io_in[s]) h->io_in[s] = static_cast<float *>(h->alloc_bytes(maxb));
+    if (!h->io_out[s]) h->io_out[s] = static_cast<float *>(h->alloc_bytes(maxb * h->cfg.num_stems));
+    if (!h->io_in[s] || !h->io_out[s]) return fail(h, MRF_ENOMEM, "device allocation failed (io buffers)");
+  }
+  mrf_status st = MRF_OK;
+  if (!h->h2d_stream && !cuda_ok(h, cudaStreamCreateWithFlags(&h->h2d_stream, cudaStreamNonBlocking), "copy stream", &st)) return st;
+  if (!h->d2h_stream && !cuda_ok(h, cudaStreamCreateWithFlags(&h->d2h_stream, cudaStreamNonBlocking), "copy stream", &st)) return st;
+  cudaEvent_t *evs[7] = {&h->ev_in[0], &h->ev_in[1], &h->ev_fwd[0], &h->ev_fwd[1], &h->ev_out[0], &h->ev_out[1], &h->ev_join};
+  for (cudaEvent_t *e : evs)
+    if (!*e && !cuda_ok(h, cudaEventCreateWithFlags(e, cudaEventDisableTiming), "event", &st)) return st;
+  return MRF_OK;
+}
+
+// One call of the pipeline on slot io_next: H2D on h2d_stream after the forward that last read
+// the slot's input; the forward on `stream` after that copy and after the copy that last read the
+// slot's output; D2H on d2h_stream after the forward.  (Waiting on an event that was never
+// recorded returns at once, which covers a slot's first use.)
+mrf_status host_pipe_call(mrf_handle *h, const float *in_host, float *out_host, int B, int T, void *stream) {
   if (!h) return fail(nullptr, MRF_EINVAL, "null handle");
   if (!in_host || !out_host) return fail(h, MRF_EINVAL, "null host buffer");
   if (B < 1 || B > h->cfg.max_batch || T < 1 || T > h->cfg.max_frames)
     return fail(h, MRF_ESHAPE, "B or T outside [1, max_batch] x [1, max_frames]");
+  mrf_status s = host_pipe_init(h);
+  if (s != MRF_OK) return s;
   const size_t bytes = (size_t)B * h->tab.n_freqs * h->tab.channels * T * 2 * sizeof(float);
   const size_t out_bytes = bytes * h->cfg.num_stems;
-  mrf_status s = MRF_OK;
-  if (!h->io_in) {
-    const size_t maxb = (size_t)h->cfg.max_batch * h->tab.n_freqs * h->tab.channels * h->cfg.max_frames * 2 * sizeof(float);
-    h->io_in = static_cast<float *>(h->alloc_bytes(maxb));
-    h->io_out = static_cast<float *>(h->alloc_bytes(maxb * h->cfg.num_stems));
-    if (!h->io_in || !h->io_out) return fail(h, MRF_ENOMEM, "device allocation failed (io buffers)");
-  }
+  const int k = h->io_next;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (!cuda_ok(h, cudaMemcpyAsync(h->io_in, in_host, bytes, cudaMemcpyHostToDevice, st), "H2D copy", &s)) return s;
-  s = mrf_forward(h, h->io_in, h->io_out, B, T, stream);
+  if (!cuda_ok(h, cudaStreamWaitEvent(h->h2d_stream, h->ev_fwd[k], 0), "copy ordering", &s) ||
+      !cuda_ok(h, cudaMemcpyAsync(h->io_in[k], in_host, bytes, cudaMemcpyHostToDevice, h->h2d_stream), "H2D copy", &s) ||
+      !cuda_ok(h, cudaEventRecord(h->ev_in[k], h->h2d_stream), "copy ordering", &s) ||
+      !cuda_ok(h, cudaStreamWaitEvent(st, h->ev_in[k], 0), "copy ordering", &s) ||
+      !cuda_ok(h, cudaStreamWaitEvent(st, h->ev_out[k], 0), "copy ordering", &s))
+    return s;
+  s = mrf_forward(h, h->io_in[k], h->io_out[k], B, T, stream);
   if (s != MRF_OK) return s;
-  if (!cuda_ok(h, cudaMemcpyAsync(out_host, h->io_out, out_bytes, cudaMemcpyDeviceToHost, st), "D2H copy", &s)) return s;
-  if (!cuda_ok(h, cudaStreamSynchronize(st), "stream sync", &s)) return s;
+  if (!cuda_ok(h, cudaEventRecord(h->ev_fwd[k], st), "copy ordering", &s) ||
+      !cuda_ok(h, cudaStreamWaitEvent(h->d2h_stream, h->ev_fwd[k], 0), "copy ordering", &s) ||
+      !cuda_ok(h, cudaMemcpyAsync(out_host, h->io_out[k], out_bytes, cudaMemcpyDeviceToHost, h->d2h_stream), "D2H copy", &s) ||
+      !cuda_ok(h, cudaEventRecord(h->ev_out[k], h->d2h_stream), "copy ordering", &s))
+    return s;
+  h->io_next = k ^ 1;
+  return MRF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mrf_status mrf_forward_host_async(mrf_handle *h, const float *in_host, float *out_host, int B, int T, void *stream) {
+  return host_pipe_call(h, in_host, out_host, B, T, stream);
+}
+
+mrf_status mrf_host_join(mrf_handle *h, void *stream) {
+  if (!h) return fail(nullptr, MRF_EINVAL, "null handle");
+  if (!h->d2h_stream) return MRF_OK;
+  mrf_status s = MRF_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!cuda_ok(h, cudaEventRecord(h->ev_join, h->d2h_stream), "join", &s) ||
+      !cuda_ok(h, cudaStreamWaitEvent(st, h->ev_join, 0), "join", &s))
+    return s;
+  return MRF_OK;
+}
+
+mrf_status mrf_forward_host(mrf_handle *h, const float *in_host, float *out_host, int B, int T,
+                            void *stream) {
+  mrf_status s = host_pipe_call(h, in_host, out_host, B, T, stream);
+  if (s != MRF_OK) return s;
+  s = mrf_host_join(h, stream);
+  if (s != MRF_OK) return s;
   return mrf_sync_status(h, stream);
 }
 
@@ -628,6 +687,10 @@ void mrf_destroy(mrf_handle *h) {
   for (void *p : h->allocs) cudaFree(p);
   for (auto &p : h->sig_scratch) cudaFree(p.first);
   if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  for (cudaStream_t c : {h->h2d_stream, h->d2h_stream})
+    if (c) { cudaStreamSynchronize(c); cudaStreamDestroy(c); }
+  for (cudaEvent_t e : {h->ev_in[0], h->ev_in[1], h->ev_fwd[0], h->ev_fwd[1], h->ev_out[0], h->ev_out[1], h->ev_join})
+    if (e) cudaEventDestroy(e);
   destroy_fp16(h);
   delete h;
 }

@@ -102,7 +102,13 @@ struct mrf_handle {
   std::vector<mrf::GraphEntry> graphs;
   int launch_counter = 0, last_launches = -1, last_B = -1, last_T = -1;
   bool last_static = false;  // the last forward ran in mrf_forward_static's shared scratch
-  float *io_in = nullptr, *io_out = nullptr;
+  // host-buffer entry points: two device input/output slots used in turn, one copy stream
+  // per direction, and the events that order copies and forwards (mrf_api.cu, host_pipe)
+  float *io_in[2] = {nullptr, nullptr}, *io_out[2] = {nullptr, nullptr};
+  cudaStream_t h2d_stream = nullptr, d2h_stream = nullptr;
+  cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_fwd[2] = {nullptr, nullptr},
+              ev_out[2] = {nullptr, nullptr}, ev_join = nullptr;
+  int io_next = 0;
   // spectral front / back end (signal_api.cu): FFT tables of n_fft and grow-only scratch
   float2 *d_tw = nullptr;
   float *d_win = nullptr;

@@ -25,7 +25,7 @@ STATUS = {0: "MRF_OK", -1: "MRF_EINVAL", -2: "MRF_ESHAPE", -3: "MRF_ENOMEM", -4:
 
 # every symbol include/mrf.h declares
 EXPORTS = ["mrf_create", "mrf_forward", "mrf_forward_separate", "mrf_stft", "mrf_istft", "mrf_separate_audio",
-           "mrf_forward_host", "mrf_sync_status", "mrf_destroy",
+           "mrf_forward_host", "mrf_forward_host_async", "mrf_host_join", "mrf_sync_status", "mrf_destroy",
            "mrf_last_error", "mrf_band_tables", "mrf_set_timing", "mrf_kernel_times",
            "mrf_set_graph", "mrf_launches_per_forward", "mrf_debug_buffer", "mrf_forward_static",
            "mrf_debug_stall_next", "mrf_chunk_plan", "mrf_separate_audio_chunked"]
@@ -83,6 +83,10 @@ def lib():
         L.mrf_forward_static.restype = I
         L.mrf_forward_host.argtypes = [P, P, P, I, I, P]
         L.mrf_forward_host.restype = I
+        L.mrf_forward_host_async.argtypes = [P, P, P, I, I, P]
+        L.mrf_forward_host_async.restype = I
+        L.mrf_host_join.argtypes = [P, P]
+        L.mrf_host_join.restype = I
         L.mrf_sync_status.argtypes = [P, P]
         L.mrf_sync_status.restype = I
         L.mrf_destroy.argtypes = [P]
@@ -193,6 +197,7 @@ class Model:
         h = ctypes.c_void_p()
         _check(lib().mrf_create(ctypes.byref(c), table, len(weights), ctypes.byref(h)))
         self._h = h
+        self._host_pending = []  # (input, output) host tensors of forward_host_async calls not yet synced
 
     @property
     def handle(self):
@@ -315,8 +320,29 @@ class Model:
                                       B, T, _stream_ptr(stream)), self._h)
         return out
 
+    def forward_host_async(self, stft_repr, out, stream=None):
+        """enqueues H2D copy, forward and D2H copy of one host tensor and returns; `out` holds the
+        masks once host_join and a stream synchronize (or sync_status) have followed.  Both
+        tensors are kept referenced here until then; pin them for copies that overlap compute."""
+        import torch
+        x = stft_repr
+        assert not x.is_cuda and x.dtype == torch.float32 and x.is_contiguous(), "stft_repr: contiguous host float32"
+        assert x.dim() == 4 and x.shape[1] == self.rows and x.shape[3] == 2, \
+            f"stft_repr must be [B, {self.rows}, T, 2], got {tuple(x.shape)}"
+        self._check_out(x, out)
+        B, R, T, _ = x.shape
+        _check(lib().mrf_forward_host_async(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
+                                            ctypes.c_void_p(out.data_ptr()), B, T, _stream_ptr(stream)), self._h)
+        self._host_pending.append((stft_repr, out))
+        return out
+
+    def host_join(self, stream=None):
+        """makes `stream` wait for every copy forward_host_async enqueued (no host wait)."""
+        _check(lib().mrf_host_join(self._h, _stream_ptr(stream)), self._h)
+
     def sync_status(self, stream=None):
         _check(lib().mrf_sync_status(self._h, _stream_ptr(stream)), self._h)
+        self._host_pending = []
 
     def set_timing(self, on: bool):
         _check(lib().mrf_set_timing(self._h, int(on)), self._h)

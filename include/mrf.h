@@ -193,6 +193,41 @@ mrf_status mrf_forward_host(mrf_handle *h, const float *stft_repr_host, float *m
                             int B, int T, void *stream);
 
 /*
+ * mrf_forward_host_async - mrf_forward_host without the wait, for a caller that feeds a
+ * stream of inputs from host memory (a file or a live source cut into windows): each call
+ * enqueues the host-to-device copy of stft_repr_host, the forward and the device-to-host copy
+ * of the masks, and returns.  Copies run on two streams of the handle's own (one per
+ * direction) and the forward on `stream`; the handle keeps two device input/output slots that
+ * calls use in turn, so call k+1's input copy and call k-1's output copy run while call k
+ * computes.  Events order the three: a slot's input is overwritten only after the forward that
+ * read it ended, and its output only after its copy to the host ended.  (The pages have no
+ * counterpart: this is an integration entry point, not a step of the method.)
+ *
+ * Shapes and layouts as for mrf_forward_host.  Ownership: the caller keeps both host buffers
+ * alive and unchanged (stft_repr_host) and unread (masks_host) until mrf_host_join's wait has
+ * returned; stft_repr_host must hold its data when the call is made, since its copy may start
+ * before work enqueued earlier on `stream` has run.  For copies that overlap compute both
+ * buffers must be pinned (cudaHostAlloc / torch pin_memory): a pageable output buffer makes the
+ * copy wait for its forward inside the call.  Not for use while `stream` is being captured.
+ * Errors: MRF_EINVAL / MRF_ESHAPE for bad arguments (nothing enqueued), MRF_ECUDA if a copy or
+ * the forward could not be enqueued; a device-side expired wait surfaces at mrf_sync_status.
+ */
+mrf_status mrf_forward_host_async(mrf_handle *h, const float *stft_repr_host, float *masks_host,
+                                  int B, int T, void *stream);
+
+/*
+ * mrf_host_join - makes `stream` wait (on the device; the host does not block) until every
+ * copy that mrf_forward_host_async has enqueued so far has ended.  After it, a
+ * cudaStreamSynchronize of `stream` (or mrf_sync_status, which does one and checks the status
+ * word) means every masks_host buffer of those calls holds its result.  Work enqueued on
+ * `stream` after the join is ordered after those copies, so CUDA events recorded on `stream`
+ * around a batch of calls and the join time the whole pipeline, copies included.  A join with
+ * no call pending does nothing.  Errors: MRF_EINVAL for a null handle, MRF_ECUDA if the wait
+ * could not be enqueued.
+ */
+mrf_status mrf_host_join(mrf_handle *h, void *stream);
+
+/*
  * mrf_forward_static - the same fp16 forward as mrf_forward, for callers that must not
  * allocate device memory while they run the model: a real-time audio callback that may not
  * block in the allocator, or a host framework that owns every device allocation and
