@@ -221,6 +221,13 @@ class Model:
         assert x.dim() == 4 and x.shape[1] == self.rows and x.shape[3] == 2, \
             f"stft_repr must be [B, {self.rows}, T, 2], got {tuple(x.shape)}"
 
+    def _check_host_input(self, x):
+        """stft_repr for the host-buffer entry points: a contiguous host float32 [B, F*C, T, 2]."""
+        import torch
+        assert not x.is_cuda and x.dtype == torch.float32 and x.is_contiguous(), "stft_repr: contiguous host float32"
+        assert x.dim() == 4 and x.shape[1] == self.rows and x.shape[3] == 2, \
+            f"stft_repr must be [B, {self.rows}, T, 2], got {tuple(x.shape)}"
+
     def _check_out(self, x, out):
         """`out` must hold exactly B * num_stems * rows * T * 2 floats, on x's device."""
         import torch
@@ -314,6 +321,7 @@ class Model:
         """masks for a host float32 array/tensor, copies inside the call; waits for the stream."""
         import torch
         x = stft_repr if isinstance(stft_repr, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(stft_repr))
+        self._check_host_input(x)
         B, R, T, _ = x.shape
         out = self._out_like(x, out)
         _check(lib().mrf_forward_host(self._h, ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(out.data_ptr()),
@@ -324,11 +332,8 @@ class Model:
         """enqueues H2D copy, forward and D2H copy of one host tensor and returns; `out` holds the
         masks once host_join and a stream synchronize (or sync_status) have followed.  Both
         tensors are kept referenced here until then; pin them for copies that overlap compute."""
-        import torch
         x = stft_repr
-        assert not x.is_cuda and x.dtype == torch.float32 and x.is_contiguous(), "stft_repr: contiguous host float32"
-        assert x.dim() == 4 and x.shape[1] == self.rows and x.shape[3] == 2, \
-            f"stft_repr must be [B, {self.rows}, T, 2], got {tuple(x.shape)}"
+        self._check_host_input(x)
         self._check_out(x, out)
         B, R, T, _ = x.shape
         _check(lib().mrf_forward_host_async(self._h, ctypes.c_void_p(stft_repr.data_ptr()),
