@@ -599,16 +599,18 @@ mrf_status host_pipe_init(mrf_handle *h) {
   mrf_status st = MRF_OK;
   if (!h->h2d_stream && !cuda_ok(h, cudaStreamCreateWithFlags(&h->h2d_stream, cudaStreamNonBlocking), "copy stream", &st)) return st;
   if (!h->d2h_stream && !cuda_ok(h, cudaStreamCreateWithFlags(&h->d2h_stream, cudaStreamNonBlocking), "copy stream", &st)) return st;
-  cudaEvent_t *evs[7] = {&h->ev_in[0], &h->ev_in[1], &h->ev_fwd[0], &h->ev_fwd[1], &h->ev_out[0], &h->ev_out[1], &h->ev_join};
+  cudaEvent_t *evs[8] = {&h->ev_in[0], &h->ev_in[1], &h->ev_fwd[0], &h->ev_fwd[1],
+                         &h->ev_out[0], &h->ev_out[1], &h->ev_join, &h->ev_start};
   for (cudaEvent_t *e : evs)
     if (!*e && !cuda_ok(h, cudaEventCreateWithFlags(e, cudaEventDisableTiming), "event", &st)) return st;
   return MRF_OK;
 }
 
 // One call of the pipeline on slot io_next: H2D on h2d_stream after the forward that last read
-// the slot's input; the forward on `stream` after that copy and after the copy that last read the
-// slot's output; D2H on d2h_stream after the forward.  (Waiting on an event that was never
-// recorded returns at once, which covers a slot's first use.)
+// the slot's input (and, for the first call of a batch, after the work already on `stream`); the
+// forward on `stream` after that copy and after the copy that last read the slot's output; D2H on
+// d2h_stream after the forward.  (Waiting on an event that was never recorded returns at once,
+// which covers a slot's first use.)
 mrf_status host_pipe_call(mrf_handle *h, const float *in_host, float *out_host, int B, int T, void *stream) {
   if (!h) return fail(nullptr, MRF_EINVAL, "null handle");
   if (!in_host || !out_host) return fail(h, MRF_EINVAL, "null host buffer");
@@ -620,6 +622,12 @@ mrf_status host_pipe_call(mrf_handle *h, const float *in_host, float *out_host, 
   const size_t out_bytes = bytes * h->cfg.num_stems;
   const int k = h->io_next;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!h->pipe_open) {  // a batch begins: its first copy follows what the caller enqueued before it
+    if (!cuda_ok(h, cudaEventRecord(h->ev_start, st), "copy ordering", &s) ||
+        !cuda_ok(h, cudaStreamWaitEvent(h->h2d_stream, h->ev_start, 0), "copy ordering", &s))
+      return s;
+    h->pipe_open = true;
+  }
   if (!cuda_ok(h, cudaStreamWaitEvent(h->h2d_stream, h->ev_fwd[k], 0), "copy ordering", &s) ||
       !cuda_ok(h, cudaMemcpyAsync(h->io_in[k], in_host, bytes, cudaMemcpyHostToDevice, h->h2d_stream), "H2D copy", &s) ||
       !cuda_ok(h, cudaEventRecord(h->ev_in[k], h->h2d_stream), "copy ordering", &s) ||
@@ -653,6 +661,7 @@ mrf_status mrf_host_join(mrf_handle *h, void *stream) {
   if (!cuda_ok(h, cudaEventRecord(h->ev_join, h->d2h_stream), "join", &s) ||
       !cuda_ok(h, cudaStreamWaitEvent(st, h->ev_join, 0), "join", &s))
     return s;
+  h->pipe_open = false;
   return MRF_OK;
 }
 
@@ -689,7 +698,8 @@ void mrf_destroy(mrf_handle *h) {
   if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
   for (cudaStream_t c : {h->h2d_stream, h->d2h_stream})
     if (c) { cudaStreamSynchronize(c); cudaStreamDestroy(c); }
-  for (cudaEvent_t e : {h->ev_in[0], h->ev_in[1], h->ev_fwd[0], h->ev_fwd[1], h->ev_out[0], h->ev_out[1], h->ev_join})
+  for (cudaEvent_t e : {h->ev_in[0], h->ev_in[1], h->ev_fwd[0], h->ev_fwd[1], h->ev_out[0], h->ev_out[1], h->ev_join,
+                        h->ev_start})
     if (e) cudaEventDestroy(e);
   destroy_fp16(h);
   delete h;

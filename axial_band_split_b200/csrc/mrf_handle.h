@@ -107,8 +107,9 @@ struct mrf_handle {
   float *io_in[2] = {nullptr, nullptr}, *io_out[2] = {nullptr, nullptr};
   cudaStream_t h2d_stream = nullptr, d2h_stream = nullptr;
   cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_fwd[2] = {nullptr, nullptr},
-              ev_out[2] = {nullptr, nullptr}, ev_join = nullptr;
+              ev_out[2] = {nullptr, nullptr}, ev_join = nullptr, ev_start = nullptr;
   int io_next = 0;
+  bool pipe_open = false;  // a batch of host-buffer calls has begun and not been joined
   // spectral front / back end (signal_api.cu): FFT tables of n_fft and grow-only scratch
   float2 *d_tw = nullptr;
   float *d_win = nullptr;

@@ -351,41 +351,49 @@ def run_ours(args):
     audio_per_rank = args.steps * accounting.audio_seconds(cfg, B, T)
     value = aggregate(audio_per_rank, world, ms_max)
 
+    # end to end through the public host-buffer entry points, from and to pinned host memory.
+    # Pipelined (mrf_forward_host_async + mrf_host_join): one event pair around all K calls and the
+    # join, so the region holds every step's H2D copy, forward, D2H copy and L2 flush; the copies
+    # of neighbouring steps run under each forward (a batch's first copy follows the start event).
+    # Synchronous (mrf_forward_host, which waits for its own copies): an event pair around each
+    # call, summed, as for `value`.
+    # `region` times the same K device-buffer forwards under one event pair with the same flushes:
+    # the pipelined figure's reference without copies.
+    xin = torch.from_numpy(x_host).pin_memory()
+    xouts = [model._out_like(xin, None) for _ in range(2)]
+
+    def one_region(steps, host):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record(stream)
+        for k in range(steps):
+            flush.zero_()
+            if host:
+                model.forward_host_async(xin, xouts[k % 2], stream=stream)
+            else:
+                fwd()
+        if host:
+            model.host_join(stream)
+        e1.record(stream)
+        barrier()
+        model.sync_status(stream)
+        return e0.elapsed_time(e1)
+
+    one_region(args.warmup, True)
+    ms_e2e = ranks.max(one_region(args.steps, True))
+    ms_region = ranks.max(one_region(args.steps, False))
+    sync_fn = lambda: model.forward_host(xin, xouts[0], stream=stream)
+    sync_fn()
+    ms_e2e_sync = ranks.max(timed(sync_fn, args.steps))
+    io_bytes = int(x_host.nbytes)
+    out_bytes = int(xouts[0].numel() * 4)
+
     # per-kernel times: the same steps launched eagerly with an event pair around each kernel
     model.set_timing(True)
     ktimed = timed(fwd, args.steps)
     kt = model.kernel_times()
     model.set_timing(False)
     model.sync_status()
-
-    # end to end through the public host-buffer entry points, from and to pinned host memory.
-    # Pipelined (mrf_forward_host_async + mrf_host_join): one event pair around all K calls and the
-    # join, so the region holds every step's H2D copy, forward, D2H copy and L2 flush; the copies
-    # of neighbouring steps run under each forward.  Synchronous (mrf_forward_host, which waits
-    # for its own copies): an event pair around each call, summed, as for `value`.
-    xin = torch.from_numpy(x_host).pin_memory()
-    xouts = [model._out_like(xin, None) for _ in range(2)]
-    sync_fn = lambda: model.forward_host(xin, xouts[0], stream=stream)
-    sync_fn()
-    ms_e2e_sync = ranks.max(timed(sync_fn, args.steps))
-
-    def pipelined(steps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
-        e0.record(stream)
-        for k in range(steps):
-            flush.zero_()
-            model.forward_host_async(xin, xouts[k % 2], stream=stream)
-        model.host_join(stream)
-        e1.record(stream)
-        barrier()
-        model.sync_status(stream)
-        return e0.elapsed_time(e1)
-
-    pipelined(args.warmup)
-    ms_e2e = ranks.max(pipelined(args.steps))
-    io_bytes = int(x_host.nbytes)
-    out_bytes = int(xouts[0].numel() * 4)
 
     # the same workload in the bf16 compute mode (weights rounded to bf16), device-timed like `value`
     bf_line = None
@@ -466,6 +474,9 @@ def run_ours(args):
                 "ms_per_step": ms_e2e / args.steps,
                 "api": "mrf_forward_host_async x K + mrf_host_join, pinned host buffers, one event pair "
                        "around the K steps (copies, forwards and the per-step L2 flush inside)",
+                "device_region_ms_per_step": ms_region / args.steps,
+                "device_region_note": "the same K forwards from device buffers under one event pair with the same "
+                                      "flushes: the pipelined figure without its copies",
                 "sync_call": {"value": aggregate(audio_per_rank, world, ms_e2e_sync),
                               "ms_per_step": ms_e2e_sync / args.steps,
                               "api": "mrf_forward_host (waits for its copies), event pair per call"}},

@@ -205,8 +205,11 @@ mrf_status mrf_forward_host(mrf_handle *h, const float *stft_repr_host, float *m
  *
  * Shapes and layouts as for mrf_forward_host.  Ownership: the caller keeps both host buffers
  * alive and unchanged (stft_repr_host) and unread (masks_host) until mrf_host_join's wait has
- * returned; stft_repr_host must hold its data when the call is made, since its copy may start
- * before work enqueued earlier on `stream` has run.  For copies that overlap compute both
+ * returned.  Calls between two joins form a batch: the batch's first copy starts after the work
+ * enqueued on `stream` before that call (so CUDA events recorded on `stream` before the batch and
+ * after its join bracket every copy); a later call's copy starts as soon as its slot is free,
+ * possibly before work enqueued on `stream` since the batch began has run, so stft_repr_host must
+ * hold its data when the call is made.  For copies that overlap compute both
  * buffers must be pinned (cudaHostAlloc / torch pin_memory): a pageable output buffer makes the
  * copy wait for its forward inside the call.  Not for use while `stream` is being captured.
  * Errors: MRF_EINVAL / MRF_ESHAPE for bad arguments (nothing enqueued), MRF_ECUDA if a copy or
@@ -217,7 +220,8 @@ mrf_status mrf_forward_host_async(mrf_handle *h, const float *stft_repr_host, fl
 
 /*
  * mrf_host_join - makes `stream` wait (on the device; the host does not block) until every
- * copy that mrf_forward_host_async has enqueued so far has ended.  After it, a
+ * copy that mrf_forward_host_async has enqueued so far has ended, and closes the batch (the
+ * next call's copy again follows the work on its stream).  After it, a
  * cudaStreamSynchronize of `stream` (or mrf_sync_status, which does one and checks the status
  * word) means every masks_host buffer of those calls holds its result.  Work enqueued on
  * `stream` after the join is ordered after those copies, so CUDA events recorded on `stream`

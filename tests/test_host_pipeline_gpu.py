@@ -7,7 +7,8 @@ the same input copied by hand (the same kernels run on the same bytes), and one 
 the fp16 parity bar against the oracle.  Cases: more calls than slots with a different input
 each (a slot overwritten before its predecessor's output was read would show up as another
 call's masks), a pageable output buffer, a synchronous call between asynchronous ones, a join
-with nothing pending, and a smaller (B, T) after a larger one in the same slot."""
+with nothing pending, a smaller (B, T) after a larger one in the same slot, and a batch whose
+input buffer is filled by work queued on its stream just before it."""
 import numpy as np
 import pytest
 
@@ -82,4 +83,32 @@ def test_small_window_in_pipeline():
     m.host_join(stream)
     m.sync_status(stream)
     assert np.array_equal(osh.numpy(), want)
+    m.close()
+
+
+@pytest.mark.parametrize("sync", [False, True])
+def test_batch_copy_follows_stream_work(sync):
+    """The first call of a batch copies its input only after the work already on its stream: the
+    input buffer is filled by a device-to-host copy queued behind a ~25 ms sleep kernel, and the
+    masks must be those of the new input, not of the zeros the buffer held before."""
+    cfg = synth.TINY
+    B, T = 2, 17
+    W, _ = case(cfg, B, T, True)
+    m = model_for(cfg, W, B, T)
+    x1 = synth.make_stft_repr(cfg, B, T, seed=31)
+    want = device_masks(m, x1)
+    stream = torch.cuda.current_stream()
+    xin = torch.zeros(x1.shape).pin_memory()
+    out = m._out_like(xin, None)
+    xd = torch.from_numpy(x1).cuda()
+    torch.cuda.synchronize()
+    torch.cuda._sleep(50_000_000)
+    xin.copy_(xd, non_blocking=True)
+    if sync:
+        m.forward_host(xin, out, stream=stream)
+    else:
+        m.forward_host_async(xin, out, stream=stream)
+        m.host_join(stream)
+        m.sync_status(stream)
+    assert np.array_equal(out.numpy(), want)
     m.close()
